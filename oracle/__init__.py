@@ -1,0 +1,206 @@
+"""fp64 CPU oracle for the SSA sparse stream -- TEST INFRASTRUCTURE.
+
+Only the tests, the smoke check and the bench's CPU-baseline leg may import
+this package.  It shares no code with the CUDA library: the arithmetic lives
+in ssa_oracle.c (plain C, fp64, pthreads); this module only widens bf16
+tensors exactly to fp64 and marshals numpy arrays through ctypes.
+
+Functions (each cites the passage it follows in ssa_oracle.c):
+  block_pool      mean of each 64-token key block; GQA-group mean of the queries
+  block_select    diagonal + top-(k-1) earlier blocks by pooled score
+  attn_rows       sparse output/LSE and, on request, full causal output/LSE and
+                  dropped mass (two routes) for a list of query rows
+  sparse_bwd_dq_rows / sparse_bwd_dkv_blocks
+                  gradient of the sparse output, by the explicit formulas
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Optional
+
+import numpy as np
+
+from . import build as _build
+
+BLOCK = 64
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        dp = ctypes.POINTER(ctypes.c_double)
+        ip = ctypes.POINTER(ctypes.c_int32)
+        lp = ctypes.POINTER(ctypes.c_int64)
+        c_int, c_dbl, c_i64 = ctypes.c_int, ctypes.c_double, ctypes.c_int64
+        lib.ora_block_pool.argtypes = [c_int] * 6 + [dp, dp, dp, dp, c_int]
+        lib.ora_block_select.argtypes = [c_int] * 5 + [dp, dp, ip, dp, c_int]
+        lib.ora_attn_rows.argtypes = ([c_int] * 7 + [c_dbl, dp, dp, dp, ip, c_i64, lp, c_int]
+                                      + [dp] * 6 + [c_int])
+        lib.ora_sparse_bwd_dq_rows.argtypes = ([c_int] * 7 + [c_dbl, dp, dp, dp, dp, ip, c_i64,
+                                                              lp, dp, c_int])
+        lib.ora_sparse_bwd_dkv_blocks.argtypes = ([c_int] * 7 + [c_dbl, dp, dp, dp, dp, ip,
+                                                                 c_i64, lp, dp, dp, c_int])
+        for f in (lib.ora_block_pool, lib.ora_block_select, lib.ora_attn_rows,
+                  lib.ora_sparse_bwd_dq_rows, lib.ora_sparse_bwd_dkv_blocks):
+            f.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def default_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def _ptr(a: Optional[np.ndarray], ctype):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+def widen(x) -> np.ndarray:
+    """Exact bf16 -> fp64 widening (a torch bf16 tensor, or fp64/fp32 array as is)."""
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            if x.dtype == torch.bfloat16:
+                bits = x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+                return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+            return x.detach().cpu().numpy().astype(np.float64)
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def _f64(x) -> np.ndarray:
+    return np.ascontiguousarray(widen(x), dtype=np.float64)
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise ValueError(f"oracle {what} rejected its arguments (rc={rc})")
+
+
+def block_pool(k, q=None, bs: int = BLOCK, nthreads: Optional[int] = None):
+    """K-bar [B,Hkv,n,D] and, if q is given, group-pooled Q-bar [B,Hkv,n,D] (fp64)."""
+    k64 = _f64(k)
+    B, S, Hkv, D = k64.shape
+    q64 = _f64(q) if q is not None else None
+    Hq = q64.shape[2] if q64 is not None else Hkv
+    n = S // bs
+    kbar = np.zeros((B, Hkv, n, D))
+    qbar = np.zeros((B, Hkv, n, D)) if q64 is not None else None
+    rc = _load().ora_block_pool(B, S, Hq, Hkv, D, bs, _ptr(k64, ctypes.c_double),
+                                _ptr(q64, ctypes.c_double), _ptr(kbar, ctypes.c_double),
+                                _ptr(qbar, ctypes.c_double), nthreads or default_threads())
+    _check(rc, "block_pool")
+    return kbar, qbar
+
+
+def block_select(qbar: np.ndarray, kbar: np.ndarray, topk: int, nthreads: Optional[int] = None):
+    """idx [B,Hkv,n,topk] int32 ascending (-1 padded) and gap [B,Hkv,n] (NaN = no boundary)."""
+    qbar = np.ascontiguousarray(qbar, dtype=np.float64)
+    kbar = np.ascontiguousarray(kbar, dtype=np.float64)
+    B, Hkv, n, D = kbar.shape
+    idx = np.zeros((B, Hkv, n, topk), dtype=np.int32)
+    gap = np.zeros((B, Hkv, n))
+    rc = _load().ora_block_select(B, Hkv, n, D, topk, _ptr(qbar, ctypes.c_double),
+                                  _ptr(kbar, ctypes.c_double), _ptr(idx, ctypes.c_int32),
+                                  _ptr(gap, ctypes.c_double), nthreads or default_threads())
+    _check(rc, "block_select")
+    return idx, gap
+
+
+def all_rows(B: int, Hq: int, S: int) -> np.ndarray:
+    """Every (b, hq, t) triple, in that nesting order."""
+    b, h, t = np.meshgrid(np.arange(B), np.arange(Hq), np.arange(S), indexing="ij")
+    return np.stack([b.ravel(), h.ravel(), t.ravel()], axis=1).astype(np.int64)
+
+
+def attn_rows(q, k, v, idx: np.ndarray, rows: np.ndarray, scale: Optional[float] = None,
+              want_full: bool = True, bs: int = BLOCK, nthreads: Optional[int] = None
+              ) -> Dict[str, np.ndarray]:
+    """Per listed query row: sparse O/LSE and (want_full) full O/LSE and dropped mass."""
+    q64, k64, v64 = _f64(q), _f64(k), _f64(v)
+    B, S, Hq, D = q64.shape
+    Hkv = k64.shape[2]
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    topk = idx.shape[-1]
+    rows = np.ascontiguousarray(rows, dtype=np.int64).reshape(-1, 3)
+    R = rows.shape[0]
+    scale = (1.0 / np.sqrt(D)) if scale is None else float(scale)
+    out = {"o_sparse": np.zeros((R, D)), "lse_sparse": np.zeros(R)}
+    if want_full:
+        out.update(o_full=np.zeros((R, D)), lse_full=np.zeros(R), delta=np.zeros(R),
+                   delta_lse=np.zeros(R))
+    g = out.get
+    rc = _load().ora_attn_rows(
+        B, S, Hq, Hkv, D, bs, topk, scale, _ptr(q64, ctypes.c_double), _ptr(k64, ctypes.c_double),
+        _ptr(v64, ctypes.c_double), _ptr(idx, ctypes.c_int32), R, _ptr(rows, ctypes.c_int64),
+        1 if want_full else 0, _ptr(out["o_sparse"], ctypes.c_double),
+        _ptr(out["lse_sparse"], ctypes.c_double), _ptr(g("o_full"), ctypes.c_double),
+        _ptr(g("lse_full"), ctypes.c_double), _ptr(g("delta"), ctypes.c_double),
+        _ptr(g("delta_lse"), ctypes.c_double), nthreads or default_threads())
+    _check(rc, "attn_rows")
+    return out
+
+
+def sparse_bwd_dq_rows(q, k, v, do, idx: np.ndarray, rows: np.ndarray,
+                       scale: Optional[float] = None, bs: int = BLOCK,
+                       nthreads: Optional[int] = None) -> np.ndarray:
+    """dQ [R, D] for the listed (b, hq, t) rows."""
+    q64, k64, v64, do64 = _f64(q), _f64(k), _f64(v), _f64(do)
+    B, S, Hq, D = q64.shape
+    Hkv = k64.shape[2]
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    rows = np.ascontiguousarray(rows, dtype=np.int64).reshape(-1, 3)
+    scale = (1.0 / np.sqrt(D)) if scale is None else float(scale)
+    dq = np.zeros((rows.shape[0], D))
+    rc = _load().ora_sparse_bwd_dq_rows(
+        B, S, Hq, Hkv, D, bs, idx.shape[-1], scale, _ptr(q64, ctypes.c_double),
+        _ptr(k64, ctypes.c_double), _ptr(v64, ctypes.c_double), _ptr(do64, ctypes.c_double),
+        _ptr(idx, ctypes.c_int32), rows.shape[0], _ptr(rows, ctypes.c_int64),
+        _ptr(dq, ctypes.c_double), nthreads or default_threads())
+    _check(rc, "sparse_bwd_dq_rows")
+    return dq
+
+
+def sparse_bwd_dkv_blocks(q, k, v, do, idx: np.ndarray, blocks: np.ndarray,
+                          scale: Optional[float] = None, bs: int = BLOCK,
+                          nthreads: Optional[int] = None):
+    """dK, dV [NB, bs, D] for the listed (b, kvh, key block j) triples."""
+    q64, k64, v64, do64 = _f64(q), _f64(k), _f64(v), _f64(do)
+    B, S, Hq, D = q64.shape
+    Hkv = k64.shape[2]
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    blocks = np.ascontiguousarray(blocks, dtype=np.int64).reshape(-1, 3)
+    scale = (1.0 / np.sqrt(D)) if scale is None else float(scale)
+    dk = np.zeros((blocks.shape[0], bs, D))
+    dv = np.zeros((blocks.shape[0], bs, D))
+    rc = _load().ora_sparse_bwd_dkv_blocks(
+        B, S, Hq, Hkv, D, bs, idx.shape[-1], scale, _ptr(q64, ctypes.c_double),
+        _ptr(k64, ctypes.c_double), _ptr(v64, ctypes.c_double), _ptr(do64, ctypes.c_double),
+        _ptr(idx, ctypes.c_int32), blocks.shape[0], _ptr(blocks, ctypes.c_int64),
+        _ptr(dk, ctypes.c_double), _ptr(dv, ctypes.c_double), nthreads or default_threads())
+    _check(rc, "sparse_bwd_dkv_blocks")
+    return dk, dv
+
+
+def sparse_forward_problem(q, k, v, topk: int, rows: Optional[np.ndarray] = None,
+                           want_full: bool = False, nthreads: Optional[int] = None):
+    """Pool -> select -> attention rows for a whole problem (or a row sample)."""
+    kbar, qbar = block_pool(k, q, nthreads=nthreads)
+    idx, gap = block_select(qbar, kbar, topk, nthreads=nthreads)
+    if rows is None:
+        B, S, Hq, _ = tuple(q.shape)
+        rows = all_rows(B, Hq, S)
+    out = attn_rows(q, k, v, idx, rows, want_full=want_full, nthreads=nthreads)
+    out.update(idx=idx, gap=gap, kbar=kbar, qbar=qbar, rows=rows)
+    return out

@@ -1,0 +1,345 @@
+"""Pins the fp64 oracle to things other than itself.
+
+Each test checks the oracle against a closed form, a brute-force enumeration,
+an independent library routine (torch float64 SDPA / autograd), a finite
+difference, or an invariant the method fixes.  Chosen so that a dropped term,
+a wrong sign or index, or a transposed operand in the oracle fails one of them.
+"""
+import itertools
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import gen
+import oracle
+
+BS = 64
+
+
+def _rand(shape, seed):
+    return np.random.Generator(np.random.PCG64(seed)).standard_normal(shape)
+
+
+def _tiny(B=1, S=256, Hq=4, Hkv=2, D=8, seed=0):
+    q = _rand((B, S, Hq, D), seed)
+    k = _rand((B, S, Hkv, D), seed + 1)
+    v = _rand((B, S, Hkv, D), seed + 2)
+    return q, k, v
+
+
+def _mask_from_idx(idx, b, h, S, complement=False):
+    """Boolean [S, S] attention mask (True = attend) built from a block table."""
+    n = S // BS
+    blk = np.zeros((n, n), dtype=bool)
+    for i in range(n):
+        for j in idx[b, h, i]:
+            if j >= 0:
+                blk[i, j] = True
+    tok = np.repeat(np.repeat(blk, BS, axis=0), BS, axis=1)
+    causal = np.tril(np.ones((S, S), dtype=bool))
+    return (causal & ~tok) if complement else (causal & tok)
+
+
+def _sdpa_rows(q, k, v, mask_fn):
+    """torch float64 SDPA per (b, hq) with an explicit boolean mask -> [B, Hq, S, D]."""
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    G = Hq // Hkv
+    out = np.zeros((B, Hq, S, D))
+    for b in range(B):
+        for hq in range(Hq):
+            h = hq // G
+            m = torch.from_numpy(mask_fn(b, h))
+            qt = torch.from_numpy(q[b, :, hq, :])[None]
+            kt = torch.from_numpy(k[b, :, h, :])[None]
+            vt = torch.from_numpy(v[b, :, h, :])[None]
+            o = F.scaled_dot_product_attention(qt, kt, vt, attn_mask=m[None])
+            out[b, hq] = o[0].numpy()
+    return out
+
+
+def _as_bhsd(flat, B, Hq, S, D):
+    return flat.reshape(B, Hq, S, D)
+
+
+# ------------------------------------------------------------------ pooling
+
+def test_pool_is_the_block_mean():
+    x = gen.make_inputs("tiny_1k")
+    kbar, qbar = oracle.block_pool(x.k, x.q)
+    k = oracle.widen(x.k)
+    q = oracle.widen(x.q)
+    B, S, Hkv, D = k.shape
+    G = q.shape[2] // Hkv
+    n = S // BS
+    ref_k = k.reshape(B, n, BS, Hkv, D).mean(axis=2).transpose(0, 2, 1, 3)
+    ref_q = q.reshape(B, n, BS, Hkv, G, D).mean(axis=(2, 4)).transpose(0, 2, 1, 3)
+    np.testing.assert_allclose(kbar, ref_k, rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(qbar, ref_q, rtol=1e-13, atol=1e-15)
+
+
+def test_group_pooled_score_equals_mean_of_per_head_scores():
+    # linearity: (mean_g qbar_g) . kbar == mean_g (qbar_g . kbar)
+    q, k, _ = _tiny(Hq=4, Hkv=1, D=8, seed=7)
+    kbar, qbar = oracle.block_pool(k, q)
+    per_head = [oracle.block_pool(k, q[:, :, g:g + 1, :])[1] for g in range(4)]
+    s_group = np.einsum("bhid,bhjd->bhij", qbar, kbar)
+    s_mean = np.mean([np.einsum("bhid,bhjd->bhij", p, kbar) for p in per_head], axis=0)
+    np.testing.assert_allclose(s_group, s_mean, rtol=1e-12, atol=1e-14)
+
+
+# ---------------------------------------------------------------- selection
+
+@pytest.mark.parametrize("topk", [1, 2, 3, 4, 9])
+def test_select_matches_brute_force_subsets(topk):
+    n, D = 9, 5
+    qbar = _rand((1, 2, n, D), 11)
+    kbar = _rand((1, 2, n, D), 12)
+    idx, gap = oracle.block_select(qbar, kbar, topk)
+    for h in range(2):
+        for i in range(n):
+            m = min(topk - 1, i)
+            best, best_sum = None, -np.inf
+            for sub in itertools.combinations(range(i), m):
+                s = sum(float(qbar[0, h, i] @ kbar[0, h, j]) for j in sub)
+                if s > best_sum:
+                    best, best_sum = sub, s
+            want = sorted(set(best) | {i})
+            got = [int(j) for j in idx[0, h, i] if j >= 0]
+            assert got == want, (h, i, got, want)
+            assert list(idx[0, h, i][len(want):]) == [-1] * (topk - len(want))
+            if topk >= 2 and i > topk - 1:
+                assert gap[0, h, i] >= 0.0
+            else:
+                assert np.isnan(gap[0, h, i])
+
+
+def test_select_tie_goes_to_lower_block_index():
+    D = 4
+    kbar = np.zeros((1, 1, 5, D))
+    kbar[0, 0, :, 0] = [1.0, 2.0, 2.0, 1.0, 0.0]   # blocks 1 and 2 tie, 0 and 3 tie
+    qbar = np.zeros((1, 1, 5, D))
+    qbar[0, 0, :, 0] = 1.0
+    idx, _ = oracle.block_select(qbar, kbar, 3)
+    assert list(idx[0, 0, 4]) == [1, 2, 4]
+    idx, _ = oracle.block_select(qbar, kbar, 4)
+    assert list(idx[0, 0, 4]) == [0, 1, 2, 4]
+
+
+def test_select_nests_in_k_and_full_budget_takes_every_causal_block():
+    x = gen.make_inputs("tiny_1k")
+    kbar, qbar = oracle.block_pool(x.k, x.q)
+    n = kbar.shape[2]
+    prev = None
+    for topk in range(1, n + 2):
+        idx, _ = oracle.block_select(qbar, kbar, topk)
+        sets = [[set(int(j) for j in idx[0, 0, i] if j >= 0) for i in range(n)]]
+        for i in range(n):
+            assert i in sets[0][i]
+            assert len(sets[0][i]) == min(topk, i + 1)
+            if prev is not None:
+                assert prev[0][i] <= sets[0][i]
+        prev = sets
+    for i in range(n):
+        assert prev[0][i] == set(range(i + 1))
+
+
+def test_select_finds_exaggerated_plants():
+    # wide head dim so that cross-talk between random directions (std ~ shift*sqrt(3/D))
+    # stays far below the planted score (~ shift)
+    x = gen.make_custom(1, 1024, 4, 2, 512, 4, seed=5, n_plant=3, plant_shift=10.0)
+    kbar, qbar = oracle.block_pool(x.k, x.q)
+    idx, _ = oracle.block_select(qbar, kbar, 4)
+    n = 1024 // BS
+    for h in range(2):
+        for i in range(4, n):
+            got = set(int(j) for j in idx[0, h, i] if j >= 0)
+            assert got == set(x.plants[(0, h, i)]) | {i}
+
+
+# ---------------------------------------------------------------- attention
+
+def test_full_budget_equals_dense_causal_sdpa():
+    q, k, v = _tiny(B=2, S=256, Hq=4, Hkv=2, D=16, seed=3)
+    out = oracle.sparse_forward_problem(q, k, v, topk=4, want_full=True)
+    B, S, Hq, D = q.shape
+    qt = torch.from_numpy(q).permute(0, 2, 1, 3)
+    kt = torch.from_numpy(k).permute(0, 2, 1, 3).repeat_interleave(2, dim=1)
+    vt = torch.from_numpy(v).permute(0, 2, 1, 3).repeat_interleave(2, dim=1)
+    ref = F.scaled_dot_product_attention(qt, kt, vt, is_causal=True).numpy()
+    np.testing.assert_allclose(_as_bhsd(out["o_sparse"], B, Hq, S, D), ref, atol=1e-12)
+    np.testing.assert_allclose(_as_bhsd(out["o_full"], B, Hq, S, D), ref, atol=1e-12)
+    assert np.all(out["delta"] == 0.0)
+    np.testing.assert_allclose(out["lse_sparse"], out["lse_full"], atol=1e-12)
+
+
+@pytest.mark.parametrize("topk", [1, 2, 3])
+def test_sparse_output_equals_masked_sdpa(topk):
+    q, k, v = _tiny(B=1, S=320, Hq=4, Hkv=2, D=16, seed=5)
+    out = oracle.sparse_forward_problem(q, k, v, topk=topk, want_full=True)
+    B, S, Hq, D = q.shape
+    idx = out["idx"]
+    ref = _sdpa_rows(q, k, v, lambda b, h: _mask_from_idx(idx, b, h, S))
+    np.testing.assert_allclose(_as_bhsd(out["o_sparse"], B, Hq, S, D), ref, atol=1e-12)
+
+
+def test_lse_matches_logsumexp():
+    q, k, v = _tiny(B=1, S=192, Hq=2, Hkv=1, D=8, seed=9)
+    out = oracle.sparse_forward_problem(q, k, v, topk=2, want_full=True)
+    S = q.shape[1]
+    scale = 1.0 / np.sqrt(8)
+    idx = out["idx"]
+    m = _mask_from_idx(idx, 0, 0, S)
+    for r, (b, hq, t) in enumerate(out["rows"]):
+        logits = scale * (k[b, :, 0, :] @ q[b, t, hq, :])
+        full = torch.logsumexp(torch.from_numpy(logits[: t + 1]), 0).item()
+        sp = torch.logsumexp(torch.from_numpy(logits[m[t]]), 0).item()
+        assert abs(out["lse_full"][r] - full) < 1e-12
+        assert abs(out["lse_sparse"][r] - sp) < 1e-12
+
+
+def test_rows_are_probability_distributions_over_selected_causal_keys():
+    # V = identity rows: O_t[s] is the attention weight P_ts itself.
+    B, S, Hq, Hkv, D = 1, 128, 2, 1, 128
+    q = _rand((B, S, Hq, D), 21) * 0.3
+    k = _rand((B, S, Hkv, D), 22) * 0.3
+    v = np.zeros((B, S, Hkv, D))
+    v[0, np.arange(S), 0, np.arange(S)] = 1.0
+    out = oracle.sparse_forward_problem(q, k, v, topk=1, want_full=True)
+    P = out["o_sparse"].reshape(Hq, S, S)
+    Pf = out["o_full"].reshape(Hq, S, S)
+    scale = 1.0 / np.sqrt(D)
+    for hq in range(Hq):
+        for t in range(S):
+            i = t // BS
+            allowed = np.zeros(S, dtype=bool)
+            allowed[i * BS:t + 1] = True          # topk=1: the diagonal block only
+            assert np.all(P[hq, t][~allowed] == 0.0)
+            assert abs(P[hq, t].sum() - 1.0) < 1e-12
+            assert np.all(Pf[hq, t][t + 1:] == 0.0)
+            assert abs(Pf[hq, t].sum() - 1.0) < 1e-12
+            s0 = i * BS
+            for s in range(s0 + 1, t + 1):
+                want = np.exp(scale * (q[0, t, hq] @ (k[0, s, 0] - k[0, s0, 0])))
+                assert abs(P[hq, t, s] / P[hq, t, s0] - want) < 1e-11 * max(1.0, want)
+
+
+def test_value_ones_gives_ones():
+    q, k, v = _tiny(B=1, S=256, Hq=4, Hkv=2, D=8, seed=31)
+    v = np.ones_like(v)
+    out = oracle.sparse_forward_problem(q, k, v, topk=2, want_full=True)
+    np.testing.assert_allclose(out["o_sparse"], 1.0, atol=1e-12)
+    np.testing.assert_allclose(out["o_full"], 1.0, atol=1e-12)
+
+
+# -------------------------------------------------------------- dropped mass
+
+def test_dropped_mass_properties_and_linear_error_identity():
+    q, k, v = _tiny(B=1, S=384, Hq=4, Hkv=2, D=16, seed=41)
+    B, S, Hq, D = q.shape
+    n = S // BS
+    prev = None
+    for topk in range(1, n + 1):
+        out = oracle.sparse_forward_problem(q, k, v, topk=topk, want_full=True)
+        d = out["delta"]
+        assert np.all(d >= 0.0) and np.all(d <= 1.0)
+        np.testing.assert_allclose(d, out["delta_lse"], atol=1e-12)
+        t = out["rows"][:, 2]
+        assert np.all(d[t // BS < topk] == 0.0)
+        if prev is not None:
+            assert np.all(d <= prev + 1e-15)
+        prev = d
+        if topk < n:
+            idx = out["idx"]
+            o_unsel = _sdpa_rows(q, k, v, lambda b, h: _mask_from_idx(idx, b, h, S, True))
+            o_unsel = o_unsel.reshape(-1, D)
+            o_sp, o_f = out["o_sparse"], out["o_full"]
+            has = d > 0
+            lhs = o_f[has]
+            rhs = (1 - d[has])[:, None] * o_sp[has] + d[has][:, None] * o_unsel[has]
+            np.testing.assert_allclose(lhs, rhs, atol=1e-12)
+            vmax = np.abs(v).max()
+            assert np.all(np.abs(o_f - o_sp).max(axis=1) <= 2 * d * vmax + 1e-12)
+    assert np.all(prev == 0.0)
+
+
+# ----------------------------------------------------------------- backward
+
+def _loss(q, k, v, do, idx):
+    B, S, Hq, D = q.shape
+    rows = oracle.all_rows(B, Hq, S)
+    o = oracle.attn_rows(q, k, v, idx, rows, want_full=False)["o_sparse"]
+    return float(np.sum(o.reshape(B, Hq, S, D).transpose(0, 2, 1, 3) * do))
+
+
+def _full_bwd(q, k, v, do, idx):
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    n = S // BS
+    rows = oracle.all_rows(B, Hq, S)
+    dq = oracle.sparse_bwd_dq_rows(q, k, v, do, idx, rows).reshape(B, Hq, S, D).transpose(0, 2, 1, 3)
+    blocks = oracle.all_rows(B, Hkv, n)
+    dk, dv = oracle.sparse_bwd_dkv_blocks(q, k, v, do, idx, blocks)
+    dk = dk.reshape(B, Hkv, n * BS, D).transpose(0, 2, 1, 3)
+    dv = dv.reshape(B, Hkv, n * BS, D).transpose(0, 2, 1, 3)
+    return dq, dk, dv
+
+
+def test_backward_matches_central_finite_differences():
+    q, k, v = _tiny(B=1, S=256, Hq=4, Hkv=2, D=8, seed=51)
+    do = _rand(q.shape, 52)
+    kbar, qbar = oracle.block_pool(k, q)
+    idx, _ = oracle.block_select(qbar, kbar, 2)   # frozen selection
+    grads = _full_bwd(q, k, v, do, idx)
+    rng = np.random.Generator(np.random.PCG64(53))
+    h = 1e-6
+    for name, arr, g in zip("qkv", (q, k, v), grads):
+        for _ in range(12):
+            pos = tuple(int(rng.integers(0, s)) for s in arr.shape)
+            plus, minus = arr.copy(), arr.copy()
+            plus[pos] += h
+            minus[pos] -= h
+            args_p = {"q": q, "k": k, "v": v}
+            args_m = dict(args_p)
+            args_p[name], args_m[name] = plus, minus
+            fd = (_loss(args_p["q"], args_p["k"], args_p["v"], do, idx)
+                  - _loss(args_m["q"], args_m["k"], args_m["v"], do, idx)) / (2 * h)
+            assert abs(fd - g[pos]) <= 1e-6 * max(1.0, abs(g[pos])), (name, pos, fd, g[pos])
+
+
+def test_backward_matches_torch_autograd_of_masked_sdpa():
+    q, k, v = _tiny(B=1, S=256, Hq=4, Hkv=2, D=8, seed=61)
+    do = _rand(q.shape, 62)
+    kbar, qbar = oracle.block_pool(k, q)
+    idx, _ = oracle.block_select(qbar, kbar, 2)
+    dq, dk, dv = _full_bwd(q, k, v, do, idx)
+    B, S, Hq, D = q.shape
+    G = 2
+    qt = torch.from_numpy(q).permute(0, 2, 1, 3).clone().requires_grad_(True)
+    kt = torch.from_numpy(k).permute(0, 2, 1, 3).clone().requires_grad_(True)
+    vt = torch.from_numpy(v).permute(0, 2, 1, 3).clone().requires_grad_(True)
+    mask = torch.stack([torch.from_numpy(_mask_from_idx(idx, 0, hq // G, S)) for hq in range(Hq)])
+    o = F.scaled_dot_product_attention(qt, kt.repeat_interleave(G, 1), vt.repeat_interleave(G, 1),
+                                       attn_mask=mask[None])
+    (o * torch.from_numpy(do).permute(0, 2, 1, 3)).sum().backward()
+    np.testing.assert_allclose(dq, qt.grad.permute(0, 2, 1, 3).numpy(), atol=1e-11)
+    np.testing.assert_allclose(dk, kt.grad.permute(0, 2, 1, 3).numpy(), atol=1e-11)
+    np.testing.assert_allclose(dv, vt.grad.permute(0, 2, 1, 3).numpy(), atol=1e-11)
+
+
+def test_unselected_block_gets_exactly_zero_gradient():
+    q, k, v = _tiny(B=1, S=640, Hq=2, Hkv=1, D=8, seed=71)
+    do = _rand(q.shape, 72)
+    kbar, qbar = oracle.block_pool(k, q)
+    idx, _ = oracle.block_select(qbar, kbar, 2)
+    n = 640 // BS
+    lonely = [j for j in range(n)
+              if not any(j in idx[0, 0, i] for i in range(j + 1, n))]
+    assert lonely, "test data should leave some block unselected by later blocks"
+    for j in lonely:
+        do_j = do.copy()
+        do_j[0, j * BS:(j + 1) * BS] = 0.0
+        dk, dv = oracle.sparse_bwd_dkv_blocks(q, k, v, do_j, idx, np.array([[0, 0, j]]))
+        assert np.all(dk == 0.0) and np.all(dv == 0.0)
