@@ -1,0 +1,357 @@
+"""Benchmark of the SSA sparse stream on B200 (one JSON line on rank 0).
+
+A step is one pass of the sparse-stream forward over one batch of the
+workload: ssa_block_pool -> ssa_block_select -> ssa_sparse_attn_fwd, with the
+inputs already resident in HBM.  The metric is TFLOP/s over the selected
+blocks: 4 * D FLOPs per unmasked (query, key) pair of the selected blocks
+(QK^T and PV), summed over batch and query heads, per second.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...     # the fp64 CPU oracle on host cores
+
+Under torchrun (N > 1) every rank runs its own replica of the workload (the
+path has no exchange step; units are independent), the timed region is
+bracketed by barriers, and the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import gen  # noqa: E402
+
+METRIC = "sparse attn fwd TFLOP/s (selected blocks) and % of B200 BF16 peak at 8k/32k"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def selected_pairs(workload) -> int:
+    """Unmasked (query, key) pairs of the selected blocks for one (b, query head)
+    summed over query blocks; selection always holds min(k, i + 1) blocks, the
+    diagonal one causally masked (64 * 65 / 2 pairs), the others full (64 * 64)."""
+    n, k = workload.n_blocks, workload.top_k
+    total = 0
+    for i in range(n):
+        m = min(k, i + 1)
+        total += (m - 1) * 64 * 64 + 64 * 65 // 2
+    return total
+
+
+def algorithmic_flops(workload) -> float:
+    w = workload
+    return 4.0 * w.head_dim * selected_pairs(w) * w.batch * w.n_q_heads
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while the timed loop runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+        return False
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, flags in rows for i, f in enumerate(flags)
+                          if f.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": rows[0][1],
+                "reasons": reasons, "samples": len(rows)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def dist_max(value: float, world: int) -> float:
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def config_of(w, l2: str):
+    return {"workload": w.name, "batch": w.batch, "seq_len": w.seq_len, "n_q_heads": w.n_q_heads,
+            "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim, "block_size": 64,
+            "top_k": w.top_k, "causal": True, "between_steps": l2}
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args, world, rank, local):
+    import block_sparse_attention_21_b200 as ssa
+    from block_sparse_attention_21_b200 import build as ssa_build
+    ssa_build.build()
+    lib = ssa.lib()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    x = gen.make_inputs(args.workload)
+    w = x.workload
+    p = ssa.problem(w.batch, w.seq_len, w.n_q_heads, w.n_kv_heads, w.head_dim, w.top_k)
+    q, k, v = (t.to(dev) for t in (x.q, x.k, x.v))
+    st = ssa.SparseStream(p, dev)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flops = algorithmic_flops(w)
+
+    def step():
+        st.forward(q, k, v)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+
+    # device-timed steps: one event pair around each step, L2 flushed between
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    fwd_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    launches0 = ssa.ssa_launch_count()
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for s in range(args.steps):
+            flush.fill_(s & 0xFF)
+            ev[s][0].record(stream)
+            st.select(q, k)
+            fwd_ev[s][0].record(stream)
+            ssa.ssa_sparse_attn_fwd(p, q, k, v, st.block_idx, st.o, st.lse)
+            fwd_ev[s][1].record(stream)
+            ev[s][1].record(stream)
+        torch.cuda.synchronize()
+    dist_barrier(world)
+    launches = ssa.ssa_launch_count() - launches0
+    step_ms = sum(a.elapsed_time(b) for a, b in ev)
+    fwd_ms = sum(a.elapsed_time(b) for a, b in fwd_ev) / args.steps
+    total_ms = dist_max(step_ms, world)
+    ms_per_step = total_ms / args.steps
+    value = flops * world / (ms_per_step * 1e-3) / 1e12
+
+    # end to end through the public API: pinned host inputs in, O and LSE out
+    hq, hk, hv = (t.pin_memory() for t in (x.q, x.k, x.v))
+    ho = torch.empty(st.o.shape, dtype=st.o.dtype).pin_memory()
+    hl = torch.empty(st.lse.shape, dtype=st.lse.dtype).pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    e2e_steps = max(1, min(args.steps, 200))
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        st.forward(dq, dk, dv)
+        ho.copy_(st.o, non_blocking=True)
+        hl.copy_(st.lse, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    dist_barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = dist_max(e0.elapsed_time(e1), world) / e2e_steps
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    achieved = flops / (fwd_ms * 1e-3) / 1e12
+    traffic = load_traffic(w.name)
+    rec = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": config_of(w, "l2_flushed"),
+        "e2e": {"value": round(flops * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(e2e_ms, 4)},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "traffic": traffic, "kernel": "attn_fwd_kernel (ssa_sparse_attn_fwd)",
+                     "peak_source": f"{peak_src} bf16_tflops (burst)",
+                     "kernel_ms": round(fwd_ms, 5)},
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+        "pct_of_peak_step": round(100.0 * value / world / peak, 2),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rec["cpu_baseline"] = cpu_baseline(x, args.cpu_sample_blocks)
+    return rec
+
+
+def load_traffic(name):
+    """dram bytes per launch of the sparse forward from the committed ncu summary
+    of this workload, or None."""
+    path = os.path.join(ROOT, "profiles", f"attn_fwd_{name}.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    return d.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------- CPU baseline
+
+def cpu_baseline(x, sample_blocks: int, want_time: float = 0.0):
+    """The fp64 oracle as it stands on the host cores: pooling and selection of
+    the whole workload plus sparse attention for every row of `sample_blocks`
+    query blocks (all heads, all batch entries), reported as TFLOP/s of the
+    selected-pair FLOPs it computed."""
+    import oracle
+    w = x.workload
+    threads = oracle.default_threads()
+    rng = np.random.Generator(np.random.PCG64(2024))
+    blocks = sorted(rng.choice(np.arange(w.top_k, w.n_blocks), size=sample_blocks, replace=False))
+    rows = []
+    for i in blocks:
+        t = np.arange(64 * i, 64 * i + 64)
+        for b in range(w.batch):
+            for hq in range(w.n_q_heads):
+                rows.append(np.stack([np.full_like(t, b), np.full_like(t, hq), t], axis=1))
+    rows = np.concatenate(rows).astype(np.int64)
+    q64, k64, v64 = oracle.widen(x.q), oracle.widen(x.k), oracle.widen(x.v)
+    t0 = time.perf_counter()
+    kbar, qbar = oracle.block_pool(k64, q64, nthreads=threads)
+    idx, _ = oracle.block_select(qbar, kbar, w.top_k, nthreads=threads)
+    oracle.attn_rows(q64, k64, v64, idx, rows, want_full=False, nthreads=threads)
+    dt = time.perf_counter() - t0
+    pairs_per_block = (w.top_k - 1) * 64 * 64 + 64 * 65 // 2
+    flops = 4.0 * w.head_dim * pairs_per_block * len(blocks) * w.batch * w.n_q_heads
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": threads,
+            "kind": "oracle", "seconds": round(dt, 2),
+            "sample": (f"pool+select of the whole workload, then sparse attention of all rows "
+                       f"of {len(blocks)} of {w.n_blocks} query blocks (all heads, all batch), "
+                       f"fp64, {threads} threads")}
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the fp64 oracle on the host cores, on this arm's
+    workload, one bounded sample per step."""
+    if rank != 0:
+        return None
+    x = gen.make_inputs(args.workload)
+    w = x.workload
+    samples = []
+    for _ in range(args.warmup):
+        cpu_baseline(x, 1)
+    for _ in range(args.steps):
+        samples.append(cpu_baseline(x, args.cpu_sample_blocks))
+    value = statistics.median(s["value"] for s in samples)
+    secs = sum(s["seconds"] for s in samples)
+    cb = dict(samples[-1])
+    cb["value"] = value
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1000.0 * secs / max(1, len(samples)), 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_of(w, "host_cpu"), "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="llama1b_8k", choices=sorted(gen.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-sample-blocks", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            rec = run_reference(args, world, rank)
+        else:
+            rec = run_ours(args, world, rank, local)
+        if rank == 0 and rec is not None:
+            print(json.dumps(rec), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

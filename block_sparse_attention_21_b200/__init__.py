@@ -1,0 +1,77 @@
+"""SSA sparse stream on B200: block-sparse causal attention with top-k KV-block
+selection, as hand-written sm_100a kernels behind a C ABI (libssa.so).
+
+The C entry points are re-exported with their own names (argument marshalling
+only, see _binding.py).  `SparseStream` strings them together over buffers it
+allocates once with torch (device memory and streams are all torch is used for).
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from ._binding import (EXPORTED, LIB_PATH, SsaError, SsaProblem, lib, problem,
+                       ssa_block_pool, ssa_block_select, ssa_debug_timeout_probe,
+                       ssa_full_attn_fwd_with_mass, ssa_get_device_error, ssa_launch_count,
+                       ssa_sparse_attn_bwd, ssa_sparse_attn_bwd_workspace,
+                       ssa_sparse_attn_fwd, ssa_status_string)
+
+__all__ = ["EXPORTED", "LIB_PATH", "SsaError", "SsaProblem", "SparseStream", "lib", "problem",
+           "ssa_block_pool", "ssa_block_select", "ssa_debug_timeout_probe",
+           "ssa_full_attn_fwd_with_mass", "ssa_get_device_error", "ssa_launch_count",
+           "ssa_sparse_attn_bwd", "ssa_sparse_attn_bwd_workspace", "ssa_sparse_attn_fwd",
+           "ssa_status_string"]
+
+
+class SparseStream:
+    """Pre-allocated buffers for one problem shape and the calls of the path.
+
+    forward():   ssa_block_pool -> ssa_block_select -> ssa_sparse_attn_fwd
+    alignment(): ssa_block_pool -> ssa_block_select -> ssa_full_attn_fwd_with_mass
+    backward():  ssa_sparse_attn_bwd (after forward())
+    """
+
+    def __init__(self, p: SsaProblem, device: Optional[torch.device] = None):
+        self.p = p
+        dev = device or torch.device("cuda", torch.cuda.current_device())
+        B, S, Hq, Hkv, D = p.batch, p.seq_len, p.n_q_heads, p.n_kv_heads, p.head_dim
+        n = S // p.block_size
+        f32, bf16 = torch.float32, torch.bfloat16
+        self.k_pooled = torch.empty(B, Hkv, n, D, dtype=f32, device=dev)
+        self.q_pooled = torch.empty(B, Hkv, n, D, dtype=f32, device=dev)
+        self.block_idx = torch.empty(B, Hkv, n, p.top_k, dtype=torch.int32, device=dev)
+        self.o = torch.empty(B, S, Hq, D, dtype=bf16, device=dev)
+        self.lse = torch.empty(B, Hq, S, dtype=f32, device=dev)
+        self._full = None
+        self._grad = None
+
+    def select(self, q, k, stream=None):
+        ssa_block_pool(self.p, k, q, self.k_pooled, self.q_pooled, stream)
+        ssa_block_select(self.p, self.q_pooled, self.k_pooled, self.block_idx, stream)
+        return self.block_idx
+
+    def forward(self, q, k, v, stream=None):
+        self.select(q, k, stream)
+        ssa_sparse_attn_fwd(self.p, q, k, v, self.block_idx, self.o, self.lse, stream)
+        return self.o
+
+    def alignment(self, q, k, v, stream=None):
+        if self._full is None:
+            self._full = (torch.empty_like(self.o), torch.empty_like(self.lse),
+                          torch.empty_like(self.lse))
+        o_full, lse_full, dropped = self._full
+        self.select(q, k, stream)
+        ssa_full_attn_fwd_with_mass(self.p, q, k, v, self.block_idx, self.o, self.lse, o_full,
+                                    lse_full, dropped, stream)
+        return self.o, o_full, dropped
+
+    def backward(self, q, k, v, d_o, stream=None):
+        if self._grad is None:
+            ws = ssa_sparse_attn_bwd_workspace(self.p)
+            self._grad = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v),
+                          torch.empty(max(ws, 256), dtype=torch.uint8, device=q.device), ws)
+        dq, dk, dv, workspace, ws = self._grad
+        ssa_sparse_attn_bwd(self.p, q, k, v, self.o, self.lse, d_o, self.block_idx, dq, dk, dv,
+                            workspace, workspace.numel(), stream)
+        return dq, dk, dv

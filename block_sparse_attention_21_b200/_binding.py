@@ -1,0 +1,204 @@
+"""ctypes binding of libssa.so -- argument marshalling only.
+
+Every function here has the name of the C entry point it calls and takes the
+same arguments, with torch tensors standing for device pointers.  No step of
+the computation happens in Python: each call validates dtypes/devices/shapes,
+passes raw pointers and the current CUDA stream, and raises SsaError on a
+non-OK status.  If libssa.so is missing the import fails loudly; there is no
+fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libssa.so")
+
+SSA_OK = 0
+STATUS_NAMES = {0: "SSA_OK", 1: "SSA_ERR_INVALID_ARG", 2: "SSA_ERR_UNSUPPORTED",
+                3: "SSA_ERR_CUDA", 4: "SSA_ERR_DEVICE_TIMEOUT", 5: "SSA_ERR_WORKSPACE"}
+
+# every symbol include/ssa.h declares
+EXPORTED = ("ssa_block_pool", "ssa_block_select", "ssa_sparse_attn_fwd",
+            "ssa_full_attn_fwd_with_mass", "ssa_sparse_attn_bwd_workspace",
+            "ssa_sparse_attn_bwd", "ssa_get_device_error", "ssa_debug_timeout_probe",
+            "ssa_status_string", "ssa_launch_count")
+
+
+class SsaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+        self.status = status
+
+
+class SsaProblem(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int), ("seq_len", ctypes.c_int), ("n_q_heads", ctypes.c_int),
+                ("n_kv_heads", ctypes.c_int), ("head_dim", ctypes.c_int),
+                ("block_size", ctypes.c_int), ("top_k", ctypes.c_int), ("causal", ctypes.c_int),
+                ("softmax_scale", ctypes.c_float)]
+
+
+def problem(batch: int, seq_len: int, n_q_heads: int, n_kv_heads: int, head_dim: int,
+            top_k: int, block_size: int = 64, causal: int = 1,
+            softmax_scale: float = 0.0) -> SsaProblem:
+    return SsaProblem(batch, seq_len, n_q_heads, n_kv_heads, head_dim, block_size, top_k,
+                      causal, softmax_scale)
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libssa.so; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libssa.so not found at {LIB_PATH}: build it with "
+                               "`python -m block_sparse_attention_21_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, P = ctypes.c_void_p, ctypes.POINTER(SsaProblem)
+        sigs = {
+            "ssa_block_pool": [P, vp, vp, vp, vp, vp],
+            "ssa_block_select": [P, vp, vp, vp, vp],
+            "ssa_sparse_attn_fwd": [P, vp, vp, vp, vp, vp, vp, vp],
+            "ssa_full_attn_fwd_with_mass": [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
+            "ssa_sparse_attn_bwd": [P] + [vp] * 11 + [ctypes.c_size_t, vp],
+            "ssa_get_device_error": [vp],
+            "ssa_debug_timeout_probe": [ctypes.c_int, vp],
+        }
+        for name, args in sigs.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = ctypes.c_int
+        L.ssa_sparse_attn_bwd_workspace.argtypes = [P]
+        L.ssa_sparse_attn_bwd_workspace.restype = ctypes.c_size_t
+        L.ssa_status_string.argtypes = [ctypes.c_int]
+        L.ssa_status_string.restype = ctypes.c_char_p
+        L.ssa_launch_count.argtypes = []
+        L.ssa_launch_count.restype = ctypes.c_uint64
+        _lib = L
+    return _lib
+
+
+def _ptr(t: Optional[torch.Tensor], dtype=None, name: str = "") -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name}: expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name}: expected {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _call(name: str, *args) -> None:
+    rc = getattr(lib(), name)(*args)
+    if rc != SSA_OK:
+        raise SsaError(rc, name)
+
+
+def _numel_check(t, shape, name):
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _shapes(p: SsaProblem):
+    B, S, Hq, Hkv, D = p.batch, p.seq_len, p.n_q_heads, p.n_kv_heads, p.head_dim
+    n = S // max(p.block_size, 1)
+    return dict(q=(B, S, Hq, D), kv=(B, S, Hkv, D), pooled=(B, Hkv, n, D),
+                idx=(B, Hkv, n, p.top_k), lse=(B, Hq, S))
+
+
+BF16, F32, I32 = torch.bfloat16, torch.float32, torch.int32
+
+
+def ssa_block_pool(p: SsaProblem, k, q, k_pooled, q_pooled, stream=None) -> None:
+    sh = _shapes(p)
+    _numel_check(k, sh["kv"], "k")
+    _numel_check(k_pooled, sh["pooled"], "k_pooled")
+    if q is not None:
+        _numel_check(q, sh["q"], "q")
+        _numel_check(q_pooled, sh["pooled"], "q_pooled")
+    _call("ssa_block_pool", ctypes.byref(p), _ptr(k, BF16, "k"), _ptr(q, BF16, "q"),
+          _ptr(k_pooled, F32, "k_pooled"), _ptr(q_pooled, F32, "q_pooled"), _stream(stream))
+
+
+def ssa_block_select(p: SsaProblem, q_pooled, k_pooled, block_idx, stream=None) -> None:
+    sh = _shapes(p)
+    _numel_check(q_pooled, sh["pooled"], "q_pooled")
+    _numel_check(k_pooled, sh["pooled"], "k_pooled")
+    _numel_check(block_idx, sh["idx"], "block_idx")
+    _call("ssa_block_select", ctypes.byref(p), _ptr(q_pooled, F32, "q_pooled"),
+          _ptr(k_pooled, F32, "k_pooled"), _ptr(block_idx, I32, "block_idx"), _stream(stream))
+
+
+def ssa_sparse_attn_fwd(p: SsaProblem, q, k, v, block_idx, o, lse, stream=None) -> None:
+    sh = _shapes(p)
+    for t, s, nm in ((q, "q", "q"), (k, "kv", "k"), (v, "kv", "v"), (block_idx, "idx", "block_idx"),
+                     (o, "q", "o"), (lse, "lse", "lse")):
+        _numel_check(t, sh[s], nm)
+    _call("ssa_sparse_attn_fwd", ctypes.byref(p), _ptr(q, BF16, "q"), _ptr(k, BF16, "k"),
+          _ptr(v, BF16, "v"), _ptr(block_idx, I32, "block_idx"), _ptr(o, BF16, "o"),
+          _ptr(lse, F32, "lse"), _stream(stream))
+
+
+def ssa_full_attn_fwd_with_mass(p: SsaProblem, q, k, v, block_idx, o_sparse, lse_sparse, o_full,
+                                lse_full, dropped, stream=None) -> None:
+    sh = _shapes(p)
+    for t, s, nm in ((q, "q", "q"), (k, "kv", "k"), (v, "kv", "v"), (block_idx, "idx", "block_idx"),
+                     (o_sparse, "q", "o_sparse"), (lse_sparse, "lse", "lse_sparse"),
+                     (o_full, "q", "o_full"), (lse_full, "lse", "lse_full"),
+                     (dropped, "lse", "dropped")):
+        _numel_check(t, sh[s], nm)
+    _call("ssa_full_attn_fwd_with_mass", ctypes.byref(p), _ptr(q, BF16, "q"), _ptr(k, BF16, "k"),
+          _ptr(v, BF16, "v"), _ptr(block_idx, I32, "block_idx"), _ptr(o_sparse, BF16, "o_sparse"),
+          _ptr(lse_sparse, F32, "lse_sparse"), _ptr(o_full, BF16, "o_full"),
+          _ptr(lse_full, F32, "lse_full"), _ptr(dropped, F32, "dropped"), _stream(stream))
+
+
+def ssa_sparse_attn_bwd_workspace(p: SsaProblem) -> int:
+    return int(lib().ssa_sparse_attn_bwd_workspace(ctypes.byref(p)))
+
+
+def ssa_sparse_attn_bwd(p: SsaProblem, q, k, v, o, lse, d_o, block_idx, dq, dk, dv, workspace,
+                        ws_bytes: int, stream=None) -> None:
+    sh = _shapes(p)
+    for t, s, nm in ((q, "q", "q"), (k, "kv", "k"), (v, "kv", "v"), (o, "q", "o"),
+                     (lse, "lse", "lse"), (d_o, "q", "d_o"), (block_idx, "idx", "block_idx"),
+                     (dq, "q", "dq"), (dk, "kv", "dk"), (dv, "kv", "dv")):
+        _numel_check(t, sh[s], nm)
+    _call("ssa_sparse_attn_bwd", ctypes.byref(p), _ptr(q, BF16, "q"), _ptr(k, BF16, "k"),
+          _ptr(v, BF16, "v"), _ptr(o, BF16, "o"), _ptr(lse, F32, "lse"), _ptr(d_o, BF16, "d_o"),
+          _ptr(block_idx, I32, "block_idx"), _ptr(dq, BF16, "dq"), _ptr(dk, BF16, "dk"),
+          _ptr(dv, BF16, "dv"), _ptr(workspace, None, "workspace"), int(ws_bytes),
+          _stream(stream))
+
+
+def ssa_get_device_error(stream=None) -> int:
+    """Status code (not raised): 0 OK, 4 a bounded device wait ran out."""
+    return int(lib().ssa_get_device_error(_stream(stream)))
+
+
+def ssa_debug_timeout_probe(timeout_us: int, stream=None) -> None:
+    _call("ssa_debug_timeout_probe", int(timeout_us), _stream(stream))
+
+
+def ssa_status_string(status: int) -> str:
+    return lib().ssa_status_string(int(status)).decode()
+
+
+def ssa_launch_count() -> int:
+    return int(lib().ssa_launch_count())

@@ -1,0 +1,385 @@
+// attn_fwd.cuh -- block-sparse causal attention forward on tcgen05 tensor cores.
+//
+// One CTA handles one query block i (64 tokens) of one batch entry for 2*T
+// query heads that share KV head h.  Its rows form T M-tiles of 128 rows
+// (2 heads x 64 tokens).  The KV blocks it visits are either the selected
+// blocks of the index table (sparse stream: "SSA: Guida a Sparse Sparse
+// Attention per LLM", section "Block-sparse attention e Receptive Field",
+// attention computed only over the tokens of the selected blocks) or, with
+// MASS, every causal block 0..i, each one's P.V going to the selected or the
+// unselected accumulator against one shared running maximum, which yields the
+// dense counterpart, the sparse output and the dropped attention mass from
+// one pass ("Resumen Tecnico: SSA", section 2, "Alineacion Bidireccional",
+// and section 1 on the dropped mass).
+//
+// Warp roles (128 * (T + 1) threads):
+//   warp 0      TMA producer: the Q tiles once, then K and V of each visited
+//               block through an NS-stage ring (index-guided loads).
+//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer:
+//               S_t = Q_t K^T (both operands in shared memory), then
+//               O_t += P_t V (P_t read from TMEM, V in shared memory).
+//   warps 2-3   build the selection bitmap (MASS), otherwise idle.
+//   warps 4..   one warpgroup per M-tile: thread r owns row r of the tile;
+//               online softmax in the exp2 domain with lazy rescaling
+//               (the running maximum only moves when it grows by > 8, i.e.
+//               a factor 256), P written back to TMEM as bf16, O rescaled in
+//               TMEM when needed, and the epilogue.
+//
+// TMEM layout per M-tile t (base t * 512 / T): S at +0 (64 columns), P at +64
+// (32 columns of bf16 pairs), O (O_selected with MASS) at +128 (D columns),
+// O_unselected at +128 + D (MASS only).
+#pragma once
+
+#include "sm100.cuh"
+
+namespace ssa {
+
+struct FwdParams {
+  int B, S, Hq, Hkv, G, n, topk, slices;
+  float scale_log2;  // softmax scale * log2(e)
+  const int32_t* idx;
+  __nv_bfloat16* o;      // sparse output
+  float* lse;            // sparse log-sum-exp (natural log)
+  __nv_bfloat16* o_full; // MASS: dense causal output
+  float* lse_full;       // MASS
+  float* dropped;        // MASS: dropped attention mass
+  uint64_t timeout_ns;
+};
+
+template <int D, int T, bool MASS>
+struct FwdConfig {
+  static constexpr int NP = D / 64;               // 64-column panels per row
+  static constexpr int QTILE = 128 * D * 2;       // bytes of one Q M-tile
+  static constexpr int KVT = 64 * D * 2;          // bytes of one K (or V) block
+  static constexpr int NS = (D == 64) ? 4 : 3;    // K/V ring stages
+  static constexpr int TSTRIDE = 512 / T;         // TMEM columns per M-tile
+  static constexpr int THREADS = 128 * (T + 1);
+  static constexpr int NBARS = 1 + 3 * NS + 4 * T + 1;
+  // shared memory: Q tiles, K ring, V ring, barriers, tmem slot, abort flag,
+  // selection bitmap (up to 8192 blocks)
+  static constexpr int SMEM_TILES = T * QTILE + 2 * NS * KVT;
+  static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + NBARS * 8 + 16 + 1024;
+  static_assert((MASS ? 128 + 2 * D : 128 + D) <= TSTRIDE, "TMEM budget per M-tile");
+};
+
+template <int D, int T, bool MASS>
+__global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using C = FwdConfig<D, T, MASS>;
+  constexpr int NP = C::NP, QTILE = C::QTILE, KVT = C::KVT, NS = C::NS, TSTRIDE = C::TSTRIDE;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sK = sQ + T * QTILE;
+  uint8_t* sV = sK + NS * KVT;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + NS * KVT);
+  uint64_t* bar_q = bars;
+  uint64_t* bar_kfull = bars + 1;
+  uint64_t* bar_vfull = bar_kfull + NS;
+  uint64_t* bar_empty = bar_vfull + NS;
+  uint64_t* bar_sfull = bar_empty + NS;
+  uint64_t* bar_sfree = bar_sfull + T;
+  uint64_t* bar_pfull = bar_sfree + T;
+  uint64_t* bar_odone = bar_pfull + T;
+  uint64_t* bar_mma_done = bar_odone + T;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint32_t* selbits = tmem_slot + 4;
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  // work unit, heaviest query blocks first
+  const int per_i = p.B * p.Hkv * p.slices;
+  const int i = p.n - 1 - static_cast<int>(blockIdx.x) / per_i;
+  int rem = static_cast<int>(blockIdx.x) % per_i;
+  const int slice = rem % p.slices;
+  rem /= p.slices;
+  const int h = rem % p.Hkv;
+  const int b = rem / p.Hkv;
+  const int hq0 = h * p.G + slice * 2 * T;
+  const int nsel = min(p.topk, i + 1);
+  const int nblk = MASS ? (i + 1) : nsel;
+  const int32_t* idx_row = p.idx + ((static_cast<size_t>(b) * p.Hkv + h) * p.n + i) * p.topk;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&bar_kfull[s], 1);
+      mbar_init(&bar_vfull[s], 1);
+      mbar_init(&bar_empty[s], 1);
+    }
+    for (int t = 0; t < T; ++t) {
+      mbar_init(&bar_sfull[t], 1);
+      mbar_init(&bar_sfree[t], 128);
+      mbar_init(&bar_pfull[t], 128);
+      mbar_init(&bar_odone[t], 1);
+    }
+    mbar_init(bar_mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (MASS && warp == 2) {
+    const int words = (p.n + 31) / 32;
+    for (int w = lane; w < words; w += 32) selbits[w] = 0u;
+    __syncwarp();
+    for (int r = lane; r < nsel; r += 32) {
+      const int j = idx_row[r];
+      if (j >= 0 && j <= i) atomicOr(&selbits[j >> 5], 1u << (j & 31));
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint64_t tmo = p.timeout_ns;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_arrive_expect_tx(bar_q, T * QTILE);
+      for (int t = 0; t < T; ++t)
+        for (int hh = 0; hh < 2; ++hh)
+          for (int pn = 0; pn < NP; ++pn)
+            tma_load_4d(sQ + t * QTILE + pn * (128 * 128) + hh * (64 * 128), &tm_q, bar_q,
+                        64 * pn, hq0 + 2 * t + hh, 64 * i, b);
+      for (int jj = 0; jj < nblk; ++jj) {
+        const int st = jj % NS, use = jj / NS;
+        if (use > 0 && !mbar_wait(&bar_empty[st], (use - 1) & 1, abort_flag, tmo, 0x101)) break;
+        const int j = MASS ? jj : idx_row[jj];
+        mbar_arrive_expect_tx(&bar_kfull[st], KVT);
+        for (int pn = 0; pn < NP; ++pn)
+          tma_load_4d(sK + st * KVT + pn * (64 * 128), &tm_k, &bar_kfull[st], 64 * pn, h, 64 * j, b);
+        mbar_arrive_expect_tx(&bar_vfull[st], KVT);
+        for (int pn = 0; pn < NP; ++pn)
+          tma_load_4d(sV + st * KVT + pn * (64 * 128), &tm_v, &bar_vfull[st], 64 * pn, h, 64 * j, b);
+      }
+      // loads are never left in flight: every issued stage is consumed by the
+      // MMA issuer, or on abort waited for here (bounded)
+      if (*abort_flag) {
+        for (int s = 0; s < NS; ++s) {
+          volatile int never = 0;
+          mbar_wait(&bar_kfull[s], 0, &never, 1000000ull, 0x1ff);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 64, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
+      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
+      bool ok = mbar_wait(bar_q, 0, abort_flag, tmo, 0x201);
+      auto issue_qk = [&](int t, int st) {
+        const uint32_t d = tmem + t * TSTRIDE;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk % 4) * 32;  // 16 bf16 = 32 B inside the 128 B row
+          const uint64_t a = sdesc_sw128(sQa + t * QTILE + (kk / 4) * (128 * 128) + off, 16, 1024);
+          const uint64_t bd = sdesc_sw128(sKa + st * KVT + (kk / 4) * (64 * 128) + off, 16, 1024);
+          mma_ss(d, a, bd, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+      };
+      if (ok && nblk > 0) {
+        ok = mbar_wait(&bar_kfull[0], 0, abort_flag, tmo, 0x202);
+        if (ok) {
+          tc_fence_after();
+          for (int t = 0; t < T; ++t) {
+            issue_qk(t, 0);
+            tc_commit(&bar_sfull[t]);
+          }
+        }
+      }
+      bool first_sel = true, first_uns = true;
+      for (int jj = 0; ok && jj < nblk; ++jj) {
+        const int st = jj % NS;
+        if (jj + 1 < nblk) {
+          const int st1 = (jj + 1) % NS;
+          if (!mbar_wait(&bar_kfull[st1], ((jj + 1) / NS) & 1, abort_flag, tmo, 0x203)) break;
+          for (int t = 0; t < T; ++t) {
+            if (!mbar_wait(&bar_sfree[t], jj & 1, abort_flag, tmo, 0x204)) { ok = false; break; }
+            tc_fence_after();
+            issue_qk(t, st1);
+            tc_commit(&bar_sfull[t]);
+          }
+          if (!ok) break;
+        }
+        if (!mbar_wait(&bar_vfull[st], (jj / NS) & 1, abort_flag, tmo, 0x205)) break;
+        bool is_sel = true;
+        if (MASS) is_sel = (selbits[jj >> 5] >> (jj & 31)) & 1u;
+        const bool first = MASS ? (is_sel ? first_sel : first_uns) : (jj == 0);
+        for (int t = 0; t < T; ++t) {
+          if (!mbar_wait(&bar_pfull[t], jj & 1, abort_flag, tmo, 0x206)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t base = tmem + t * TSTRIDE;
+          const uint32_t o_col = base + 128 + ((MASS && !is_sel) ? D : 0);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t bd = sdesc_sw128(sVa + st * KVT + kk * (16 * 128), 64 * 128, 1024);
+            mma_ts(o_col, base + 64 + kk * 8, bd, idesc_pv, (first && kk == 0) ? 0u : 1u);
+          }
+          tc_commit(&bar_odone[t]);
+        }
+        if (!ok) break;
+        if (MASS) {
+          if (is_sel) first_sel = false; else first_uns = false;
+        }
+        tc_commit(&bar_empty[st]);
+      }
+      // every issued MMA has completed before TMEM is released
+      tc_commit(bar_mma_done);
+      volatile int never = 0;
+      mbar_wait(bar_mma_done, 0, &never, tmo, 0x2ff);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax
+    const int t = (warp - 4) / 4;
+    const int wq = warp % 4;
+    const int r = wq * 32 + lane;
+    const int hh = r / 64, tq = r % 64;
+    const int hq = hq0 + 2 * t + hh;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16) + t * TSTRIDE;
+    const uint32_t tS = lane_base, tP = lane_base + 64, tO = lane_base + 128;
+    const uint32_t tOu = tO + D;
+    float m_ref = -INFINITY, l_sel = 0.f, l_uns = 0.f;
+    bool ok = true;
+    for (int jj = 0; jj < nblk; ++jj) {
+      // waits are made warp-uniform: the tcgen05.ld/st below are .sync.aligned
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar_sfull[t], jj & 1, abort_flag, tmo, 0x301))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float s[64];
+      {
+        float a[32], c2[32];
+        tmem_ld32(tS, a);
+        tmem_ld32(tS + 32, c2);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) { s[c] = a[c]; s[32 + c] = c2[c]; }
+      }
+      tc_fence_before();
+      mbar_arrive(&bar_sfree[t]);
+      const bool diag = (jj == nblk - 1);
+      bool is_sel = true;
+      if (MASS) is_sel = (selbits[jj >> 5] >> (jj & 31)) & 1u;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        float x = s[c] * p.scale_log2;
+        if (diag && c > tq) x = -INFINITY;
+        s[c] = x;
+        mx = fmaxf(mx, x);
+      }
+      float alpha = 1.f;
+      bool resc = false;
+      if (mx > m_ref + 8.f) {
+        alpha = ex2(m_ref - mx);
+        m_ref = mx;
+        resc = (jj > 0);
+      }
+      float rs = 0.f;
+      uint32_t pk[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const float p0 = ex2(s[2 * c] - m_ref);
+        const float p1 = ex2(s[2 * c + 1] - m_ref);
+        rs += p0 + p1;
+        pk[c] = pack_bf16x2(p0, p1);
+      }
+      l_sel *= alpha;
+      l_uns *= alpha;
+      if (is_sel) l_sel += rs; else l_uns += rs;
+      if (jj > 0) {
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(&bar_odone[t], (jj - 1) & 1, abort_flag, tmo, 0x302))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, resc)) {
+#pragma unroll
+          for (int acc = 0; acc < (MASS ? 2 : 1); ++acc) {
+            const uint32_t base = acc ? tOu : tO;
+#pragma unroll
+            for (int ch = 0; ch < D / 32; ++ch) {
+              float o[32];
+              uint32_t w[32];
+              tmem_ld32(base + ch * 32, o);
+#pragma unroll
+              for (int c = 0; c < 32; ++c) w[c] = __float_as_uint(o[c] * alpha);
+              tmem_st32(base + ch * 32, w);
+            }
+          }
+        }
+      }
+      tmem_st32(tP, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bar_pfull[t]);
+    }
+    // ---------------------------------------------------------- epilogue
+    if (ok && __all_sync(0xffffffffu,
+                         mbar_wait(&bar_odone[t], (nblk - 1) & 1, abort_flag, tmo, 0x303))) {
+      tc_fence_after();
+      const int tok = 64 * i + tq;
+      const size_t orow = ((static_cast<size_t>(b) * p.S + tok) * p.Hq + hq) * D;
+      const size_t lrow = (static_cast<size_t>(b) * p.Hq + hq) * p.S + tok;
+      const bool has_uns = MASS && (nblk > nsel);
+      const float inv_sel = 1.f / l_sel;
+      const float l_all = l_sel + (has_uns ? l_uns : 0.f);
+      const float inv_all = 1.f / l_all;
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) {
+        float o[32];
+        tmem_ld32(tO + ch * 32, o);
+        uint32_t w[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) w[c] = pack_bf16x2(o[2 * c] * inv_sel, o[2 * c + 1] * inv_sel);
+        uint4* dst = reinterpret_cast<uint4*>(p.o + orow + ch * 32);
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4)
+          dst[v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+        if (MASS) {
+          if (has_uns) {
+            float ou[32];
+            tmem_ld32(tOu + ch * 32, ou);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] += ou[c];
+          }
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            w[c] = pack_bf16x2(o[2 * c] * inv_all, o[2 * c + 1] * inv_all);
+          uint4* dstf = reinterpret_cast<uint4*>(p.o_full + orow + ch * 32);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            dstf[v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+        }
+      }
+      constexpr float kLn2 = 0.69314718055994530942f;
+      p.lse[lrow] = (m_ref + log2f(l_sel)) * kLn2;
+      if (MASS) {
+        p.lse_full[lrow] = (m_ref + log2f(l_all)) * kLn2;
+        p.dropped[lrow] = has_uns ? (l_uns / l_all) : 0.f;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace ssa

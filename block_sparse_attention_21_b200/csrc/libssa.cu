@@ -1,0 +1,323 @@
+// libssa.cu -- host side of the C ABI declared in include/ssa.h: argument
+// validation, TMA tensor-map construction, kernel dispatch and the device
+// error word.  The whole library is one translation unit so that every kernel
+// shares the one device error word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdlib>
+#include <mutex>
+
+#include "ssa.h"
+#include "sm100.cuh"
+#include "pool_select.cuh"
+#include "attn_fwd.cuh"
+#include "attn_bwd.cuh"
+
+namespace {
+
+std::atomic<uint64_t> g_launches{0};
+
+constexpr int kMaxDevices = 64;
+constexpr int kMaxSeqLen = 524288;
+
+uint64_t wait_timeout_ns() {
+  static uint64_t ns = [] {
+    const char* env = std::getenv("SSA_WAIT_TIMEOUT_MS");
+    long ms = env ? std::atol(env) : 0;
+    if (ms <= 0) ms = 2000;
+    return static_cast<uint64_t>(ms) * 1000000ull;
+  }();
+  return ns;
+}
+
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+struct Dims {
+  int B, S, Hq, Hkv, D, G, n, topk;
+  float scale;
+};
+
+// Host-side validation shared by every entry point.
+ssa_status check_problem(const ssa_problem* p, Dims* d) {
+  if (p == nullptr) return SSA_ERR_INVALID_ARG;
+  if (p->batch < 1 || p->seq_len < 1 || p->n_q_heads < 1 || p->n_kv_heads < 1 ||
+      p->head_dim < 1 || p->block_size < 1 || p->top_k < 1)
+    return SSA_ERR_INVALID_ARG;
+  if (p->n_q_heads % p->n_kv_heads != 0) return SSA_ERR_INVALID_ARG;
+  if (p->seq_len % p->block_size != 0) return SSA_ERR_INVALID_ARG;
+  if (!std::isfinite(p->softmax_scale)) return SSA_ERR_INVALID_ARG;
+  if (p->block_size != 64) return SSA_ERR_UNSUPPORTED;
+  if (p->causal != 1) return SSA_ERR_UNSUPPORTED;
+  if (p->head_dim != 64 && p->head_dim != 128) return SSA_ERR_UNSUPPORTED;
+  const int G = p->n_q_heads / p->n_kv_heads;
+  if (G != 2 && G != 4 && G != 8 && G != 16) return SSA_ERR_UNSUPPORTED;
+  if (p->seq_len > kMaxSeqLen) return SSA_ERR_UNSUPPORTED;
+  // grid and element counts stay far inside 32-bit launch limits
+  const double rows = static_cast<double>(p->batch) * p->n_kv_heads * (p->seq_len / 64) * G;
+  if (rows > 1.0e9) return SSA_ERR_UNSUPPORTED;
+  d->B = p->batch;
+  d->S = p->seq_len;
+  d->Hq = p->n_q_heads;
+  d->Hkv = p->n_kv_heads;
+  d->D = p->head_dim;
+  d->G = G;
+  d->n = p->seq_len / 64;
+  d->topk = p->top_k;
+  d->scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt(static_cast<float>(p->head_dim));
+  return SSA_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// bf16 tensor [d3][d2][d1][d0] (d0 innermost), box of 64 x 1 x 64 x 1 elements
+// (64 columns of one head for 64 consecutive tokens), 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, int d0, int d1, int d2, int d3) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d0), static_cast<cuuint64_t>(d1),
+                              static_cast<cuuint64_t>(d2), static_cast<cuuint64_t>(d3)};
+  const cuuint64_t strides[3] = {dims[0] * 2, dims[0] * dims[1] * 2, dims[0] * dims[1] * dims[2] * 2};
+  const cuuint32_t box[4] = {64, 1, 64, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (kernel, device).
+template <typename K>
+ssa_status ensure_smem(K kernel, int bytes, std::atomic<uint64_t>* done_mask) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return SSA_ERR_CUDA;
+  const uint64_t bit = 1ull << dev;
+  if (done_mask->load() & bit) return SSA_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return SSA_ERR_CUDA;
+  done_mask->fetch_or(bit);
+  return SSA_OK;
+}
+
+ssa_status launch_result() {
+  g_launches.fetch_add(1);
+  return cudaGetLastError() == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;
+}
+
+template <int D>
+ssa_status launch_pool(const Dims& d, const void* k, const void* q, float* kb, float* qb,
+                       cudaStream_t st) {
+  ssa::PoolParams pp;
+  pp.k = static_cast<const __nv_bfloat16*>(k);
+  pp.q = static_cast<const __nv_bfloat16*>(q);
+  pp.kbar = kb;
+  pp.qbar = qb;
+  pp.S = d.S;
+  pp.Hq = d.Hq;
+  pp.Hkv = d.Hkv;
+  pp.G = d.G;
+  pp.n = d.n;
+  ssa::block_pool_kernel<D><<<dim3(d.n, d.Hkv, d.B), 256, 0, st>>>(pp);
+  return launch_result();
+}
+
+template <int D, int T, bool MASS>
+ssa_status launch_fwd(const Dims& d, const void* q, const void* k, const void* v,
+                      const int32_t* idx, void* o, float* lse, void* of, float* lsef,
+                      float* dropped, cudaStream_t st) {
+  using C = ssa::FwdConfig<D, T, MASS>;
+  static std::atomic<uint64_t> smem_done{0};
+  auto kernel = ssa::attn_fwd_kernel<D, T, MASS>;
+  ssa_status s = ensure_smem(kernel, C::SMEM_BYTES, &smem_done);
+  if (s != SSA_OK) return s;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, D, d.Hq, d.S, d.B) || !make_map(&mk, k, D, d.Hkv, d.S, d.B) ||
+      !make_map(&mv, v, D, d.Hkv, d.S, d.B))
+    return SSA_ERR_CUDA;
+  ssa::FwdParams fp;
+  fp.B = d.B;
+  fp.S = d.S;
+  fp.Hq = d.Hq;
+  fp.Hkv = d.Hkv;
+  fp.G = d.G;
+  fp.n = d.n;
+  fp.topk = d.topk;
+  fp.slices = (d.G / 2) / T;
+  fp.scale_log2 = d.scale * 1.4426950408889634f;
+  fp.idx = idx;
+  fp.o = static_cast<__nv_bfloat16*>(o);
+  fp.lse = lse;
+  fp.o_full = static_cast<__nv_bfloat16*>(of);
+  fp.lse_full = lsef;
+  fp.dropped = dropped;
+  fp.timeout_ns = wait_timeout_ns();
+  const unsigned grid = static_cast<unsigned>(d.B) * d.Hkv * d.n * fp.slices;
+  kernel<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, mv, fp);
+  return launch_result();
+}
+
+__global__ void timeout_probe_kernel(uint64_t timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    ssa::mbar_init(&bar, 1);
+    abort_flag = 0;
+    ssa::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) ssa::mbar_wait(&bar, 0, &abort_flag, timeout_ns, 0x900);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ssa_status_string(ssa_status s) {
+  switch (s) {
+    case SSA_OK: return "SSA_OK";
+    case SSA_ERR_INVALID_ARG: return "SSA_ERR_INVALID_ARG";
+    case SSA_ERR_UNSUPPORTED: return "SSA_ERR_UNSUPPORTED";
+    case SSA_ERR_CUDA: return "SSA_ERR_CUDA";
+    case SSA_ERR_DEVICE_TIMEOUT: return "SSA_ERR_DEVICE_TIMEOUT";
+    case SSA_ERR_WORKSPACE: return "SSA_ERR_WORKSPACE";
+  }
+  return "SSA_ERR_UNKNOWN";
+}
+
+uint64_t ssa_launch_count(void) { return g_launches.load(); }
+
+ssa_status ssa_block_pool(const ssa_problem* p, const ssa_bf16* k, const ssa_bf16* q,
+                          float* k_pooled, float* q_pooled, ssa_stream stream) {
+  Dims d;
+  ssa_status s = check_problem(p, &d);
+  if (s != SSA_OK) return s;
+  if (k == nullptr || k_pooled == nullptr) return SSA_ERR_INVALID_ARG;
+  if ((q == nullptr) != (q_pooled == nullptr)) return SSA_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(k_pooled) || !aligned16(q) || !aligned16(q_pooled))
+    return SSA_ERR_INVALID_ARG;
+  auto st = reinterpret_cast<cudaStream_t>(stream);
+  return d.D == 64 ? launch_pool<64>(d, k, q, k_pooled, q_pooled, st)
+                   : launch_pool<128>(d, k, q, k_pooled, q_pooled, st);
+}
+
+ssa_status ssa_block_select(const ssa_problem* p, const float* q_pooled, const float* k_pooled,
+                            int32_t* block_idx, ssa_stream stream) {
+  Dims d;
+  ssa_status s = check_problem(p, &d);
+  if (s != SSA_OK) return s;
+  if (q_pooled == nullptr || k_pooled == nullptr || block_idx == nullptr) return SSA_ERR_INVALID_ARG;
+  if (!aligned16(q_pooled) || !aligned16(k_pooled) || !aligned16(block_idx)) return SSA_ERR_INVALID_ARG;
+  static std::atomic<uint64_t> smem_done{0};
+  const int words = (d.n + 31) / 32;
+  const int smem = ssa::kSelectWarps * (d.n + words + d.D) * 4;
+  s = ensure_smem(ssa::block_select_kernel, 227 * 1024, &smem_done);
+  if (s != SSA_OK) return s;
+  ssa::SelectParams sp;
+  sp.qbar = q_pooled;
+  sp.kbar = k_pooled;
+  sp.idx = block_idx;
+  sp.n = d.n;
+  sp.D = d.D;
+  sp.topk = d.topk;
+  sp.rows = d.B * d.Hkv * d.n;
+  const unsigned grid = static_cast<unsigned>((sp.rows + ssa::kSelectWarps - 1) / ssa::kSelectWarps);
+  ssa::block_select_kernel<<<grid, 32 * ssa::kSelectWarps, smem,
+                             reinterpret_cast<cudaStream_t>(stream)>>>(sp);
+  return launch_result();
+}
+
+ssa_status ssa_sparse_attn_fwd(const ssa_problem* p, const ssa_bf16* q, const ssa_bf16* k,
+                               const ssa_bf16* v, const int32_t* block_idx, ssa_bf16* o,
+                               float* lse, ssa_stream stream) {
+  Dims d;
+  ssa_status s = check_problem(p, &d);
+  if (s != SSA_OK) return s;
+  const void* ptrs[] = {q, k, v, block_idx, o, lse};
+  for (const void* ptr : ptrs)
+    if (ptr == nullptr || !aligned16(ptr)) return SSA_ERR_INVALID_ARG;
+  auto st = reinterpret_cast<cudaStream_t>(stream);
+  if (d.D == 64)
+    return d.G >= 4 ? launch_fwd<64, 2, false>(d, q, k, v, block_idx, o, lse, nullptr, nullptr, nullptr, st)
+                    : launch_fwd<64, 1, false>(d, q, k, v, block_idx, o, lse, nullptr, nullptr, nullptr, st);
+  return d.G >= 4 ? launch_fwd<128, 2, false>(d, q, k, v, block_idx, o, lse, nullptr, nullptr, nullptr, st)
+                  : launch_fwd<128, 1, false>(d, q, k, v, block_idx, o, lse, nullptr, nullptr, nullptr, st);
+}
+
+ssa_status ssa_full_attn_fwd_with_mass(const ssa_problem* p, const ssa_bf16* q, const ssa_bf16* k,
+                                       const ssa_bf16* v, const int32_t* block_idx,
+                                       ssa_bf16* o_sparse, float* lse_sparse, ssa_bf16* o_full,
+                                       float* lse_full, float* dropped, ssa_stream stream) {
+  Dims d;
+  ssa_status s = check_problem(p, &d);
+  if (s != SSA_OK) return s;
+  const void* ptrs[] = {q, k, v, block_idx, o_sparse, lse_sparse, o_full, lse_full, dropped};
+  for (const void* ptr : ptrs)
+    if (ptr == nullptr || !aligned16(ptr)) return SSA_ERR_INVALID_ARG;
+  auto st = reinterpret_cast<cudaStream_t>(stream);
+  if (d.D == 64)
+    return d.G >= 4
+               ? launch_fwd<64, 2, true>(d, q, k, v, block_idx, o_sparse, lse_sparse, o_full, lse_full, dropped, st)
+               : launch_fwd<64, 1, true>(d, q, k, v, block_idx, o_sparse, lse_sparse, o_full, lse_full, dropped, st);
+  return launch_fwd<128, 1, true>(d, q, k, v, block_idx, o_sparse, lse_sparse, o_full, lse_full, dropped, st);
+}
+
+size_t ssa_sparse_attn_bwd_workspace(const ssa_problem* p) {
+  Dims d;
+  if (check_problem(p, &d) != SSA_OK) return 0;
+  return ssa_bwd_workspace_bytes(d.B, d.S, d.Hq, d.Hkv, d.n, d.topk);
+}
+
+ssa_status ssa_sparse_attn_bwd(const ssa_problem* p, const ssa_bf16* q, const ssa_bf16* k,
+                               const ssa_bf16* v, const ssa_bf16* o, const float* lse,
+                               const ssa_bf16* d_o, const int32_t* block_idx, ssa_bf16* dq,
+                               ssa_bf16* dk, ssa_bf16* dv, void* workspace, size_t ws_bytes,
+                               ssa_stream stream) {
+  Dims d;
+  ssa_status s = check_problem(p, &d);
+  if (s != SSA_OK) return s;
+  const void* ptrs[] = {q, k, v, o, lse, d_o, block_idx, dq, dk, dv};
+  for (const void* ptr : ptrs)
+    if (ptr == nullptr || !aligned16(ptr)) return SSA_ERR_INVALID_ARG;
+  const size_t need = ssa_bwd_workspace_bytes(d.B, d.S, d.Hq, d.Hkv, d.n, d.topk);
+  if (workspace == nullptr || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return SSA_ERR_WORKSPACE;
+  return ssa_bwd_launch(d.B, d.S, d.Hq, d.Hkv, d.D, d.G, d.n, d.topk, d.scale, q, k, v, o, lse, d_o,
+                        block_idx, dq, dk, dv, workspace, reinterpret_cast<cudaStream_t>(stream),
+                        wait_timeout_ns());
+}
+
+ssa_status ssa_get_device_error(ssa_stream stream) {
+  const cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  unsigned int word = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&word, ssa::g_error_word, sizeof(word)) != cudaSuccess)
+    return SSA_ERR_CUDA;
+  if (word != 0 && cudaMemcpyToSymbol(ssa::g_error_word, &zero, sizeof(zero)) != cudaSuccess)
+    return SSA_ERR_CUDA;
+  if (word & ssa::kErrTimeout) return SSA_ERR_DEVICE_TIMEOUT;
+  return e == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;
+}
+
+ssa_status ssa_debug_timeout_probe(int timeout_us, ssa_stream stream) {
+  if (timeout_us < 1 || timeout_us > 10000000) return SSA_ERR_INVALID_ARG;
+  timeout_probe_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint64_t>(timeout_us) * 1000ull);
+  return launch_result();
+}
+
+}  // extern "C"

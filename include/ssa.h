@@ -1,0 +1,180 @@
+/*
+ * ssa.h -- C ABI of libssa, the B200 (sm_100a) SSA sparse-stream kernels.
+ *
+ * SSA ("Sparse Sparse Attention") trains a model with a block-sparse attention
+ * stream and a full attention stream side by side.  This library implements
+ * the data-parallel hot path of the sparse stream on one GPU:
+ *
+ *   ssa_block_pool               mean-pooled block summaries of K (and of the
+ *                                GQA-group queries)
+ *   ssa_block_select             top-k block selection per query block, the
+ *                                diagonal block always kept
+ *   ssa_sparse_attn_fwd          exact softmax attention over the selected
+ *                                blocks only (online softmax, tcgen05 + TMEM)
+ *   ssa_full_attn_fwd_with_mass  the dense causal counterpart, the sparse
+ *                                output and the dropped attention mass, all
+ *                                from one launch
+ *   ssa_sparse_attn_bwd          dQ, dK, dV over the selected pairs only
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Pointers named q, k, v, o, d_o, dq, dk, dv, ... are DEVICE pointers owned
+ *    by the caller.  The library never allocates, frees or retains device
+ *    memory.  bf16 tensors are passed as ssa_bf16 (the 16-bit storage of
+ *    IEEE-754 bfloat16); every tensor is dense and contiguous.
+ *  - Layouts (row-major):
+ *        q, o, d_o, dq           [B][S][Hq][D]     bf16
+ *        k, v, dk, dv            [B][S][Hkv][D]    bf16
+ *        k_pooled, q_pooled      [B][Hkv][n][D]    fp32    n = S / block_size
+ *        block_idx               [B][Hkv][n][top_k] int32
+ *        lse, lse_*, dropped     [B][Hq][S]        fp32
+ *    Query head hq uses KV head hq / (Hq / Hkv).  Token t belongs to block
+ *    t / block_size.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream).  Arguments are validated on the host before anything is
+ *    launched: a bad argument returns SSA_ERR_INVALID_ARG and a shape this
+ *    build does not implement returns SSA_ERR_UNSUPPORTED, in both cases with
+ *    nothing launched and no output touched.  A launch failure returns
+ *    SSA_ERR_CUDA.  A kernel whose bounded wait ran out records the fact in a
+ *    device error word and exits early; ssa_get_device_error() reports it.
+ *  - Outputs are fully overwritten (dk and dv are written, not accumulated).
+ *  - Device pointers must be 16-byte aligned (TMA and vector accesses).
+ *
+ * Supported shapes in this build: block_size = 64, head_dim in {64, 128},
+ * causal = 1, seq_len a positive multiple of 64 up to 524288, Hq a multiple
+ * of Hkv with an even group size G = Hq / Hkv (2, 4, 8 or 16), top_k >= 1.
+ *
+ * Passages cited below are from the pages this method is described on:
+ *  [SSA-es]  "Resumen Tecnico: SSA (Sparse Sparse Attention)"
+ *  [SSA-it]  "SSA: Guida a Sparse Sparse Attention per LLM"
+ *  [Dash]    the DashAttention summary (hierarchical routing)
+ */
+#ifndef SSA_H_
+#define SSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SSA_OK = 0,
+  SSA_ERR_INVALID_ARG = 1,     /* null/misaligned pointer, inconsistent sizes     */
+  SSA_ERR_UNSUPPORTED = 2,     /* valid problem that this build does not implement */
+  SSA_ERR_CUDA = 3,            /* a CUDA runtime/driver call or launch failed      */
+  SSA_ERR_DEVICE_TIMEOUT = 4,  /* a kernel's bounded wait ran out (see below)      */
+  SSA_ERR_WORKSPACE = 5        /* workspace missing or smaller than required        */
+} ssa_status;
+
+typedef uint16_t ssa_bf16;               /* bfloat16 storage                       */
+typedef struct CUstream_st *ssa_stream;  /* same type as cudaStream_t              */
+
+/* The problem statement: Q/K/V shapes, block size, top-k budget, causal mask
+ * ([SSA-it] "Block-sparse attention e Receptive Field": contiguous blocks,
+ * top-k blocks per query, receptive field = block size x blocks selected). */
+typedef struct {
+  int batch;          /* B  >= 1                                                */
+  int seq_len;        /* S, multiple of block_size                               */
+  int n_q_heads;      /* Hq, multiple of n_kv_heads                              */
+  int n_kv_heads;     /* Hkv (GQA: fewer KV heads than query heads, [SSA-it]
+                         "Approccio generale" / "Training recipe")               */
+  int head_dim;       /* D                                                       */
+  int block_size;     /* query block == key block; 64 in this build              */
+  int top_k;          /* blocks per query block INCLUDING the diagonal, >= 1     */
+  int causal;         /* must be 1                                               */
+  float softmax_scale;/* <= 0 selects 1/sqrt(head_dim)                           */
+} ssa_problem;
+
+/* Mean pooling of blocks ([SSA-it] "Block-sparse attention e Receptive Field":
+ * a mean representation of each block; [Dash] Stage 0: a zero-initialised
+ * summary query is a uniform mean).
+ *   k_pooled[b,h,j,:] = (1/64) * sum_{t in block j} k[b,t,h,:]
+ *   q_pooled[b,h,i,:] = (1/(64*G)) * sum_{g<G} sum_{t in block i} q[b,t,h*G+g,:]
+ * Sums and outputs are fp32.  q and q_pooled may both be NULL (keys only). */
+ssa_status ssa_block_pool(const ssa_problem *p, const ssa_bf16 *k, const ssa_bf16 *q,
+                          float *k_pooled, float *q_pooled, ssa_stream stream);
+
+/* Top-k block selection ([SSA-it] same section: keep only the top-k most
+ * relevant earlier blocks; [Dash] Stage 1: heads sharing a KV head share one
+ * support, here by scoring the group-pooled query).  For query block i:
+ *   score(i, j) = q_pooled[i] . k_pooled[j]  (fp32) for j < i;
+ *   selected = {i} + the top_k - 1 highest-scoring j < i (ties: lower j first);
+ *   when i + 1 <= top_k every block 0..i is selected.
+ * block_idx[b,h,i,:] lists the selected blocks in ascending order, padded with
+ * -1 after the min(top_k, i + 1) valid entries. */
+ssa_status ssa_block_select(const ssa_problem *p, const float *q_pooled, const float *k_pooled,
+                            int32_t *block_idx, ssa_stream stream);
+
+/* Sparse attention forward ([SSA-es] section 2, sparse stream; [SSA-it]: the
+ * attention is computed only over the tokens of the selected blocks).
+ * For query t of block i and head hq (KV head h):
+ *   o[t]   = sum_{s in sel(i), s <= t} softmax_s(scale * q_t . k_s) * v_s
+ *   lse[t] = ln sum_{s in sel(i), s <= t} exp(scale * q_t . k_s)
+ * block_idx must satisfy the ssa_block_select output contract (ascending,
+ * diagonal present, min(top_k, i + 1) valid entries); it is trusted.
+ * o is rounded to bf16 (nearest even); lse is the natural log, fp32. */
+ssa_status ssa_sparse_attn_fwd(const ssa_problem *p, const ssa_bf16 *q, const ssa_bf16 *k,
+                               const ssa_bf16 *v, const int32_t *block_idx, ssa_bf16 *o,
+                               float *lse, ssa_stream stream);
+
+/* Full causal attention with its sparse counterpart and the dropped mass, in
+ * one launch ([SSA-es] section 2 "Alineacion Bidireccional": the opposite-mode
+ * output is computed alongside, for the alignment only; section 1: the error
+ * of sparse attention grows linearly with the attention mass it drops).
+ * Every causal block's contribution is accumulated either into the selected
+ * or into the unselected accumulator, against one shared running maximum:
+ *   o_sparse, lse_sparse  as ssa_sparse_attn_fwd
+ *   o_full, lse_full      dense causal attention over all s <= t
+ *   dropped[t]            = 1 - exp(lse_sparse[t] - lse_full[t])
+ *                         = full-softmax weight on the causal tokens not selected */
+ssa_status ssa_full_attn_fwd_with_mass(const ssa_problem *p, const ssa_bf16 *q,
+                                       const ssa_bf16 *k, const ssa_bf16 *v,
+                                       const int32_t *block_idx, ssa_bf16 *o_sparse,
+                                       float *lse_sparse, ssa_bf16 *o_full, float *lse_full,
+                                       float *dropped, ssa_stream stream);
+
+/* Bytes of device workspace ssa_sparse_attn_bwd needs for problem p (0 on an
+ * invalid problem). */
+size_t ssa_sparse_attn_bwd_workspace(const ssa_problem *p);
+
+/* Sparse attention backward ([SSA-es] section 1: keys outside the selected
+ * blocks receive zero gradient; the selection itself is not differentiated).
+ * With P_ts = exp(scale * q_t . k_s - lse_t) over the selected causal pairs:
+ *   D_t = d_o_t . o_t;  dv_s = sum_t P_ts d_o_t;  dS_ts = P_ts (d_o_t . v_s - D_t)
+ *   dq_t = scale sum_s dS_ts k_s;  dk_s = scale sum_t dS_ts q_t
+ * (sums over the G heads of a group go into dk, dv).  o and lse are the
+ * outputs of ssa_sparse_attn_fwd for the same inputs.  `workspace` is a
+ * caller-owned device buffer of at least ssa_sparse_attn_bwd_workspace(p)
+ * bytes, 256-byte aligned; its contents on entry do not matter. */
+ssa_status ssa_sparse_attn_bwd(const ssa_problem *p, const ssa_bf16 *q, const ssa_bf16 *k,
+                               const ssa_bf16 *v, const ssa_bf16 *o, const float *lse,
+                               const ssa_bf16 *d_o, const int32_t *block_idx, ssa_bf16 *dq,
+                               ssa_bf16 *dk, ssa_bf16 *dv, void *workspace, size_t ws_bytes,
+                               ssa_stream stream);
+
+/* Synchronises `stream`, then reports and clears the device error word of the
+ * current device: SSA_ERR_DEVICE_TIMEOUT if a kernel's bounded wait ran out
+ * since the last call, SSA_ERR_CUDA if the stream reported an error, else
+ * SSA_OK. */
+ssa_status ssa_get_device_error(ssa_stream stream);
+
+/* Launches one tiny kernel whose single wait can never be satisfied (an
+ * mbarrier that nothing arrives on), bounded by timeout_us microseconds of
+ * %globaltimer.  It exercises the timeout path without any fault: the kernel
+ * records SSA_ERR_DEVICE_TIMEOUT in the device error word and returns. */
+ssa_status ssa_debug_timeout_probe(int timeout_us, ssa_stream stream);
+
+/* Static, human-readable name of a status code. */
+const char *ssa_status_string(ssa_status s);
+
+/* Number of kernels this library has launched since it was loaded (all
+ * devices, all entry points); for accounting in benchmarks. */
+uint64_t ssa_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSA_H_ */

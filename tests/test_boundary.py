@@ -1,0 +1,105 @@
+"""The C ABI boundary, without a GPU: the library loads, exports every symbol
+include/ssa.h declares, and rejects bad arguments on the host before launching
+anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_sparse_attention_21_b200 as ssa
+from block_sparse_attention_21_b200 import build as ssa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ssa.h")
+
+INVALID, UNSUPPORTED, WORKSPACE = 1, 2, 5
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails first
+
+
+@pytest.fixture(scope="module")
+def lib():
+    ssa_build.build()
+    return ssa.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ssa_[a-z_]+)\s*\(", text)))
+
+
+def test_header_and_binding_agree():
+    assert sorted(ssa.EXPORTED) == declared_functions()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code, name in ssa._binding.STATUS_NAMES.items():
+        assert ssa.ssa_status_string(code) == name
+
+
+def _p(**kw):
+    base = dict(batch=1, seq_len=1024, n_q_heads=8, n_kv_heads=2, head_dim=64, top_k=4)
+    base.update(kw)
+    return ssa.problem(**base)
+
+
+BAD_PROBLEMS = [
+    (dict(batch=0), INVALID),
+    (dict(seq_len=1000), INVALID),          # not a multiple of the block
+    (dict(n_q_heads=6, n_kv_heads=4), INVALID),
+    (dict(top_k=0), INVALID),
+    (dict(head_dim=96), UNSUPPORTED),
+    (dict(block_size=128), UNSUPPORTED),
+    (dict(causal=0), UNSUPPORTED),
+    (dict(n_q_heads=2, n_kv_heads=2), UNSUPPORTED),   # G = 1
+    (dict(n_q_heads=64, n_kv_heads=2), UNSUPPORTED),  # G = 32
+    (dict(seq_len=1048576), UNSUPPORTED),
+    (dict(softmax_scale=float("nan")), INVALID),
+]
+
+
+@pytest.mark.parametrize("kw,code", BAD_PROBLEMS)
+def test_bad_problem_is_rejected_by_every_entry_point(lib, kw, code):
+    p = ctypes.byref(_p(**kw))
+    f = FAKE
+    assert lib.ssa_block_pool(p, f, f, f, f, None) == code
+    assert lib.ssa_block_select(p, f, f, f, None) == code
+    assert lib.ssa_sparse_attn_fwd(p, f, f, f, f, f, f, None) == code
+    assert lib.ssa_full_attn_fwd_with_mass(p, f, f, f, f, f, f, f, f, f, None) == code
+    assert lib.ssa_sparse_attn_bwd(p, f, f, f, f, f, f, f, f, f, f, f, 1 << 30, None) == code
+    assert lib.ssa_sparse_attn_bwd_workspace(p) == 0
+
+
+def test_null_problem(lib):
+    assert lib.ssa_sparse_attn_fwd(None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None) == INVALID
+
+
+def test_null_and_misaligned_pointers(lib):
+    p = ctypes.byref(_p())
+    f = FAKE
+    assert lib.ssa_sparse_attn_fwd(p, None, f, f, f, f, f, None) == INVALID
+    assert lib.ssa_sparse_attn_fwd(p, f, f, f, f, f + 2, f, None) == INVALID
+    assert lib.ssa_block_pool(p, f, f, f, None, None) == INVALID   # q without q_pooled
+    assert lib.ssa_block_select(p, f, None, f, None) == INVALID
+    assert lib.ssa_full_attn_fwd_with_mass(p, f, f, f, f, f, f, f, f, None, None) == INVALID
+
+
+def test_backward_workspace_is_checked_before_launch(lib):
+    p = ctypes.byref(_p())
+    need = lib.ssa_sparse_attn_bwd_workspace(p)
+    f = FAKE
+    args = [p] + [f] * 10
+    assert lib.ssa_sparse_attn_bwd(*args, None, need, None) == WORKSPACE
+    if need > 0:
+        assert lib.ssa_sparse_attn_bwd(*args, f, need - 1, None) == WORKSPACE
+    assert lib.ssa_sparse_attn_bwd(*args, f + 16, need, None) == WORKSPACE   # not 256-aligned
+
+
+def test_timeout_probe_rejects_bad_limit(lib):
+    assert lib.ssa_debug_timeout_probe(0, None) == INVALID

@@ -1,0 +1,249 @@
+"""GPU parity of the forward path (pool, select, sparse attention, full attention
+with dropped mass) against the fp64 oracle, through the C ABI.
+
+Tolerances: selected indices bit-exact (the generator guarantees a score gap
+> 1e-3 at the k-th boundary); outputs max-abs <= 2e-2 (bf16 in/out, fp32
+accumulation); dropped mass max-abs <= 1e-3; log-sum-exp max-abs <= 1e-3.
+"""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_21_b200 as ssa
+import gen
+import oracle
+from conftest import workload_inputs
+
+pytestmark = pytest.mark.gpu
+
+O_TOL, LSE_TOL, DELTA_TOL, POOL_TOL = 2e-2, 1e-3, 1e-3, 1e-5
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    from block_sparse_attention_21_b200 import build
+    build.build()
+    ssa.lib()
+
+
+def _prob(x, topk=None):
+    w = x.workload
+    return ssa.problem(w.batch, w.seq_len, w.n_q_heads, w.n_kv_heads, w.head_dim,
+                       topk or w.top_k)
+
+
+def _dev(x):
+    return x.q.to(DEV), x.k.to(DEV), x.v.to(DEV)
+
+
+def _gpu_select(p, q, k):
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    n = S // 64
+    kb = torch.empty(B, Hkv, n, D, device=DEV)
+    qb = torch.empty(B, Hkv, n, D, device=DEV)
+    idx = torch.empty(B, Hkv, n, p.top_k, dtype=torch.int32, device=DEV)
+    ssa.ssa_block_pool(p, k, q, kb, qb)
+    ssa.ssa_block_select(p, qb, kb, idx)
+    torch.cuda.synchronize()
+    return kb, qb, idx
+
+
+def _gpu_sparse(p, q, k, v, idx, pad=0):
+    B, S, Hq, D = q.shape
+    o = torch.empty(B * S * Hq * D + pad, dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty(B * Hq * S + pad, dtype=torch.float32, device=DEV)
+    if pad:
+        o[-pad:] = 7.0
+        lse[-pad:] = 7.0
+    ov = o[: B * S * Hq * D].view(B, S, Hq, D)
+    lv = lse[: B * Hq * S].view(B, Hq, S)
+    ssa.ssa_sparse_attn_fwd(p, q, k, v, idx, ov, lv)
+    torch.cuda.synchronize()
+    if pad:
+        assert torch.all(o[-pad:] == 7.0) and torch.all(lse[-pad:] == 7.0), "wrote past the end"
+    return ov, lv
+
+
+def _gpu_mass(p, q, k, v, idx):
+    B, S, Hq, D = q.shape
+    o = torch.empty(B, S, Hq, D, dtype=torch.bfloat16, device=DEV)
+    of = torch.empty_like(o)
+    lse = torch.empty(B, Hq, S, device=DEV)
+    lsef = torch.empty_like(lse)
+    dm = torch.empty_like(lse)
+    ssa.ssa_full_attn_fwd_with_mass(p, q, k, v, idx, o, lse, of, lsef, dm)
+    torch.cuda.synchronize()
+    return o, lse, of, lsef, dm
+
+
+def _rows_of(o, lse, rows):
+    """Gather [R, D] outputs and [R] lse for (b, hq, t) rows."""
+    r = torch.as_tensor(rows, device=DEV, dtype=torch.long)
+    ov = o[r[:, 0], r[:, 2], r[:, 1]].float().cpu().numpy()
+    lv = lse[r[:, 0], r[:, 1], r[:, 2]].cpu().numpy()
+    return ov, lv
+
+
+def _sample_rows(B, Hq, S, n_random, seed, blocks=()):
+    rng = np.random.Generator(np.random.PCG64(seed))
+    rows = [np.stack([rng.integers(0, B, n_random), rng.integers(0, Hq, n_random),
+                      rng.integers(0, S, n_random)], axis=1)]
+    for i in blocks:        # every row of a few whole query blocks (all heads of batch 0)
+        t = np.arange(64 * i, 64 * i + 64)
+        for hq in range(Hq):
+            rows.append(np.stack([np.zeros_like(t), np.full_like(t, hq), t], axis=1))
+    return np.concatenate(rows).astype(np.int64)
+
+
+def _check_select(x, p, kb, qb, idx):
+    okb, oqb = oracle.block_pool(x.k, x.q)
+    np.testing.assert_allclose(kb.cpu().numpy(), okb, atol=POOL_TOL, rtol=0)
+    np.testing.assert_allclose(qb.cpu().numpy(), oqb, atol=POOL_TOL, rtol=0)
+    oidx, _ = oracle.block_select(oqb, okb, p.top_k)
+    gidx = idx.cpu().numpy()
+    mism = np.argwhere(gidx != oidx)
+    assert mism.size == 0, f"{len(mism)} index mismatches, first {mism[:3].tolist()}"
+    return oidx
+
+
+# ------------------------------------------------------------ small, every row
+
+SMALL = [
+    # (B, S, Hq, Hkv, D, topk, n_plant)   several tiles, early rows with < k blocks
+    (1, 1024, 4, 1, 64, 4, 0),      # the tiny workload's shape, T = 2
+    (2, 320, 8, 2, 64, 3, 2),       # 5 blocks, B = 2, G = 4
+    (1, 576, 4, 2, 128, 4, 3),      # D = 128, G = 2 (one M-tile per CTA)
+    (1, 512, 16, 1, 64, 2, 3),      # G = 16 (two CTAs per group)
+    (1, 384, 8, 1, 128, 3, 2),      # D = 128, G = 8
+    (2, 256, 4, 2, 64, 1, 0),       # diagonal block only
+    (1, 448, 4, 1, 64, 16, 0),      # budget above the block count: dense causal
+]
+
+
+@pytest.mark.parametrize("shape", SMALL, ids=lambda s: "x".join(map(str, s)))
+def test_small_problems_every_row(shape):
+    B, S, Hq, Hkv, D, topk, npl = shape
+    x = gen.make_custom(B, S, Hq, Hkv, D, topk, seed=100 + S + D + topk, n_plant=npl)
+    p = ssa.problem(B, S, Hq, Hkv, D, topk)
+    q, k, v = _dev(x)
+    kb, qb, idx = _gpu_select(p, q, k)
+    okb, oqb = oracle.block_pool(x.k, x.q)
+    oidx, gap = oracle.block_select(oqb, okb, topk)
+    gidx = idx.cpu().numpy()
+    # rows whose boundary is closer than the guaranteed gap may legitimately differ
+    close = ~np.isnan(gap) & (gap <= 1e-3)
+    assert np.array_equal(gidx[~close], oidx[~close])
+    rows = oracle.all_rows(B, Hq, S)
+    ref = oracle.attn_rows(x.q, x.k, x.v, gidx, rows, want_full=True)
+    o, lse = _gpu_sparse(p, q, k, v, idx, pad=4096)
+    ov, lv = _rows_of(o, lse, rows)
+    assert np.abs(ov - ref["o_sparse"]).max() <= O_TOL
+    assert np.abs(lv - ref["lse_sparse"]).max() <= LSE_TOL
+    mo, ml, mof, mlf, mdm = _gpu_mass(p, q, k, v, idx)
+    mov, mlv = _rows_of(mo, ml, rows)
+    fov, flv = _rows_of(mof, mlf, rows)
+    _, dmv = _rows_of(mof, mdm, rows)
+    assert np.abs(mov - ref["o_sparse"]).max() <= O_TOL
+    assert np.abs(mlv - ref["lse_sparse"]).max() <= LSE_TOL
+    assert np.abs(fov - ref["o_full"]).max() <= O_TOL
+    assert np.abs(flv - ref["lse_full"]).max() <= LSE_TOL
+    assert np.abs(dmv - ref["delta"]).max() <= DELTA_TOL
+
+
+def test_tiny_workload_every_row_and_deterministic():
+    x = workload_inputs("tiny_1k")
+    p = _prob(x)
+    q, k, v = _dev(x)
+    kb, qb, idx = _gpu_select(p, q, k)
+    oidx = _check_select(x, p, kb, qb, idx)
+    rows = oracle.all_rows(1, 4, 1024)
+    ref = oracle.attn_rows(x.q, x.k, x.v, oidx, rows, want_full=True)
+    o, lse = _gpu_sparse(p, q, k, v, idx)
+    o2, lse2 = _gpu_sparse(p, q, k, v, idx)
+    assert torch.equal(o.view(torch.int16), o2.view(torch.int16)) and torch.equal(lse, lse2)
+    ov, lv = _rows_of(o, lse, rows)
+    assert np.abs(ov - ref["o_sparse"]).max() <= O_TOL
+    assert np.abs(lv - ref["lse_sparse"]).max() <= LSE_TOL
+    mo, ml, mof, mlf, mdm = _gpu_mass(p, q, k, v, idx)
+    fov, flv = _rows_of(mof, mlf, rows)
+    _, dmv = _rows_of(mof, mdm, rows)
+    assert np.abs(fov - ref["o_full"]).max() <= O_TOL
+    assert np.abs(flv - ref["lse_full"]).max() <= LSE_TOL
+    assert np.abs(dmv - ref["delta"]).max() <= DELTA_TOL
+    # sparse output of the alignment launch equals the sparse launch's
+    assert torch.equal(mo.view(torch.int16), o.view(torch.int16)) or \
+        (mo.float() - o.float()).abs().max().item() <= 2 * O_TOL
+
+
+# -------------------------------------------------------- full-size workloads
+
+@pytest.mark.parametrize("name", ["llama1b_8k", "train_8k"])
+def test_sparse_forward_full_size_sampled(name):
+    x = workload_inputs(name)
+    p = _prob(x)
+    q, k, v = _dev(x)
+    kb, qb, idx = _gpu_select(p, q, k)
+    oidx = _check_select(x, p, kb, qb, idx)
+    w = x.workload
+    rows = _sample_rows(w.batch, w.n_q_heads, w.seq_len, 3000, seed=7, blocks=(0, 17, w.n_blocks - 1))
+    ref = oracle.attn_rows(x.q, x.k, x.v, oidx, rows, want_full=False)
+    o, lse = _gpu_sparse(p, q, k, v, idx)
+    ov, lv = _rows_of(o, lse, rows)
+    assert np.abs(ov - ref["o_sparse"]).max() <= O_TOL
+    assert np.abs(lv - ref["lse_sparse"]).max() <= LSE_TOL
+    assert torch.isfinite(o.float()).all()
+
+
+@pytest.mark.parametrize("topk", [8, 16, 32, 64, 128])
+def test_long_context_budget_sweep_sampled(topk):
+    x = workload_inputs("long_32k")
+    p = _prob(x, topk)
+    q, k, v = _dev(x)
+    kb, qb, idx = _gpu_select(p, q, k)
+    oidx = _check_select(x, p, kb, qb, idx)
+    rows = _sample_rows(1, 16, 32768, 1500, seed=topk, blocks=(0, 511))
+    ref = oracle.attn_rows(x.q, x.k, x.v, oidx, rows, want_full=False)
+    o, lse = _gpu_sparse(p, q, k, v, idx)
+    ov, lv = _rows_of(o, lse, rows)
+    assert np.abs(ov - ref["o_sparse"]).max() <= O_TOL
+    assert np.abs(lv - ref["lse_sparse"]).max() <= LSE_TOL
+
+
+def test_alignment_pass_full_size_sampled():
+    x = workload_inputs("align_8k")
+    p = _prob(x)
+    q, k, v = _dev(x)
+    kb, qb, idx = _gpu_select(p, q, k)
+    oidx = _check_select(x, p, kb, qb, idx)
+    rows = _sample_rows(2, 32, 8192, 1500, seed=3, blocks=(0, 127))
+    ref = oracle.attn_rows(x.q, x.k, x.v, oidx, rows, want_full=True)
+    o, lse, of, lsef, dm = _gpu_mass(p, q, k, v, idx)
+    ov, lv = _rows_of(o, lse, rows)
+    fov, flv = _rows_of(of, lsef, rows)
+    _, dmv = _rows_of(of, dm, rows)
+    assert np.abs(ov - ref["o_sparse"]).max() <= O_TOL
+    assert np.abs(lv - ref["lse_sparse"]).max() <= LSE_TOL
+    assert np.abs(fov - ref["o_full"]).max() <= O_TOL
+    assert np.abs(flv - ref["lse_full"]).max() <= LSE_TOL
+    assert np.abs(dmv - ref["delta"]).max() <= DELTA_TOL
+    # properties at every position: 0 <= delta <= 1, delta = 0 where i < k
+    dmc = dm.cpu()
+    assert float(dmc.min()) >= 0.0 and float(dmc.max()) <= 1.0
+    assert torch.all(dmc[:, :, : 64 * 16] == 0.0)
+
+
+def test_device_timeout_is_reported_and_context_survives():
+    ssa.ssa_debug_timeout_probe(2000)
+    assert ssa.ssa_get_device_error() == 4
+    assert ssa.ssa_get_device_error() == 0
+    x = gen.make_custom(1, 256, 4, 1, 64, 2, seed=1)
+    p = ssa.problem(1, 256, 4, 1, 64, 2)
+    q, k, v = _dev(x)
+    _, _, idx = _gpu_select(p, q, k)
+    o, _ = _gpu_sparse(p, q, k, v, idx)
+    assert torch.isfinite(o.float()).all()
+    assert ssa.ssa_get_device_error() == 0
