@@ -15,19 +15,24 @@
 // Warp roles (128 * (T + 1) threads):
 //   warp 0      TMA producer: the Q tiles once, then K and V of each visited
 //               block through an NS-stage ring (index-guided loads).
-//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer:
-//               S_t = Q_t K^T (both operands in shared memory), then
-//               O_t += P_t V (P_t read from TMEM, V in shared memory).
+//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer.  Per
+//               visited block jj and M-tile t, in this order:
+//                 wait P_t(jj);  O_t += P_t(jj) V(jj);  S_t = Q_t K(jj+1)^T
+//               so one commit of S_t(jj+1) also tells the softmax warps that
+//               O_t is stable.  P_t lives in the first 32 TMEM columns of S_t;
+//               the tensor pipe executes one thread's MMAs in issue order, so
+//               S_t(jj+1) overwrites P_t(jj) only after P.V has read it.
 //   warps 2-3   build the selection bitmap (MASS), otherwise idle.
 //   warps 4..   one warpgroup per M-tile: thread r owns row r of the tile;
-//               online softmax in the exp2 domain with lazy rescaling
-//               (the running maximum only moves when it grows by > 8, i.e.
-//               a factor 256), P written back to TMEM as bf16, O rescaled in
-//               TMEM when needed, and the epilogue.
+//               online softmax in the exp2 domain with lazy rescaling (the
+//               reference maximum only moves when the row maximum exceeds it
+//               by more than 8, i.e. a factor 256), P written back to TMEM as
+//               bf16 pairs, O rescaled in TMEM when the maximum moved, and
+//               the epilogue.
 //
-// TMEM layout per M-tile t (base t * 512 / T): S at +0 (64 columns), P at +64
-// (32 columns of bf16 pairs), O (O_selected with MASS) at +128 (D columns),
-// O_unselected at +128 + D (MASS only).
+// TMEM per M-tile t (stride 64 + D, or 64 + 2D with MASS): S/P at +0
+// (64 columns of fp32 scores; P overwrites columns 0..31 as bf16 pairs),
+// O (O_selected with MASS) at +64, O_unselected at +64 + D (MASS only).
 #pragma once
 
 #include "sm100.cuh"
@@ -46,21 +51,92 @@ struct FwdParams {
   uint64_t timeout_ns;
 };
 
+__host__ __device__ constexpr int pow2_at_least(int x) {
+  return x <= 32 ? 32 : x <= 64 ? 64 : x <= 128 ? 128 : x <= 256 ? 256 : 512;
+}
+
 template <int D, int T, bool MASS>
 struct FwdConfig {
   static constexpr int NP = D / 64;               // 64-column panels per row
   static constexpr int QTILE = 128 * D * 2;       // bytes of one Q M-tile
   static constexpr int KVT = 64 * D * 2;          // bytes of one K (or V) block
   static constexpr int NS = (D == 64) ? 4 : 3;    // K/V ring stages
-  static constexpr int TSTRIDE = 512 / T;         // TMEM columns per M-tile
+  static constexpr int TSTRIDE = 64 + (MASS ? 2 : 1) * D;  // TMEM columns per M-tile
+  static constexpr int TMEM_COLS = pow2_at_least(T * TSTRIDE);
   static constexpr int THREADS = 128 * (T + 1);
-  static constexpr int NBARS = 1 + 3 * NS + 4 * T + 1;
+  static constexpr int NBARS = 2 + 3 * NS + 3 * T;
   // shared memory: Q tiles, K ring, V ring, barriers, tmem slot, abort flag,
   // selection bitmap (up to 8192 blocks)
   static constexpr int SMEM_TILES = T * QTILE + 2 * NS * KVT;
   static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + NBARS * 8 + 16 + 1024;
-  static_assert((MASS ? 128 + 2 * D : 128 + D) <= TSTRIDE, "TMEM budget per M-tile");
+  static_assert(T * TSTRIDE <= 512, "TMEM budget");
 };
+
+// Packed fp32 pair helpers (Blackwell f32x2 FMA-pipe instructions).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Row maximum of 32 raw scores; on the diagonal block keys past the row's own
+// token (column c0 + c > tq) are excluded.
+template <bool DIAG>
+__device__ __forceinline__ float row_max32(const float (&s)[32], int c0, int tq, float m) {
+#pragma unroll
+  for (int c = 0; c < 32; c += 2) {
+    float a = s[c], b = s[c + 1];
+    if (DIAG) {
+      if (c0 + c > tq) a = -INFINITY;
+      if (c0 + c + 1 > tq) b = -INFINITY;
+    }
+    m = max3f(m, a, b);
+  }
+  return m;
+}
+
+// p = 2^(s * scale_log2 - m_ref) for 32 scores, summed into the pair
+// accumulator and packed to 16 bf16 pairs.
+template <bool DIAG>
+__device__ __forceinline__ void exp_pack32(const float (&s)[32], int c0, int tq, uint64_t scale2,
+                                           uint64_t negm2, uint64_t& acc, uint32_t (&pk)[16]) {
+#pragma unroll
+  for (int c = 0; c < 32; c += 2) {
+    const uint64_t x = f2_fma(f2_pack(s[c], s[c + 1]), scale2, negm2);
+    float x0, x1;
+    f2_unpack(x, x0, x1);
+    if (DIAG) {
+      if (c0 + c > tq) x0 = -INFINITY;
+      if (c0 + c + 1 > tq) x1 = -INFINITY;
+    }
+    const float p0 = ex2(x0), p1 = ex2(x1);
+    acc = f2_add(acc, f2_pack(p0, p1));
+    pk[c / 2] = pack_bf16x2(p0, p1);
+  }
+}
 
 template <int D, int T, bool MASS>
 __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, 1)
@@ -81,11 +157,10 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, 1)
   uint64_t* bar_vfull = bar_kfull + NS;
   uint64_t* bar_empty = bar_vfull + NS;
   uint64_t* bar_sfull = bar_empty + NS;
-  uint64_t* bar_sfree = bar_sfull + T;
-  uint64_t* bar_pfull = bar_sfree + T;
+  uint64_t* bar_pfull = bar_sfull + T;
   uint64_t* bar_odone = bar_pfull + T;
-  uint64_t* bar_mma_done = bar_odone + T;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_mma_done + 1);
+  uint64_t* bar_drain = bar_odone + T;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint32_t* selbits = tmem_slot + 4;
 
@@ -113,11 +188,10 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, 1)
     }
     for (int t = 0; t < T; ++t) {
       mbar_init(&bar_sfull[t], 1);
-      mbar_init(&bar_sfree[t], 128);
       mbar_init(&bar_pfull[t], 128);
       mbar_init(&bar_odone[t], 1);
     }
-    mbar_init(bar_mma_done, 1);
+    mbar_init(bar_drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -131,7 +205,7 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, 1)
     }
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 512);
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -152,6 +226,7 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, 1)
           for (int pn = 0; pn < NP; ++pn)
             tma_load_4d(sQ + t * QTILE + pn * (128 * 128) + hh * (64 * 128), &tm_q, bar_q,
                         64 * pn, hq0 + 2 * t + hh, 64 * i, b);
+      int issued = 0;
       for (int jj = 0; jj < nblk; ++jj) {
         const int st = jj % NS, use = jj / NS;
         if (use > 0 && !mbar_wait(&bar_empty[st], (use - 1) & 1, abort_flag, tmo, 0x101)) break;
@@ -162,14 +237,13 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, 1)
         mbar_arrive_expect_tx(&bar_vfull[st], KVT);
         for (int pn = 0; pn < NP; ++pn)
           tma_load_4d(sV + st * KVT + pn * (64 * 128), &tm_v, &bar_vfull[st], 64 * pn, h, 64 * j, b);
+        ++issued;
       }
-      // loads are never left in flight: every issued stage is consumed by the
-      // MMA issuer, or on abort waited for here (bounded)
+      // on abort, loads already issued are waited for (bounded) before exit
       if (*abort_flag) {
-        for (int s = 0; s < NS; ++s) {
-          volatile int never = 0;
-          mbar_wait(&bar_kfull[s], 0, &never, 1000000ull, 0x1ff);
-        }
+        volatile int never = 0;
+        for (int jj = (issued > NS ? issued - NS : 0); jj < issued; ++jj)
+          mbar_wait(&bar_vfull[jj % NS], (jj / NS) & 1, &never, 1000000ull, 0x1ff);
       }
     }
   } else if (warp == 1) {
@@ -178,7 +252,6 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, 1)
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 64, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
-      bool ok = mbar_wait(bar_q, 0, abort_flag, tmo, 0x201);
       auto issue_qk = [&](int t, int st) {
         const uint32_t d = tmem + t * TSTRIDE;
 #pragma unroll
@@ -189,45 +262,41 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, 1)
           mma_ss(d, a, bd, idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
-      if (ok && nblk > 0) {
-        ok = mbar_wait(&bar_kfull[0], 0, abort_flag, tmo, 0x202);
-        if (ok) {
-          tc_fence_after();
-          for (int t = 0; t < T; ++t) {
-            issue_qk(t, 0);
-            tc_commit(&bar_sfull[t]);
-          }
+      bool ok = mbar_wait(bar_q, 0, abort_flag, tmo, 0x201) &&
+                mbar_wait(&bar_kfull[0], 0, abort_flag, tmo, 0x202);
+      if (ok) {
+        tc_fence_after();
+        for (int t = 0; t < T; ++t) {
+          issue_qk(t, 0);
+          tc_commit(&bar_sfull[t]);
         }
       }
       bool first_sel = true, first_uns = true;
       for (int jj = 0; ok && jj < nblk; ++jj) {
         const int st = jj % NS;
-        if (jj + 1 < nblk) {
-          const int st1 = (jj + 1) % NS;
-          if (!mbar_wait(&bar_kfull[st1], ((jj + 1) / NS) & 1, abort_flag, tmo, 0x203)) break;
-          for (int t = 0; t < T; ++t) {
-            if (!mbar_wait(&bar_sfree[t], jj & 1, abort_flag, tmo, 0x204)) { ok = false; break; }
-            tc_fence_after();
-            issue_qk(t, st1);
-            tc_commit(&bar_sfull[t]);
-          }
-          if (!ok) break;
-        }
-        if (!mbar_wait(&bar_vfull[st], (jj / NS) & 1, abort_flag, tmo, 0x205)) break;
+        const bool more = jj + 1 < nblk;
+        const int st1 = (jj + 1) % NS;
+        if (!mbar_wait(&bar_vfull[st], (jj / NS) & 1, abort_flag, tmo, 0x203)) break;
+        if (more && !mbar_wait(&bar_kfull[st1], ((jj + 1) / NS) & 1, abort_flag, tmo, 0x204)) break;
         bool is_sel = true;
         if (MASS) is_sel = (selbits[jj >> 5] >> (jj & 31)) & 1u;
         const bool first = MASS ? (is_sel ? first_sel : first_uns) : (jj == 0);
         for (int t = 0; t < T; ++t) {
-          if (!mbar_wait(&bar_pfull[t], jj & 1, abort_flag, tmo, 0x206)) { ok = false; break; }
+          if (!mbar_wait(&bar_pfull[t], jj & 1, abort_flag, tmo, 0x205)) { ok = false; break; }
           tc_fence_after();
           const uint32_t base = tmem + t * TSTRIDE;
-          const uint32_t o_col = base + 128 + ((MASS && !is_sel) ? D : 0);
+          const uint32_t o_col = base + 64 + ((MASS && !is_sel) ? D : 0);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t bd = sdesc_sw128(sVa + st * KVT + kk * (16 * 128), 64 * 128, 1024);
-            mma_ts(o_col, base + 64 + kk * 8, bd, idesc_pv, (first && kk == 0) ? 0u : 1u);
+            mma_ts(o_col, base + kk * 8, bd, idesc_pv, (first && kk == 0) ? 0u : 1u);
           }
-          tc_commit(&bar_odone[t]);
+          if (more) {
+            issue_qk(t, st1);
+            tc_commit(&bar_sfull[t]);
+          } else {
+            tc_commit(&bar_odone[t]);
+          }
         }
         if (!ok) break;
         if (MASS) {
@@ -235,10 +304,12 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, 1)
         }
         tc_commit(&bar_empty[st]);
       }
-      // every issued MMA has completed before TMEM is released
-      tc_commit(bar_mma_done);
-      volatile int never = 0;
-      mbar_wait(bar_mma_done, 0, &never, tmo, 0x2ff);
+      if (!ok) {
+        // every issued MMA completes before TMEM is released (bounded wait)
+        tc_commit(bar_drain);
+        volatile int never = 0;
+        mbar_wait(bar_drain, 0, &never, tmo, 0x2ff);
+      }
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax
@@ -248,9 +319,12 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, 1)
     const int hh = r / 64, tq = r % 64;
     const int hq = hq0 + 2 * t + hh;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16) + t * TSTRIDE;
-    const uint32_t tS = lane_base, tP = lane_base + 64, tO = lane_base + 128;
+    const uint32_t tS = lane_base, tO = lane_base + 64;
     const uint32_t tOu = tO + D;
-    float m_ref = -INFINITY, l_sel = 0.f, l_uns = 0.f;
+    const float sl2 = p.scale_log2;
+    const uint64_t scale2 = f2_pack(sl2, sl2);
+    float m_ref = -INFINITY;  // reference maximum, scaled (log2) units
+    float l_sel = 0.f, l_uns = 0.f;
     bool ok = true;
     for (int jj = 0; jj < nblk; ++jj) {
       // waits are made warp-uniform: the tcgen05.ld/st below are .sync.aligned
@@ -259,77 +333,73 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, 1)
         break;
       }
       tc_fence_after();
-      float s[64];
-      {
-        float a[32], c2[32];
-        tmem_ld32(tS, a);
-        tmem_ld32(tS + 32, c2);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) { s[c] = a[c]; s[32 + c] = c2[c]; }
-      }
-      tc_fence_before();
-      mbar_arrive(&bar_sfree[t]);
       const bool diag = (jj == nblk - 1);
       bool is_sel = true;
       if (MASS) is_sel = (selbits[jj >> 5] >> (jj & 31)) & 1u;
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        float x = s[c] * p.scale_log2;
-        if (diag && c > tq) x = -INFINITY;
-        s[c] = x;
-        mx = fmaxf(mx, x);
+      // raw row maximum over both halves; half A (columns 0..31) stays in registers
+      float sA[32];
+      float mx;
+      {
+        float sB[32];
+        tmem_ld32(tS + 32, sB);
+        mx = diag ? row_max32<true>(sB, 32, tq, -INFINITY) : row_max32<false>(sB, 32, tq, -INFINITY);
       }
+      tmem_ld32(tS, sA);
+      mx = diag ? row_max32<true>(sA, 0, tq, mx) : row_max32<false>(sA, 0, tq, mx);
+      const float mx_s = mx * sl2;
       float alpha = 1.f;
-      bool resc = false;
-      if (mx > m_ref + 8.f) {
-        alpha = ex2(m_ref - mx);
-        m_ref = mx;
-        resc = (jj > 0);
+      const bool moved = mx_s > m_ref + 8.f;
+      if (moved) {
+        alpha = ex2(m_ref - mx_s);
+        m_ref = mx_s;
       }
-      float rs = 0.f;
-      uint32_t pk[32];
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float p0 = ex2(s[2 * c] - m_ref);
-        const float p1 = ex2(s[2 * c + 1] - m_ref);
-        rs += p0 + p1;
-        pk[c] = pack_bf16x2(p0, p1);
+      const uint64_t negm2 = f2_pack(-m_ref, -m_ref);
+      uint64_t acc2 = f2_pack(0.f, 0.f);
+      uint32_t pk[16];
+      if (diag) exp_pack32<true>(sA, 0, tq, scale2, negm2, acc2, pk);
+      else exp_pack32<false>(sA, 0, tq, scale2, negm2, acc2, pk);
+      tmem_st16(tS, pk);  // P columns 0..15 over S columns 0..15 (already read)
+      {
+        float sB[32];
+        tmem_ld32(tS + 32, sB);
+        if (diag) exp_pack32<true>(sB, 32, tq, scale2, negm2, acc2, pk);
+        else exp_pack32<false>(sB, 32, tq, scale2, negm2, acc2, pk);
       }
+      tmem_st16(tS + 16, pk);  // P columns 16..31
+      float r0, r1;
+      f2_unpack(acc2, r0, r1);
       l_sel *= alpha;
       l_uns *= alpha;
-      if (is_sel) l_sel += rs; else l_uns += rs;
-      if (jj > 0) {
-        if (!__all_sync(0xffffffffu,
-                        mbar_wait(&bar_odone[t], (jj - 1) & 1, abort_flag, tmo, 0x302))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, resc)) {
+      if (is_sel) l_sel += r0 + r1; else l_uns += r0 + r1;
+      // O is stable here (S(jj) was committed after P(jj-1).V) and is read by
+      // the tensor core only after pfull: rescale it when the maximum moved
+      if (jj > 0 && __any_sync(0xffffffffu, moved)) {
+        const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
-          for (int acc = 0; acc < (MASS ? 2 : 1); ++acc) {
-            const uint32_t base = acc ? tOu : tO;
+        for (int acc = 0; acc < (MASS ? 2 : 1); ++acc) {
+          const uint32_t base = acc ? tOu : tO;
 #pragma unroll
-            for (int ch = 0; ch < D / 32; ++ch) {
-              float o[32];
-              uint32_t w[32];
-              tmem_ld32(base + ch * 32, o);
+          for (int ch = 0; ch < D / 16; ++ch) {
+            float o[16];
+            uint32_t w[16];
+            tmem_ld16(base + ch * 16, o);
 #pragma unroll
-              for (int c = 0; c < 32; ++c) w[c] = __float_as_uint(o[c] * alpha);
-              tmem_st32(base + ch * 32, w);
+            for (int c = 0; c < 16; c += 2) {
+              float lo, hi;
+              f2_unpack(f2_mul(f2_pack(o[c], o[c + 1]), a2), lo, hi);
+              w[c] = __float_as_uint(lo);
+              w[c + 1] = __float_as_uint(hi);
             }
+            tmem_st16(base + ch * 16, w);
           }
         }
       }
-      tmem_st32(tP, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bar_pfull[t]);
     }
     // ---------------------------------------------------------- epilogue
-    if (ok && __all_sync(0xffffffffu,
-                         mbar_wait(&bar_odone[t], (nblk - 1) & 1, abort_flag, tmo, 0x303))) {
+    if (ok && __all_sync(0xffffffffu, mbar_wait(&bar_odone[t], 0, abort_flag, tmo, 0x303))) {
       tc_fence_after();
       const int tok = 64 * i + tq;
       const size_t orow = ((static_cast<size_t>(b) * p.S + tok) * p.Hq + hq) * D;
@@ -378,7 +448,7 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 

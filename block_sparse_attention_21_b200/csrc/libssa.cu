@@ -252,11 +252,15 @@ ssa_status ssa_sparse_attn_fwd(const ssa_problem* p, const ssa_bf16* q, const ss
   for (const void* ptr : ptrs)
     if (ptr == nullptr || !aligned16(ptr)) return SSA_ERR_INVALID_ARG;
   auto st = reinterpret_cast<cudaStream_t>(stream);
-  if (d.D == 64)
-    return d.G >= 4 ? launch_fwd<64, 2, false>(d, q, k, v, block_idx, o, lse, nullptr, nullptr, nullptr, st)
-                    : launch_fwd<64, 1, false>(d, q, k, v, block_idx, o, lse, nullptr, nullptr, nullptr, st);
-  return d.G >= 4 ? launch_fwd<128, 2, false>(d, q, k, v, block_idx, o, lse, nullptr, nullptr, nullptr, st)
-                  : launch_fwd<128, 1, false>(d, q, k, v, block_idx, o, lse, nullptr, nullptr, nullptr, st);
+  // M-tiles per CTA: as many head pairs of the group as TMEM holds (4 at D=64,
+  // 2 at D=128)
+  if (d.D == 64) {
+    if (d.G >= 8) return launch_fwd<64, 4, false>(d, q, k, v, block_idx, o, lse, nullptr, nullptr, nullptr, st);
+    if (d.G == 4) return launch_fwd<64, 2, false>(d, q, k, v, block_idx, o, lse, nullptr, nullptr, nullptr, st);
+    return launch_fwd<64, 1, false>(d, q, k, v, block_idx, o, lse, nullptr, nullptr, nullptr, st);
+  }
+  if (d.G >= 4) return launch_fwd<128, 2, false>(d, q, k, v, block_idx, o, lse, nullptr, nullptr, nullptr, st);
+  return launch_fwd<128, 1, false>(d, q, k, v, block_idx, o, lse, nullptr, nullptr, nullptr, st);
 }
 
 ssa_status ssa_full_attn_fwd_with_mass(const ssa_problem* p, const ssa_bf16* q, const ssa_bf16* k,
