@@ -13,13 +13,15 @@ import torch
 
 from ._binding import (EXPORTED, LIB_PATH, SsaError, SsaProblem, lib, problem,
                        ssa_block_pool, ssa_block_select, ssa_debug_timeout_probe,
-                       ssa_full_attn_fwd_with_mass, ssa_get_device_error, ssa_launch_count,
+                       ssa_full_attn_fwd_with_mass, ssa_get_device_error,
+                       ssa_get_device_error_site, ssa_launch_count,
                        ssa_sparse_attn_bwd, ssa_sparse_attn_bwd_workspace,
                        ssa_sparse_attn_fwd, ssa_status_string)
 
 __all__ = ["EXPORTED", "LIB_PATH", "SsaError", "SsaProblem", "SparseStream", "lib", "problem",
            "ssa_block_pool", "ssa_block_select", "ssa_debug_timeout_probe",
-           "ssa_full_attn_fwd_with_mass", "ssa_get_device_error", "ssa_launch_count",
+           "ssa_full_attn_fwd_with_mass", "ssa_get_device_error", "ssa_get_device_error_site",
+           "ssa_launch_count",
            "ssa_sparse_attn_bwd", "ssa_sparse_attn_bwd_workspace", "ssa_sparse_attn_fwd",
            "ssa_status_string"]
 
@@ -65,6 +67,20 @@ class SparseStream:
         ssa_full_attn_fwd_with_mass(self.p, q, k, v, self.block_idx, self.o, self.lse, o_full,
                                     lse_full, dropped, stream)
         return self.o, o_full, dropped
+
+    def capture_forward(self, q, k, v) -> "torch.cuda.CUDAGraph":
+        """A CUDA graph of forward() over these exact buffers (pool, select and
+        sparse attention: three kernel launches); graph.replay() reruns it on
+        the current stream.  Refill q, k, v in place to run on new data."""
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            self.forward(q, k, v)          # first call sets kernel attributes
+        torch.cuda.current_stream().wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            self.forward(q, k, v)
+        return graph
 
     def backward(self, q, k, v, d_o, stream=None):
         if self._grad is None:

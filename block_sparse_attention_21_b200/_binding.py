@@ -25,7 +25,8 @@ STATUS_NAMES = {0: "SSA_OK", 1: "SSA_ERR_INVALID_ARG", 2: "SSA_ERR_UNSUPPORTED",
 # every symbol include/ssa.h declares
 EXPORTED = ("ssa_block_pool", "ssa_block_select", "ssa_sparse_attn_fwd",
             "ssa_full_attn_fwd_with_mass", "ssa_sparse_attn_bwd_workspace",
-            "ssa_sparse_attn_bwd", "ssa_get_device_error", "ssa_debug_timeout_probe",
+            "ssa_sparse_attn_bwd", "ssa_get_device_error", "ssa_get_device_error_site",
+            "ssa_debug_timeout_probe",
             "ssa_status_string", "ssa_launch_count")
 
 
@@ -78,6 +79,8 @@ def lib():
         L.ssa_sparse_attn_bwd_workspace.restype = ctypes.c_size_t
         L.ssa_status_string.argtypes = [ctypes.c_int]
         L.ssa_status_string.restype = ctypes.c_char_p
+        L.ssa_get_device_error_site.argtypes = []
+        L.ssa_get_device_error_site.restype = ctypes.c_uint
         L.ssa_launch_count.argtypes = []
         L.ssa_launch_count.restype = ctypes.c_uint64
         _lib = L
@@ -190,6 +193,10 @@ def ssa_sparse_attn_bwd(p: SsaProblem, q, k, v, o, lse, d_o, block_idx, dq, dk, 
 def ssa_get_device_error(stream=None) -> int:
     """Status code (not raised): 0 OK, 4 a bounded device wait ran out."""
     return int(lib().ssa_get_device_error(_stream(stream)))
+
+
+def ssa_get_device_error_site() -> int:
+    return int(lib().ssa_get_device_error_site())
 
 
 def ssa_debug_timeout_probe(timeout_us: int, stream=None) -> None:

@@ -12,17 +12,24 @@
 // one pass ("Resumen Tecnico: SSA", section 2, "Alineacion Bidireccional",
 // and section 1 on the dropped mass).
 //
+// Two CTAs share an SM when T = 2 (256 TMEM columns each), so one CTA's
+// prologue and epilogue overlap the other's main loop.
+//
 // Warp roles (128 * (T + 1) threads):
 //   warp 0      TMA producer: the Q tiles once, then K and V of each visited
 //               block through an NS-stage ring (index-guided loads).
-//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer.  Per
-//               visited block jj and M-tile t, in this order:
+//   warps 1-2   TMEM allocation (warp 1) and the tcgen05.mma issuers (two
+//               when T = 4, else one), one elected thread each, owning
+//               alternate M-tiles; an issuer polls its tiles and issues for
+//               whichever is ready, and releases a K/V stage with one commit
+//               once all its tiles are done with it.  Per visited block jj
+//               and M-tile t, in this order:
 //                 wait P_t(jj);  O_t += P_t(jj) V(jj);  S_t = Q_t K(jj+1)^T
 //               so one commit of S_t(jj+1) also tells the softmax warps that
 //               O_t is stable.  P_t lives in the first 32 TMEM columns of S_t;
 //               the tensor pipe executes one thread's MMAs in issue order, so
 //               S_t(jj+1) overwrites P_t(jj) only after P.V has read it.
-//   warps 2-3   build the selection bitmap (MASS), otherwise idle.
+//   warp 3      builds the selection bitmap (MASS), otherwise idle.
 //   warps 4..   one warpgroup per M-tile: thread r owns row r of the tile;
 //               online softmax in the exp2 domain with lazy rescaling (the
 //               reference maximum only moves when the row maximum exceeds it
@@ -36,24 +43,9 @@
 #pragma once
 
 #include "sm100.cuh"
+#include "softmax_util.cuh"
 
 namespace ssa {
-
-struct FwdParams {
-  int B, S, Hq, Hkv, G, n, topk, slices;
-  float scale_log2;  // softmax scale * log2(e)
-  const int32_t* idx;
-  __nv_bfloat16* o;      // sparse output
-  float* lse;            // sparse log-sum-exp (natural log)
-  __nv_bfloat16* o_full; // MASS: dense causal output
-  float* lse_full;       // MASS
-  float* dropped;        // MASS: dropped attention mass
-  uint64_t timeout_ns;
-};
-
-__host__ __device__ constexpr int pow2_at_least(int x) {
-  return x <= 32 ? 32 : x <= 64 ? 64 : x <= 128 ? 128 : x <= 256 ? 256 : 512;
-}
 
 template <int D, int T, bool MASS>
 struct FwdConfig {
@@ -64,82 +56,20 @@ struct FwdConfig {
   static constexpr int TSTRIDE = 64 + (MASS ? 2 : 1) * D;  // TMEM columns per M-tile
   static constexpr int TMEM_COLS = pow2_at_least(T * TSTRIDE);
   static constexpr int THREADS = 128 * (T + 1);
-  static constexpr int NBARS = 2 + 3 * NS + 3 * T;
+  static constexpr int ISS = T >= 4 ? 2 : 1;      // MMA issuer warps (warps 1..ISS)
+  static constexpr int NBARS = 1 + ISS + 3 * NS + 3 * T;
   // shared memory: Q tiles, K ring, V ring, barriers, tmem slot, abort flag,
   // selection bitmap (up to 8192 blocks)
   static constexpr int SMEM_TILES = T * QTILE + 2 * NS * KVT;
   static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + NBARS * 8 + 16 + 1024;
+  // two CTAs share an SM when both fit in TMEM (256 columns each) and in
+  // shared memory: one CTA's prologue and epilogue overlap the other's loop
+  static constexpr int MIN_CTAS = (TMEM_COLS <= 256 && SMEM_BYTES <= 113 * 1024) ? 2 : 1;
   static_assert(T * TSTRIDE <= 512, "TMEM budget");
 };
 
-// Packed fp32 pair helpers (Blackwell f32x2 FMA-pipe instructions).
-__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
-}
-__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ float max3f(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-
-// Row maximum of 32 raw scores; on the diagonal block keys past the row's own
-// token (column c0 + c > tq) are excluded.
-template <bool DIAG>
-__device__ __forceinline__ float row_max32(const float (&s)[32], int c0, int tq, float m) {
-#pragma unroll
-  for (int c = 0; c < 32; c += 2) {
-    float a = s[c], b = s[c + 1];
-    if (DIAG) {
-      if (c0 + c > tq) a = -INFINITY;
-      if (c0 + c + 1 > tq) b = -INFINITY;
-    }
-    m = max3f(m, a, b);
-  }
-  return m;
-}
-
-// p = 2^(s * scale_log2 - m_ref) for 32 scores, summed into the pair
-// accumulator and packed to 16 bf16 pairs.
-template <bool DIAG>
-__device__ __forceinline__ void exp_pack32(const float (&s)[32], int c0, int tq, uint64_t scale2,
-                                           uint64_t negm2, uint64_t& acc, uint32_t (&pk)[16]) {
-#pragma unroll
-  for (int c = 0; c < 32; c += 2) {
-    const uint64_t x = f2_fma(f2_pack(s[c], s[c + 1]), scale2, negm2);
-    float x0, x1;
-    f2_unpack(x, x0, x1);
-    if (DIAG) {
-      if (c0 + c > tq) x0 = -INFINITY;
-      if (c0 + c + 1 > tq) x1 = -INFINITY;
-    }
-    const float p0 = ex2(x0), p1 = ex2(x1);
-    acc = f2_add(acc, f2_pack(p0, p1));
-    pk[c / 2] = pack_bf16x2(p0, p1);
-  }
-}
-
 template <int D, int T, bool MASS>
-__global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, 1)
+__global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, FwdConfig<D, T, MASS>::MIN_CTAS)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   using C = FwdConfig<D, T, MASS>;
@@ -160,7 +90,7 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, 1)
   uint64_t* bar_pfull = bar_sfull + T;
   uint64_t* bar_odone = bar_pfull + T;
   uint64_t* bar_drain = bar_odone + T;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_drain + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_drain + C::ISS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint32_t* selbits = tmem_slot + 4;
 
@@ -184,18 +114,18 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, 1)
     for (int s = 0; s < NS; ++s) {
       mbar_init(&bar_kfull[s], 1);
       mbar_init(&bar_vfull[s], 1);
-      mbar_init(&bar_empty[s], 1);
+      mbar_init(&bar_empty[s], C::ISS);  // released once per issuer
     }
     for (int t = 0; t < T; ++t) {
       mbar_init(&bar_sfull[t], 1);
       mbar_init(&bar_pfull[t], 128);
       mbar_init(&bar_odone[t], 1);
     }
-    mbar_init(bar_drain, 1);
+    for (int x = 0; x < C::ISS; ++x) mbar_init(&bar_drain[x], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (MASS && warp == 2) {
+  if (MASS && warp == 3) {
     const int words = (p.n + 31) / 32;
     for (int w = lane; w < words; w += 32) selbits[w] = 0u;
     __syncwarp();
@@ -246,9 +176,16 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, 1)
           mbar_wait(&bar_vfull[jj % NS], (jj / NS) & 1, &never, 1000000ull, 0x1ff);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp >= 1 && warp <= C::ISS) {
+    // ------------------------------------------------------------ MMA issuers
+    // Issuer warp w owns M-tiles t = w - 1, w - 1 + ISS, ...; it polls their
+    // P-ready barriers and issues for whichever tile is ready, so a slow tile
+    // does not hold up the others.  A K/V stage is released after all T
+    // tiles committed their use of it.
     if (lane == 0) {
+      constexpr int ISS = C::ISS;
+      constexpr int MT = (T + ISS - 1) / ISS;  // tiles per issuer
+      const int me = warp - 1;
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 64, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
@@ -266,24 +203,45 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, 1)
                 mbar_wait(&bar_kfull[0], 0, abort_flag, tmo, 0x202);
       if (ok) {
         tc_fence_after();
-        for (int t = 0; t < T; ++t) {
+        for (int t = me; t < T; t += ISS) {
           issue_qk(t, 0);
           tc_commit(&bar_sfull[t]);
         }
       }
-      bool first_sel = true, first_uns = true;
-      for (int jj = 0; ok && jj < nblk; ++jj) {
-        const int st = jj % NS;
-        const bool more = jj + 1 < nblk;
-        const int st1 = (jj + 1) % NS;
-        if (!mbar_wait(&bar_vfull[st], (jj / NS) & 1, abort_flag, tmo, 0x203)) break;
-        if (more && !mbar_wait(&bar_kfull[st1], ((jj + 1) / NS) & 1, abort_flag, tmo, 0x204)) break;
-        bool is_sel = true;
-        if (MASS) is_sel = (selbits[jj >> 5] >> (jj & 31)) & 1u;
-        const bool first = MASS ? (is_sel ? first_sel : first_uns) : (jj == 0);
-        for (int t = 0; t < T; ++t) {
-          if (!mbar_wait(&bar_pfull[t], jj & 1, abort_flag, tmo, 0x205)) { ok = false; break; }
+      int next[MT];
+      bool first_sel[MT], first_uns[MT];
+      int remaining = 0, own = 0;
+      uint32_t stage_uses = 0;  // per K/V stage (8 bits each): own tiles done with its current use
+#pragma unroll
+      for (int x = 0; x < MT; ++x) {
+        next[x] = 0;
+        first_sel[x] = first_uns[x] = true;
+        if (me + x * ISS < T) {
+          remaining += nblk;
+          ++own;
+        }
+      }
+      uint64_t t_last = globaltimer_ns();
+      while (ok && remaining > 0) {
+        bool progressed = false;
+#pragma unroll
+        for (int x = 0; x < MT; ++x) {
+          const int t = me + x * ISS;
+          const int jj = next[x];
+          if (t >= T || jj >= nblk || !ok) continue;
+          if (!mbar_test(&bar_pfull[t], jj & 1)) continue;
+          const int st = jj % NS;
+          const bool more = jj + 1 < nblk;
+          const int st1 = (jj + 1) % NS;
+          if (!mbar_wait(&bar_vfull[st], (jj / NS) & 1, abort_flag, tmo, 0x203) ||
+              (more && !mbar_wait(&bar_kfull[st1], ((jj + 1) / NS) & 1, abort_flag, tmo, 0x204))) {
+            ok = false;
+            continue;
+          }
           tc_fence_after();
+          bool is_sel = true;
+          if (MASS) is_sel = (selbits[jj >> 5] >> (jj & 31)) & 1u;
+          const bool first = MASS ? (is_sel ? first_sel[x] : first_uns[x]) : (jj == 0);
           const uint32_t base = tmem + t * TSTRIDE;
           const uint32_t o_col = base + 64 + ((MASS && !is_sel) ? D : 0);
 #pragma unroll
@@ -297,18 +255,37 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, 1)
           } else {
             tc_commit(&bar_odone[t]);
           }
+          stage_uses += 1u << (8 * st);
+          if (((stage_uses >> (8 * st)) & 0xffu) == static_cast<uint32_t>(own)) {
+            tc_commit(&bar_empty[st]);  // this issuer's tiles are all done with the stage
+            stage_uses &= ~(0xffu << (8 * st));
+          }
+          if (MASS) {
+            if (is_sel) first_sel[x] = false; else first_uns[x] = false;
+          }
+          next[x] = jj + 1;
+          --remaining;
+          progressed = true;
         }
-        if (!ok) break;
-        if (MASS) {
-          if (is_sel) first_sel = false; else first_uns = false;
+        if (progressed) {
+          t_last = globaltimer_ns();
+        } else if (MT == 1 && ok && remaining > 0) {
+          // one tile: a suspending wait costs the softmax warps no issue slots
+          ok = mbar_wait(&bar_pfull[me], next[0] & 1, abort_flag, tmo, 0x205);
+        } else if (*abort_flag) {
+          ok = false;
+        } else if (globaltimer_ns() - t_last > tmo) {
+          report_timeout(abort_flag, 0x205);
+          ok = false;
+        } else {
+          __nanosleep(32);  // back off: the softmax warps share this scheduler
         }
-        tc_commit(&bar_empty[st]);
       }
       if (!ok) {
-        // every issued MMA completes before TMEM is released (bounded wait)
-        tc_commit(bar_drain);
+        // every MMA this thread issued completes before TMEM is released
+        tc_commit(&bar_drain[me]);
         volatile int never = 0;
-        mbar_wait(bar_drain, 0, &never, tmo, 0x2ff);
+        mbar_wait(&bar_drain[me], 0, &never, tmo, 0x2ff);
       }
     }
   } else if (warp >= 4) {

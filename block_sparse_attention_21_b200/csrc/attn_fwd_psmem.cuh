@@ -1,0 +1,415 @@
+// attn_fwd_psmem.cuh -- block-sparse causal attention forward on tcgen05 tensor
+// cores, with P staged in shared memory (the variant used at head_dim 128).
+//
+// One CTA handles one query block i (64 tokens) of one batch entry for 2*T
+// query heads that share KV head h.  Its rows form T M-tiles of 128 rows
+// (2 heads x 64 tokens).  The KV blocks it visits are either the selected
+// blocks of the index table (sparse stream: "SSA: Guida a Sparse Sparse
+// Attention per LLM", section "Block-sparse attention e Receptive Field",
+// attention computed only over the tokens of the selected blocks) or, with
+// MASS, every causal block 0..i, each one's P.V going to the selected or the
+// unselected accumulator against one shared running maximum, which yields the
+// dense counterpart, the sparse output and the dropped attention mass from
+// one pass ("Resumen Tecnico: SSA", section 2, "Alineacion Bidireccional",
+// and section 1 on the dropped mass).
+//
+// Pipeline per M-tile t and visited block jj:
+//   S_t(jj) = Q_t K(jj)^T          tensor core, fp32 in TMEM
+//   softmax warps load S_t(jj) into registers and release it at once, so the
+//   issuer can start S_t(jj+1) while they exponentiate
+//   P_t(jj) (bf16) -> shared memory, 128-byte swizzled like Q
+//   O_t += P_t(jj) V(jj)           tensor core, A and B from shared memory
+// so the score MMA of the next block and the P.V of this block both overlap
+// the softmax.  O is rescaled in TMEM (lazily, see below) after the previous
+// P.V has completed.
+//
+// Warp roles (128 * (T + 1) threads):
+//   warp 0      TMA producer: the Q tiles once, then K and V of each visited
+//               block through an NS-stage ring (index-guided loads).
+//   issuers     one warp per M-tile (warps 1, 2, 3 and, for a fourth tile,
+//               the warp after the softmax warpgroups); one elected thread
+//               issues that tile's tcgen05.mma in order, waiting (suspended,
+//               no issue slots taken) on its "S consumed" and "P ready"
+//               barriers.  Warp 1 also allocates TMEM; warp 3 first builds
+//               the selection bitmap (MASS).
+//   warps 4..   one warpgroup per M-tile: thread r owns row r of the tile;
+//               online softmax in the exp2 domain with lazy rescaling (the
+//               reference maximum only moves when the row maximum exceeds it
+//               by more than 8, i.e. a factor 256), and the epilogue.
+//
+// TMEM per M-tile t (stride 64 + D, or 64 + 2D with MASS): S at +0 (64 fp32
+// columns), O (O_selected with MASS) at +64, O_unselected at +64 + D.
+#pragma once
+
+#include "sm100.cuh"
+#include "softmax_util.cuh"
+
+namespace ssa {
+
+template <int D, int T, bool MASS>
+struct PsFwdConfig {
+  static constexpr int NP = D / 64;               // 64-column panels per row
+  static constexpr int QTILE = 128 * D * 2;       // bytes of one Q M-tile
+  static constexpr int KVT = 64 * D * 2;          // bytes of one K (or V) block
+  static constexpr int PTILE = 128 * 64 * 2;      // bytes of one P tile (128 rows x 64 keys)
+  static constexpr int NS = (D == 64) ? 4 : 3;    // K/V ring stages
+  static constexpr int TSTRIDE = 64 + (MASS ? 2 : 1) * D;  // TMEM columns per M-tile
+  static constexpr int TMEM_COLS = pow2_at_least(T * TSTRIDE);
+  // warps: 0 producer, 1..3 issuers, 4.. softmax (4 per tile), then the
+  // issuer of a fourth tile
+  static constexpr int THREADS = 128 * (T + 1) + (T > 3 ? 32 : 0);
+  // barriers: q, kfull/vfull/empty[NS], sfull/sfree/pfull/pvdone/odone/drain[T]
+  static constexpr int NBARS = 1 + 3 * NS + 6 * T;
+  // shared memory: Q tiles, K ring, V ring, P tiles, barriers, tmem slot,
+  // abort flag, selection bitmap (up to 8192 blocks)
+  static constexpr int SMEM_TILES = T * QTILE + 2 * NS * KVT + T * PTILE;
+  static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + NBARS * 8 + 16 + 1024;
+  static_assert(T * TSTRIDE <= 512, "TMEM budget");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+// Warp that issues the MMAs of M-tile t.
+template <int T>
+__device__ __forceinline__ int ps_issuer_warp(int t) {
+  return t < 3 ? 1 + t : 4 + 4 * T;
+}
+
+template <int D, int T, bool MASS>
+__global__ void __launch_bounds__(PsFwdConfig<D, T, MASS>::THREADS, 1)
+    attn_fwd_psmem_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using C = PsFwdConfig<D, T, MASS>;
+  constexpr int NP = C::NP, QTILE = C::QTILE, KVT = C::KVT, PTILE = C::PTILE, NS = C::NS,
+                TSTRIDE = C::TSTRIDE;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem;                 // [T][QTILE]
+  uint8_t* sK = sQ + T * QTILE;       // [NS][KVT]
+  uint8_t* sV = sK + NS * KVT;        // [NS][KVT]
+  uint8_t* sP = sV + NS * KVT;        // [T][PTILE]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + T * PTILE);
+  uint64_t* bar_q = bars;
+  uint64_t* bar_kfull = bar_q + 1;              // [NS]
+  uint64_t* bar_vfull = bar_kfull + NS;
+  uint64_t* bar_empty = bar_vfull + NS;
+  uint64_t* bar_sfull = bar_empty + NS;         // [T] scores in TMEM
+  uint64_t* bar_sfree = bar_sfull + T;          // [T] scores read by the softmax
+  uint64_t* bar_pfull = bar_sfree + T;          // [T] P in shared memory (O rescaled)
+  uint64_t* bar_pvdone = bar_pfull + T;         // [T] P.V completed
+  uint64_t* bar_odone = bar_pvdone + T;         // [T] last P.V completed
+  uint64_t* bar_drain = bar_odone + T;          // [T] issuer's MMAs drained (abort)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_drain + T);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint32_t* selbits = tmem_slot + 4;
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  // work unit, heaviest query blocks first
+  const int per_i = p.B * p.Hkv * p.slices;
+  const int i = p.n - 1 - static_cast<int>(blockIdx.x) / per_i;
+  int rem = static_cast<int>(blockIdx.x) % per_i;
+  const int slice = rem % p.slices;
+  rem /= p.slices;
+  const int h = rem % p.Hkv;
+  const int b = rem / p.Hkv;
+  const int hq0 = h * p.G + slice * 2 * T;
+  const int nsel = min(p.topk, i + 1);
+  const int nblk = MASS ? (i + 1) : nsel;
+  const int32_t* idx_row = p.idx + ((static_cast<size_t>(b) * p.Hkv + h) * p.n + i) * p.topk;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&bar_kfull[s], 1);
+      mbar_init(&bar_vfull[s], 1);
+      mbar_init(&bar_empty[s], T);  // released by each tile's issuer
+    }
+    for (int t = 0; t < T; ++t) {
+      mbar_init(&bar_sfull[t], 1);
+      mbar_init(&bar_sfree[t], 128);
+      mbar_init(&bar_pfull[t], 128);
+      mbar_init(&bar_pvdone[t], 1);
+      mbar_init(&bar_odone[t], 1);
+      mbar_init(&bar_drain[t], 1);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (MASS && warp == 3) {
+    const int words = (p.n + 31) / 32;
+    for (int w = lane; w < words; w += 32) selbits[w] = 0u;
+    __syncwarp();
+    for (int r = lane; r < nsel; r += 32) {
+      const int j = idx_row[r];
+      if (j >= 0 && j <= i) atomicOr(&selbits[j >> 5], 1u << (j & 31));
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint64_t tmo = p.timeout_ns;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_arrive_expect_tx(bar_q, T * QTILE);
+      for (int t = 0; t < T; ++t)
+        for (int hh = 0; hh < 2; ++hh)
+          for (int pn = 0; pn < NP; ++pn)
+            tma_load_4d(sQ + t * QTILE + pn * (128 * 128) + hh * (64 * 128), &tm_q, bar_q,
+                        64 * pn, hq0 + 2 * t + hh, 64 * i, b);
+      int issued = 0;
+      for (int jj = 0; jj < nblk; ++jj) {
+        const int st = jj % NS, use = jj / NS;
+        if (use > 0 && !mbar_wait(&bar_empty[st], (use - 1) & 1, abort_flag, tmo, 0x101)) break;
+        const int j = MASS ? jj : idx_row[jj];
+        mbar_arrive_expect_tx(&bar_kfull[st], KVT);
+        for (int pn = 0; pn < NP; ++pn)
+          tma_load_4d(sK + st * KVT + pn * (64 * 128), &tm_k, &bar_kfull[st], 64 * pn, h, 64 * j, b);
+        mbar_arrive_expect_tx(&bar_vfull[st], KVT);
+        for (int pn = 0; pn < NP; ++pn)
+          tma_load_4d(sV + st * KVT + pn * (64 * 128), &tm_v, &bar_vfull[st], 64 * pn, h, 64 * j, b);
+        ++issued;
+      }
+      // on abort, loads already issued are waited for (bounded) before exit
+      if (*abort_flag) {
+        volatile int never = 0;
+        for (int jj = (issued > NS ? issued - NS : 0); jj < issued; ++jj)
+          mbar_wait(&bar_vfull[jj % NS], (jj / NS) & 1, &never, 1000000ull, 0x1ff);
+      }
+    }
+  } else if (warp != 0 && (warp < 4 || warp >= 4 + 4 * T)) {
+    // ------------------------------------------------------------ MMA issuers
+    // The issuer of tile t walks  S(0);  then for s = 0, 1, ...:
+    //   [S(s) read]  S(s+1);   [P(s) in shared memory]  O += P(s) V(s)
+    int t = -1;
+#pragma unroll
+    for (int x = 0; x < T; ++x)
+      if (ps_issuer_warp<T>(x) == warp) t = x;
+    if (lane == 0 && t >= 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 64, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
+      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV), sPa = smem_u32(sP);
+      const uint32_t s_tmem = tmem + t * TSTRIDE;
+      auto issue_qk = [&](int st) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk % 4) * 32;  // 16 bf16 = 32 B inside the 128 B row
+          const uint64_t a = sdesc_sw128(sQa + t * QTILE + (kk / 4) * (128 * 128) + off, 16, 1024);
+          const uint64_t bd = sdesc_sw128(sKa + st * KVT + (kk / 4) * (64 * 128) + off, 16, 1024);
+          mma_ss(s_tmem, a, bd, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(bar_q, 0, abort_flag, tmo, 0x201) &&
+                mbar_wait(&bar_kfull[0], 0, abort_flag, tmo, 0x202);
+      if (ok) {
+        tc_fence_after();
+        issue_qk(0);
+        tc_commit(&bar_sfull[t]);
+      }
+      bool first_sel = true, first_uns = true;
+      for (int s = 0; ok && s < nblk; ++s) {
+        if (s + 1 < nblk) {
+          // S(s+1) as soon as the softmax has read S(s)
+          const int st1 = (s + 1) % NS;
+          if (!mbar_wait(&bar_sfree[t], s & 1, abort_flag, tmo, 0x203) ||
+              !mbar_wait(&bar_kfull[st1], ((s + 1) / NS) & 1, abort_flag, tmo, 0x204)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_qk(st1);
+          tc_commit(&bar_sfull[t]);
+        }
+        // P(s).V once P(s) is in shared memory
+        const int st = s % NS;
+        if (!mbar_wait(&bar_pfull[t], s & 1, abort_flag, tmo, 0x205) ||
+            !mbar_wait(&bar_vfull[st], (s / NS) & 1, abort_flag, tmo, 0x206)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        bool is_sel = true;
+        if (MASS) is_sel = (selbits[s >> 5] >> (s & 31)) & 1u;
+        const bool first = MASS ? (is_sel ? first_sel : first_uns) : (s == 0);
+        const uint32_t o_col = s_tmem + 64 + ((MASS && !is_sel) ? D : 0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t a = sdesc_sw128(sPa + t * PTILE + kk * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(sVa + st * KVT + kk * (16 * 128), 64 * 128, 1024);
+          mma_ss(o_col, a, bd, idesc_pv, (first && kk == 0) ? 0u : 1u);
+        }
+        tc_commit(&bar_pvdone[t]);
+        if (s + 1 == nblk) tc_commit(&bar_odone[t]);
+        tc_commit(&bar_empty[st]);
+        if (MASS) {
+          if (is_sel) first_sel = false; else first_uns = false;
+        }
+      }
+      if (!ok) {
+        // every MMA this thread issued completes before TMEM is released
+        tc_commit(&bar_drain[t]);
+        volatile int never = 0;
+        mbar_wait(&bar_drain[t], 0, &never, tmo, 0x2ff);
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax
+    const int t = (warp - 4) / 4;
+    const int wq = warp % 4;
+    const int r = wq * 32 + lane;
+    const int hh = r / 64, tq = r % 64;
+    const int hq = hq0 + 2 * t + hh;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16) + t * TSTRIDE;
+    const uint32_t tS = lane_base, tO = lane_base + 64;
+    const uint32_t tOu = tO + D;
+    // this row of the P tile: 8 chunks of 16 B (8 keys each), 128-byte swizzle
+    uint8_t* prow = sP + t * PTILE + r * 128;
+    const float sl2 = p.scale_log2;
+    const uint64_t scale2 = f2_pack(sl2, sl2);
+    float m_ref = -INFINITY;  // reference maximum, scaled (log2) units
+    float l_sel = 0.f, l_uns = 0.f;
+    bool ok = true;
+    for (int jj = 0; jj < nblk; ++jj) {
+      // waits are made warp-uniform: the tcgen05.ld/st below are .sync.aligned
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar_sfull[t], jj & 1, abort_flag, tmo, 0x301))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float sA[32], sB[32];
+      tmem_ld32(tS, sA);
+      tmem_ld32(tS + 32, sB);
+      // the scores are in registers: the issuer may overwrite S with the next block's
+      tc_fence_before();
+      mbar_arrive(&bar_sfree[t]);
+      const bool diag = (jj == nblk - 1);
+      bool is_sel = true;
+      if (MASS) is_sel = (selbits[jj >> 5] >> (jj & 31)) & 1u;
+      float mx = diag ? row_max32<true>(sB, 32, tq, -INFINITY) : row_max32<false>(sB, 32, tq, -INFINITY);
+      mx = diag ? row_max32<true>(sA, 0, tq, mx) : row_max32<false>(sA, 0, tq, mx);
+      const float mx_s = mx * sl2;
+      float alpha = 1.f;
+      const bool moved = mx_s > m_ref + 8.f;
+      if (moved) {
+        alpha = ex2(m_ref - mx_s);
+        m_ref = mx_s;
+      }
+      const uint64_t negm2 = f2_pack(-m_ref, -m_ref);
+      uint64_t acc2 = f2_pack(0.f, 0.f);
+      uint32_t pk[32];
+      if (diag) {
+        exp_pack32<true>(sA, 0, tq, scale2, negm2, acc2, pk);
+        exp_pack32<true>(sB, 32, tq, scale2, negm2, acc2, pk + 16);
+      } else {
+        exp_pack32<false>(sA, 0, tq, scale2, negm2, acc2, pk);
+        exp_pack32<false>(sB, 32, tq, scale2, negm2, acc2, pk + 16);
+      }
+      float r0, r1;
+      f2_unpack(acc2, r0, r1);
+      l_sel *= alpha;
+      l_uns *= alpha;
+      if (is_sel) l_sel += r0 + r1; else l_uns += r0 + r1;
+      if (jj > 0) {
+        // P(jj-1).V has finished: the P tile may be overwritten and O is stable
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar_pvdone[t], (jj - 1) & 1, abort_flag, tmo, 0x302))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, moved)) {
+          const uint64_t a2 = f2_pack(alpha, alpha);
+#pragma unroll
+          for (int acc = 0; acc < (MASS ? 2 : 1); ++acc) {
+            const uint32_t base = acc ? tOu : tO;
+#pragma unroll
+            for (int ch = 0; ch < D / 16; ++ch) {
+              float o[16];
+              uint32_t w[16];
+              tmem_ld16(base + ch * 16, o);
+#pragma unroll
+              for (int c = 0; c < 16; c += 2) {
+                float lo, hi;
+                f2_unpack(f2_mul(f2_pack(o[c], o[c + 1]), a2), lo, hi);
+                w[c] = __float_as_uint(lo);
+                w[c + 1] = __float_as_uint(hi);
+              }
+              tmem_st16(base + ch * 16, w);
+            }
+          }
+          tmem_wait_st();
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) =
+            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bar_pfull[t]);
+    }
+    // ---------------------------------------------------------- epilogue
+    if (ok && __all_sync(0xffffffffu, mbar_wait(&bar_odone[t], 0, abort_flag, tmo, 0x303))) {
+      tc_fence_after();
+      const int tok = 64 * i + tq;
+      const size_t orow = ((static_cast<size_t>(b) * p.S + tok) * p.Hq + hq) * D;
+      const size_t lrow = (static_cast<size_t>(b) * p.Hq + hq) * p.S + tok;
+      const bool has_uns = MASS && (nblk > nsel);
+      const float inv_sel = 1.f / l_sel;
+      const float l_all = l_sel + (has_uns ? l_uns : 0.f);
+      const float inv_all = 1.f / l_all;
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) {
+        float o[32];
+        tmem_ld32(tO + ch * 32, o);
+        uint32_t w[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) w[c] = pack_bf16x2(o[2 * c] * inv_sel, o[2 * c + 1] * inv_sel);
+        uint4* dst = reinterpret_cast<uint4*>(p.o + orow + ch * 32);
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4)
+          dst[v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+        if (MASS) {
+          if (has_uns) {
+            float ou[32];
+            tmem_ld32(tOu + ch * 32, ou);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] += ou[c];
+          }
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            w[c] = pack_bf16x2(o[2 * c] * inv_all, o[2 * c + 1] * inv_all);
+          uint4* dstf = reinterpret_cast<uint4*>(p.o_full + orow + ch * 32);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            dstf[v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+        }
+      }
+      constexpr float kLn2 = 0.69314718055994530942f;
+      p.lse[lrow] = (m_ref + log2f(l_sel)) * kLn2;
+      if (MASS) {
+        p.lse_full[lrow] = (m_ref + log2f(l_all)) * kLn2;
+        p.dropped[lrow] = has_uns ? (l_uns / l_all) : 0.f;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace ssa

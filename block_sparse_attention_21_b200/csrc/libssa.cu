@@ -15,6 +15,7 @@
 #include "sm100.cuh"
 #include "pool_select.cuh"
 #include "attn_fwd.cuh"
+#include "attn_fwd_psmem.cuh"
 #include "attn_bwd.cuh"
 
 namespace {
@@ -133,7 +134,7 @@ ssa_status launch_pool(const Dims& d, const void* k, const void* q, float* kb, f
   pp.Hkv = d.Hkv;
   pp.G = d.G;
   pp.n = d.n;
-  ssa::block_pool_kernel<D><<<dim3(d.n, d.Hkv, d.B), 256, 0, st>>>(pp);
+  ssa::block_pool_kernel<D><<<dim3(d.n, 2 * d.Hkv, d.B), 256, 0, st>>>(pp);
   return launch_result();
 }
 
@@ -144,6 +145,42 @@ ssa_status launch_fwd(const Dims& d, const void* q, const void* k, const void* v
   using C = ssa::FwdConfig<D, T, MASS>;
   static std::atomic<uint64_t> smem_done{0};
   auto kernel = ssa::attn_fwd_kernel<D, T, MASS>;
+  ssa_status s = ensure_smem(kernel, C::SMEM_BYTES, &smem_done);
+  if (s != SSA_OK) return s;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, D, d.Hq, d.S, d.B) || !make_map(&mk, k, D, d.Hkv, d.S, d.B) ||
+      !make_map(&mv, v, D, d.Hkv, d.S, d.B))
+    return SSA_ERR_CUDA;
+  ssa::FwdParams fp;
+  fp.B = d.B;
+  fp.S = d.S;
+  fp.Hq = d.Hq;
+  fp.Hkv = d.Hkv;
+  fp.G = d.G;
+  fp.n = d.n;
+  fp.topk = d.topk;
+  fp.slices = (d.G / 2) / T;
+  fp.scale_log2 = d.scale * 1.4426950408889634f;
+  fp.idx = idx;
+  fp.o = static_cast<__nv_bfloat16*>(o);
+  fp.lse = lse;
+  fp.o_full = static_cast<__nv_bfloat16*>(of);
+  fp.lse_full = lsef;
+  fp.dropped = dropped;
+  fp.timeout_ns = wait_timeout_ns();
+  const unsigned grid = static_cast<unsigned>(d.B) * d.Hkv * d.n * fp.slices;
+  kernel<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, mv, fp);
+  return launch_result();
+}
+
+// The same launch for the kernel that stages P in shared memory.
+template <int D, int T, bool MASS>
+ssa_status launch_psfwd(const Dims& d, const void* q, const void* k, const void* v,
+                      const int32_t* idx, void* o, float* lse, void* of, float* lsef,
+                      float* dropped, cudaStream_t st) {
+  using C = ssa::PsFwdConfig<D, T, MASS>;
+  static std::atomic<uint64_t> smem_done{0};
+  auto kernel = ssa::attn_fwd_psmem_kernel<D, T, MASS>;
   ssa_status s = ensure_smem(kernel, C::SMEM_BYTES, &smem_done);
   if (s != SSA_OK) return s;
   CUtensorMap mq, mk, mv;
@@ -223,22 +260,27 @@ ssa_status ssa_block_select(const ssa_problem* p, const float* q_pooled, const f
   if (s != SSA_OK) return s;
   if (q_pooled == nullptr || k_pooled == nullptr || block_idx == nullptr) return SSA_ERR_INVALID_ARG;
   if (!aligned16(q_pooled) || !aligned16(k_pooled) || !aligned16(block_idx)) return SSA_ERR_INVALID_ARG;
-  static std::atomic<uint64_t> smem_done{0};
-  const int words = (d.n + 31) / 32;
-  const int smem = ssa::kSelectWarps * (d.n + words + d.D) * 4;
-  s = ensure_smem(ssa::block_select_kernel, 227 * 1024, &smem_done);
-  if (s != SSA_OK) return s;
   ssa::SelectParams sp;
   sp.qbar = q_pooled;
   sp.kbar = k_pooled;
   sp.idx = block_idx;
   sp.n = d.n;
-  sp.D = d.D;
   sp.topk = d.topk;
   sp.rows = d.B * d.Hkv * d.n;
+  const size_t smem = static_cast<size_t>(ssa::kSelectWarps) * d.n * 4;
   const unsigned grid = static_cast<unsigned>((sp.rows + ssa::kSelectWarps - 1) / ssa::kSelectWarps);
-  ssa::block_select_kernel<<<grid, 32 * ssa::kSelectWarps, smem,
-                             reinterpret_cast<cudaStream_t>(stream)>>>(sp);
+  auto st = reinterpret_cast<cudaStream_t>(stream);
+  if (d.D == 64) {
+    static std::atomic<uint64_t> done{0};
+    s = ensure_smem(ssa::block_select_kernel<64>, 200 * 1024, &done);
+    if (s != SSA_OK) return s;
+    ssa::block_select_kernel<64><<<grid, 32 * ssa::kSelectWarps, smem, st>>>(sp);
+  } else {
+    static std::atomic<uint64_t> done{0};
+    s = ensure_smem(ssa::block_select_kernel<128>, 200 * 1024, &done);
+    if (s != SSA_OK) return s;
+    ssa::block_select_kernel<128><<<grid, 32 * ssa::kSelectWarps, smem, st>>>(sp);
+  }
   return launch_result();
 }
 
@@ -252,15 +294,15 @@ ssa_status ssa_sparse_attn_fwd(const ssa_problem* p, const ssa_bf16* q, const ss
   for (const void* ptr : ptrs)
     if (ptr == nullptr || !aligned16(ptr)) return SSA_ERR_INVALID_ARG;
   auto st = reinterpret_cast<cudaStream_t>(stream);
-  // M-tiles per CTA: as many head pairs of the group as TMEM holds (4 at D=64,
-  // 2 at D=128)
-  if (d.D == 64) {
-    if (d.G >= 8) return launch_fwd<64, 4, false>(d, q, k, v, block_idx, o, lse, nullptr, nullptr, nullptr, st);
-    if (d.G == 4) return launch_fwd<64, 2, false>(d, q, k, v, block_idx, o, lse, nullptr, nullptr, nullptr, st);
-    return launch_fwd<64, 1, false>(d, q, k, v, block_idx, o, lse, nullptr, nullptr, nullptr, st);
-  }
-  if (d.G >= 4) return launch_fwd<128, 2, false>(d, q, k, v, block_idx, o, lse, nullptr, nullptr, nullptr, st);
-  return launch_fwd<128, 1, false>(d, q, k, v, block_idx, o, lse, nullptr, nullptr, nullptr, st);
+  // head_dim 64: two M-tiles (4 query heads) per CTA and two CTAs per SM;
+  // head_dim 128: P staged in shared memory, two M-tiles per CTA
+  if (d.D == 64)
+    return d.G >= 4
+               ? launch_fwd<64, 2, false>(d, q, k, v, block_idx, o, lse, nullptr, nullptr, nullptr, st)
+               : launch_fwd<64, 1, false>(d, q, k, v, block_idx, o, lse, nullptr, nullptr, nullptr, st);
+  return d.G >= 4
+             ? launch_psfwd<128, 2, false>(d, q, k, v, block_idx, o, lse, nullptr, nullptr, nullptr, st)
+             : launch_psfwd<128, 1, false>(d, q, k, v, block_idx, o, lse, nullptr, nullptr, nullptr, st);
 }
 
 ssa_status ssa_full_attn_fwd_with_mass(const ssa_problem* p, const ssa_bf16* q, const ssa_bf16* k,
@@ -315,6 +357,12 @@ ssa_status ssa_get_device_error(ssa_stream stream) {
     return SSA_ERR_CUDA;
   if (word & ssa::kErrTimeout) return SSA_ERR_DEVICE_TIMEOUT;
   return e == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;
+}
+
+unsigned int ssa_get_device_error_site(void) {
+  unsigned int site = 0;
+  if (cudaMemcpyFromSymbol(&site, ssa::g_error_site, sizeof(site)) != cudaSuccess) return 0;
+  return site;
 }
 
 ssa_status ssa_debug_timeout_probe(int timeout_us, ssa_stream stream) {

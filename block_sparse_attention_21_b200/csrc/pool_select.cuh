@@ -38,63 +38,49 @@ __device__ __forceinline__ uint4 ld_stream16(const void* p) {
   return r;
 }
 
-// One CTA of 256 threads per (block j, KV head h, batch b).  Each thread owns
-// one 16-byte chunk column of the 64-row slab and sums a strided subset of the
-// rows in fp32; a shared-memory pass then adds the row lanes (and, for Q, the
-// G heads of the group).  Requires CH = (row width)/8 to divide 256.
+// One CTA of 256 threads per (block j, KV head h, batch b, role): role 0 pools
+// the 64 keys of block j, role 1 the 64 queries x G heads of query block j.
+// Each thread owns one 16-byte chunk column of the slab and sums a strided
+// subset of its rows in fp32 (8 loads in flight); a shared-memory pass then
+// adds the row lanes (and, for queries, the G heads of the group).  Requires
+// CH = (row width in elements) / 8 to divide 256.
 template <int D>
 __global__ void __launch_bounds__(256) block_pool_kernel(const PoolParams p) {
   __shared__ float part[256][9];
-  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int j = blockIdx.x, h = blockIdx.y >> 1, role = blockIdx.y & 1, b = blockIdx.z;
   const int tid = threadIdx.x;
   const size_t out_off = ((static_cast<size_t>(b) * p.Hkv + h) * p.n + j) * D;
-
-  // ---- keys: slab of 64 rows x D, row stride Hkv*D
-  {
-    constexpr int CH = D / 8;
-    constexpr int NTL = 256 / CH;
-    const int ch = tid % CH, tl = tid / CH;
-    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    const __nv_bfloat16* base =
-        p.k + ((static_cast<size_t>(b) * p.S + 64 * j) * p.Hkv + h) * D + ch * 8;
+  if (role == 1 && (p.q == nullptr || p.qbar == nullptr)) return;
+  const int width = role ? p.G * D : D;                     // elements per row of the slab
+  const size_t row_stride = role ? static_cast<size_t>(p.Hq) * D : static_cast<size_t>(p.Hkv) * D;
+  const __nv_bfloat16* slab =
+      role ? p.q + ((static_cast<size_t>(b) * p.S + 64 * j) * p.Hq + h * p.G) * D
+           : p.k + ((static_cast<size_t>(b) * p.S + 64 * j) * p.Hkv + h) * D;
+  const int CH = width / 8;
+  const int NTL = 256 / CH;
+  const int ch = tid % CH, tl = tid / CH;
+  float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  const __nv_bfloat16* base = slab + ch * 8;
+  for (int t0 = tl; t0 < 64; t0 += 8 * NTL) {
+    uint4 v[8];
 #pragma unroll
-    for (int t = tl; t < 64; t += NTL)
-      add_bf16x8(acc, ld_stream16(base + static_cast<size_t>(t) * p.Hkv * D));
+    for (int x = 0; x < 8; ++x)
+      if (t0 + x * NTL < 64) v[x] = ld_stream16(base + static_cast<size_t>(t0 + x * NTL) * row_stride);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) part[tid][e] = acc[e];
-    __syncthreads();
-    for (int d = tid; d < D; d += 256) {
-      float s = 0.f;
-      for (int l = 0; l < NTL; ++l) s += part[l * CH + d / 8][d % 8];
-      p.kbar[out_off + d] = s * (1.0f / 64.0f);
-    }
-    __syncthreads();
+    for (int x = 0; x < 8; ++x)
+      if (t0 + x * NTL < 64) add_bf16x8(acc, v[x]);
   }
-  if (p.q == nullptr || p.qbar == nullptr) return;
-
-  // ---- queries: slab of 64 rows x (G*D) contiguous, row stride Hq*D
-  {
-    const int CH = p.G * (D / 8);
-    const int NTL = 256 / CH;
-    const int ch = tid % CH, tl = tid / CH;
-    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    const __nv_bfloat16* base =
-        p.q + ((static_cast<size_t>(b) * p.S + 64 * j) * p.Hq + h * p.G) * D + ch * 8;
-    if (tl < NTL) {
-#pragma unroll 4
-      for (int t = tl; t < 64; t += NTL)
-        add_bf16x8(acc, ld_stream16(base + static_cast<size_t>(t) * p.Hq * D));
-    }
 #pragma unroll
-    for (int e = 0; e < 8; ++e) part[tid][e] = acc[e];
-    __syncthreads();
-    const float inv = 1.0f / (64.0f * static_cast<float>(p.G));
-    for (int d = tid; d < D; d += 256) {
-      float s = 0.f;
-      for (int l = 0; l < NTL; ++l)
-        for (int g = 0; g < p.G; ++g) s += part[l * CH + g * (D / 8) + d / 8][d % 8];
-      p.qbar[out_off + d] = s * inv;
-    }
+  for (int e = 0; e < 8; ++e) part[tid][e] = acc[e];
+  __syncthreads();
+  const int G = role ? p.G : 1;
+  const float inv = role ? 1.0f / (64.0f * static_cast<float>(p.G)) : 1.0f / 64.0f;
+  float* out = role ? p.qbar : p.kbar;
+  for (int d = tid; d < D; d += 256) {
+    float s = 0.f;
+    for (int l = 0; l < NTL; ++l)
+      for (int g = 0; g < G; ++g) s += part[l * CH + g * (D / 8) + d / 8][d % 8];
+    out[out_off + d] = s * inv;
   }
 }
 
@@ -102,71 +88,95 @@ struct SelectParams {
   const float* qbar;
   const float* kbar;
   int32_t* idx;
-  int n, D, topk, rows;  // rows = B * Hkv * n
+  int n, topk, rows;  // rows = B * Hkv * n
 };
 
 constexpr int kSelectWarps = 4;
+constexpr int kSelectMaxPerLane = 256;  // n <= 8192
 
-// One warp per (b, h, query block i).  Scores q_pooled[i] . k_pooled[j] for
-// j < i in fp32, then k-1 rounds of a warp arg-max (higher score first, lower
-// j on ties), then the chosen set plus i written in ascending order, -1 padded.
-// Dynamic shared memory per warp: n scores, n/32 taken-bits, D pooled query.
+// Order-preserving map of fp32 onto uint32 (larger float -> larger key).
+__device__ __forceinline__ uint32_t f32_order_key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// One warp per (b, h, query block i).
+//  1. score(i, j) = q_pooled[i] . k_pooled[j] in fp32 for j < i; lane l owns
+//     the candidates j = l, l + 32, ... (kept in shared memory), each dot
+//     product over D with all loads of four candidates in flight.
+//  2. The (k-1)-th largest score T is found exactly by a 32-step radix search
+//     on order-preserving keys: the largest key T with #(key >= T) >= k-1.
+//  3. Chosen = {j : key > T} plus the lowest j with key == T up to k-1 in all
+//     (higher score first, lower block index on ties), plus i itself; written
+//     in ascending order and -1 padded.
+template <int D>
 __global__ void __launch_bounds__(32 * kSelectWarps) block_select_kernel(const SelectParams p) {
-  extern __shared__ float sel_smem[];
+  extern __shared__ uint32_t sel_keys[];  // [warps][n] order keys of the scores
+  __shared__ float4 qs_all[kSelectWarps][D / 4];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int row = blockIdx.x * kSelectWarps + warp;
   if (row >= p.rows) return;
-  const int words = (p.n + 31) / 32;
-  float* sc = sel_smem + static_cast<size_t>(warp) * (p.n + words + p.D);
-  uint32_t* taken = reinterpret_cast<uint32_t*>(sc + p.n);
-  float* qs = sc + p.n + words;
   const int i = row % p.n;
   const size_t bh = static_cast<size_t>(row / p.n);
   int32_t* out = p.idx + static_cast<size_t>(row) * p.topk;
-
   if (i + 1 <= p.topk) {  // every causal block
     for (int r = lane; r < p.topk; r += 32) out[r] = (r <= i) ? r : -1;
     return;
   }
-  for (int d = lane; d < p.D; d += 32) qs[d] = p.qbar[static_cast<size_t>(row) * p.D + d];
-  for (int w = lane; w < words; w += 32) taken[w] = 0u;
+  float4* qs = qs_all[warp];
+  const float4* qrow = reinterpret_cast<const float4*>(p.qbar + static_cast<size_t>(row) * D);
+  for (int d4 = lane; d4 < D / 4; d4 += 32) qs[d4] = __ldg(qrow + d4);
   __syncwarp();
-  for (int j = lane; j < i; j += 32) {
-    const float4* kj = reinterpret_cast<const float4*>(p.kbar + (bh * p.n + j) * p.D);
-    float s = 0.f;
-    for (int d4 = 0; d4 < p.D / 4; ++d4) {
-      const float4 kv = __ldg(kj + d4);
-      s = fmaf(qs[4 * d4 + 0], kv.x, s);
-      s = fmaf(qs[4 * d4 + 1], kv.y, s);
-      s = fmaf(qs[4 * d4 + 2], kv.z, s);
-      s = fmaf(qs[4 * d4 + 3], kv.w, s);
-    }
-    sc[j] = s;
-  }
-  __syncwarp();
-  for (int r = 0; r < p.topk - 1; ++r) {
-    float bs = -INFINITY;
-    int bj = 0x7fffffff;
-    for (int j = lane; j < i; j += 32) {
-      if (taken[j >> 5] & (1u << (j & 31))) continue;
-      const float s = sc[j];
-      if (s > bs || (s == bs && j < bj)) { bs = s; bj = j; }
+  uint32_t* key = sel_keys + static_cast<size_t>(warp) * p.n;
+  const float* kb = p.kbar + bh * p.n * D;
+  for (int j0 = lane; j0 < i; j0 += 4 * 32) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int d4 = 0; d4 < D / 4; ++d4) {
+      const float4 q4 = qs[d4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = j0 + 32 * u;
+        if (j < i) {
+          const float4 k4 = __ldg(reinterpret_cast<const float4*>(kb + static_cast<size_t>(j) * D) + d4);
+          acc[u] = fmaf(q4.x, k4.x, acc[u]);
+          acc[u] = fmaf(q4.y, k4.y, acc[u]);
+          acc[u] = fmaf(q4.z, k4.z, acc[u]);
+          acc[u] = fmaf(q4.w, k4.w, acc[u]);
+        }
+      }
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float os = __shfl_xor_sync(0xffffffffu, bs, off);
-      const int oj = __shfl_xor_sync(0xffffffffu, bj, off);
-      if (os > bs || (os == bs && oj < bj)) { bs = os; bj = oj; }
-    }
-    if (bj >= i) break;  // nothing comparable left (non-finite scores)
-    if (lane == 0) taken[bj >> 5] |= 1u << (bj & 31);
-    __syncwarp();
+    for (int u = 0; u < 4; ++u)
+      if (j0 + 32 * u < i) key[j0 + 32 * u] = f32_order_key(acc[u]);
   }
   __syncwarp();
+  // radix search for the (k-1)-th largest key
+  const int need = p.topk - 1;
+  uint32_t T = 0;
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = T | (1u << bit);
+    int cnt = 0;
+    for (int j = lane; j < i; j += 32) cnt += (key[j] >= cand) ? 1 : 0;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
+    if (cnt >= need) T = cand;
+  }
+  // ties at T: the lowest block indices first
+  int above = 0;
+  for (int j = lane; j < i; j += 32) above += (key[j] > T) ? 1 : 0;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) above += __shfl_xor_sync(0xffffffffu, above, off);
+  int ties_left = need - above;
   int written = 0;
   for (int c = 0; c * 32 <= i; ++c) {
     const int j = c * 32 + lane;
-    const bool chosen = (j == i) || (j < i && (taken[j >> 5] & (1u << (j & 31))));
+    const uint32_t kj = (j < i) ? key[j] : 0u;
+    const bool tie = (j < i) && kj == T;
+    const uint32_t tm = __ballot_sync(0xffffffffu, tie);
+    const int tie_rank = __popc(tm & ((1u << lane) - 1u));
+    const bool chosen = (j == i) || (j < i && (kj > T || (tie && tie_rank < ties_left)));
+    ties_left -= __popc(tm);
     const uint32_t m = __ballot_sync(0xffffffffu, chosen);
     const int pos = written + __popc(m & ((1u << lane) - 1u));
     if (chosen && pos < p.topk) out[pos] = j;

@@ -64,6 +64,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of whether the phase with the given parity has completed.
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Records a timed-out wait: raises the CTA abort flag and the device error word.
+__device__ __forceinline__ void report_timeout(volatile int* abort_flag, unsigned int site) {
+  *abort_flag = 1;
+  atomicOr(&g_error_word, kErrTimeout);
+  atomicExch(&g_error_site, site);
+}
+
 // Waits for the phase with the given parity to complete.  Gives up when the
 // CTA's abort flag is raised by another thread, or after timeout_ns of
 // %globaltimer, in which case it raises the abort flag and records the site in
@@ -82,6 +102,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
       return false;
     }
   }
+}
+
+// Named barrier among `nthreads` threads (a multiple of 32) of the CTA.
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // ----------------------------------------------------------------------- TMA

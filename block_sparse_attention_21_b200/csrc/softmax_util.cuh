@@ -1,0 +1,109 @@
+// softmax_util.cuh -- pieces shared by the forward attention kernels: the
+// parameter block, packed-fp32 helpers and the per-row online-softmax steps
+// (row maximum, exp2 with the scale folded into one packed FMA, bf16 packing).
+#pragma once
+
+#include "sm100.cuh"
+
+namespace ssa {
+
+struct FwdParams {
+  int B, S, Hq, Hkv, G, n, topk, slices;
+  float scale_log2;  // softmax scale * log2(e)
+  const int32_t* idx;
+  __nv_bfloat16* o;      // sparse output
+  float* lse;            // sparse log-sum-exp (natural log)
+  __nv_bfloat16* o_full; // MASS: dense causal output
+  float* lse_full;       // MASS
+  float* dropped;        // MASS: dropped attention mass
+  uint64_t timeout_ns;
+};
+
+__host__ __device__ constexpr int pow2_at_least(int x) {
+  return x <= 32 ? 32 : x <= 64 ? 64 : x <= 128 ? 128 : x <= 256 ? 256 : 512;
+}
+
+// Packed fp32 pair helpers (Blackwell f32x2 FMA-pipe instructions).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Row maximum of 32 raw scores; on the diagonal block keys past the row's own
+// token (column c0 + c > tq) are excluded.  Four independent max3 chains keep
+// the dependency depth short.
+template <bool DIAG>
+__device__ __forceinline__ float row_max32(const float* s, int c0, int tq, float m) {
+  float x[32];
+#pragma unroll
+  for (int c = 0; c < 32; ++c) x[c] = (DIAG && c0 + c > tq) ? -INFINITY : s[c];
+  float m0 = max3f(m, x[0], x[1]), m1 = max3f(x[2], x[3], x[4]);
+  float m2 = max3f(x[5], x[6], x[7]), m3 = max3f(x[8], x[9], x[10]);
+#pragma unroll
+  for (int c = 11; c + 7 < 32; c += 8) {
+    m0 = max3f(m0, x[c], x[c + 1]);
+    m1 = max3f(m1, x[c + 2], x[c + 3]);
+    m2 = max3f(m2, x[c + 4], x[c + 5]);
+    m3 = max3f(m3, x[c + 6], x[c + 7]);
+  }
+  // c = 27..31
+  m0 = max3f(m0, x[27], x[28]);
+  m1 = max3f(m1, x[29], x[30]);
+  m2 = fmaxf(m2, x[31]);
+  return max3f(m0, m1, fmaxf(m2, m3));
+}
+
+// p = 2^(s * scale_log2 - m_ref) for 32 scores, summed into the pair
+// accumulator (two independent partial sums) and packed to 16 bf16 pairs.
+template <bool DIAG>
+__device__ __forceinline__ void exp_pack32(const float* s, int c0, int tq, uint64_t scale2,
+                                           uint64_t negm2, uint64_t& acc, uint32_t* pk) {
+  uint64_t acc_b = f2_pack(0.f, 0.f);
+#pragma unroll
+  for (int c = 0; c < 32; c += 2) {
+    const uint64_t x = f2_fma(f2_pack(s[c], s[c + 1]), scale2, negm2);
+    float x0, x1;
+    f2_unpack(x, x0, x1);
+    if (DIAG) {
+      if (c0 + c > tq) x0 = -INFINITY;
+      if (c0 + c + 1 > tq) x1 = -INFINITY;
+    }
+    const float p0 = ex2(x0), p1 = ex2(x1);
+    if ((c / 2) & 1) acc_b = f2_add(acc_b, f2_pack(p0, p1));
+    else acc = f2_add(acc, f2_pack(p0, p1));
+    pk[c / 2] = pack_bf16x2(p0, p1);
+  }
+  acc = f2_add(acc, acc_b);
+}
+
+// Makes this thread's generic-proxy shared-memory writes visible to the async
+// proxy (the tensor core reads P through a shared-memory descriptor).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+}  // namespace ssa

@@ -160,6 +160,12 @@ ssa_status ssa_sparse_attn_bwd(const ssa_problem *p, const ssa_bf16 *q, const ss
  * SSA_OK. */
 ssa_status ssa_get_device_error(ssa_stream stream);
 
+/* Site code of the most recent bounded wait that ran out on the current
+ * device (0 if none since the library was loaded); for diagnostics.  The code
+ * names the kernel role and the barrier; it is not cleared by
+ * ssa_get_device_error. */
+unsigned int ssa_get_device_error_site(void);
+
 /* Launches one tiny kernel whose single wait can never be satisfied (an
  * mbarrier that nothing arrives on), bounded by timeout_us microseconds of
  * %globaltimer.  It exercises the timeout path without any fault: the kernel
