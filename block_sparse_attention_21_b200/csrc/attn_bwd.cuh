@@ -1,16 +1,681 @@
-// attn_bwd.cuh -- sparse attention backward (dQ, dK, dV over selected pairs).
+// attn_bwd.cuh -- sparse attention backward: dQ, dK, dV over the selected
+// (query block, key block) pairs only.
+//
+// The gradient of exact softmax attention restricted to the selected blocks
+// ("Resumen Tecnico: SSA", section 1: tokens the sparse stream drops receive
+// zero gradient; the top-k selection itself is not differentiated).  With
+// P_ts = exp(scale q_t.k_s - LSE_t) from the forward's log-sum-exp:
+//   D_t  = dO_t . O_t
+//   dV_s = sum_t P_ts dO_t            dS_ts = P_ts (dO_t . v_s - D_t)
+//   dK_s = scale sum_t dS_ts q_t      dQ_t  = scale sum_s dS_ts k_s
+// where t runs over the query rows of every head of the KV head's group.
+//
+// Three launches, no atomics (results are deterministic):
+//   bwd_prep_kernel    D_t for every row, and the reverse index: for each key
+//                      block j the query blocks whose selection contains j,
+//                      ascending (CSR in the workspace).
+//   attn_bwd_dkdv_kernel  one CTA per (batch, KV head, key block j): walks the
+//                      query tiles (query block x head pair) of j's reverse
+//                      list; S = Q K_j^T and dP = dO V_j^T on tcgen05, the
+//                      elementwise warps form P and dS into shared memory,
+//                      then dV += P^T dO and dK += dS^T Q as M = 64 MMAs with
+//                      both operands MN-major in shared memory.
+//   attn_bwd_dq_kernel one CTA per (batch, KV head, query block, head pairs):
+//                      walks the selected blocks like the forward; dS goes to
+//                      TMEM over S and dQ += dS K_j reads it as the A operand.
 #pragma once
 
 #include "sm100.cuh"
+#include "softmax_util.cuh"
 
-static size_t ssa_bwd_workspace_bytes(int B, int S, int Hq, int Hkv, int n, int topk) {
-  (void)B; (void)S; (void)Hq; (void)Hkv; (void)n; (void)topk;
-  return 0;
+namespace ssa {
+
+struct BwdParams {
+  int B, S, Hq, Hkv, G, n, topk, slices;
+  float scale;       // softmax scale
+  float scale_log2;  // softmax scale * log2(e)
+  const __nv_bfloat16* o;
+  const __nv_bfloat16* d_o;
+  const float* lse;       // [B][Hq][S] natural log
+  const int32_t* idx;     // [B][Hkv][n][topk]
+  float* dt;              // workspace: D_t [B][Hq][S]
+  int32_t* rev_off;       // workspace: [B][Hkv][n + 1]
+  int32_t* rev;           // workspace: [B][Hkv][n * topk]
+  __nv_bfloat16* dq;
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  uint64_t timeout_ns;
+};
+
+__host__ __device__ inline size_t bwd_align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct BwdWorkspace {
+  size_t dt, rev_off, rev, total;
+};
+
+__host__ __device__ inline BwdWorkspace bwd_workspace_layout(int B, int S, int Hq, int Hkv, int n,
+                                                            int topk) {
+  BwdWorkspace w;
+  w.dt = 0;
+  w.rev_off = bwd_align256(static_cast<size_t>(B) * Hq * S * sizeof(float));
+  w.rev = w.rev_off + bwd_align256(static_cast<size_t>(B) * Hkv * (n + 1) * sizeof(int32_t));
+  w.total = w.rev + bwd_align256(static_cast<size_t>(B) * Hkv * n * topk * sizeof(int32_t));
+  return w;
 }
 
-static ssa_status ssa_bwd_launch(int, int, int, int, int, int, int, int, float, const void*,
-                                 const void*, const void*, const void*, const float*,
-                                 const void*, const int32_t*, void*, void*, void*, void*,
-                                 cudaStream_t, uint64_t) {
-  return SSA_ERR_UNSUPPORTED;
+// Whether key block j is in query block i's selection (ascending row of
+// min(topk, i + 1) valid entries).
+__device__ __forceinline__ bool row_selects(const int32_t* row, int nvalid, int j) {
+  int lo = 0, hi = nvalid - 1;
+  while (lo <= hi) {
+    const int mid = (lo + hi) >> 1;
+    const int v = row[mid];
+    if (v == j) return true;
+    if (v < j) lo = mid + 1; else hi = mid - 1;
+  }
+  return false;
 }
+
+// Block 0..(rowsD - 1): D_t for 8 rows per warp-iteration...; the last
+// B * Hkv blocks: the reverse index of one (b, KV head).
+//  - D_t: each row's D elements are read by D / 8 lanes (16 B each) and
+//    reduced with shuffles.
+//  - reverse index: thread per key block j counts, then (after an exclusive
+//    scan in shared memory) lists, the query blocks i >= j selecting j, in
+//    ascending order.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p, int dt_blocks) {
+  if (static_cast<int>(blockIdx.x) < dt_blocks) {
+    constexpr int LPR = D / 8;            // lanes per row
+    constexpr int RPW = 32 / LPR;         // rows per warp per iteration
+    const int warp_global = (blockIdx.x * blockDim.x + threadIdx.x) / 32;
+    const int nwarps = dt_blocks * (blockDim.x / 32);
+    const int lane = threadIdx.x % 32;
+    const int sub = lane / LPR, part = lane % LPR;
+    const long long rows = static_cast<long long>(p.B) * p.S * p.Hq;  // (b, t, hq) row-major
+    for (long long r0 = static_cast<long long>(warp_global) * RPW; r0 < rows;
+         r0 += static_cast<long long>(nwarps) * RPW) {
+      const long long r = r0 + sub;
+      float acc = 0.f;
+      if (r < rows) {
+        const uint4 a = *reinterpret_cast<const uint4*>(p.o + r * D + part * 8);
+        const uint4 g = *reinterpret_cast<const uint4*>(p.d_o + r * D + part * 8);
+        const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wg[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          acc = fmaf(__uint_as_float(wa[e] << 16), __uint_as_float(wg[e] << 16), acc);
+          acc = fmaf(__uint_as_float(wa[e] & 0xFFFF0000u), __uint_as_float(wg[e] & 0xFFFF0000u), acc);
+        }
+      }
+#pragma unroll
+      for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      if (r < rows && part == 0) {
+        const int hq = static_cast<int>(r % p.Hq);
+        const long long bt = r / p.Hq;
+        const int t = static_cast<int>(bt % p.S), b = static_cast<int>(bt / p.S);
+        p.dt[(static_cast<size_t>(b) * p.Hq + hq) * p.S + t] = acc;
+      }
+    }
+    return;
+  }
+  // ---- reverse index of (b, h)
+  extern __shared__ int32_t rev_count[];  // n + 1
+  const int bh = blockIdx.x - dt_blocks;
+  const int32_t* idx = p.idx + static_cast<size_t>(bh) * p.n * p.topk;
+  for (int j = threadIdx.x; j < p.n; j += blockDim.x) {
+    int cnt = 0;
+    for (int i = j; i < p.n; ++i)
+      cnt += row_selects(idx + static_cast<size_t>(i) * p.topk, min(p.topk, i + 1), j) ? 1 : 0;
+    rev_count[j + 1] = cnt;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    rev_count[0] = 0;
+    for (int j = 0; j < p.n; ++j) rev_count[j + 1] += rev_count[j];
+  }
+  __syncthreads();
+  int32_t* off = p.rev_off + static_cast<size_t>(bh) * (p.n + 1);
+  int32_t* rev = p.rev + static_cast<size_t>(bh) * p.n * p.topk;
+  for (int j = threadIdx.x; j <= p.n; j += blockDim.x) off[j] = rev_count[j];
+  for (int j = threadIdx.x; j < p.n; j += blockDim.x) {
+    int w = rev_count[j];
+    for (int i = j; i < p.n; ++i)
+      if (row_selects(idx + static_cast<size_t>(i) * p.topk, min(p.topk, i + 1), j)) rev[w++] = i;
+  }
+}
+
+template <int D>
+struct DkdvConfig {
+  static constexpr int NP = D / 64;
+  static constexpr int QTILE = 128 * D * 2;    // Q or dO tile: 128 rows = 2 heads x 64 tokens
+  static constexpr int KVT = 64 * D * 2;       // K or V block
+  static constexpr int PTILE = 128 * 64 * 2;   // P or dS tile
+  static constexpr int NQ = 2;                 // Q/dO ring stages
+  static constexpr int TMEM_COLS = pow2_at_least(128 + 2 * D);
+  static constexpr int THREADS = 256;          // warp 0 producer, 1 issuer, 4..7 elementwise
+  static constexpr int NBARS = 1 + 2 * NQ + 7;
+  static constexpr int SMEM_BYTES = 1024 + 2 * KVT + NQ * 2 * QTILE + 2 * PTILE + NBARS * 8 + 16;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+// One CTA per (batch b, KV head h, key block j), heaviest first is not known
+// in advance; blocks are taken in index order.  TMEM: S at +0 and dP at +64
+// (128 lanes x 64 fp32 each), dV at +128 and dK at +128 + D (M = 64
+// accumulators: key row r sits in lane (r % 16) + 32 * (r / 16)).
+template <int D>
+__global__ void __launch_bounds__(256, 1)
+    attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                         const BwdParams p) {
+  using C = DkdvConfig<D>;
+  constexpr int NP = C::NP, QTILE = C::QTILE, KVT = C::KVT, PTILE = C::PTILE, NQ = C::NQ;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sK = smem;
+  uint8_t* sV = sK + KVT;
+  uint8_t* sQ = sV + KVT;              // [NQ][QTILE]
+  uint8_t* sdO = sQ + NQ * QTILE;      // [NQ][QTILE]
+  uint8_t* sP = sdO + NQ * QTILE;      // P tile, then dS tile
+  uint8_t* sdS = sP + PTILE;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sdS + PTILE);
+  uint64_t* kv_full = bars;
+  uint64_t* q_full = kv_full + 1;      // [NQ]
+  uint64_t* q_empty = q_full + NQ;     // [NQ]
+  uint64_t* s_full = q_empty + NQ;     // S and dP of a tile in TMEM
+  uint64_t* s_free = s_full + 1;       // ... read by the elementwise warps
+  uint64_t* p_full = s_free + 1;       // P and dS in shared memory
+  uint64_t* p_done = p_full + 1;       // dV, dK MMAs of the tile completed
+  uint64_t* o_done = p_done + 1;       // all MMAs completed
+  uint64_t* drain = o_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int bhn = blockIdx.x;
+  const int j = bhn % p.n;
+  const int h = (bhn / p.n) % p.Hkv;
+  const int b = bhn / (p.n * p.Hkv);
+  const int HP = p.G / 2;                                   // head pairs per group
+  const size_t bh = static_cast<size_t>(b) * p.Hkv + h;
+  const int32_t* off = p.rev_off + bh * (p.n + 1);
+  const int32_t* rev = p.rev + bh * p.n * p.topk;
+  const int first_q = off[j];
+  const int ntiles = (off[j + 1] - first_q) * HP;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < NQ; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 128);
+    mbar_init(p_full, 128);
+    mbar_init(p_done, 1);
+    mbar_init(o_done, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint64_t tmo = p.timeout_ns;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && ntiles > 0) {
+      mbar_arrive_expect_tx(kv_full, 2 * KVT);
+      for (int pn = 0; pn < NP; ++pn) {
+        tma_load_4d(sK + pn * (64 * 128), &tm_k, kv_full, 64 * pn, h, 64 * j, b);
+        tma_load_4d(sV + pn * (64 * 128), &tm_v, kv_full, 64 * pn, h, 64 * j, b);
+      }
+      int issued = 0;
+      for (int x = 0; x < ntiles; ++x) {
+        const int qs = x % NQ;
+        if (x >= NQ && !mbar_wait(&q_empty[qs], ((x / NQ) - 1) & 1, abort_flag, tmo, 0x801)) break;
+        const int i = rev[first_q + x / HP];
+        const int hq0 = h * p.G + 2 * (x % HP);
+        mbar_arrive_expect_tx(&q_full[qs], 2 * QTILE);
+        for (int hh = 0; hh < 2; ++hh)
+          for (int pn = 0; pn < NP; ++pn) {
+            tma_load_4d(sQ + qs * QTILE + pn * (128 * 128) + hh * (64 * 128), &tm_q, &q_full[qs],
+                        64 * pn, hq0 + hh, 64 * i, b);
+            tma_load_4d(sdO + qs * QTILE + pn * (128 * 128) + hh * (64 * 128), &tm_do, &q_full[qs],
+                        64 * pn, hq0 + hh, 64 * i, b);
+          }
+        ++issued;
+      }
+      if (*abort_flag) {  // loads already issued land before the CTA exits
+        volatile int never = 0;
+        mbar_wait(kv_full, 0, &never, 1000000ull, 0x8ff);
+        for (int x = (issued > NQ ? issued - NQ : 0); x < issued; ++x)
+          mbar_wait(&q_full[x % NQ], (x / NQ) & 1, &never, 1000000ull, 0x8ff);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && ntiles > 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, false);
+      // M = 64 keys, N = D, both operands MN-major (bit 15: A, bit 16: B)
+      constexpr uint32_t idesc_kv = idesc_bf16_f32(64, D, true) | (1u << 15);
+      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), adO = smem_u32(sdO),
+                     aP = smem_u32(sP), adS = smem_u32(sdS);
+      const uint32_t tS = tmem, tdP = tmem + 64, tdV = tmem + 128, tdK = tmem + 128 + D;
+      auto issue_scores = [&](int x) {
+        const int qs = x % NQ;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t o = (kk / 4) * (128 * 128) + (kk % 4) * 32;
+          const uint32_t ok_ = (kk / 4) * (64 * 128) + (kk % 4) * 32;
+          mma_ss(tS, sdesc_sw128(aQ + qs * QTILE + o, 16, 1024), sdesc_sw128(aK + ok_, 16, 1024),
+                 idesc_s, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t o = (kk / 4) * (128 * 128) + (kk % 4) * 32;
+          const uint32_t ok_ = (kk / 4) * (64 * 128) + (kk % 4) * 32;
+          mma_ss(tdP, sdesc_sw128(adO + qs * QTILE + o, 16, 1024), sdesc_sw128(aV + ok_, 16, 1024),
+                 idesc_s, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(s_full);
+      };
+      bool ok = mbar_wait(kv_full, 0, abort_flag, tmo, 0x901) &&
+                mbar_wait(&q_full[0], 0, abort_flag, tmo, 0x902);
+      if (ok) {
+        tc_fence_after();
+        issue_scores(0);
+      }
+      for (int x = 0; ok && x < ntiles; ++x) {
+        const int qs = x % NQ;
+        if (x + 1 < ntiles) {
+          // the next tile's S and dP once the elementwise warps hold this one's
+          if (!mbar_wait(s_free, x & 1, abort_flag, tmo, 0x903) ||
+              !mbar_wait(&q_full[(x + 1) % NQ], ((x + 1) / NQ) & 1, abort_flag, tmo, 0x904)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_scores(x + 1);
+        }
+        if (!mbar_wait(p_full, x & 1, abort_flag, tmo, 0x905)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // dV += P^T dO and dK += dS^T Q over the tile's 128 rows (8 K-steps)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t acc = (x > 0 || kk > 0) ? 1u : 0u;
+          mma_ss(tdV, sdesc_sw128(aP + kk * 2048, PTILE, 1024),
+                 sdesc_sw128(adO + qs * QTILE + kk * 2048, 128 * 128, 1024), idesc_kv, acc);
+          mma_ss(tdK, sdesc_sw128(adS + kk * 2048, PTILE, 1024),
+                 sdesc_sw128(aQ + qs * QTILE + kk * 2048, 128 * 128, 1024), idesc_kv, acc);
+        }
+        tc_commit(p_done);
+        tc_commit(&q_empty[qs]);
+      }
+      if (ok) {
+        tc_commit(o_done);
+      } else {
+        tc_commit(drain);
+        volatile int never = 0;
+        mbar_wait(drain, 0, &never, tmo, 0x9ff);
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------- elementwise warps
+    const int wq = warp % 4;
+    const int r = wq * 32 + lane;
+    const int hh = r / 64, tq = r % 64;
+    const uint32_t row = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    uint8_t* prow = sP + r * 128;
+    uint8_t* dsrow = sdS + r * 128;
+    constexpr float kLog2e = 1.4426950408889634f;
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+    for (int x = 0; x < ntiles; ++x) {
+      const int i = rev[first_q + x / HP];
+      const int hq = h * p.G + 2 * (x % HP) + hh;
+      const size_t lrow = (static_cast<size_t>(b) * p.Hq + hq) * p.S + 64 * i + tq;
+      const float nlse = -p.lse[lrow] * kLog2e;
+      const float dt = p.dt[lrow];
+      if (!__all_sync(0xffffffffu, mbar_wait(s_full, x & 1, abort_flag, tmo, 0xa01))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float s[64], dp[64];
+      tmem_ld32_to(row, s);
+      tmem_ld32_to(row + 32, s + 32);
+      tmem_ld32_to(row + 64, dp);
+      tmem_ld32_to(row + 96, dp + 32);
+      tc_fence_before();
+      mbar_arrive(s_free);
+      const bool diag = (i == j);
+      uint32_t pp[32], dd[32];
+#pragma unroll
+      for (int c = 0; c < 64; c += 2) {
+        float p0 = ex2(fmaf(s[c], sl2, nlse)), p1 = ex2(fmaf(s[c + 1], sl2, nlse));
+        if (diag) {
+          if (c > tq) p0 = 0.f;
+          if (c + 1 > tq) p1 = 0.f;
+        }
+        pp[c / 2] = pack_bf16x2(p0, p1);
+        dd[c / 2] = pack_bf16x2(p0 * (dp[c] - dt), p1 * (dp[c + 1] - dt));
+      }
+      if (x > 0 && !__all_sync(0xffffffffu, mbar_wait(p_done, (x - 1) & 1, abort_flag, tmo, 0xa02))) {
+        ok = false;
+        break;
+      }
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc) {
+        const int sw = (cc ^ (r & 7)) << 4;
+        *reinterpret_cast<uint4*>(prow + sw) = make_uint4(pp[4 * cc], pp[4 * cc + 1], pp[4 * cc + 2], pp[4 * cc + 3]);
+        *reinterpret_cast<uint4*>(dsrow + sw) = make_uint4(dd[4 * cc], dd[4 * cc + 1], dd[4 * cc + 2], dd[4 * cc + 3]);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(p_full);
+    }
+    // ---------------------------------------------------------- epilogue
+    // key row kr = 16 * wq + lane (lanes 0..15 of each quadrant hold the M = 64 rows)
+    const int kr = 16 * wq + lane;
+    const size_t grow = ((static_cast<size_t>(b) * p.S + 64 * j + kr) * p.Hkv + h) * D;
+    if (ntiles == 0) {
+      if (lane < 16)
+        for (int d = 0; d < D; d += 8) {
+          *reinterpret_cast<uint4*>(p.dv + grow + d) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(p.dk + grow + d) = make_uint4(0, 0, 0, 0);
+        }
+    } else if (ok && __all_sync(0xffffffffu, mbar_wait(o_done, 0, abort_flag, tmo, 0xa03))) {
+      tc_fence_after();
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t base = row + 128 + which * D;
+        const float mul = which ? p.scale : 1.f;
+        __nv_bfloat16* dst = which ? p.dk : p.dv;
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) {
+          float o[32];
+          tmem_ld32(base + ch * 32, o);
+          if (lane < 16) {
+            uint32_t w[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) w[c] = pack_bf16x2(o[2 * c] * mul, o[2 * c + 1] * mul);
+            uint4* out = reinterpret_cast<uint4*>(dst + grow + ch * 32);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4) out[v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int D, int T_>
+struct DqConfig {
+  static constexpr int T = T_;                 // M-tiles (head pairs) per CTA
+  static constexpr int NP = D / 64;
+  static constexpr int QTILE = 128 * D * 2;
+  static constexpr int KVT = 64 * D * 2;
+  static constexpr int NS = (D == 64) ? 4 : 2;
+  static constexpr int TSTRIDE = 128 + D;      // S (dS over it) +0, dP +64, dQ +128
+  static constexpr int TMEM_COLS = pow2_at_least(T * TSTRIDE);
+  static constexpr int THREADS = 128 * (T + 1);
+  static constexpr int NBARS = 1 + 3 * NS + 3 * T + 1;
+  static constexpr int SMEM_BYTES = 1024 + 2 * T * QTILE + 2 * NS * KVT + NBARS * 8 + 16;
+  static_assert(T * TSTRIDE <= 512, "TMEM budget");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+// One CTA per (batch b, KV head h, query block i, T head pairs of h's group).
+// For each selected block jj (in the index table's order) and tile t:
+//   issuer:      wait dS_t(jj);  dQ_t += dS_t(jj) K(jj);  S_t = Q_t K(jj+1)^T,
+//                dP_t = dO_t V(jj+1)^T
+//   elementwise: S_t, dP_t -> P = exp2(S scale log2e - LSE log2e),
+//                dS = P (dP - D) -> bf16 over S's first 32 TMEM columns.
+// dS(jj) is overwritten by S(jj+1) only after the dQ MMA read it (the tensor
+// pipe runs one thread's MMAs in issue order).
+template <int D, int T_>
+__global__ void __launch_bounds__(DqConfig<D, T_>::THREADS, 1)
+    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                       const BwdParams p) {
+  using C = DqConfig<D, T_>;
+  constexpr int T = C::T, NP = C::NP, QTILE = C::QTILE, KVT = C::KVT, NS = C::NS, TS = C::TSTRIDE;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem;                  // [T][QTILE]
+  uint8_t* sdO = sQ + T * QTILE;       // [T][QTILE]
+  uint8_t* sK = sdO + T * QTILE;       // [NS][KVT]
+  uint8_t* sV = sK + NS * KVT;         // [NS][KVT]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + NS * KVT);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = q_full + 1;       // [NS]
+  uint64_t* v_full = k_full + NS;
+  uint64_t* kv_empty = v_full + NS;
+  uint64_t* s_full = kv_empty + NS;    // [T]
+  uint64_t* ds_full = s_full + T;      // [T]
+  uint64_t* q_done = ds_full + T;      // [T] last dQ MMA completed
+  uint64_t* drain = q_done + T;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int per_i = p.B * p.Hkv * p.slices;
+  const int i = p.n - 1 - static_cast<int>(blockIdx.x) / per_i;
+  int rem = static_cast<int>(blockIdx.x) % per_i;
+  const int slice = rem % p.slices;
+  rem /= p.slices;
+  const int h = rem % p.Hkv;
+  const int b = rem / p.Hkv;
+  const int hq0 = h * p.G + slice * 2 * T;
+  const int nblk = min(p.topk, i + 1);
+  const int32_t* idx_row = p.idx + ((static_cast<size_t>(b) * p.Hkv + h) * p.n + i) * p.topk;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int t = 0; t < T; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&ds_full[t], 128);
+      mbar_init(&q_done[t], 1);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint64_t tmo = p.timeout_ns;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, 2 * T * QTILE);
+      for (int t = 0; t < T; ++t)
+        for (int hh = 0; hh < 2; ++hh)
+          for (int pn = 0; pn < NP; ++pn) {
+            const uint32_t o = t * QTILE + pn * (128 * 128) + hh * (64 * 128);
+            tma_load_4d(sQ + o, &tm_q, q_full, 64 * pn, hq0 + 2 * t + hh, 64 * i, b);
+            tma_load_4d(sdO + o, &tm_do, q_full, 64 * pn, hq0 + 2 * t + hh, 64 * i, b);
+          }
+      int issued = 0;
+      for (int jj = 0; jj < nblk; ++jj) {
+        const int st = jj % NS, use = jj / NS;
+        if (use > 0 && !mbar_wait(&kv_empty[st], (use - 1) & 1, abort_flag, tmo, 0xb01)) break;
+        const int j = idx_row[jj];
+        mbar_arrive_expect_tx(&k_full[st], KVT);
+        for (int pn = 0; pn < NP; ++pn)
+          tma_load_4d(sK + st * KVT + pn * (64 * 128), &tm_k, &k_full[st], 64 * pn, h, 64 * j, b);
+        mbar_arrive_expect_tx(&v_full[st], KVT);
+        for (int pn = 0; pn < NP; ++pn)
+          tma_load_4d(sV + st * KVT + pn * (64 * 128), &tm_v, &v_full[st], 64 * pn, h, 64 * j, b);
+        ++issued;
+      }
+      if (*abort_flag) {
+        volatile int never = 0;
+        for (int jj = (issued > NS ? issued - NS : 0); jj < issued; ++jj)
+          mbar_wait(&v_full[jj % NS], (jj / NS) & 1, &never, 1000000ull, 0xbff);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, false);
+      constexpr uint32_t idesc_dq = idesc_bf16_f32(128, D, true);  // B = K block, MN-major
+      const uint32_t aQ = smem_u32(sQ), adO = smem_u32(sdO), aK = smem_u32(sK), aV = smem_u32(sV);
+      auto issue_scores = [&](int t, int st) {
+        const uint32_t tS = tmem + t * TS;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t oq = t * QTILE + (kk / 4) * (128 * 128) + (kk % 4) * 32;
+          const uint32_t ok_ = st * KVT + (kk / 4) * (64 * 128) + (kk % 4) * 32;
+          mma_ss(tS, sdesc_sw128(aQ + oq, 16, 1024), sdesc_sw128(aK + ok_, 16, 1024), idesc_s,
+                 kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t oq = t * QTILE + (kk / 4) * (128 * 128) + (kk % 4) * 32;
+          const uint32_t ok_ = st * KVT + (kk / 4) * (64 * 128) + (kk % 4) * 32;
+          mma_ss(tS + 64, sdesc_sw128(adO + oq, 16, 1024), sdesc_sw128(aV + ok_, 16, 1024), idesc_s,
+                 kk > 0 ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(q_full, 0, abort_flag, tmo, 0xc01) &&
+                mbar_wait(&k_full[0], 0, abort_flag, tmo, 0xc02) &&
+                mbar_wait(&v_full[0], 0, abort_flag, tmo, 0xc03);
+      if (ok) {
+        tc_fence_after();
+        for (int t = 0; t < T; ++t) {
+          issue_scores(t, 0);
+          tc_commit(&s_full[t]);
+        }
+      }
+      for (int jj = 0; ok && jj < nblk; ++jj) {
+        const int st = jj % NS;
+        const bool more = jj + 1 < nblk;
+        const int st1 = (jj + 1) % NS;
+        if (more && (!mbar_wait(&k_full[st1], ((jj + 1) / NS) & 1, abort_flag, tmo, 0xc04) ||
+                     !mbar_wait(&v_full[st1], ((jj + 1) / NS) & 1, abort_flag, tmo, 0xc05)))
+          break;
+        for (int t = 0; t < T; ++t) {
+          if (!mbar_wait(&ds_full[t], jj & 1, abort_flag, tmo, 0xc06)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t tS = tmem + t * TS;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t bd = sdesc_sw128(aK + st * KVT + kk * (16 * 128), 64 * 128, 1024);
+            mma_ts(tS + 128, tS + kk * 8, bd, idesc_dq, (jj == 0 && kk == 0) ? 0u : 1u);
+          }
+          if (more) {
+            issue_scores(t, st1);
+            tc_commit(&s_full[t]);
+          } else {
+            tc_commit(&q_done[t]);
+          }
+        }
+        if (!ok) break;
+        tc_commit(&kv_empty[st]);
+      }
+      if (!ok || *abort_flag) {
+        tc_commit(drain);
+        volatile int never = 0;
+        mbar_wait(drain, 0, &never, tmo, 0xcff);
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------- elementwise warps
+    const int t = (warp - 4) / 4;
+    const int wq = warp % 4;
+    const int r = wq * 32 + lane;
+    const int hh = r / 64, tq = r % 64;
+    const int hq = hq0 + 2 * t + hh;
+    const int tok = 64 * i + tq;
+    const uint32_t row = tmem + (static_cast<uint32_t>(wq * 32) << 16) + t * TS;
+    constexpr float kLog2e = 1.4426950408889634f;
+    const float sl2 = p.scale_log2;
+    const size_t lrow = (static_cast<size_t>(b) * p.Hq + hq) * p.S + tok;
+    const float nlse = -p.lse[lrow] * kLog2e;
+    const float dt = p.dt[lrow];
+    bool ok = true;
+    for (int jj = 0; jj < nblk; ++jj) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[t], jj & 1, abort_flag, tmo, 0xd01))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float s[64], dp[64];
+      tmem_ld32_to(row, s);
+      tmem_ld32_to(row + 32, s + 32);
+      tmem_ld32_to(row + 64, dp);
+      tmem_ld32_to(row + 96, dp + 32);
+      const bool diag = (jj == nblk - 1);
+      uint32_t dd[32];
+#pragma unroll
+      for (int c = 0; c < 64; c += 2) {
+        float p0 = ex2(fmaf(s[c], sl2, nlse)), p1 = ex2(fmaf(s[c + 1], sl2, nlse));
+        if (diag) {
+          if (c > tq) p0 = 0.f;
+          if (c + 1 > tq) p1 = 0.f;
+        }
+        dd[c / 2] = pack_bf16x2(p0 * (dp[c] - dt), p1 * (dp[c + 1] - dt));
+      }
+      tmem_st32(row, dd);  // dS (bf16 pairs) over S columns 0..31, already read
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&ds_full[t]);
+    }
+    if (ok && __all_sync(0xffffffffu, mbar_wait(&q_done[t], 0, abort_flag, tmo, 0xd02))) {
+      tc_fence_after();
+      const size_t orow = ((static_cast<size_t>(b) * p.S + tok) * p.Hq + hq) * D;
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) {
+        float o[32];
+        tmem_ld32(row + 128 + ch * 32, o);
+        uint32_t w[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) w[c] = pack_bf16x2(o[2 * c] * p.scale, o[2 * c + 1] * p.scale);
+        uint4* dst = reinterpret_cast<uint4*>(p.dq + orow + ch * 32);
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4) dst[v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace ssa

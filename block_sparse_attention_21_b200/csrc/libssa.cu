@@ -209,6 +209,81 @@ ssa_status launch_psfwd(const Dims& d, const void* q, const void* k, const void*
   return launch_result();
 }
 
+// ---------------------------------------------------------------- backward
+
+size_t bwd_workspace_bytes(const Dims& d) {
+  return ssa::bwd_workspace_layout(d.B, d.S, d.Hq, d.Hkv, d.n, d.topk).total;
+}
+
+template <int D, int TQ>
+ssa_status launch_bwd(const Dims& d, const void* q, const void* k, const void* v, const void* o,
+                      const float* lse, const void* d_o, const int32_t* idx, void* dq, void* dk,
+                      void* dv, void* workspace, cudaStream_t st) {
+  const ssa::BwdWorkspace ws = ssa::bwd_workspace_layout(d.B, d.S, d.Hq, d.Hkv, d.n, d.topk);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  ssa::BwdParams bp;
+  bp.B = d.B;
+  bp.S = d.S;
+  bp.Hq = d.Hq;
+  bp.Hkv = d.Hkv;
+  bp.G = d.G;
+  bp.n = d.n;
+  bp.topk = d.topk;
+  bp.slices = (d.G / 2) / TQ;
+  bp.scale = d.scale;
+  bp.scale_log2 = d.scale * 1.4426950408889634f;
+  bp.o = static_cast<const __nv_bfloat16*>(o);
+  bp.d_o = static_cast<const __nv_bfloat16*>(d_o);
+  bp.lse = lse;
+  bp.idx = idx;
+  bp.dt = reinterpret_cast<float*>(base + ws.dt);
+  bp.rev_off = reinterpret_cast<int32_t*>(base + ws.rev_off);
+  bp.rev = reinterpret_cast<int32_t*>(base + ws.rev);
+  bp.dq = static_cast<__nv_bfloat16*>(dq);
+  bp.dk = static_cast<__nv_bfloat16*>(dk);
+  bp.dv = static_cast<__nv_bfloat16*>(dv);
+  bp.timeout_ns = wait_timeout_ns();
+  if (bp.slices < 1) return SSA_ERR_UNSUPPORTED;
+
+  CUtensorMap mq, mk, mv, mdo;
+  if (!make_map(&mq, q, D, d.Hq, d.S, d.B) || !make_map(&mk, k, D, d.Hkv, d.S, d.B) ||
+      !make_map(&mv, v, D, d.Hkv, d.S, d.B) || !make_map(&mdo, d_o, D, d.Hq, d.S, d.B))
+    return SSA_ERR_CUDA;
+
+  // 1. D_t and the reverse index
+  // (its dynamic shared memory, 4 (n + 1) bytes <= 32 KB, is under the default limit)
+  const long long rows = static_cast<long long>(d.B) * d.S * d.Hq;
+  const int rows_per_block = 8 * (32 / (D / 8));
+  long long dt_blocks_ll = (rows + rows_per_block - 1) / rows_per_block;
+  const int dt_blocks = static_cast<int>(dt_blocks_ll < 4096 ? dt_blocks_ll : 4096);
+  ssa::bwd_prep_kernel<D><<<dt_blocks + d.B * d.Hkv, 256, 4 * (d.n + 1), st>>>(bp, dt_blocks);
+  ssa_status s = launch_result();
+  if (s != SSA_OK) return s;
+
+  // 2. dK, dV: one CTA per (b, KV head, key block)
+  {
+    using C = ssa::DkdvConfig<D>;
+    static std::atomic<uint64_t> done{0};
+    auto kernel = ssa::attn_bwd_dkdv_kernel<D>;
+    s = ensure_smem(kernel, C::SMEM_BYTES, &done);
+    if (s != SSA_OK) return s;
+    kernel<<<static_cast<unsigned>(d.B) * d.Hkv * d.n, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, mv, mdo, bp);
+    s = launch_result();
+    if (s != SSA_OK) return s;
+  }
+  // 3. dQ: one CTA per (b, KV head, query block, head pairs)
+  {
+    using C = ssa::DqConfig<D, TQ>;
+    static std::atomic<uint64_t> done{0};
+    auto kernel = ssa::attn_bwd_dq_kernel<D, TQ>;
+    s = ensure_smem(kernel, C::SMEM_BYTES, &done);
+    if (s != SSA_OK) return s;
+    kernel<<<static_cast<unsigned>(d.B) * d.Hkv * d.n * bp.slices, C::THREADS, C::SMEM_BYTES, st>>>(
+        mq, mk, mv, mdo, bp);
+    return launch_result();
+  }
+}
+
 __global__ void timeout_probe_kernel(uint64_t timeout_ns) {
   __shared__ uint64_t bar;
   __shared__ int abort_flag;
@@ -326,7 +401,7 @@ ssa_status ssa_full_attn_fwd_with_mass(const ssa_problem* p, const ssa_bf16* q, 
 size_t ssa_sparse_attn_bwd_workspace(const ssa_problem* p) {
   Dims d;
   if (check_problem(p, &d) != SSA_OK) return 0;
-  return ssa_bwd_workspace_bytes(d.B, d.S, d.Hq, d.Hkv, d.n, d.topk);
+  return bwd_workspace_bytes(d);
 }
 
 ssa_status ssa_sparse_attn_bwd(const ssa_problem* p, const ssa_bf16* q, const ssa_bf16* k,
@@ -340,12 +415,16 @@ ssa_status ssa_sparse_attn_bwd(const ssa_problem* p, const ssa_bf16* q, const ss
   const void* ptrs[] = {q, k, v, o, lse, d_o, block_idx, dq, dk, dv};
   for (const void* ptr : ptrs)
     if (ptr == nullptr || !aligned16(ptr)) return SSA_ERR_INVALID_ARG;
-  const size_t need = ssa_bwd_workspace_bytes(d.B, d.S, d.Hq, d.Hkv, d.n, d.topk);
+  const size_t need = bwd_workspace_bytes(d);
   if (workspace == nullptr || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return SSA_ERR_WORKSPACE;
-  return ssa_bwd_launch(d.B, d.S, d.Hq, d.Hkv, d.D, d.G, d.n, d.topk, d.scale, q, k, v, o, lse, d_o,
-                        block_idx, dq, dk, dv, workspace, reinterpret_cast<cudaStream_t>(stream),
-                        wait_timeout_ns());
+  auto st = reinterpret_cast<cudaStream_t>(stream);
+  // dQ kernel: two head pairs per CTA when the group has them
+  if (d.D == 64)
+    return d.G >= 4 ? launch_bwd<64, 2>(d, q, k, v, o, lse, d_o, block_idx, dq, dk, dv, workspace, st)
+                    : launch_bwd<64, 1>(d, q, k, v, o, lse, d_o, block_idx, dq, dk, dv, workspace, st);
+  return d.G >= 4 ? launch_bwd<128, 2>(d, q, k, v, o, lse, d_o, block_idx, dq, dk, dv, workspace, st)
+                  : launch_bwd<128, 1>(d, q, k, v, o, lse, d_o, block_idx, dq, dk, dv, workspace, st);
 }
 
 ssa_status ssa_get_device_error(ssa_stream stream) {

@@ -239,6 +239,14 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   for (int c = 0; c < 16; ++c) v[c] = __uint_as_float(r[c]);
 }
 
+// Same as tmem_ld32, into v[0..31] of a larger register array.
+__device__ __forceinline__ void tmem_ld32_to(uint32_t taddr, float* v) {
+  float t[32];
+  tmem_ld32(taddr, *reinterpret_cast<float(*)[32]>(t));
+#pragma unroll
+  for (int c = 0; c < 32; ++c) v[c] = t[c];
+}
+
 // registers -> TMEM, 32 lanes x 32 bit, 32 consecutive columns (no wait).
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
