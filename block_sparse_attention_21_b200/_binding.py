@@ -25,7 +25,8 @@ STATUS_NAMES = {0: "SSA_OK", 1: "SSA_ERR_INVALID_ARG", 2: "SSA_ERR_UNSUPPORTED",
 # every symbol include/ssa.h declares
 EXPORTED = ("ssa_block_pool", "ssa_block_select", "ssa_sparse_attn_fwd",
             "ssa_full_attn_fwd_with_mass", "ssa_sparse_attn_bwd_workspace",
-            "ssa_sparse_attn_bwd", "ssa_get_device_error", "ssa_get_device_error_site",
+            "ssa_sparse_attn_bwd", "ssa_sparse_attn_bwd_noalloc", "ssa_get_device_error",
+            "ssa_get_device_error_site",
             "ssa_debug_timeout_probe",
             "ssa_status_string", "ssa_launch_count")
 
@@ -68,6 +69,7 @@ def lib():
             "ssa_sparse_attn_fwd": [P, vp, vp, vp, vp, vp, vp, vp],
             "ssa_full_attn_fwd_with_mass": [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
             "ssa_sparse_attn_bwd": [P] + [vp] * 11 + [ctypes.c_size_t, vp],
+            "ssa_sparse_attn_bwd_noalloc": [P] + [vp] * 11,
             "ssa_get_device_error": [vp],
             "ssa_debug_timeout_probe": [ctypes.c_int, vp],
         }
@@ -188,6 +190,22 @@ def ssa_sparse_attn_bwd(p: SsaProblem, q, k, v, o, lse, d_o, block_idx, dq, dk, 
           _ptr(block_idx, I32, "block_idx"), _ptr(dq, BF16, "dq"), _ptr(dk, BF16, "dk"),
           _ptr(dv, BF16, "dv"), _ptr(workspace, None, "workspace"), int(ws_bytes),
           _stream(stream))
+
+
+def ssa_sparse_attn_bwd_noalloc(p: SsaProblem, q, k, v, o, lse, d_o, block_idx, dq, dk, dv,
+                                stream=None) -> None:
+    """ssa_sparse_attn_bwd for callers that cannot allocate: the library's own
+    fixed scratch (SSA_NOALLOC_SCRATCH_BYTES per device) replaces the
+    workspace; calls that overlap on the GPU race on it."""
+    sh = _shapes(p)
+    for t, s, nm in ((q, "q", "q"), (k, "kv", "k"), (v, "kv", "v"), (o, "q", "o"),
+                     (lse, "lse", "lse"), (d_o, "q", "d_o"), (block_idx, "idx", "block_idx"),
+                     (dq, "q", "dq"), (dk, "kv", "dk"), (dv, "kv", "dv")):
+        _numel_check(t, sh[s], nm)
+    _call("ssa_sparse_attn_bwd_noalloc", ctypes.byref(p), _ptr(q, BF16, "q"), _ptr(k, BF16, "k"),
+          _ptr(v, BF16, "v"), _ptr(o, BF16, "o"), _ptr(lse, F32, "lse"), _ptr(d_o, BF16, "d_o"),
+          _ptr(block_idx, I32, "block_idx"), _ptr(dq, BF16, "dq"), _ptr(dk, BF16, "dk"),
+          _ptr(dv, BF16, "dv"), _stream(stream))
 
 
 def ssa_get_device_error(stream=None) -> int:

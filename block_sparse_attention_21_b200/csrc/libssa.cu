@@ -284,6 +284,26 @@ ssa_status launch_bwd(const Dims& d, const void* q, const void* k, const void* v
   }
 }
 
+// ------------------------------------------- backward without an allocation
+// Scratch of ssa_sparse_attn_bwd_noalloc: one file-scope array per device.
+// Host code must not use its name as a device address; the address is looked
+// up once per device with cudaGetSymbolAddress and passed to the kernels.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[SSA_NOALLOC_SCRATCH_BYTES];
+
+void* noalloc_scratch_address() {
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    addr[dev] = ptr;
+  }
+  return addr[dev];
+}
+
 __global__ void timeout_probe_kernel(uint64_t timeout_ns) {
   __shared__ uint64_t bar;
   __shared__ int abort_flag;
@@ -425,6 +445,27 @@ ssa_status ssa_sparse_attn_bwd(const ssa_problem* p, const ssa_bf16* q, const ss
                     : launch_bwd<64, 1>(d, q, k, v, o, lse, d_o, block_idx, dq, dk, dv, workspace, st);
   return d.G >= 4 ? launch_bwd<128, 2>(d, q, k, v, o, lse, d_o, block_idx, dq, dk, dv, workspace, st)
                   : launch_bwd<128, 1>(d, q, k, v, o, lse, d_o, block_idx, dq, dk, dv, workspace, st);
+}
+
+ssa_status ssa_sparse_attn_bwd_noalloc(const ssa_problem* p, const ssa_bf16* q, const ssa_bf16* k,
+                                       const ssa_bf16* v, const ssa_bf16* o, const float* lse,
+                                       const ssa_bf16* d_o, const int32_t* block_idx, ssa_bf16* dq,
+                                       ssa_bf16* dk, ssa_bf16* dv, ssa_stream stream) {
+  Dims d;
+  ssa_status s = check_problem(p, &d);
+  if (s != SSA_OK) return s;
+  const void* ptrs[] = {q, k, v, o, lse, d_o, block_idx, dq, dk, dv};
+  for (const void* ptr : ptrs)
+    if (ptr == nullptr || !aligned16(ptr)) return SSA_ERR_INVALID_ARG;
+  if (bwd_workspace_bytes(d) > SSA_NOALLOC_SCRATCH_BYTES) return SSA_ERR_WORKSPACE;
+  void* scratch = noalloc_scratch_address();
+  if (scratch == nullptr) return SSA_ERR_CUDA;
+  auto st = reinterpret_cast<cudaStream_t>(stream);
+  if (d.D == 64)
+    return d.G >= 4 ? launch_bwd<64, 2>(d, q, k, v, o, lse, d_o, block_idx, dq, dk, dv, scratch, st)
+                    : launch_bwd<64, 1>(d, q, k, v, o, lse, d_o, block_idx, dq, dk, dv, scratch, st);
+  return d.G >= 4 ? launch_bwd<128, 2>(d, q, k, v, o, lse, d_o, block_idx, dq, dk, dv, scratch, st)
+                  : launch_bwd<128, 1>(d, q, k, v, o, lse, d_o, block_idx, dq, dk, dv, scratch, st);
 }
 
 ssa_status ssa_get_device_error(ssa_stream stream) {

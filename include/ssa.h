@@ -154,6 +154,37 @@ ssa_status ssa_sparse_attn_bwd(const ssa_problem *p, const ssa_bf16 *q, const ss
                                ssa_bf16 *dk, ssa_bf16 *dv, void *workspace, size_t ws_bytes,
                                ssa_stream stream);
 
+/* Largest scratch (in bytes) that ssa_sparse_attn_bwd_noalloc can use. */
+#define SSA_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* ssa_sparse_attn_bwd without a workspace argument, for callers that cannot
+ * allocate device memory: a plugin or runtime that is handed only its input
+ * and output buffers, or a service that reserves all of its memory up front
+ * and must not call an allocator while it serves (an allocation can block,
+ * synchronise the device, fragment the heap or fail under memory pressure).
+ * The pages have no counterpart for this call; it exists for such callers.
+ *
+ * Same arguments, layouts, results and errors as ssa_sparse_attn_bwd, minus
+ * the workspace.  Its scratch is one array of SSA_NOALLOC_SCRATCH_BYTES that
+ * the library holds in device memory on every GPU that loads it, for the
+ * life of the process.  It allocates nothing and calls no allocator.
+ *  - A problem whose scratch (ssa_sparse_attn_bwd_workspace) exceeds
+ *    SSA_NOALLOC_SCRATCH_BYTES is rejected with SSA_ERR_WORKSPACE before
+ *    anything is launched.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture on the device.  A failed look-up returns
+ *    SSA_ERR_CUDA.
+ *  - Every call on a device shares the one array and leaves its contents
+ *    behind; nothing in it has to start at zero.  Calls whose kernels
+ *    overlap on the GPU (on different streams, or from several threads)
+ *    race on it: order them on one stream or synchronise between them. */
+ssa_status ssa_sparse_attn_bwd_noalloc(const ssa_problem *p, const ssa_bf16 *q, const ssa_bf16 *k,
+                                       const ssa_bf16 *v, const ssa_bf16 *o, const float *lse,
+                                       const ssa_bf16 *d_o, const int32_t *block_idx,
+                                       ssa_bf16 *dq, ssa_bf16 *dk, ssa_bf16 *dv,
+                                       ssa_stream stream);
+
 /* Synchronises `stream`, then reports and clears the device error word of the
  * current device: SSA_ERR_DEVICE_TIMEOUT if a kernel's bounded wait ran out
  * since the last call, SSA_ERR_CUDA if the stream reported an error, else
