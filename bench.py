@@ -273,77 +273,102 @@ def run_ours(args, world, rank, local):
         "pct_of_peak_step": round(100.0 * value / world / peak, 2),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rec["cpu_baseline"] = cpu_baseline(x, args.cpu_sample_blocks)
+        rec["cpu_baseline"] = cpu_baseline(x)
     return rec
 
 
 def load_traffic(name):
-    """dram bytes per launch of the sparse forward from the committed ncu summary
-    of this workload, or None."""
-    path = os.path.join(ROOT, "profiles", f"attn_fwd_{name}.json")
+    """DRAM bytes per launch of the sparse forward (dram__bytes_read.sum +
+    dram__bytes_write.sum from one ncu capture) from the committed summary of
+    this workload, or None."""
+    path = os.path.join(ROOT, "profiles", f"attn_fwd_{name}.md")
     if not os.path.exists(path):
         return None
+    import re
     with open(path) as f:
-        d = json.load(f)
-    return d.get("dram_bytes_per_launch")
+        m = re.search(r"^dram_bytes_per_launch:\s*(\d+)", f.read(), re.M)
+    return int(m.group(1)) if m else None
 
 
 # ----------------------------------------------------------- CPU baseline
 
-def cpu_baseline(x, sample_blocks: int, want_time: float = 0.0):
-    """The fp64 oracle as it stands on the host cores: pooling and selection of
-    the whole workload plus sparse attention for every row of `sample_blocks`
-    query blocks (all heads, all batch entries), reported as TFLOP/s of the
-    selected-pair FLOPs it computed."""
+def _row_flops(workload, idx, rows):
+    """Selected-pair FLOPs (4 * D per unmasked pair) of each (b, hq, t) row."""
+    nsel = np.minimum(workload.top_k, rows[:, 2] // 64 + 1)
+    return 4.0 * workload.head_dim * ((nsel - 1) * 64 + rows[:, 2] % 64 + 1)
+
+
+def cpu_baseline(x):
+    """The fp64 oracle as it stands on the host cores, on the whole workload:
+    pooling, selection and sparse attention of every row, reported as TFLOP/s
+    of the selected-pair FLOPs."""
     import oracle
     w = x.workload
     threads = oracle.default_threads()
-    rng = np.random.Generator(np.random.PCG64(2024))
-    blocks = sorted(rng.choice(np.arange(w.top_k, w.n_blocks), size=sample_blocks, replace=False))
-    rows = []
-    for i in blocks:
-        t = np.arange(64 * i, 64 * i + 64)
-        for b in range(w.batch):
-            for hq in range(w.n_q_heads):
-                rows.append(np.stack([np.full_like(t, b), np.full_like(t, hq), t], axis=1))
-    rows = np.concatenate(rows).astype(np.int64)
     q64, k64, v64 = oracle.widen(x.q), oracle.widen(x.k), oracle.widen(x.v)
+    rows = oracle.all_rows(w.batch, w.n_q_heads, w.seq_len)
     t0 = time.perf_counter()
     kbar, qbar = oracle.block_pool(k64, q64, nthreads=threads)
     idx, _ = oracle.block_select(qbar, kbar, w.top_k, nthreads=threads)
     oracle.attn_rows(q64, k64, v64, idx, rows, want_full=False, nthreads=threads)
     dt = time.perf_counter() - t0
-    pairs_per_block = (w.top_k - 1) * 64 * 64 + 64 * 65 // 2
-    flops = 4.0 * w.head_dim * pairs_per_block * len(blocks) * w.batch * w.n_q_heads
+    flops = algorithmic_flops(w)
     return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": threads,
             "kind": "oracle", "seconds": round(dt, 2),
-            "sample": (f"pool+select of the whole workload, then sparse attention of all rows "
-                       f"of {len(blocks)} of {w.n_blocks} query blocks (all heads, all batch), "
-                       f"fp64, {threads} threads")}
+            "sample": (f"the whole workload: pooling, selection and sparse attention of all "
+                       f"{len(rows)} rows, fp64, {threads} threads")}
 
 
 def run_reference(args, world, rank):
     """The reference arm: the fp64 oracle on the host cores, on this arm's
-    workload, one bounded sample per step."""
+    workload.  Pooling and selection of the whole workload run once (timed and
+    reported); each step then computes the sparse attention of a random sample
+    of query rows, sized so that the whole run takes about two minutes."""
     if rank != 0:
         return None
+    import oracle
     x = gen.make_inputs(args.workload)
     w = x.workload
-    samples = []
+    threads = oracle.default_threads()
+    q64, k64, v64 = oracle.widen(x.q), oracle.widen(x.k), oracle.widen(x.v)
+    t0 = time.perf_counter()
+    kbar, qbar = oracle.block_pool(k64, q64, nthreads=threads)
+    idx, _ = oracle.block_select(qbar, kbar, w.top_k, nthreads=threads)
+    select_s = time.perf_counter() - t0
+    rng = np.random.Generator(np.random.PCG64(4242))
+
+    def sample(nrows):
+        return np.stack([rng.integers(0, w.batch, nrows), rng.integers(0, w.n_q_heads, nrows),
+                         rng.integers(0, w.seq_len, nrows)], axis=1).astype(np.int64)
+
+    def run(rows):
+        t = time.perf_counter()
+        oracle.attn_rows(q64, k64, v64, idx, rows, want_full=False, nthreads=threads)
+        return time.perf_counter() - t
+
+    cal = sample(4 * threads)
+    rate = _row_flops(w, idx, cal).sum() / max(run(cal), 1e-6)
+    mean_row = algorithmic_flops(w) / (w.batch * w.n_q_heads * w.seq_len)
+    budget = 120.0 / (args.steps + args.warmup)
+    nrows = int(np.clip(budget * rate / mean_row, 8, 1 << 16))
     for _ in range(args.warmup):
-        cpu_baseline(x, 1)
+        run(sample(nrows))
+    flops = secs = 0.0
     for _ in range(args.steps):
-        samples.append(cpu_baseline(x, args.cpu_sample_blocks))
-    value = statistics.median(s["value"] for s in samples)
-    secs = sum(s["seconds"] for s in samples)
-    cb = dict(samples[-1])
-    cb["value"] = value
-    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        rows = sample(nrows)
+        secs += run(rows)
+        flops += _row_flops(w, idx, rows).sum()
+    value = flops / secs / 1e12
+    cb = {"value": round(value, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+          "sample": (f"per step the sparse attention of {nrows} random query rows "
+                     f"(fp64, {threads} threads); pooling and selection of the whole workload "
+                     f"once beforehand ({select_s:.2f} s)")}
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(1000.0 * secs / max(1, len(samples)), 2),
+            "ms_per_step": round(1000.0 * secs / max(1, args.steps), 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": config_of(w, "host_cpu"), "cpu_baseline": cb,
-            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
 
@@ -354,7 +379,6 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="llama1b_8k", choices=sorted(gen.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--cpu-sample-blocks", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
