@@ -137,6 +137,9 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS>::THREADS, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
+  // launched with programmatic serialization: the index table may still be
+  // in flight from the selection kernel until here
+  pdl_wait();
   if (MASS && warp == 3) {
     const int words = (p.n + 31) / 32;
     for (int w = lane; w < words; w += 32) selbits[w] = 0u;

@@ -121,6 +121,31 @@ ssa_status launch_result() {
   return cudaGetLastError() == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;
 }
 
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel on the stream finishes; it calls pdl_wait before
+// touching global memory.
+template <typename... KArgs, typename... Args>
+ssa_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                      cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  g_launches.fetch_add(1);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return SSA_ERR_CUDA;
+  }
+  return cudaGetLastError() == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;
+}
+
 template <int D>
 ssa_status launch_pool(const Dims& d, const void* k, const void* q, float* kb, float* qb,
                        cudaStream_t st) {
@@ -134,8 +159,19 @@ ssa_status launch_pool(const Dims& d, const void* k, const void* q, float* kb, f
   pp.Hkv = d.Hkv;
   pp.G = d.G;
   pp.n = d.n;
-  ssa::block_pool_kernel<D><<<dim3(d.n, 2 * d.Hkv, d.B), 256, 0, st>>>(pp);
-  return launch_result();
+  return launch_pdl(ssa::block_pool_kernel<D>, dim3(d.n, d.Hkv, d.B), dim3(ssa::PoolConfig<D>::THREADS), 0,
+                    st, pp);
+}
+
+template <int D, int KPL>
+ssa_status launch_select(const Dims& d, const ssa::SelectParams& sp, cudaStream_t st) {
+  static std::atomic<uint64_t> done{0};
+  auto kernel = ssa::block_select_kernel<D, KPL>;
+  const ssa_status s = ensure_smem(kernel, 200 * 1024, &done);
+  if (s != SSA_OK) return s;
+  const dim3 grid((d.n + ssa::kSelectWarps - 1) / ssa::kSelectWarps, d.B * d.Hkv);
+  return launch_pdl(kernel, grid, dim3(32 * ssa::kSelectWarps), ssa::SelectConfig<D>::smem_bytes(d.n), st,
+                    sp);
 }
 
 template <int D, int T, bool MASS>
@@ -169,8 +205,7 @@ ssa_status launch_fwd(const Dims& d, const void* q, const void* k, const void* v
   fp.dropped = dropped;
   fp.timeout_ns = wait_timeout_ns();
   const unsigned grid = static_cast<unsigned>(d.B) * d.Hkv * d.n * fp.slices;
-  kernel<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, mv, fp);
-  return launch_result();
+  return launch_pdl(kernel, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, st, mq, mk, mv, fp);
 }
 
 // The same launch for the kernel that stages P in shared memory.
@@ -205,8 +240,7 @@ ssa_status launch_psfwd(const Dims& d, const void* q, const void* k, const void*
   fp.dropped = dropped;
   fp.timeout_ns = wait_timeout_ns();
   const unsigned grid = static_cast<unsigned>(d.B) * d.Hkv * d.n * fp.slices;
-  kernel<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, mv, fp);
-  return launch_result();
+  return launch_pdl(kernel, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, st, mq, mk, mv, fp);
 }
 
 // ---------------------------------------------------------------- backward
@@ -361,22 +395,13 @@ ssa_status ssa_block_select(const ssa_problem* p, const float* q_pooled, const f
   sp.idx = block_idx;
   sp.n = d.n;
   sp.topk = d.topk;
-  sp.rows = d.B * d.Hkv * d.n;
-  const size_t smem = static_cast<size_t>(ssa::kSelectWarps) * d.n * 4;
-  const unsigned grid = static_cast<unsigned>((sp.rows + ssa::kSelectWarps - 1) / ssa::kSelectWarps);
   auto st = reinterpret_cast<cudaStream_t>(stream);
-  if (d.D == 64) {
-    static std::atomic<uint64_t> done{0};
-    s = ensure_smem(ssa::block_select_kernel<64>, 200 * 1024, &done);
-    if (s != SSA_OK) return s;
-    ssa::block_select_kernel<64><<<grid, 32 * ssa::kSelectWarps, smem, st>>>(sp);
-  } else {
-    static std::atomic<uint64_t> done{0};
-    s = ensure_smem(ssa::block_select_kernel<128>, 200 * 1024, &done);
-    if (s != SSA_OK) return s;
-    ssa::block_select_kernel<128><<<grid, 32 * ssa::kSelectWarps, smem, st>>>(sp);
-  }
-  return launch_result();
+  // keys in registers while a lane's share (n / 32) is small
+  if (d.D == 64)
+    return d.n <= 128 ? launch_select<64, 4>(d, sp, st)
+                      : (d.n <= 512 ? launch_select<64, 16>(d, sp, st) : launch_select<64, 0>(d, sp, st));
+  return d.n <= 128 ? launch_select<128, 4>(d, sp, st)
+                    : (d.n <= 512 ? launch_select<128, 16>(d, sp, st) : launch_select<128, 0>(d, sp, st));
 }
 
 ssa_status ssa_sparse_attn_fwd(const ssa_problem* p, const ssa_bf16* q, const ssa_bf16* k,

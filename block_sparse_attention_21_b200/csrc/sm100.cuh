@@ -25,6 +25,20 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// ------------------------------------------- programmatic dependent launch
+// Kernels launched with the programmatic-serialization attribute may start
+// while the previous kernel on the stream is still running.  pdl_wait blocks
+// until that kernel has completed and its memory is visible; every kernel of
+// the library calls it before its first global-memory access, so the overlap
+// is only its prologue.  pdl_launch_dependents lets the next kernel start its
+// own prologue early.  Both are no-ops for a normal launch.
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
