@@ -12,7 +12,7 @@ from typing import Optional
 import torch
 
 from ._binding import (EXPORTED, LIB_PATH, SsaError, SsaProblem, lib, problem,
-                       ssa_block_pool, ssa_block_select, ssa_debug_timeout_probe,
+                       ssa_block_pool, ssa_block_select, ssa_debug_exp2_poly, ssa_debug_timeout_probe,
                        ssa_full_attn_fwd_with_mass, ssa_get_device_error,
                        ssa_get_device_error_site, ssa_launch_count,
                        ssa_sparse_attn_bwd, ssa_sparse_attn_bwd_noalloc,
@@ -20,7 +20,7 @@ from ._binding import (EXPORTED, LIB_PATH, SsaError, SsaProblem, lib, problem,
                        ssa_sparse_attn_fwd, ssa_status_string)
 
 __all__ = ["EXPORTED", "LIB_PATH", "SsaError", "SsaProblem", "SparseStream", "lib", "problem",
-           "ssa_block_pool", "ssa_block_select", "ssa_debug_timeout_probe",
+           "ssa_block_pool", "ssa_block_select", "ssa_debug_exp2_poly", "ssa_debug_timeout_probe",
            "ssa_full_attn_fwd_with_mass", "ssa_get_device_error", "ssa_get_device_error_site",
            "ssa_launch_count",
            "ssa_sparse_attn_bwd", "ssa_sparse_attn_bwd_noalloc", "ssa_sparse_attn_bwd_workspace",

@@ -27,7 +27,7 @@ EXPORTED = ("ssa_block_pool", "ssa_block_select", "ssa_sparse_attn_fwd",
             "ssa_full_attn_fwd_with_mass", "ssa_sparse_attn_bwd_workspace",
             "ssa_sparse_attn_bwd", "ssa_sparse_attn_bwd_noalloc", "ssa_get_device_error",
             "ssa_get_device_error_site",
-            "ssa_debug_timeout_probe",
+            "ssa_debug_timeout_probe", "ssa_debug_exp2_poly",
             "ssa_status_string", "ssa_launch_count")
 
 
@@ -72,6 +72,7 @@ def lib():
             "ssa_sparse_attn_bwd_noalloc": [P] + [vp] * 11,
             "ssa_get_device_error": [vp],
             "ssa_debug_timeout_probe": [ctypes.c_int, vp],
+            "ssa_debug_exp2_poly": [vp, vp, ctypes.c_int, vp],
         }
         for name, args in sigs.items():
             f = getattr(L, name)
@@ -219,6 +220,14 @@ def ssa_get_device_error_site() -> int:
 
 def ssa_debug_timeout_probe(timeout_us: int, stream=None) -> None:
     _call("ssa_debug_timeout_probe", int(timeout_us), _stream(stream))
+
+
+def ssa_debug_exp2_poly(x: torch.Tensor, y: torch.Tensor, stream=None) -> None:
+    """y = 2^x by the forward kernels' FMA-pipe polynomial (fp32 CUDA tensors)."""
+    n = x.numel()
+    if y.numel() != n:
+        raise ValueError("x and y differ in size")
+    _call("ssa_debug_exp2_poly", _ptr(x, F32, "x"), _ptr(y, F32, "y"), int(n), _stream(stream))
 
 
 def ssa_status_string(status: int) -> str:

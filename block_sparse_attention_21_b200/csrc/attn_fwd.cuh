@@ -20,10 +20,10 @@
 //               block through an NS-stage ring (index-guided loads).
 //   warps 1-2   TMEM allocation (warp 1) and the tcgen05.mma issuers (two
 //               when T = 4, else one), one elected thread each, owning
-//               alternate M-tiles; an issuer polls its tiles and issues for
-//               whichever is ready, and releases a K/V stage with one commit
-//               once all its tiles are done with it.  Per visited block jj
-//               and M-tile t, in this order:
+//               alternate M-tiles; an issuer serves its tiles round-robin
+//               with suspending waits, and releases a K/V stage with one
+//               commit once all its tiles are done with it.  Per visited
+//               block jj and M-tile t, in this order:
 //                 wait P_t(jj);  O_t += P_t(jj) V(jj);  S_t = Q_t K(jj+1)^T
 //               so one commit of S_t(jj+1) also tells the softmax warps that
 //               O_t is stable.  P_t lives in the first 32 TMEM columns of S_t;
@@ -57,6 +57,7 @@ struct FwdConfig {
   static constexpr int TMEM_COLS = pow2_at_least(T * TSTRIDE);
   static constexpr int THREADS = 128 * (T + 1);
   static constexpr int ISS = T >= 4 ? 2 : 1;      // MMA issuer warps (warps 1..ISS)
+  static constexpr int POLY = (D == 128) ? 3 : 0; // exp2 pairs of 8 on the FMA pipe
   static constexpr int NBARS = 1 + ISS + 3 * NS + 3 * T;
   // shared memory: Q tiles, K ring, V ring, barriers, tmem slot, abort flag,
   // selection bitmap (up to 8192 blocks)
@@ -181,25 +182,30 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, FwdConfig<D, T
     }
   } else if (warp >= 1 && warp <= C::ISS) {
     // ------------------------------------------------------------ MMA issuers
-    // Issuer warp w owns M-tiles t = w - 1, w - 1 + ISS, ...; it polls their
-    // P-ready barriers and issues for whichever tile is ready, so a slow tile
-    // does not hold up the others.  A K/V stage is released after all T
-    // tiles committed their use of it.
+    // Issuer warp w owns M-tiles t = w - 1, w - 1 + ISS, ...  Every tile
+    // advances one block per round, so the issuer serves its tiles round-robin
+    // with suspending waits (no issue slots taken from the softmax warps while
+    // it waits).  Operand descriptors are built once; an operand offset is
+    // added to the descriptor's address field (byte offset / 16).  A K/V stage
+    // is released once all of the issuer's tiles committed their P.V on it.
     if (lane == 0) {
       constexpr int ISS = C::ISS;
       constexpr int MT = (T + ISS - 1) / ISS;  // tiles per issuer
       const int me = warp - 1;
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 64, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
-      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
+      const uint64_t dQ = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dK = sdesc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t dV = sdesc_sw128(smem_u32(sV), 64 * 128, 1024);
       auto issue_qk = [&](int t, int st) {
         const uint32_t d = tmem + t * TSTRIDE;
+        const uint64_t a0 = dQ + ((t * QTILE) >> 4), b0 = dK + ((st * KVT) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk % 4) * 32;  // 16 bf16 = 32 B inside the 128 B row
-          const uint64_t a = sdesc_sw128(sQa + t * QTILE + (kk / 4) * (128 * 128) + off, 16, 1024);
-          const uint64_t bd = sdesc_sw128(sKa + st * KVT + (kk / 4) * (64 * 128) + off, 16, 1024);
-          mma_ss(d, a, bd, idesc_qk, kk > 0 ? 1u : 0u);
+          // 16 bf16 = 32 B inside a 128 B row; 64-column panels
+          const uint32_t oa = ((kk / 4) * (128 * 128) + (kk % 4) * 32) >> 4;
+          const uint32_t ob = ((kk / 4) * (64 * 128) + (kk % 4) * 32) >> 4;
+          mma_ss(d, a0 + oa, b0 + ob, idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
       bool ok = mbar_wait(bar_q, 0, abort_flag, tmo, 0x201) &&
@@ -211,78 +217,48 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, FwdConfig<D, T
           tc_commit(&bar_sfull[t]);
         }
       }
-      int next[MT];
       bool first_sel[MT], first_uns[MT];
-      int remaining = 0, own = 0;
-      uint32_t stage_uses = 0;  // per K/V stage (8 bits each): own tiles done with its current use
 #pragma unroll
-      for (int x = 0; x < MT; ++x) {
-        next[x] = 0;
-        first_sel[x] = first_uns[x] = true;
-        if (me + x * ISS < T) {
-          remaining += nblk;
-          ++own;
+      for (int x = 0; x < MT; ++x) first_sel[x] = first_uns[x] = true;
+      for (int jj = 0; ok && jj < nblk; ++jj) {
+        const int st = jj % NS;
+        const bool more = jj + 1 < nblk;
+        const int st1 = (jj + 1) % NS;
+        if (!mbar_wait(&bar_vfull[st], (jj / NS) & 1, abort_flag, tmo, 0x203) ||
+            (more && !mbar_wait(&bar_kfull[st1], ((jj + 1) / NS) & 1, abort_flag, tmo, 0x204))) {
+          ok = false;
+          break;
         }
-      }
-      uint64_t t_last = globaltimer_ns();
-      while (ok && remaining > 0) {
-        bool progressed = false;
+        bool is_sel = true;
+        if (MASS) is_sel = (selbits[jj >> 5] >> (jj & 31)) & 1u;
+        const uint64_t v0 = dV + ((st * KVT) >> 4);
 #pragma unroll
         for (int x = 0; x < MT; ++x) {
           const int t = me + x * ISS;
-          const int jj = next[x];
-          if (t >= T || jj >= nblk || !ok) continue;
-          if (!mbar_test(&bar_pfull[t], jj & 1)) continue;
-          const int st = jj % NS;
-          const bool more = jj + 1 < nblk;
-          const int st1 = (jj + 1) % NS;
-          if (!mbar_wait(&bar_vfull[st], (jj / NS) & 1, abort_flag, tmo, 0x203) ||
-              (more && !mbar_wait(&bar_kfull[st1], ((jj + 1) / NS) & 1, abort_flag, tmo, 0x204))) {
+          if (t >= T || !ok) continue;
+          if (!mbar_wait(&bar_pfull[t], jj & 1, abort_flag, tmo, 0x205)) {
             ok = false;
             continue;
           }
           tc_fence_after();
-          bool is_sel = true;
-          if (MASS) is_sel = (selbits[jj >> 5] >> (jj & 31)) & 1u;
           const bool first = MASS ? (is_sel ? first_sel[x] : first_uns[x]) : (jj == 0);
           const uint32_t base = tmem + t * TSTRIDE;
           const uint32_t o_col = base + 64 + ((MASS && !is_sel) ? D : 0);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t bd = sdesc_sw128(sVa + st * KVT + kk * (16 * 128), 64 * 128, 1024);
-            mma_ts(o_col, base + kk * 8, bd, idesc_pv, (first && kk == 0) ? 0u : 1u);
-          }
+          for (int kk = 0; kk < 4; ++kk)  // 16 keys per MMA: 16 rows of 128 B
+            mma_ts(o_col, base + kk * 8, v0 + ((kk * (16 * 128)) >> 4), idesc_pv,
+                   (first && kk == 0) ? 0u : 1u);
           if (more) {
             issue_qk(t, st1);
             tc_commit(&bar_sfull[t]);
           } else {
             tc_commit(&bar_odone[t]);
           }
-          stage_uses += 1u << (8 * st);
-          if (((stage_uses >> (8 * st)) & 0xffu) == static_cast<uint32_t>(own)) {
-            tc_commit(&bar_empty[st]);  // this issuer's tiles are all done with the stage
-            stage_uses &= ~(0xffu << (8 * st));
-          }
           if (MASS) {
             if (is_sel) first_sel[x] = false; else first_uns[x] = false;
           }
-          next[x] = jj + 1;
-          --remaining;
-          progressed = true;
         }
-        if (progressed) {
-          t_last = globaltimer_ns();
-        } else if (MT == 1 && ok && remaining > 0) {
-          // one tile: a suspending wait costs the softmax warps no issue slots
-          ok = mbar_wait(&bar_pfull[me], next[0] & 1, abort_flag, tmo, 0x205);
-        } else if (*abort_flag) {
-          ok = false;
-        } else if (globaltimer_ns() - t_last > tmo) {
-          report_timeout(abort_flag, 0x205);
-          ok = false;
-        } else {
-          __nanosleep(32);  // back off: the softmax warps share this scheduler
-        }
+        if (ok) tc_commit(&bar_empty[st]);  // this issuer's tiles are all done with the stage
       }
       if (!ok) {
         // every MMA this thread issued completes before TMEM is released
@@ -337,13 +313,13 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, FwdConfig<D, T
       uint64_t acc2 = f2_pack(0.f, 0.f);
       uint32_t pk[16];
       if (diag) exp_pack32<true>(sA, 0, tq, scale2, negm2, acc2, pk);
-      else exp_pack32<false>(sA, 0, tq, scale2, negm2, acc2, pk);
+      else exp_pack32<false, C::POLY>(sA, 0, tq, scale2, negm2, acc2, pk);
       tmem_st16(tS, pk);  // P columns 0..15 over S columns 0..15 (already read)
       {
         float sB[32];
         tmem_ld32(tS + 32, sB);
         if (diag) exp_pack32<true>(sB, 32, tq, scale2, negm2, acc2, pk);
-        else exp_pack32<false>(sB, 32, tq, scale2, negm2, acc2, pk);
+        else exp_pack32<false, C::POLY>(sB, 32, tq, scale2, negm2, acc2, pk);
       }
       tmem_st16(tS + 16, pk);  // P columns 16..31
       float r0, r1;

@@ -55,6 +55,7 @@ struct PsFwdConfig {
   static constexpr int NS = (D == 64) ? 4 : 3;    // K/V ring stages
   static constexpr int TSTRIDE = 64 + (MASS ? 2 : 1) * D;  // TMEM columns per M-tile
   static constexpr int TMEM_COLS = pow2_at_least(T * TSTRIDE);
+  static constexpr int POLY = 3;                  // exp2 pairs of 8 on the FMA pipe
   // warps: 0 producer, 1..3 issuers, 4.. softmax (4 per tile), then the
   // issuer of a fourth tile
   static constexpr int THREADS = 128 * (T + 1) + (T > 3 ? 32 : 0);
@@ -315,8 +316,8 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS>::THREADS, 1)
         exp_pack32<true>(sA, 0, tq, scale2, negm2, acc2, pk);
         exp_pack32<true>(sB, 32, tq, scale2, negm2, acc2, pk + 16);
       } else {
-        exp_pack32<false>(sA, 0, tq, scale2, negm2, acc2, pk);
-        exp_pack32<false>(sB, 32, tq, scale2, negm2, acc2, pk + 16);
+        exp_pack32<false, C::POLY>(sA, 0, tq, scale2, negm2, acc2, pk);
+        exp_pack32<false, C::POLY>(sB, 32, tq, scale2, negm2, acc2, pk + 16);
       }
       float r0, r1;
       f2_unpack(acc2, r0, r1);

@@ -350,6 +350,17 @@ __global__ void timeout_probe_kernel(uint64_t timeout_ns) {
   if (threadIdx.x == 0) ssa::mbar_wait(&bar, 0, &abort_flag, timeout_ns, 0x900);
 }
 
+// Applies the forward kernels' FMA-pipe exp2 to n inputs (pairs per thread).
+__global__ void exp2_poly_kernel(const float* x, float* y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float x0 = x[i], x1 = (i + 1 < n) ? x[i + 1] : 0.f;
+  float p0, p1;
+  ssa::exp2_poly2(x0, x1, p0, p1);
+  y[i] = p0;
+  if (i + 1 < n) y[i + 1] = p1;
+}
+
 }  // namespace
 
 extern "C" {
@@ -514,6 +525,14 @@ ssa_status ssa_debug_timeout_probe(int timeout_us, ssa_stream stream) {
   if (timeout_us < 1 || timeout_us > 10000000) return SSA_ERR_INVALID_ARG;
   timeout_probe_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       static_cast<uint64_t>(timeout_us) * 1000ull);
+  return launch_result();
+}
+
+ssa_status ssa_debug_exp2_poly(const float* x, float* y, int n, ssa_stream stream) {
+  if (n < 0 || (n > 0 && (x == nullptr || y == nullptr))) return SSA_ERR_INVALID_ARG;
+  if (n == 0) return SSA_OK;
+  const int pairs = (n + 1) / 2;
+  exp2_poly_kernel<<<(pairs + 255) / 256, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n);
   return launch_result();
 }
 

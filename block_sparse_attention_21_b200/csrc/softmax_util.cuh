@@ -77,9 +77,37 @@ __device__ __forceinline__ float row_max32(const float* s, int c0, int tq, float
   return max3f(m0, m1, fmaxf(m2, m3));
 }
 
+// 2^x for a pair of inputs on the FMA pipe, to take part of the softmax's
+// exponentials off the MUFU unit.  x = j + f with j = round(x) and f in
+// [-1/2, 1/2]: adding 1.5 * 2^23 rounds x to an integer held in the low
+// mantissa bits, so j << 23 is those bits shifted into the exponent field;
+// 2^f is a degree-3 polynomial whose coefficients were fitted to minimise the
+// relative error on [-1/2, 1/2] by Lawson's iteratively reweighted least
+// squares (maximum relative error 7.5e-5, well below half a bf16 ulp, 2^-9).
+// Inputs below -125 are clamped: 2^-125 (about 2e-38) stands in for 0.
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& p0, float& p1) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  const uint64_t x = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t t = f2_add(x, f2_pack(kRound, kRound));
+  const uint64_t j = f2_add(t, f2_pack(-kRound, -kRound));            // round(x), exact
+  const uint64_t f = f2_fma(j, f2_pack(-1.f, -1.f), x);               // x - round(x), exact
+  uint64_t q = f2_fma(f2_pack(0.0551716685f, 0.0551716685f), f, f2_pack(0.2426111400f, 0.2426111400f));
+  q = f2_fma(q, f, f2_pack(0.6932609677f, 0.6932609677f));
+  q = f2_fma(q, f, f2_pack(0.9999280572f, 0.9999280572f));
+  float q0, q1, t0, t1;
+  f2_unpack(q, q0, q1);
+  f2_unpack(t, t0, t1);
+  p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+  p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
 // p = 2^(s * scale_log2 - m_ref) for 32 scores, summed into the pair
 // accumulator (two independent partial sums) and packed to 16 bf16 pairs.
-template <bool DIAG>
+// POLY of every 8 pairs take the FMA-pipe polynomial instead of MUFU ex2
+// (off the diagonal block only, where no score is masked): it pays where the
+// softmax is bound by the MUFU rate (head_dim 128), not where it is bound by
+// latency (head_dim 64).
+template <bool DIAG, int POLY = 0>
 __device__ __forceinline__ void exp_pack32(const float* s, int c0, int tq, uint64_t scale2,
                                            uint64_t negm2, uint64_t& acc, uint32_t* pk) {
   uint64_t acc_b = f2_pack(0.f, 0.f);
@@ -88,11 +116,18 @@ __device__ __forceinline__ void exp_pack32(const float* s, int c0, int tq, uint6
     const uint64_t x = f2_fma(f2_pack(s[c], s[c + 1]), scale2, negm2);
     float x0, x1;
     f2_unpack(x, x0, x1);
+    float p0, p1;
     if (DIAG) {
       if (c0 + c > tq) x0 = -INFINITY;
       if (c0 + c + 1 > tq) x1 = -INFINITY;
+      p0 = ex2(x0);
+      p1 = ex2(x1);
+    } else if ((c / 2) % 8 >= 8 - POLY) {
+      exp2_poly2(x0, x1, p0, p1);
+    } else {
+      p0 = ex2(x0);
+      p1 = ex2(x1);
     }
-    const float p0 = ex2(x0), p1 = ex2(x1);
     if ((c / 2) & 1) acc_b = f2_add(acc_b, f2_pack(p0, p1));
     else acc = f2_add(acc, f2_pack(p0, p1));
     pk[c / 2] = pack_bf16x2(p0, p1);

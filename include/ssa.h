@@ -203,6 +203,14 @@ unsigned int ssa_get_device_error_site(void);
  * records SSA_ERR_DEVICE_TIMEOUT in the device error word and returns. */
 ssa_status ssa_debug_timeout_probe(int timeout_us, ssa_stream stream);
 
+/* y[i] = 2^x[i] for n device floats, computed by the FMA-pipe polynomial the
+ * forward kernels use for part of the softmax exponentials (instead of the
+ * MUFU ex2 unit): maximum relative error 7.5e-5 for x in [-125, 64]; inputs
+ * below -125 give 2^-125.  The pages have no counterpart: this call exists so
+ * tests can check that approximation against exp2f.  INVALID_ARG for n < 0 or
+ * null pointers with n > 0. */
+ssa_status ssa_debug_exp2_poly(const float *x, float *y, int n, ssa_stream stream);
+
 /* Static, human-readable name of a status code. */
 const char *ssa_status_string(ssa_status s);
 
