@@ -15,27 +15,29 @@
 // Two CTAs share an SM when T = 2 (256 TMEM columns each), so one CTA's
 // prologue and epilogue overlap the other's main loop.
 //
-// Warp roles (128 * (T + 1) threads):
-//   warp 0      TMA producer: the Q tiles once, then K and V of each visited
-//               block through an NS-stage ring (index-guided loads).
-//   warps 1-2   TMEM allocation (warp 1) and the tcgen05.mma issuers (two
-//               when T = 4, else one), one elected thread each, owning
-//               alternate M-tiles; an issuer serves its tiles round-robin
-//               with suspending waits, and releases a K/V stage with one
-//               commit once all its tiles are done with it.  Per visited
-//               block jj and M-tile t, in this order:
-//                 wait P_t(jj);  O_t += P_t(jj) V(jj);  S_t = Q_t K(jj+1)^T
+// Warp roles (64 + 128 * T threads):
+//   warp 0      builds the selection bitmap (MASS), then is the TMA producer:
+//               the Q tiles once, then K and V of each visited block through
+//               an NS-stage ring (index-guided loads).
+//   warp 1      TMEM allocation and the tcgen05.mma issuer (one elected
+//               thread), serving the M-tiles round-robin with suspending
+//               waits; it releases a K/V stage with one commit once all
+//               tiles are done with it.  Per visited block jj and M-tile t,
+//               in this order:
+//                 wait P_t(jj) keys 0..31;   O_t += P_t V(jj) over them;
+//                 wait P_t(jj) keys 32..63;  O_t += P_t V(jj) over them;
+//                 S_t = Q_t K(jj+1)^T
 //               so one commit of S_t(jj+1) also tells the softmax warps that
 //               O_t is stable.  P_t lives in the first 32 TMEM columns of S_t;
 //               the tensor pipe executes one thread's MMAs in issue order, so
 //               S_t(jj+1) overwrites P_t(jj) only after P.V has read it.
-//   warp 3      builds the selection bitmap (MASS), otherwise idle.
-//   warps 4..   one warpgroup per M-tile: thread r owns row r of the tile;
-//               online softmax in the exp2 domain with lazy rescaling (the
-//               reference maximum only moves when the row maximum exceeds it
-//               by more than 8, i.e. a factor 256), P written back to TMEM as
-//               bf16 pairs, O rescaled in TMEM when the maximum moved, and
-//               the epilogue.
+//   warps 2..   one warpgroup per M-tile (TMEM lane quarter = warp % 4):
+//               thread r owns row r of the tile; all 64 scores of a block
+//               come in with one TMEM load; online softmax in the exp2 domain
+//               with lazy rescaling (the reference maximum only moves when the
+//               row maximum exceeds it by more than 8, i.e. a factor 256), P
+//               written back to TMEM as bf16 pairs in two halves, O rescaled in
+//               TMEM when the maximum moved, and the epilogue.
 //
 // TMEM per M-tile t (stride 64 + D, or 64 + 2D with MASS): S/P at +0
 // (64 columns of fp32 scores; P overwrites columns 0..31 as bf16 pairs),
@@ -55,10 +57,10 @@ struct FwdConfig {
   static constexpr int NS = (D == 64) ? 4 : 3;    // K/V ring stages
   static constexpr int TSTRIDE = 64 + (MASS ? 2 : 1) * D;  // TMEM columns per M-tile
   static constexpr int TMEM_COLS = pow2_at_least(T * TSTRIDE);
-  static constexpr int THREADS = 128 * (T + 1);
-  static constexpr int ISS = T >= 4 ? 2 : 1;      // MMA issuer warps (warps 1..ISS)
+  static constexpr int THREADS = 64 + 128 * T;
+  static constexpr int ISS = 1;                   // MMA issuer warps (warp 1)
   static constexpr int POLY = (D == 128) ? 3 : 0; // exp2 pairs of 8 on the FMA pipe
-  static constexpr int NBARS = 1 + ISS + 3 * NS + 3 * T;
+  static constexpr int NBARS = 1 + ISS + 3 * NS + 4 * T;
   // shared memory: Q tiles, K ring, V ring, barriers, tmem slot, abort flag,
   // selection bitmap (up to 8192 blocks)
   static constexpr int SMEM_TILES = T * QTILE + 2 * NS * KVT;
@@ -88,7 +90,8 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, FwdConfig<D, T
   uint64_t* bar_vfull = bar_kfull + NS;
   uint64_t* bar_empty = bar_vfull + NS;
   uint64_t* bar_sfull = bar_empty + NS;
-  uint64_t* bar_pfull = bar_sfull + T;
+  uint64_t* bar_phalf = bar_sfull + T;  // P columns 0..15 (keys 0..31) stored, O rescaled
+  uint64_t* bar_pfull = bar_phalf + T;  // all of P stored
   uint64_t* bar_odone = bar_pfull + T;
   uint64_t* bar_drain = bar_odone + T;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_drain + C::ISS);
@@ -119,6 +122,7 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, FwdConfig<D, T
     }
     for (int t = 0; t < T; ++t) {
       mbar_init(&bar_sfull[t], 1);
+      mbar_init(&bar_phalf[t], 128);
       mbar_init(&bar_pfull[t], 128);
       mbar_init(&bar_odone[t], 1);
     }
@@ -129,7 +133,7 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, FwdConfig<D, T
   // launched with programmatic serialization: the index table may still be
   // in flight from the selection kernel until here
   pdl_wait();
-  if (MASS && warp == 3) {
+  if (MASS && warp == 0) {
     const int words = (p.n + 31) / 32;
     for (int w = lane; w < words; w += 32) selbits[w] = 0u;
     __syncwarp();
@@ -236,7 +240,8 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, FwdConfig<D, T
         for (int x = 0; x < MT; ++x) {
           const int t = me + x * ISS;
           if (t >= T || !ok) continue;
-          if (!mbar_wait(&bar_pfull[t], jj & 1, abort_flag, tmo, 0x205)) {
+          // keys 0..31 as soon as the first half of P is stored
+          if (!mbar_wait(&bar_phalf[t], jj & 1, abort_flag, tmo, 0x205)) {
             ok = false;
             continue;
           }
@@ -245,9 +250,17 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, FwdConfig<D, T
           const uint32_t base = tmem + t * TSTRIDE;
           const uint32_t o_col = base + 64 + ((MASS && !is_sel) ? D : 0);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)  // 16 keys per MMA: 16 rows of 128 B
+          for (int kk = 0; kk < 2; ++kk)  // 16 keys per MMA: 16 rows of 128 B
             mma_ts(o_col, base + kk * 8, v0 + ((kk * (16 * 128)) >> 4), idesc_pv,
                    (first && kk == 0) ? 0u : 1u);
+          if (!mbar_wait(&bar_pfull[t], jj & 1, abort_flag, tmo, 0x206)) {
+            ok = false;
+            continue;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 2; kk < 4; ++kk)
+            mma_ts(o_col, base + kk * 8, v0 + ((kk * (16 * 128)) >> 4), idesc_pv, 1u);
           if (more) {
             issue_qk(t, st1);
             tc_commit(&bar_sfull[t]);
@@ -267,9 +280,9 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, FwdConfig<D, T
         mbar_wait(&bar_drain[me], 0, &never, tmo, 0x2ff);
       }
     }
-  } else if (warp >= 4) {
+  } else if (warp >= 2) {
     // ------------------------------------------------------------ softmax
-    const int t = (warp - 4) / 4;
+    const int t = (warp - 2) / 4;
     const int wq = warp % 4;
     const int r = wq * 32 + lane;
     const int hh = r / 64, tq = r % 64;
@@ -292,16 +305,12 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, FwdConfig<D, T
       const bool diag = (jj == nblk - 1);
       bool is_sel = true;
       if (MASS) is_sel = (selbits[jj >> 5] >> (jj & 31)) & 1u;
-      // raw row maximum over both halves; half A (columns 0..31) stays in registers
-      float sA[32];
-      float mx;
-      {
-        float sB[32];
-        tmem_ld32(tS + 32, sB);
-        mx = diag ? row_max32<true>(sB, 32, tq, -INFINITY) : row_max32<false>(sB, 32, tq, -INFINITY);
-      }
-      tmem_ld32(tS, sA);
-      mx = diag ? row_max32<true>(sA, 0, tq, mx) : row_max32<false>(sA, 0, tq, mx);
+      // all 64 scores with one TMEM round trip, then the raw row maximum
+      float sv[64];
+      tmem_ld64(tS, sv);
+      float mx = diag ? row_max32<true>(sv + 32, 32, tq, -INFINITY)
+                      : row_max32<false>(sv + 32, 32, tq, -INFINITY);
+      mx = diag ? row_max32<true>(sv, 0, tq, mx) : row_max32<false>(sv, 0, tq, mx);
       const float mx_s = mx * sl2;
       float alpha = 1.f;
       const bool moved = mx_s > m_ref + 8.f;
@@ -312,23 +321,10 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, FwdConfig<D, T
       const uint64_t negm2 = f2_pack(-m_ref, -m_ref);
       uint64_t acc2 = f2_pack(0.f, 0.f);
       uint32_t pk[16];
-      if (diag) exp_pack32<true>(sA, 0, tq, scale2, negm2, acc2, pk);
-      else exp_pack32<false, C::POLY>(sA, 0, tq, scale2, negm2, acc2, pk);
-      tmem_st16(tS, pk);  // P columns 0..15 over S columns 0..15 (already read)
-      {
-        float sB[32];
-        tmem_ld32(tS + 32, sB);
-        if (diag) exp_pack32<true>(sB, 32, tq, scale2, negm2, acc2, pk);
-        else exp_pack32<false, C::POLY>(sB, 32, tq, scale2, negm2, acc2, pk);
-      }
-      tmem_st16(tS + 16, pk);  // P columns 16..31
-      float r0, r1;
-      f2_unpack(acc2, r0, r1);
-      l_sel *= alpha;
-      l_uns *= alpha;
-      if (is_sel) l_sel += r0 + r1; else l_uns += r0 + r1;
+      if (diag) exp_pack32<true>(sv, 0, tq, scale2, negm2, acc2, pk);
+      else exp_pack32<false, C::POLY>(sv, 0, tq, scale2, negm2, acc2, pk);
       // O is stable here (S(jj) was committed after P(jj-1).V) and is read by
-      // the tensor core only after pfull: rescale it when the maximum moved
+      // the tensor core only after phalf: rescale it when the maximum moved
       if (jj > 0 && __any_sync(0xffffffffu, moved)) {
         const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
@@ -350,6 +346,18 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, FwdConfig<D, T
           }
         }
       }
+      tmem_st16(tS, pk);  // P columns 0..15 over S columns 0..15 (already read)
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bar_phalf[t]);
+      if (diag) exp_pack32<true>(sv + 32, 32, tq, scale2, negm2, acc2, pk);
+      else exp_pack32<false, C::POLY>(sv + 32, 32, tq, scale2, negm2, acc2, pk);
+      tmem_st16(tS + 16, pk);  // P columns 16..31
+      float r0, r1;
+      f2_unpack(acc2, r0, r1);
+      l_sel *= alpha;
+      l_uns *= alpha;
+      if (is_sel) l_sel += r0 + r1; else l_uns += r0 + r1;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bar_pfull[t]);
