@@ -60,7 +60,7 @@ struct PsFwdConfig {
   // issuer of a fourth tile
   static constexpr int THREADS = 128 * (T + 1) + (T > 3 ? 32 : 0);
   // barriers: q, kfull/vfull/empty[NS], sfull/sfree/pfull/pvdone/odone/drain[T]
-  static constexpr int NBARS = 1 + 3 * NS + 6 * T;
+  static constexpr int NBARS = 1 + 3 * NS + 7 * T;
   // shared memory: Q tiles, K ring, V ring, P tiles, barriers, tmem slot,
   // abort flag, selection bitmap (up to 8192 blocks)
   static constexpr int SMEM_TILES = T * QTILE + 2 * NS * KVT + T * PTILE;
@@ -101,7 +101,8 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS>::THREADS, 1)
   uint64_t* bar_pvdone = bar_pfull + T;         // [T] P.V completed
   uint64_t* bar_odone = bar_pvdone + T;         // [T] last P.V completed
   uint64_t* bar_drain = bar_odone + T;          // [T] issuer's MMAs drained (abort)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_drain + T);
+  uint64_t* bar_turn = bar_drain + T;           // [T] tile t may exponentiate (T = 2)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_turn + T);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint32_t* selbits = tmem_slot + 4;
 
@@ -134,6 +135,7 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS>::THREADS, 1)
       mbar_init(&bar_pvdone[t], 1);
       mbar_init(&bar_odone[t], 1);
       mbar_init(&bar_drain[t], 1);
+      mbar_init(&bar_turn[t], 128);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -300,6 +302,15 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS>::THREADS, 1)
       const bool diag = (jj == nblk - 1);
       bool is_sel = true;
       if (MASS) is_sel = (selbits[jj >> 5] >> (jj & 31)) & 1u;
+      // with two tiles, their exponential phases alternate: tile 1's block jj
+      // follows tile 0's block jj, tile 0's block jj + 1 follows tile 1's
+      // block jj, so one tile's MMAs run while the other exponentiates
+      if (T == 2 && (t == 1 || jj > 0) &&
+          !__all_sync(0xffffffffu, mbar_wait(&bar_turn[t], (t == 1 ? jj : jj - 1) & 1, abort_flag, tmo,
+                                             0x305))) {
+        ok = false;
+        break;
+      }
       float mx = diag ? row_max32<true>(sB, 32, tq, -INFINITY) : row_max32<false>(sB, 32, tq, -INFINITY);
       mx = diag ? row_max32<true>(sA, 0, tq, mx) : row_max32<false>(sA, 0, tq, mx);
       const float mx_s = mx * sl2;
@@ -319,6 +330,7 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS>::THREADS, 1)
         exp_pack32<false, C::POLY>(sA, 0, tq, scale2, negm2, acc2, pk);
         exp_pack32<false, C::POLY>(sB, 32, tq, scale2, negm2, acc2, pk + 16);
       }
+      if (T == 2) mbar_arrive(&bar_turn[1 - t]);
       float r0, r1;
       f2_unpack(acc2, r0, r1);
       l_sel *= alpha;
