@@ -53,6 +53,15 @@ def algorithmic_flops(workload) -> float:
     return 4.0 * w.head_dim * selected_pairs(w) * w.batch * w.n_q_heads
 
 
+def causal_flops(workload) -> float:
+    """FLOPs of dense causal attention (the alignment pass's full stream):
+    4 D per unmasked (query, key) pair over all causal blocks."""
+    w = workload
+    n = w.n_blocks
+    pairs = n * (n - 1) // 2 * 64 * 64 + n * (64 * 65 // 2)
+    return 4.0 * w.head_dim * pairs * w.batch * w.n_q_heads
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -249,6 +258,26 @@ def run_ours(args, world, rank, local):
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
     d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
 
+    # the other rows of the path on the same workload, outside the step: the
+    # alignment pass (dense causal attention, counterpart sparse output and
+    # dropped mass in one launch) and the sparse backward with a seeded dO
+    of, lsef, dmass = torch.empty_like(st.o), torch.empty_like(st.lse), torch.empty_like(st.lse)
+    ssa.ssa_full_attn_fwd_with_mass(p, q, k, v, st.block_idx, st.o, st.lse, of, lsef, dmass)
+    g_mass = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_mass):
+        ssa.ssa_full_attn_fwd_with_mass(p, q, k, v, st.block_idx, st.o, st.lse, of, lsef, dmass)
+    g_step.replay()
+    gen_do = torch.Generator().manual_seed(7)
+    d_o = torch.randn(st.o.shape, generator=gen_do).to(torch.bfloat16).to(dev)
+    st.backward(q, k, v, d_o)
+    g_bwd = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_bwd):
+        st.backward(q, k, v, d_o)
+    mass_ms = timed(g_mass, n_k) / n_k
+    bwd_ms = timed(g_bwd, n_k) / n_k
+    torch.cuda.synchronize()
+    assert ssa.ssa_get_device_error() == 0
+
     peaks, peak_src = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     achieved = flops / (fwd_ms * 1e-3) / 1e12
@@ -268,6 +297,13 @@ def run_ours(args, world, rank, local):
                      "kernel_ms": round(fwd_ms, 5)},
         "kernels_ms": {"block_pool": round(pool_ms, 5), "block_select": round(sel_ms, 5),
                        "sparse_attn_fwd": round(fwd_ms, 5)},
+        "other_rows": {
+            "full_attn_fwd_with_mass": {
+                "ms": round(mass_ms, 5), "flops": "4 D per causal (query, key) pair",
+                "tflops": round(causal_flops(w) / (mass_ms * 1e-3) / 1e12, 2)},
+            "sparse_attn_bwd": {
+                "ms": round(bwd_ms, 5), "flops": "10 D per selected (query, key) pair",
+                "tflops": round(2.5 * flops / (bwd_ms * 1e-3) / 1e12, 2)}},
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
         "pct_of_peak_step": round(100.0 * value / world / peak, 2),
