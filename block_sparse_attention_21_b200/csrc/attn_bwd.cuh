@@ -10,7 +10,7 @@
 //   dK_s = scale sum_t dS_ts q_t      dQ_t  = scale sum_s dS_ts k_s
 // where t runs over the query rows of every head of the KV head's group.
 //
-// Three launches, no atomics (results are deterministic):
+// Three launches, no floating-point atomics (results are deterministic):
 //   bwd_prep_kernel    D_t for every row, and the reverse index: for each key
 //                      block j the query blocks whose selection contains j,
 //                      ascending (CSR in the workspace).
@@ -63,84 +63,118 @@ __host__ __device__ inline BwdWorkspace bwd_workspace_layout(int B, int S, int H
   return w;
 }
 
-// Whether key block j is in query block i's selection (ascending row of
-// min(topk, i + 1) valid entries).
-__device__ __forceinline__ bool row_selects(const int32_t* row, int nvalid, int j) {
-  int lo = 0, hi = nvalid - 1;
-  while (lo <= hi) {
-    const int mid = (lo + hi) >> 1;
-    const int v = row[mid];
-    if (v == j) return true;
-    if (v < j) lo = mid + 1; else hi = mid - 1;
-  }
-  return false;
+// Index-table entries the reverse-index CTAs stage in shared memory at a time.
+constexpr int kRevStage = 2048;
+
+// Dynamic shared memory of bwd_prep_kernel for n key blocks.
+__host__ __device__ inline size_t bwd_prep_smem(int n) {
+  return static_cast<size_t>(2 * n + 1 + kRevStage) * sizeof(int32_t);
 }
 
-// Block 0..(rowsD - 1): D_t for 8 rows per warp-iteration...; the last
-// B * Hkv blocks: the reverse index of one (b, KV head).
+// Blocks 0 .. B*Hkv - 1: the reverse index of one (b, KV head); the rest: D_t.
+//  - reverse index: for each key block j, the query blocks i whose selection
+//    holds j, ascending (CSR).  Counts come from shared-memory atomics over
+//    the table, offsets from a warp scan; then one warp walks the rows in
+//    ascending i (staged through shared memory) and appends i to the list of
+//    each of its blocks.  A row's blocks are distinct, so the lanes of one row
+//    never touch the same list, and the lists come out in ascending order
+//    without sorting: deterministic.
 //  - D_t: each row's D elements are read by D / 8 lanes (16 B each) and
-//    reduced with shuffles.
-//  - reverse index: thread per key block j counts, then (after an exclusive
-//    scan in shared memory) lists, the query blocks i >= j selecting j, in
-//    ascending order.
+//    reduced with shuffles, 8 rows per warp-iteration.
 template <int D>
-__global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p, int dt_blocks) {
-  if (static_cast<int>(blockIdx.x) < dt_blocks) {
-    constexpr int LPR = D / 8;            // lanes per row
-    constexpr int RPW = 32 / LPR;         // rows per warp per iteration
-    const int warp_global = (blockIdx.x * blockDim.x + threadIdx.x) / 32;
-    const int nwarps = dt_blocks * (blockDim.x / 32);
-    const int lane = threadIdx.x % 32;
-    const int sub = lane / LPR, part = lane % LPR;
-    const long long rows = static_cast<long long>(p.B) * p.S * p.Hq;  // (b, t, hq) row-major
-    for (long long r0 = static_cast<long long>(warp_global) * RPW; r0 < rows;
-         r0 += static_cast<long long>(nwarps) * RPW) {
-      const long long r = r0 + sub;
-      float acc = 0.f;
-      if (r < rows) {
-        const uint4 a = *reinterpret_cast<const uint4*>(p.o + r * D + part * 8);
-        const uint4 g = *reinterpret_cast<const uint4*>(p.d_o + r * D + part * 8);
-        const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wg[4] = {g.x, g.y, g.z, g.w};
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p, int rev_blocks) {
+  if (static_cast<int>(blockIdx.x) < rev_blocks) {
+    extern __shared__ int32_t rsm[];
+    const int n = p.n, k = p.topk;
+    int32_t* off = rsm;             // [n + 1]: counts, then offsets
+    int32_t* fill = off + n + 1;    // [n]
+    int32_t* stage = fill + n;      // [kRevStage]
+    const int bh = blockIdx.x;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int32_t* idx = p.idx + static_cast<size_t>(bh) * n * k;
+    for (int j = threadIdx.x; j <= n; j += blockDim.x) off[j] = 0;
+    for (int j = threadIdx.x; j < n; j += blockDim.x) fill[j] = 0;
+    __syncthreads();
+    for (int e = threadIdx.x; e < n * k; e += blockDim.x) {
+      const int j = idx[e];
+      if (j >= 0 && j < n) atomicAdd(&off[j + 1], 1);
+    }
+    __syncthreads();
+    if (warp == 0) {  // inclusive scan of off[1..n]
+      const int per = (n + 31) / 32, base = 1 + lane * per;
+      int sum = 0;
+      for (int x = 0; x < per; ++x)
+        if (base + x <= n) sum += off[base + x];
+      int incl = sum;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          acc = fmaf(__uint_as_float(wa[e] << 16), __uint_as_float(wg[e] << 16), acc);
-          acc = fmaf(__uint_as_float(wa[e] & 0xFFFF0000u), __uint_as_float(wg[e] & 0xFFFF0000u), acc);
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int run = incl - sum;
+      for (int x = 0; x < per; ++x)
+        if (base + x <= n) {
+          run += off[base + x];
+          off[base + x] = run;
+        }
+    }
+    __syncthreads();
+    int32_t* goff = p.rev_off + static_cast<size_t>(bh) * (n + 1);
+    for (int j = threadIdx.x; j <= n; j += blockDim.x) goff[j] = off[j];
+    int32_t* rev = p.rev + static_cast<size_t>(bh) * n * k;
+    const int rows_per_chunk = k <= kRevStage ? kRevStage / k : 1;
+    for (int i0 = 0; i0 < n; i0 += rows_per_chunk) {
+      const int rows = min(rows_per_chunk, n - i0);
+      for (int e = threadIdx.x; e < rows * k; e += blockDim.x)
+        stage[e] = idx[static_cast<size_t>(i0) * k + e];
+      __syncthreads();
+      if (warp == 0) {
+        for (int ii = 0; ii < rows; ++ii) {
+          for (int r = lane; r < k; r += 32) {
+            const int j = stage[ii * k + r];
+            if (j >= 0 && j < n) {
+              rev[off[j] + fill[j]] = i0 + ii;
+              fill[j] += 1;
+            }
+          }
+          __syncwarp();
         }
       }
-#pragma unroll
-      for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-      if (r < rows && part == 0) {
-        const int hq = static_cast<int>(r % p.Hq);
-        const long long bt = r / p.Hq;
-        const int t = static_cast<int>(bt % p.S), b = static_cast<int>(bt / p.S);
-        p.dt[(static_cast<size_t>(b) * p.Hq + hq) * p.S + t] = acc;
-      }
+      __syncthreads();
     }
     return;
   }
-  // ---- reverse index of (b, h)
-  extern __shared__ int32_t rev_count[];  // n + 1
-  const int bh = blockIdx.x - dt_blocks;
-  const int32_t* idx = p.idx + static_cast<size_t>(bh) * p.n * p.topk;
-  for (int j = threadIdx.x; j < p.n; j += blockDim.x) {
-    int cnt = 0;
-    for (int i = j; i < p.n; ++i)
-      cnt += row_selects(idx + static_cast<size_t>(i) * p.topk, min(p.topk, i + 1), j) ? 1 : 0;
-    rev_count[j + 1] = cnt;
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    rev_count[0] = 0;
-    for (int j = 0; j < p.n; ++j) rev_count[j + 1] += rev_count[j];
-  }
-  __syncthreads();
-  int32_t* off = p.rev_off + static_cast<size_t>(bh) * (p.n + 1);
-  int32_t* rev = p.rev + static_cast<size_t>(bh) * p.n * p.topk;
-  for (int j = threadIdx.x; j <= p.n; j += blockDim.x) off[j] = rev_count[j];
-  for (int j = threadIdx.x; j < p.n; j += blockDim.x) {
-    int w = rev_count[j];
-    for (int i = j; i < p.n; ++i)
-      if (row_selects(idx + static_cast<size_t>(i) * p.topk, min(p.topk, i + 1), j)) rev[w++] = i;
+  // ---- D_t
+  constexpr int LPR = D / 8;            // lanes per row
+  constexpr int RPW = 32 / LPR;         // rows per warp per iteration
+  const int dt_blocks = static_cast<int>(gridDim.x) - rev_blocks;
+  const int warp_global = ((blockIdx.x - rev_blocks) * blockDim.x + threadIdx.x) / 32;
+  const int nwarps = dt_blocks * (blockDim.x / 32);
+  const int lane = threadIdx.x % 32;
+  const int sub = lane / LPR, part = lane % LPR;
+  const long long rows = static_cast<long long>(p.B) * p.S * p.Hq;  // (b, t, hq) row-major
+  for (long long r0 = static_cast<long long>(warp_global) * RPW; r0 < rows;
+       r0 += static_cast<long long>(nwarps) * RPW) {
+    const long long r = r0 + sub;
+    float acc = 0.f;
+    if (r < rows) {
+      const uint4 a = *reinterpret_cast<const uint4*>(p.o + r * D + part * 8);
+      const uint4 g = *reinterpret_cast<const uint4*>(p.d_o + r * D + part * 8);
+      const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wg[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        acc = fmaf(__uint_as_float(wa[e] << 16), __uint_as_float(wg[e] << 16), acc);
+        acc = fmaf(__uint_as_float(wa[e] & 0xFFFF0000u), __uint_as_float(wg[e] & 0xFFFF0000u), acc);
+      }
+    }
+#pragma unroll
+    for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (r < rows && part == 0) {
+      const int hq = static_cast<int>(r % p.Hq);
+      const long long bt = r / p.Hq;
+      const int t = static_cast<int>(bt % p.S), b = static_cast<int>(bt / p.S);
+      p.dt[(static_cast<size_t>(b) * p.Hq + hq) * p.S + t] = acc;
+    }
   }
 }
 

@@ -290,8 +290,15 @@ ssa_status launch_bwd(const Dims& d, const void* q, const void* k, const void* v
   const int rows_per_block = 8 * (32 / (D / 8));
   long long dt_blocks_ll = (rows + rows_per_block - 1) / rows_per_block;
   const int dt_blocks = static_cast<int>(dt_blocks_ll < 4096 ? dt_blocks_ll : 4096);
-  ssa::bwd_prep_kernel<D><<<dt_blocks + d.B * d.Hkv, 256, 4 * (d.n + 1), st>>>(bp, dt_blocks);
-  ssa_status s = launch_result();
+  // the reverse-index CTAs first (they run longest), then the D_t CTAs; the
+  // shared-memory attribute is set once, for the largest supported n
+  static std::atomic<uint64_t> prep_done{0};
+  ssa_status s = ensure_smem(ssa::bwd_prep_kernel<D>, static_cast<int>(ssa::bwd_prep_smem(kMaxSeqLen / 64)),
+                             &prep_done);
+  if (s != SSA_OK) return s;
+  const int rev_blocks = d.B * d.Hkv;
+  ssa::bwd_prep_kernel<D><<<rev_blocks + dt_blocks, 256, ssa::bwd_prep_smem(d.n), st>>>(bp, rev_blocks);
+  s = launch_result();
   if (s != SSA_OK) return s;
 
   // 2. dK, dV: one CTA per (b, KV head, key block)
