@@ -10,16 +10,18 @@
 //   dK_s = scale sum_t dS_ts q_t      dQ_t  = scale sum_s dS_ts k_s
 // where t runs over the query rows of every head of the KV head's group.
 //
-// Three launches, no floating-point atomics (results are deterministic):
+// Four launches, no floating-point atomics (results are deterministic):
 //   bwd_prep_kernel    D_t for every row, and the reverse index: for each key
 //                      block j the query blocks whose selection contains j,
 //                      ascending (CSR in the workspace).
-//   attn_bwd_dkdv_kernel  one CTA per (batch, KV head, key block j): walks the
-//                      query tiles (query block x head pair) of j's reverse
-//                      list; S = Q K_j^T and dP = dO V_j^T on tcgen05, the
-//                      elementwise warps form P and dS into shared memory,
-//                      then dV += P^T dO and dK += dS^T Q as M = 64 MMAs with
-//                      both operands MN-major in shared memory.
+//   attn_bwd_dkdv_kernel  kDkdvSplit CTAs per (batch, KV head, key block j),
+//                      sharing out the query tiles (query block x head pair)
+//                      of j's reverse list; S = Q K_j^T and dP = dO V_j^T on
+//                      tcgen05, the elementwise warps form P and dS into shared
+//                      memory, then dV += P^T dO and dK += dS^T Q as M = 64 MMAs
+//                      with both operands MN-major in shared memory; each CTA
+//                      writes fp32 partial sums.
+//   bwd_dkdv_reduce_kernel  adds the partials in a fixed order into dK, dV.
 //   attn_bwd_dq_kernel one CTA per (batch, KV head, query block, head pairs):
 //                      walks the selected blocks like the forward; dS goes to
 //                      TMEM over S and dQ += dS K_j reads it as the A operand.
@@ -29,6 +31,12 @@
 #include "softmax_util.cuh"
 
 namespace ssa {
+
+// The dK/dV work of one key block is split into this many CTAs (tile x goes
+// to CTA x % kDkdvSplit), so the key blocks that many query blocks select do
+// not leave one CTA running long after the rest; each CTA writes fp32 partial
+// sums, which a reduction kernel adds in a fixed order.
+constexpr int kDkdvSplit = 4;
 
 struct BwdParams {
   int B, S, Hq, Hkv, G, n, topk, slices;
@@ -41,6 +49,7 @@ struct BwdParams {
   float* dt;              // workspace: D_t [B][Hq][S]
   int32_t* rev_off;       // workspace: [B][Hkv][n + 1]
   int32_t* rev;           // workspace: [B][Hkv][n * topk]
+  float* part;            // workspace: [B][Hkv][n][kDkdvSplit][dV, dK][64][D]
   __nv_bfloat16* dq;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
@@ -50,16 +59,17 @@ struct BwdParams {
 __host__ __device__ inline size_t bwd_align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct BwdWorkspace {
-  size_t dt, rev_off, rev, total;
+  size_t dt, rev_off, rev, part, total;
 };
 
 __host__ __device__ inline BwdWorkspace bwd_workspace_layout(int B, int S, int Hq, int Hkv, int n,
-                                                            int topk) {
+                                                            int topk, int D) {
   BwdWorkspace w;
   w.dt = 0;
   w.rev_off = bwd_align256(static_cast<size_t>(B) * Hq * S * sizeof(float));
   w.rev = w.rev_off + bwd_align256(static_cast<size_t>(B) * Hkv * (n + 1) * sizeof(int32_t));
-  w.total = w.rev + bwd_align256(static_cast<size_t>(B) * Hkv * n * topk * sizeof(int32_t));
+  w.part = w.rev + bwd_align256(static_cast<size_t>(B) * Hkv * n * topk * sizeof(int32_t));
+  w.total = w.part + bwd_align256(static_cast<size_t>(B) * Hkv * n * kDkdvSplit * 2 * 64 * D * sizeof(float));
   return w;
 }
 
@@ -188,24 +198,34 @@ struct DkdvConfig {
   static constexpr int TMEM_COLS = pow2_at_least(128 + 2 * D);
   static constexpr int THREADS = 256;          // warp 0 producer, 1 issuer, 4..7 elementwise
   static constexpr int NBARS = 1 + 2 * NQ + 7;
-  static constexpr int SMEM_BYTES = 1024 + 2 * KVT + NQ * 2 * QTILE + 2 * PTILE + NBARS * 8 + 16;
+  // no alignment slack: the dynamic shared memory of a kernel without static
+  // shared memory starts 1024-byte aligned (the kernel checks it), which lets
+  // two CTAs share an SM at head_dim 64 (TMEM 256 columns each)
+  static constexpr int SMEM_BYTES = 2 * KVT + NQ * 2 * QTILE + 2 * PTILE + NBARS * 8 + 16;
+  static constexpr int MIN_CTAS = (TMEM_COLS <= 256 && SMEM_BYTES + 1024 <= 116736) ? 2 : 1;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-// One CTA per (batch b, KV head h, key block j), heaviest first is not known
-// in advance; blocks are taken in index order.  TMEM: S at +0 and dP at +64
+// kDkdvSplit CTAs per (batch b, KV head h, key block j), CTA sp taking tiles
+// sp, sp + kDkdvSplit, ... of j's list.  TMEM: S at +0 and dP at +64
 // (128 lanes x 64 fp32 each), dV at +128 and dK at +128 + D (M = 64
 // accumulators: key row r sits in lane (r % 16) + 32 * (r / 16)).
 template <int D>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(256, DkdvConfig<D>::MIN_CTAS)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                          const BwdParams p) {
   using C = DkdvConfig<D>;
   constexpr int NP = C::NP, QTILE = C::QTILE, KVT = C::KVT, PTILE = C::PTILE, NQ = C::NQ;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if ((smem_u32(smem_raw) & 1023u) != 0) {  // the 128-byte swizzle needs 1024-byte aligned tiles
+    if (threadIdx.x == 0) {
+      atomicOr(&g_error_word, kErrTimeout);
+      atomicExch(&g_error_site, 0x8fe);
+    }
+    return;
+  }
+  uint8_t* smem = smem_raw;
   uint8_t* sK = smem;
   uint8_t* sV = sK + KVT;
   uint8_t* sQ = sV + KVT;              // [NQ][QTILE]
@@ -226,7 +246,8 @@ __global__ void __launch_bounds__(256, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int bhn = blockIdx.x;
+  const int sp = blockIdx.x % kDkdvSplit;  // this CTA's share: tiles sp, sp + kDkdvSplit, ...
+  const int bhn = blockIdx.x / kDkdvSplit;
   const int j = bhn % p.n;
   const int h = (bhn / p.n) % p.Hkv;
   const int b = bhn / (p.n * p.Hkv);
@@ -235,7 +256,8 @@ __global__ void __launch_bounds__(256, 1)
   const int32_t* off = p.rev_off + bh * (p.n + 1);
   const int32_t* rev = p.rev + bh * p.n * p.topk;
   const int first_q = off[j];
-  const int ntiles = (off[j + 1] - first_q) * HP;
+  const int ntiles_all = (off[j + 1] - first_q) * HP;
+  const int ntiles = ntiles_all > sp ? (ntiles_all - sp + kDkdvSplit - 1) / kDkdvSplit : 0;
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
@@ -274,8 +296,9 @@ __global__ void __launch_bounds__(256, 1)
       for (int x = 0; x < ntiles; ++x) {
         const int qs = x % NQ;
         if (x >= NQ && !mbar_wait(&q_empty[qs], ((x / NQ) - 1) & 1, abort_flag, tmo, 0x801)) break;
-        const int i = rev[first_q + x / HP];
-        const int hq0 = h * p.G + 2 * (x % HP);
+        const int gx = sp + x * kDkdvSplit;
+        const int i = rev[first_q + gx / HP];
+        const int hq0 = h * p.G + 2 * (gx % HP);
         mbar_arrive_expect_tx(&q_full[qs], 2 * QTILE);
         for (int hh = 0; hh < 2; ++hh)
           for (int pn = 0; pn < NP; ++pn) {
@@ -375,8 +398,9 @@ __global__ void __launch_bounds__(256, 1)
     const float sl2 = p.scale_log2;
     bool ok = true;
     for (int x = 0; x < ntiles; ++x) {
-      const int i = rev[first_q + x / HP];
-      const int hq = h * p.G + 2 * (x % HP) + hh;
+      const int gx = sp + x * kDkdvSplit;
+      const int i = rev[first_q + gx / HP];
+      const int hq = h * p.G + 2 * (gx % HP) + hh;
       const size_t lrow = (static_cast<size_t>(b) * p.Hq + hq) * p.S + 64 * i + tq;
       const float nlse = -p.lse[lrow] * kLog2e;
       const float dt = p.dt[lrow];
@@ -418,33 +442,29 @@ __global__ void __launch_bounds__(256, 1)
       mbar_arrive(p_full);
     }
     // ---------------------------------------------------------- epilogue
-    // key row kr = 16 * wq + lane (lanes 0..15 of each quadrant hold the M = 64 rows)
+    // key row kr = 16 * wq + lane (lanes 0..15 of each quadrant hold the M = 64
+    // rows); this CTA's fp32 partial sums of dV and dK (dK not yet scaled)
     const int kr = 16 * wq + lane;
-    const size_t grow = ((static_cast<size_t>(b) * p.S + 64 * j + kr) * p.Hkv + h) * D;
+    float* part = p.part + (static_cast<size_t>(bhn) * kDkdvSplit + sp) * 2 * 64 * D;
     if (ntiles == 0) {
       if (lane < 16)
-        for (int d = 0; d < D; d += 8) {
-          *reinterpret_cast<uint4*>(p.dv + grow + d) = make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>(p.dk + grow + d) = make_uint4(0, 0, 0, 0);
-        }
+        for (int which = 0; which < 2; ++which)
+          for (int d = 0; d < D; d += 4)
+            *reinterpret_cast<float4*>(part + (which * 64 + kr) * D + d) = make_float4(0.f, 0.f, 0.f, 0.f);
     } else if (ok && __all_sync(0xffffffffu, mbar_wait(o_done, 0, abort_flag, tmo, 0xa03))) {
       tc_fence_after();
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
         const uint32_t base = row + 128 + which * D;
-        const float mul = which ? p.scale : 1.f;
-        __nv_bfloat16* dst = which ? p.dk : p.dv;
 #pragma unroll
         for (int ch = 0; ch < D / 32; ++ch) {
           float o[32];
           tmem_ld32(base + ch * 32, o);
           if (lane < 16) {
-            uint32_t w[16];
+            float4* out = reinterpret_cast<float4*>(part + (which * 64 + kr) * D + ch * 32);
 #pragma unroll
-            for (int c = 0; c < 16; ++c) w[c] = pack_bf16x2(o[2 * c] * mul, o[2 * c + 1] * mul);
-            uint4* out = reinterpret_cast<uint4*>(dst + grow + ch * 32);
-#pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4) out[v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+            for (int v4 = 0; v4 < 8; ++v4)
+              out[v4] = make_float4(o[4 * v4], o[4 * v4 + 1], o[4 * v4 + 2], o[4 * v4 + 3]);
           }
         }
       }
@@ -456,6 +476,33 @@ __global__ void __launch_bounds__(256, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// dV = sum of the kDkdvSplit partials, dK = scale * sum, in a fixed order
+// (deterministic); one CTA per (b, KV head, key block).
+template <int D>
+__global__ void __launch_bounds__(256) bwd_dkdv_reduce_kernel(const BwdParams p) {
+  const int bhn = blockIdx.x;
+  const int j = bhn % p.n, h = (bhn / p.n) % p.Hkv, b = bhn / (p.n * p.Hkv);
+  constexpr int PER = 2 * 64 * D / 4;  // float4 per partial
+  const float4* part = reinterpret_cast<const float4*>(p.part + static_cast<size_t>(bhn) * kDkdvSplit * 2 * 64 * D);
+  for (int e = threadIdx.x; e < PER; e += blockDim.x) {
+    float4 a = part[e];
+#pragma unroll
+    for (int x = 1; x < kDkdvSplit; ++x) {
+      const float4 c = part[x * PER + e];
+      a.x += c.x;
+      a.y += c.y;
+      a.z += c.z;
+      a.w += c.w;
+    }
+    const int which = e / (64 * D / 4);  // 0: dV, 1: dK
+    const int rem = e % (64 * D / 4);
+    const int kr = rem / (D / 4), d4 = rem % (D / 4);
+    const float mul = which ? p.scale : 1.f;
+    __nv_bfloat16* dst = (which ? p.dk : p.dv) + ((static_cast<size_t>(b) * p.S + 64 * j + kr) * p.Hkv + h) * D + 4 * d4;
+    *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(a.x * mul, a.y * mul), pack_bf16x2(a.z * mul, a.w * mul));
   }
 }
 

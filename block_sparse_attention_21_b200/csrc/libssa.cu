@@ -246,14 +246,14 @@ ssa_status launch_psfwd(const Dims& d, const void* q, const void* k, const void*
 // ---------------------------------------------------------------- backward
 
 size_t bwd_workspace_bytes(const Dims& d) {
-  return ssa::bwd_workspace_layout(d.B, d.S, d.Hq, d.Hkv, d.n, d.topk).total;
+  return ssa::bwd_workspace_layout(d.B, d.S, d.Hq, d.Hkv, d.n, d.topk, d.D).total;
 }
 
 template <int D, int TQ>
 ssa_status launch_bwd(const Dims& d, const void* q, const void* k, const void* v, const void* o,
                       const float* lse, const void* d_o, const int32_t* idx, void* dq, void* dk,
                       void* dv, void* workspace, cudaStream_t st) {
-  const ssa::BwdWorkspace ws = ssa::bwd_workspace_layout(d.B, d.S, d.Hq, d.Hkv, d.n, d.topk);
+  const ssa::BwdWorkspace ws = ssa::bwd_workspace_layout(d.B, d.S, d.Hq, d.Hkv, d.n, d.topk, d.D);
   uint8_t* base = static_cast<uint8_t*>(workspace);
   ssa::BwdParams bp;
   bp.B = d.B;
@@ -273,6 +273,7 @@ ssa_status launch_bwd(const Dims& d, const void* q, const void* k, const void* v
   bp.dt = reinterpret_cast<float*>(base + ws.dt);
   bp.rev_off = reinterpret_cast<int32_t*>(base + ws.rev_off);
   bp.rev = reinterpret_cast<int32_t*>(base + ws.rev);
+  bp.part = reinterpret_cast<float*>(base + ws.part);
   bp.dq = static_cast<__nv_bfloat16*>(dq);
   bp.dk = static_cast<__nv_bfloat16*>(dk);
   bp.dv = static_cast<__nv_bfloat16*>(dv);
@@ -285,7 +286,6 @@ ssa_status launch_bwd(const Dims& d, const void* q, const void* k, const void* v
     return SSA_ERR_CUDA;
 
   // 1. D_t and the reverse index
-  // (its dynamic shared memory, 4 (n + 1) bytes <= 32 KB, is under the default limit)
   const long long rows = static_cast<long long>(d.B) * d.S * d.Hq;
   const int rows_per_block = 8 * (32 / (D / 8));
   long long dt_blocks_ll = (rows + rows_per_block - 1) / rows_per_block;
@@ -301,14 +301,18 @@ ssa_status launch_bwd(const Dims& d, const void* q, const void* k, const void* v
   s = launch_result();
   if (s != SSA_OK) return s;
 
-  // 2. dK, dV: one CTA per (b, KV head, key block)
+  // 2. dK, dV: kDkdvSplit CTAs per (b, KV head, key block), then their sum
   {
     using C = ssa::DkdvConfig<D>;
     static std::atomic<uint64_t> done{0};
     auto kernel = ssa::attn_bwd_dkdv_kernel<D>;
     s = ensure_smem(kernel, C::SMEM_BYTES, &done);
     if (s != SSA_OK) return s;
-    kernel<<<static_cast<unsigned>(d.B) * d.Hkv * d.n, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, mv, mdo, bp);
+    kernel<<<static_cast<unsigned>(d.B) * d.Hkv * d.n * ssa::kDkdvSplit, C::THREADS, C::SMEM_BYTES, st>>>(
+        mq, mk, mv, mdo, bp);
+    s = launch_result();
+    if (s != SSA_OK) return s;
+    ssa::bwd_dkdv_reduce_kernel<D><<<static_cast<unsigned>(d.B) * d.Hkv * d.n, 256, 0, st>>>(bp);
     s = launch_result();
     if (s != SSA_OK) return s;
   }
