@@ -50,7 +50,8 @@ def _p(**kw):
 
 
 BAD_PROBLEMS = [
-    (dict(batch=0), INVALID),
+    (dict(batch=0), INVALID),               # empty batch
+    (dict(seq_len=0), INVALID),             # empty sequence
     (dict(seq_len=1000), INVALID),          # not a multiple of the block
     (dict(n_q_heads=6, n_kv_heads=4), INVALID),
     (dict(top_k=0), INVALID),
