@@ -90,7 +90,7 @@ __host__ __device__ inline size_t bwd_prep_smem(int n) {
 //    never touch the same list, and the lists come out in ascending order
 //    without sorting: deterministic.
 //  - D_t: each row's D elements are read by D / 8 lanes (16 B each) and
-//    reduced with shuffles, 8 rows per warp-iteration.
+//    reduced with shuffles; every lane group has four rows' loads in flight.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p, int rev_blocks) {
   if (static_cast<int>(blockIdx.x) < rev_blocks) {
@@ -154,36 +154,47 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p, int re
     }
     return;
   }
-  // ---- D_t
+  // ---- D_t: four rows per lane group in flight
   constexpr int LPR = D / 8;            // lanes per row
   constexpr int RPW = 32 / LPR;         // rows per warp per iteration
+  constexpr int U = 4;                  // iterations whose loads are in flight together
   const int dt_blocks = static_cast<int>(gridDim.x) - rev_blocks;
   const int warp_global = ((blockIdx.x - rev_blocks) * blockDim.x + threadIdx.x) / 32;
   const int nwarps = dt_blocks * (blockDim.x / 32);
   const int lane = threadIdx.x % 32;
   const int sub = lane / LPR, part = lane % LPR;
   const long long rows = static_cast<long long>(p.B) * p.S * p.Hq;  // (b, t, hq) row-major
-  for (long long r0 = static_cast<long long>(warp_global) * RPW; r0 < rows;
-       r0 += static_cast<long long>(nwarps) * RPW) {
-    const long long r = r0 + sub;
-    float acc = 0.f;
-    if (r < rows) {
-      const uint4 a = *reinterpret_cast<const uint4*>(p.o + r * D + part * 8);
-      const uint4 g = *reinterpret_cast<const uint4*>(p.d_o + r * D + part * 8);
-      const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wg[4] = {g.x, g.y, g.z, g.w};
+  const long long stride = static_cast<long long>(nwarps) * RPW;
+  for (long long r0 = static_cast<long long>(warp_global) * RPW; r0 < rows; r0 += U * stride) {
+    uint4 a[U], g[U];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        acc = fmaf(__uint_as_float(wa[e] << 16), __uint_as_float(wg[e] << 16), acc);
-        acc = fmaf(__uint_as_float(wa[e] & 0xFFFF0000u), __uint_as_float(wg[e] & 0xFFFF0000u), acc);
+    for (int u = 0; u < U; ++u) {
+      const long long r = r0 + u * stride + sub;
+      if (r < rows) {
+        a[u] = *reinterpret_cast<const uint4*>(p.o + r * D + part * 8);
+        g[u] = *reinterpret_cast<const uint4*>(p.d_o + r * D + part * 8);
       }
     }
 #pragma unroll
-    for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (r < rows && part == 0) {
-      const int hq = static_cast<int>(r % p.Hq);
-      const long long bt = r / p.Hq;
-      const int t = static_cast<int>(bt % p.S), b = static_cast<int>(bt / p.S);
-      p.dt[(static_cast<size_t>(b) * p.Hq + hq) * p.S + t] = acc;
+    for (int u = 0; u < U; ++u) {
+      const long long r = r0 + u * stride + sub;
+      float acc = 0.f;
+      if (r < rows) {
+        const uint32_t wa[4] = {a[u].x, a[u].y, a[u].z, a[u].w}, wg[4] = {g[u].x, g[u].y, g[u].z, g[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          acc = fmaf(__uint_as_float(wa[e] << 16), __uint_as_float(wg[e] << 16), acc);
+          acc = fmaf(__uint_as_float(wa[e] & 0xFFFF0000u), __uint_as_float(wg[e] & 0xFFFF0000u), acc);
+        }
+      }
+#pragma unroll
+      for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      if (r < rows && part == 0) {
+        const int hq = static_cast<int>(r % p.Hq);
+        const long long bt = r / p.Hq;
+        const int t = static_cast<int>(bt % p.S), b = static_cast<int>(bt / p.S);
+        p.dt[(static_cast<size_t>(b) * p.Hq + hq) * p.S + t] = acc;
+      }
     }
   }
 }
