@@ -273,8 +273,15 @@ def run_ours(args, world, rank, local):
     g_bwd = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_bwd):
         st.backward(q, k, v, d_o)
+    # the alignment objective's backward (mode 0: d_o belongs to the sparse output)
+    st.alignment(q, k, v)
+    st.alignment_backward(q, k, v, d_o, 0, 1.0)
+    g_abwd = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_abwd):
+        st.alignment_backward(q, k, v, d_o, 0, 1.0)
     mass_ms = timed(g_mass, n_k) / n_k
     bwd_ms = timed(g_bwd, n_k) / n_k
+    abwd_ms = timed(g_abwd, n_k) / n_k
     torch.cuda.synchronize()
     assert ssa.ssa_get_device_error() == 0
 
@@ -303,7 +310,11 @@ def run_ours(args, world, rank, local):
                 "tflops": round(causal_flops(w) / (mass_ms * 1e-3) / 1e12, 2)},
             "sparse_attn_bwd": {
                 "ms": round(bwd_ms, 5), "flops": "10 D per selected (query, key) pair",
-                "tflops": round(2.5 * flops / (bwd_ms * 1e-3) / 1e12, 2)}},
+                "tflops": round(2.5 * flops / (bwd_ms * 1e-3) / 1e12, 2)},
+            "alignment_bwd": {
+                "ms": round(abwd_ms, 5),
+                "flops": "10 D per selected pair (sparse stream) + 10 D per causal pair (full stream)",
+                "tflops": round(2.5 * (flops + causal_flops(w)) / (abwd_ms * 1e-3) / 1e12, 2)}},
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
         "pct_of_peak_step": round(100.0 * value / world / peak, 2),

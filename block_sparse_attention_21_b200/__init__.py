@@ -12,6 +12,7 @@ from typing import Optional
 import torch
 
 from ._binding import (EXPORTED, LIB_PATH, SsaError, SsaProblem, lib, problem,
+                       ssa_alignment_bwd, ssa_alignment_bwd_workspace,
                        ssa_block_pool, ssa_block_select, ssa_debug_exp2_poly, ssa_debug_timeout_probe,
                        ssa_full_attn_fwd_with_mass, ssa_get_device_error,
                        ssa_get_device_error_site, ssa_launch_count,
@@ -20,6 +21,7 @@ from ._binding import (EXPORTED, LIB_PATH, SsaError, SsaProblem, lib, problem,
                        ssa_sparse_attn_fwd, ssa_status_string)
 
 __all__ = ["EXPORTED", "LIB_PATH", "SsaError", "SsaProblem", "SparseStream", "lib", "problem",
+           "ssa_alignment_bwd", "ssa_alignment_bwd_workspace",
            "ssa_block_pool", "ssa_block_select", "ssa_debug_exp2_poly", "ssa_debug_timeout_probe",
            "ssa_full_attn_fwd_with_mass", "ssa_get_device_error", "ssa_get_device_error_site",
            "ssa_launch_count",
@@ -49,6 +51,7 @@ class SparseStream:
         self.lse = torch.empty(B, Hq, S, dtype=f32, device=dev)
         self._full = None
         self._grad = None
+        self._agrad = None
 
     def select(self, q, k, stream=None):
         ssa_block_pool(self.p, k, q, self.k_pooled, self.q_pooled, stream)
@@ -92,4 +95,20 @@ class SparseStream:
         dq, dk, dv, workspace, ws = self._grad
         ssa_sparse_attn_bwd(self.p, q, k, v, self.o, self.lse, d_o, self.block_idx, dq, dk, dv,
                             workspace, workspace.numel(), stream)
+        return dq, dk, dv
+
+    def alignment_backward(self, q, k, v, d_o, mode: int = 0, alpha: float = 1.0, stream=None):
+        """Gradients with respect to q, k, v of <d_o, h_mode> + alpha * (L_sparsity +
+        L_commit) after alignment() ran on the same inputs (mode 0: d_o is the
+        gradient of the sparse output, 1: of the full output)."""
+        if self._full is None:
+            raise RuntimeError("alignment() must run before alignment_backward()")
+        if self._agrad is None:
+            ws = ssa_alignment_bwd_workspace(self.p)
+            self._agrad = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v),
+                           torch.empty(max(ws, 256), dtype=torch.uint8, device=q.device))
+        dq, dk, dv, workspace = self._agrad
+        o_full, lse_full, _ = self._full
+        ssa_alignment_bwd(self.p, q, k, v, self.o, self.lse, o_full, lse_full, d_o, mode, alpha,
+                          self.block_idx, dq, dk, dv, workspace, workspace.numel(), stream)
         return dq, dk, dv

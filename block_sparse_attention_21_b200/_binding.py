@@ -25,7 +25,8 @@ STATUS_NAMES = {0: "SSA_OK", 1: "SSA_ERR_INVALID_ARG", 2: "SSA_ERR_UNSUPPORTED",
 # every symbol include/ssa.h declares
 EXPORTED = ("ssa_block_pool", "ssa_block_select", "ssa_sparse_attn_fwd",
             "ssa_full_attn_fwd_with_mass", "ssa_sparse_attn_bwd_workspace",
-            "ssa_sparse_attn_bwd", "ssa_sparse_attn_bwd_noalloc", "ssa_get_device_error",
+            "ssa_sparse_attn_bwd", "ssa_sparse_attn_bwd_noalloc", "ssa_alignment_bwd_workspace",
+            "ssa_alignment_bwd", "ssa_get_device_error",
             "ssa_get_device_error_site",
             "ssa_debug_timeout_probe", "ssa_debug_exp2_poly",
             "ssa_status_string", "ssa_launch_count")
@@ -70,6 +71,8 @@ def lib():
             "ssa_full_attn_fwd_with_mass": [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
             "ssa_sparse_attn_bwd": [P] + [vp] * 11 + [ctypes.c_size_t, vp],
             "ssa_sparse_attn_bwd_noalloc": [P] + [vp] * 11,
+            "ssa_alignment_bwd": [P] + [vp] * 8 + [ctypes.c_int, ctypes.c_float] + [vp] * 5
+                                 + [ctypes.c_size_t, vp],
             "ssa_get_device_error": [vp],
             "ssa_debug_timeout_probe": [ctypes.c_int, vp],
             "ssa_debug_exp2_poly": [vp, vp, ctypes.c_int, vp],
@@ -78,8 +81,9 @@ def lib():
             f = getattr(L, name)
             f.argtypes = args
             f.restype = ctypes.c_int
-        L.ssa_sparse_attn_bwd_workspace.argtypes = [P]
-        L.ssa_sparse_attn_bwd_workspace.restype = ctypes.c_size_t
+        for name in ("ssa_sparse_attn_bwd_workspace", "ssa_alignment_bwd_workspace"):
+            getattr(L, name).argtypes = [P]
+            getattr(L, name).restype = ctypes.c_size_t
         L.ssa_status_string.argtypes = [ctypes.c_int]
         L.ssa_status_string.restype = ctypes.c_char_p
         L.ssa_get_device_error_site.argtypes = []
@@ -191,6 +195,30 @@ def ssa_sparse_attn_bwd(p: SsaProblem, q, k, v, o, lse, d_o, block_idx, dq, dk, 
           _ptr(block_idx, I32, "block_idx"), _ptr(dq, BF16, "dq"), _ptr(dk, BF16, "dk"),
           _ptr(dv, BF16, "dv"), _ptr(workspace, None, "workspace"), int(ws_bytes),
           _stream(stream))
+
+
+def ssa_alignment_bwd_workspace(p: SsaProblem) -> int:
+    return int(lib().ssa_alignment_bwd_workspace(ctypes.byref(p)))
+
+
+def ssa_alignment_bwd(p: SsaProblem, q, k, v, o_sparse, lse_sparse, o_full, lse_full, d_o,
+                      mode: int, alpha: float, block_idx, dq, dk, dv, workspace, ws_bytes: int,
+                      stream=None) -> None:
+    """Backward of <d_o, h_mode> + alpha (L_sparsity + L_commit) (mode 0: d_o is
+    the sparse output's gradient, 1: the full output's); see include/ssa.h."""
+    sh = _shapes(p)
+    for t, s, nm in ((q, "q", "q"), (k, "kv", "k"), (v, "kv", "v"), (o_sparse, "q", "o_sparse"),
+                     (lse_sparse, "lse", "lse_sparse"), (o_full, "q", "o_full"),
+                     (lse_full, "lse", "lse_full"), (d_o, "q", "d_o"),
+                     (block_idx, "idx", "block_idx"), (dq, "q", "dq"), (dk, "kv", "dk"),
+                     (dv, "kv", "dv")):
+        _numel_check(t, sh[s], nm)
+    _call("ssa_alignment_bwd", ctypes.byref(p), _ptr(q, BF16, "q"), _ptr(k, BF16, "k"),
+          _ptr(v, BF16, "v"), _ptr(o_sparse, BF16, "o_sparse"), _ptr(lse_sparse, F32, "lse_sparse"),
+          _ptr(o_full, BF16, "o_full"), _ptr(lse_full, F32, "lse_full"), _ptr(d_o, BF16, "d_o"),
+          int(mode), float(alpha), _ptr(block_idx, I32, "block_idx"), _ptr(dq, BF16, "dq"),
+          _ptr(dk, BF16, "dk"), _ptr(dv, BF16, "dv"), _ptr(workspace, None, "workspace"),
+          int(ws_bytes), _stream(stream))
 
 
 def ssa_sparse_attn_bwd_noalloc(p: SsaProblem, q, k, v, o, lse, d_o, block_idx, dq, dk, dv,

@@ -40,6 +40,8 @@ constexpr int kDkdvSplit = 4;
 
 struct BwdParams {
   int B, S, Hq, Hkv, G, n, topk, slices;
+  int dense;         // 1: every causal block counts as selected (dense causal
+                     // attention): no index table and no reverse index are read
   float scale;       // softmax scale
   float scale_log2;  // softmax scale * log2(e)
   const __nv_bfloat16* o;
@@ -266,8 +268,10 @@ __global__ void __launch_bounds__(256, DkdvConfig<D>::MIN_CTAS)
   const size_t bh = static_cast<size_t>(b) * p.Hkv + h;
   const int32_t* off = p.rev_off + bh * (p.n + 1);
   const int32_t* rev = p.rev + bh * p.n * p.topk;
-  const int first_q = off[j];
-  const int ntiles_all = (off[j + 1] - first_q) * HP;
+  // query blocks whose selection holds j: the reverse list, or all i >= j (dense)
+  const int first_q = p.dense ? 0 : off[j];
+  const int nq = p.dense ? (p.n - j) : (off[j + 1] - first_q);
+  const int ntiles_all = nq * HP;
   const int ntiles = ntiles_all > sp ? (ntiles_all - sp + kDkdvSplit - 1) / kDkdvSplit : 0;
 
   if (threadIdx.x == 0) {
@@ -308,7 +312,7 @@ __global__ void __launch_bounds__(256, DkdvConfig<D>::MIN_CTAS)
         const int qs = x % NQ;
         if (x >= NQ && !mbar_wait(&q_empty[qs], ((x / NQ) - 1) & 1, abort_flag, tmo, 0x801)) break;
         const int gx = sp + x * kDkdvSplit;
-        const int i = rev[first_q + gx / HP];
+        const int i = p.dense ? j + gx / HP : rev[first_q + gx / HP];
         const int hq0 = h * p.G + 2 * (gx % HP);
         mbar_arrive_expect_tx(&q_full[qs], 2 * QTILE);
         for (int hh = 0; hh < 2; ++hh)
@@ -410,7 +414,7 @@ __global__ void __launch_bounds__(256, DkdvConfig<D>::MIN_CTAS)
     bool ok = true;
     for (int x = 0; x < ntiles; ++x) {
       const int gx = sp + x * kDkdvSplit;
-      const int i = rev[first_q + gx / HP];
+      const int i = p.dense ? j + gx / HP : rev[first_q + gx / HP];
       const int hq = h * p.G + 2 * (gx % HP) + hh;
       const size_t lrow = (static_cast<size_t>(b) * p.Hq + hq) * p.S + 64 * i + tq;
       const float nlse = -p.lse[lrow] * kLog2e;
@@ -620,7 +624,7 @@ __global__ void __launch_bounds__(DqConfig<D, T_>::THREADS, 1)
       for (int jj = 0; jj < nblk; ++jj) {
         const int st = jj % NS, use = jj / NS;
         if (use > 0 && !mbar_wait(&kv_empty[st], (use - 1) & 1, abort_flag, tmo, 0xb01)) break;
-        const int j = idx_row[jj];
+        const int j = p.dense ? jj : idx_row[jj];
         mbar_arrive_expect_tx(&k_full[st], KVT);
         for (int pn = 0; pn < NP; ++pn)
           tma_load_4d(sK + st * KVT + pn * (64 * 128), &tm_k, &k_full[st], 64 * pn, h, 64 * j, b);

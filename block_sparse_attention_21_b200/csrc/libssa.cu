@@ -17,6 +17,7 @@
 #include "attn_fwd.cuh"
 #include "attn_fwd_psmem.cuh"
 #include "attn_bwd.cuh"
+#include "align_bwd.cuh"
 
 namespace {
 
@@ -249,11 +250,19 @@ size_t bwd_workspace_bytes(const Dims& d) {
   return ssa::bwd_workspace_layout(d.B, d.S, d.Hq, d.Hkv, d.n, d.topk, d.D).total;
 }
 
+// The dense causal backward needs no reverse index: its workspace layout is
+// the sparse one with a one-entry table.
+size_t dense_bwd_workspace_bytes(const Dims& d) {
+  return ssa::bwd_workspace_layout(d.B, d.S, d.Hq, d.Hkv, d.n, 1, d.D).total;
+}
+
 template <int D, int TQ>
 ssa_status launch_bwd(const Dims& d, const void* q, const void* k, const void* v, const void* o,
                       const float* lse, const void* d_o, const int32_t* idx, void* dq, void* dk,
-                      void* dv, void* workspace, cudaStream_t st) {
-  const ssa::BwdWorkspace ws = ssa::bwd_workspace_layout(d.B, d.S, d.Hq, d.Hkv, d.n, d.topk, d.D);
+                      void* dv, void* workspace, cudaStream_t st, bool dense = false) {
+  // dense: every causal block counts as selected; idx is not read
+  const ssa::BwdWorkspace ws =
+      ssa::bwd_workspace_layout(d.B, d.S, d.Hq, d.Hkv, d.n, dense ? 1 : d.topk, d.D);
   uint8_t* base = static_cast<uint8_t*>(workspace);
   ssa::BwdParams bp;
   bp.B = d.B;
@@ -262,14 +271,15 @@ ssa_status launch_bwd(const Dims& d, const void* q, const void* k, const void* v
   bp.Hkv = d.Hkv;
   bp.G = d.G;
   bp.n = d.n;
-  bp.topk = d.topk;
+  bp.topk = dense ? d.n : d.topk;
+  bp.dense = dense ? 1 : 0;
   bp.slices = (d.G / 2) / TQ;
   bp.scale = d.scale;
   bp.scale_log2 = d.scale * 1.4426950408889634f;
   bp.o = static_cast<const __nv_bfloat16*>(o);
   bp.d_o = static_cast<const __nv_bfloat16*>(d_o);
   bp.lse = lse;
-  bp.idx = idx;
+  bp.idx = dense ? reinterpret_cast<const int32_t*>(base) : idx;
   bp.dt = reinterpret_cast<float*>(base + ws.dt);
   bp.rev_off = reinterpret_cast<int32_t*>(base + ws.rev_off);
   bp.rev = reinterpret_cast<int32_t*>(base + ws.rev);
@@ -296,7 +306,7 @@ ssa_status launch_bwd(const Dims& d, const void* q, const void* k, const void* v
   ssa_status s = ensure_smem(ssa::bwd_prep_kernel<D>, static_cast<int>(ssa::bwd_prep_smem(kMaxSeqLen / 64)),
                              &prep_done);
   if (s != SSA_OK) return s;
-  const int rev_blocks = d.B * d.Hkv;
+  const int rev_blocks = dense ? 0 : d.B * d.Hkv;
   ssa::bwd_prep_kernel<D><<<rev_blocks + dt_blocks, 256, ssa::bwd_prep_smem(d.n), st>>>(bp, rev_blocks);
   s = launch_result();
   if (s != SSA_OK) return s;
@@ -370,6 +380,66 @@ __global__ void exp2_poly_kernel(const float* x, float* y, int n) {
   ssa::exp2_poly2(x0, x1, p0, p1);
   y[i] = p0;
   if (i + 1 < n) y[i + 1] = p1;
+}
+
+// Workspace of ssa_alignment_bwd: both streams' output gradients, the dense
+// pass's input gradients, then the backward workspace both passes share.
+struct AlignLayout {
+  size_t do_s, do_f, dq2, dk2, dv2, bwd, total;
+};
+
+AlignLayout align_layout(const Dims& d) {
+  auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  const size_t eq = static_cast<size_t>(d.B) * d.S * d.Hq * d.D * 2;
+  const size_t ekv = static_cast<size_t>(d.B) * d.S * d.Hkv * d.D * 2;
+  AlignLayout L;
+  L.do_s = 0;
+  L.do_f = L.do_s + al(eq);
+  L.dq2 = L.do_f + al(eq);
+  L.dk2 = L.dq2 + al(eq);
+  L.dv2 = L.dk2 + al(ekv);
+  L.bwd = L.dv2 + al(ekv);
+  const size_t wb = bwd_workspace_bytes(d), wd = dense_bwd_workspace_bytes(d);
+  L.total = L.bwd + (wb > wd ? wb : wd);
+  return L;
+}
+
+template <int D, int TQ>
+ssa_status launch_align_bwd(const Dims& d, const void* q, const void* k, const void* v,
+                            const void* o_s, const float* lse_s, const void* o_f, const float* lse_f,
+                            const void* d_o, int mode, float alpha, const int32_t* idx, void* dq,
+                            void* dk, void* dv, void* workspace, cudaStream_t st) {
+  const AlignLayout L = align_layout(d);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  auto* do_s = reinterpret_cast<__nv_bfloat16*>(ws + L.do_s);
+  auto* do_f = reinterpret_cast<__nv_bfloat16*>(ws + L.do_f);
+  const long long nq8 = static_cast<long long>(d.B) * d.S * d.Hq * d.D / 8;
+  const long long nkv8 = static_cast<long long>(d.B) * d.S * d.Hkv * d.D / 8;
+  const float c = static_cast<float>(2.0 * alpha / (8.0 * static_cast<double>(nq8)));
+  auto grid_of = [](long long n8) {
+    const long long g = (n8 + 255) / 256;
+    return static_cast<unsigned>(g < 148 * 16 ? g : 148 * 16);
+  };
+  ssa::align_grad_kernel<<<grid_of(nq8), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(o_s), static_cast<const __nv_bfloat16*>(o_f),
+      static_cast<const __nv_bfloat16*>(d_o), mode, c, do_s, do_f, nq8);
+  ssa_status s = launch_result();
+  if (s != SSA_OK) return s;
+  // the sparse stream over the selected blocks, the full stream over every causal block
+  s = launch_bwd<D, TQ>(d, q, k, v, o_s, lse_s, do_s, idx, dq, dk, dv, ws + L.bwd, st);
+  if (s != SSA_OK) return s;
+  s = launch_bwd<D, TQ>(d, q, k, v, o_f, lse_f, do_f, nullptr, ws + L.dq2, ws + L.dk2, ws + L.dv2,
+                        ws + L.bwd, st, true);
+  if (s != SSA_OK) return s;
+  ssa::add_bf16_kernel<<<grid_of(nq8), 256, 0, st>>>(static_cast<__nv_bfloat16*>(dq),
+                                                     reinterpret_cast<const __nv_bfloat16*>(ws + L.dq2), nq8);
+  if ((s = launch_result()) != SSA_OK) return s;
+  ssa::add_bf16_kernel<<<grid_of(nkv8), 256, 0, st>>>(static_cast<__nv_bfloat16*>(dk),
+                                                      reinterpret_cast<const __nv_bfloat16*>(ws + L.dk2), nkv8);
+  if ((s = launch_result()) != SSA_OK) return s;
+  ssa::add_bf16_kernel<<<grid_of(nkv8), 256, 0, st>>>(static_cast<__nv_bfloat16*>(dv),
+                                                      reinterpret_cast<const __nv_bfloat16*>(ws + L.dv2), nkv8);
+  return launch_result();
 }
 
 }  // namespace
@@ -513,6 +583,39 @@ ssa_status ssa_sparse_attn_bwd_noalloc(const ssa_problem* p, const ssa_bf16* q, 
                     : launch_bwd<64, 1>(d, q, k, v, o, lse, d_o, block_idx, dq, dk, dv, scratch, st);
   return d.G >= 4 ? launch_bwd<128, 2>(d, q, k, v, o, lse, d_o, block_idx, dq, dk, dv, scratch, st)
                   : launch_bwd<128, 1>(d, q, k, v, o, lse, d_o, block_idx, dq, dk, dv, scratch, st);
+}
+
+size_t ssa_alignment_bwd_workspace(const ssa_problem* p) {
+  Dims d;
+  if (check_problem(p, &d) != SSA_OK) return 0;
+  return align_layout(d).total;
+}
+
+ssa_status ssa_alignment_bwd(const ssa_problem* p, const ssa_bf16* q, const ssa_bf16* k,
+                             const ssa_bf16* v, const ssa_bf16* o_sparse, const float* lse_sparse,
+                             const ssa_bf16* o_full, const float* lse_full, const ssa_bf16* d_o,
+                             int mode, float alpha, const int32_t* block_idx, ssa_bf16* dq,
+                             ssa_bf16* dk, ssa_bf16* dv, void* workspace, size_t ws_bytes,
+                             ssa_stream stream) {
+  Dims d;
+  ssa_status s = check_problem(p, &d);
+  if (s != SSA_OK) return s;
+  const void* ptrs[] = {q, k, v, o_sparse, lse_sparse, o_full, lse_full, d_o, block_idx, dq, dk, dv};
+  for (const void* ptr : ptrs)
+    if (ptr == nullptr || !aligned16(ptr)) return SSA_ERR_INVALID_ARG;
+  if ((mode != 0 && mode != 1) || !std::isfinite(alpha)) return SSA_ERR_INVALID_ARG;
+  if (workspace == nullptr || !aligned16(workspace) || ws_bytes < align_layout(d).total)
+    return SSA_ERR_WORKSPACE;
+  auto st = reinterpret_cast<cudaStream_t>(stream);
+  if (d.D == 64)
+    return d.G >= 4 ? launch_align_bwd<64, 2>(d, q, k, v, o_sparse, lse_sparse, o_full, lse_full, d_o, mode,
+                                              alpha, block_idx, dq, dk, dv, workspace, st)
+                    : launch_align_bwd<64, 1>(d, q, k, v, o_sparse, lse_sparse, o_full, lse_full, d_o, mode,
+                                              alpha, block_idx, dq, dk, dv, workspace, st);
+  return d.G >= 4 ? launch_align_bwd<128, 2>(d, q, k, v, o_sparse, lse_sparse, o_full, lse_full, d_o, mode,
+                                             alpha, block_idx, dq, dk, dv, workspace, st)
+                  : launch_align_bwd<128, 1>(d, q, k, v, o_sparse, lse_sparse, o_full, lse_full, d_o, mode,
+                                             alpha, block_idx, dq, dk, dv, workspace, st);
 }
 
 ssa_status ssa_get_device_error(ssa_stream stream) {

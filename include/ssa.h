@@ -154,6 +154,40 @@ ssa_status ssa_sparse_attn_bwd(const ssa_problem *p, const ssa_bf16 *q, const ss
                                ssa_bf16 *dk, ssa_bf16 *dv, void *workspace, size_t ws_bytes,
                                ssa_stream stream);
 
+/* Bytes of device workspace ssa_alignment_bwd needs for problem p (0 on an
+ * invalid problem). */
+size_t ssa_alignment_bwd_workspace(const ssa_problem *p);
+
+/* Backward of one layer of SSA's training objective with the bidirectional
+ * alignment loss ([SSA-es] section 2, "Alineacion Bidireccional"): the
+ * gradient of
+ *     <d_o, h_mode> + alpha * (L_sparsity + L_commit)
+ * with respect to q, k and v, where h_sparse and h_full are the sparse and
+ * the full (dense causal) attention outputs, d_o is the upstream gradient of
+ * the stream this step trains (mode 0: the sparse output; mode 1: the full
+ * output; the other output is the counterpart, computed for the alignment
+ * only), and, reading the pages' unspecified distance as the mean squared
+ * error over the N = B*S*Hq*D output elements with a stop-gradient (sg) on
+ * the target,
+ *     L_sparsity = mean (h_full - sg(h_sparse))^2   (full pulled to sparse)
+ *     L_commit   = mean (h_sparse - sg(h_full))^2   (sparse pulled to full).
+ * The output gradients are then d_o + c (h_sparse - h_full) for the sparse
+ * stream (d_o only in mode 0) and c (h_full - h_sparse) for the full one
+ * (plus d_o in mode 1), c = 2 alpha / N; each goes back through its stream's
+ * attention (the full stream over every causal block) and dq, dk, dv are the
+ * sums.  o_sparse/lse_sparse and o_full/lse_full are the outputs of
+ * ssa_full_attn_fwd_with_mass for the same inputs and block_idx.  `workspace`
+ * is a caller-owned device buffer of at least ssa_alignment_bwd_workspace(p)
+ * bytes, 256-byte aligned; its contents on entry do not matter.
+ * Errors: INVALID_ARG for a null or misaligned pointer, mode outside {0, 1}
+ * or a non-finite alpha; WORKSPACE for a missing or short workspace. */
+ssa_status ssa_alignment_bwd(const ssa_problem *p, const ssa_bf16 *q, const ssa_bf16 *k,
+                             const ssa_bf16 *v, const ssa_bf16 *o_sparse, const float *lse_sparse,
+                             const ssa_bf16 *o_full, const float *lse_full, const ssa_bf16 *d_o,
+                             int mode, float alpha, const int32_t *block_idx, ssa_bf16 *dq,
+                             ssa_bf16 *dk, ssa_bf16 *dv, void *workspace, size_t ws_bytes,
+                             ssa_stream stream);
+
 /* Largest scratch (in bytes) that ssa_sparse_attn_bwd_noalloc can use. */
 #define SSA_NOALLOC_SCRATCH_BYTES (16u << 20)
 

@@ -1,9 +1,10 @@
 """fp64 CPU oracle for the SSA sparse stream -- TEST INFRASTRUCTURE.
 
 Only the tests, the smoke check and the bench's CPU-baseline leg may import
-this package.  It shares no code with the CUDA library: the arithmetic lives
-in ssa_oracle.c (plain C, fp64, pthreads); this module only widens bf16
-tensors exactly to fp64 and marshals numpy arrays through ctypes.
+this package.  It shares no code with the CUDA library: the attention
+arithmetic lives in ssa_oracle.c (plain C, fp64, pthreads); this module widens
+bf16 tensors exactly to fp64, marshals numpy arrays through ctypes, and holds
+the alignment objective's elementwise output gradients (fp64 numpy).
 
 Functions (each cites the passage it follows in ssa_oracle.c):
   block_pool      mean of each 64-token key block; GQA-group mean of the queries
@@ -12,6 +13,11 @@ Functions (each cites the passage it follows in ssa_oracle.c):
                   dropped mass (two routes) for a list of query rows
   sparse_bwd_dq_rows / sparse_bwd_dkv_blocks
                   gradient of the sparse output, by the explicit formulas
+  dense_causal_table
+                  the index table of every causal block (dense attention)
+  alignment_output_grads
+                  output gradients of the alignment objective (a formula,
+                  written here; pinned by finite differences with stop-gradient)
 """
 from __future__ import annotations
 
@@ -191,6 +197,38 @@ def sparse_bwd_dkv_blocks(q, k, v, do, idx: np.ndarray, blocks: np.ndarray,
         _ptr(dk, ctypes.c_double), _ptr(dv, ctypes.c_double), nthreads or default_threads())
     _check(rc, "sparse_bwd_dkv_blocks")
     return dk, dv
+
+
+def dense_causal_table(B: int, Hkv: int, n: int) -> np.ndarray:
+    """Index table [B, Hkv, n, n] that selects every causal block: row i holds
+    0..i, then -1.  With it the sparse functions compute dense causal attention."""
+    idx = np.full((B, Hkv, n, n), -1, dtype=np.int32)
+    for i in range(n):
+        idx[:, :, i, :i + 1] = np.arange(i + 1, dtype=np.int32)
+    return idx
+
+
+def alignment_output_grads(o_sparse, o_full, d_o, mode: int, alpha: float):
+    """Output gradients of  <d_o, h_mode> + alpha (L_sparsity + L_commit)
+    ("Resumen Tecnico: SSA", section 2, "Alineacion Bidireccional").
+
+    The pages do not fix the distance; read as the mean squared error over the
+    N elements of h with a stop-gradient (sg) on the target:
+        L_sparsity = mean (h_full - sg(h_sparse))^2   (full pulled to sparse)
+        L_commit   = mean (h_sparse - sg(h_full))^2   (sparse pulled to full)
+    mode 0: d_o is the sparse output's upstream gradient; 1: the full one's.
+    Returns (dO_sparse, dO_full) in fp64, shaped like the inputs."""
+    o_s, o_f, g = widen(o_sparse), widen(o_full), widen(d_o)
+    c = 2.0 * float(alpha) / o_s.size
+    d_s = c * (o_s - o_f)          # from L_commit, through h_sparse
+    d_f = c * (o_f - o_s)          # from L_sparsity, through h_full
+    if mode == 0:
+        d_s = d_s + g
+    elif mode == 1:
+        d_f = d_f + g
+    else:
+        raise ValueError("mode must be 0 or 1")
+    return d_s, d_f
 
 
 def sparse_forward_problem(q, k, v, topk: int, rows: Optional[np.ndarray] = None,

@@ -75,6 +75,8 @@ def test_bad_problem_is_rejected_by_every_entry_point(lib, kw, code):
     assert lib.ssa_full_attn_fwd_with_mass(p, f, f, f, f, f, f, f, f, f, None) == code
     assert lib.ssa_sparse_attn_bwd(p, f, f, f, f, f, f, f, f, f, f, f, 1 << 30, None) == code
     assert lib.ssa_sparse_attn_bwd_workspace(p) == 0
+    assert lib.ssa_alignment_bwd(p, f, f, f, f, f, f, f, f, 0, 1.0, f, f, f, f, f, 1 << 30, None) == code
+    assert lib.ssa_alignment_bwd_workspace(p) == 0
 
 
 def test_null_problem(lib):
@@ -104,3 +106,15 @@ def test_backward_workspace_is_checked_before_launch(lib):
 
 def test_timeout_probe_rejects_bad_limit(lib):
     assert lib.ssa_debug_timeout_probe(0, None) == INVALID
+
+
+def test_alignment_backward_arguments_are_checked_before_launch(lib):
+    p = ctypes.byref(_p())
+    f = FAKE
+    ws = lib.ssa_alignment_bwd_workspace(p)
+    assert ws > lib.ssa_sparse_attn_bwd_workspace(p) > 0
+    assert lib.ssa_alignment_bwd(p, f, f, f, f, f, f, f, f, 2, 1.0, f, f, f, f, f, ws, None) == INVALID
+    assert lib.ssa_alignment_bwd(p, f, f, f, f, f, f, f, f, 0, float("inf"), f, f, f, f, f, ws, None) == INVALID
+    assert lib.ssa_alignment_bwd(p, f, f, f, f, f, f, f, f, 0, 1.0, f, f, f, f, f, ws - 1, None) == WORKSPACE
+    assert lib.ssa_alignment_bwd(p, f, f, f, f, f, f, f, f, 0, 1.0, f, f, f, f, None, ws, None) == WORKSPACE
+    assert lib.ssa_alignment_bwd(p, f, f, f, f, None, f, f, f, 0, 1.0, f, f, f, f, f, ws, None) == INVALID

@@ -343,3 +343,62 @@ def test_unselected_block_gets_exactly_zero_gradient():
         do_j[0, j * BS:(j + 1) * BS] = 0.0
         dk, dv = oracle.sparse_bwd_dkv_blocks(q, k, v, do_j, idx, np.array([[0, 0, j]]))
         assert np.all(dk == 0.0) and np.all(dv == 0.0)
+
+
+# ---------------------------------------------------- alignment objective
+
+def _outputs(q, k, v, idx):
+    """Sparse and full outputs [B, S, Hq, D] of every row (fp64)."""
+    B, S, Hq, D = q.shape
+    rows = oracle.all_rows(B, Hq, S)
+    r = oracle.attn_rows(q, k, v, idx, rows, want_full=True)
+    to = lambda a: a.reshape(B, Hq, S, D).transpose(0, 2, 1, 3)  # noqa: E731
+    return to(r["o_sparse"]), to(r["o_full"])
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_alignment_gradient_matches_finite_differences_with_stop_gradient(mode):
+    # J = <G, h_mode> + alpha (mean (h_full - C_s)^2 + mean (h_sparse - C_f)^2),
+    # C_s, C_f frozen at the unperturbed outputs (the stop-gradients); the
+    # analytic gradient is the oracle's output gradients pushed back through
+    # the sparse stream (selected blocks) and the full stream (every causal block)
+    q, k, v = _tiny(B=1, S=256, Hq=4, Hkv=2, D=8, seed=81)
+    G_ = _rand(q.shape, 82)
+    kbar, qbar = oracle.block_pool(k, q)
+    idx, _ = oracle.block_select(qbar, kbar, 2)   # frozen selection
+    B, S, Hq, D = q.shape
+    dense = oracle.dense_causal_table(B, k.shape[2], S // BS)
+    o_s0, o_f0 = _outputs(q, k, v, idx)
+    alpha = 0.3 * q.size   # alignment terms of the same order as <G, h>
+    d_s, d_f = oracle.alignment_output_grads(o_s0, o_f0, G_, mode, alpha)
+    gs = _full_bwd(q, k, v, d_s, idx)
+    gf = _full_bwd(q, k, v, d_f, dense)
+    grads = [a + b for a, b in zip(gs, gf)]
+
+    def J(q_, k_, v_):
+        o_s, o_f = _outputs(q_, k_, v_, idx)
+        lin = np.sum(G_ * (o_s if mode == 0 else o_f))
+        return lin + alpha * (np.mean((o_f - o_s0) ** 2) + np.mean((o_s - o_f0) ** 2))
+
+    rng = np.random.Generator(np.random.PCG64(83 + mode))
+    h = 1e-6
+    for name, arr, g in zip("qkv", (q, k, v), grads):
+        for _ in range(8):
+            pos = tuple(int(rng.integers(0, s)) for s in arr.shape)
+            plus, minus = arr.copy(), arr.copy()
+            plus[pos] += h
+            minus[pos] -= h
+            args_p = {"q": q, "k": k, "v": v}
+            args_m = dict(args_p)
+            args_p[name], args_m[name] = plus, minus
+            fd = (J(args_p["q"], args_p["k"], args_p["v"]) - J(args_m["q"], args_m["k"], args_m["v"])) / (2 * h)
+            assert abs(fd - g[pos]) <= 2e-6 * max(1.0, abs(g[pos])), (name, pos, fd, g[pos])
+
+
+def test_dense_table_gives_dense_causal_attention():
+    q, k, v = _tiny(B=1, S=256, Hq=2, Hkv=1, D=8, seed=91)
+    dense = oracle.dense_causal_table(1, 1, 4)
+    o_s, o_f = _outputs(q, k, v, dense)
+    np.testing.assert_allclose(o_s, o_f, atol=1e-13)
+    ref = _sdpa_rows(q, k, v, lambda b, h: np.tril(np.ones((256, 256), dtype=bool)))
+    np.testing.assert_allclose(o_s.transpose(0, 2, 1, 3), ref, atol=1e-12)
