@@ -26,7 +26,8 @@ STATUS_NAMES = {0: "SSA_OK", 1: "SSA_ERR_INVALID_ARG", 2: "SSA_ERR_UNSUPPORTED",
 EXPORTED = ("ssa_block_pool", "ssa_block_select", "ssa_sparse_attn_fwd",
             "ssa_full_attn_fwd_with_mass", "ssa_sparse_attn_bwd_workspace",
             "ssa_sparse_attn_bwd", "ssa_sparse_attn_bwd_noalloc", "ssa_alignment_bwd_workspace",
-            "ssa_alignment_bwd", "ssa_get_device_error",
+            "ssa_alignment_bwd", "ssa_decode_attn_workspace", "ssa_decode_attn",
+            "ssa_get_device_error",
             "ssa_get_device_error_site",
             "ssa_debug_timeout_probe", "ssa_debug_exp2_poly",
             "ssa_status_string", "ssa_launch_count")
@@ -71,6 +72,7 @@ def lib():
             "ssa_full_attn_fwd_with_mass": [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
             "ssa_sparse_attn_bwd": [P] + [vp] * 11 + [ctypes.c_size_t, vp],
             "ssa_sparse_attn_bwd_noalloc": [P] + [vp] * 11,
+            "ssa_decode_attn": [P] + [vp] * 9 + [ctypes.c_size_t, vp],
             "ssa_alignment_bwd": [P] + [vp] * 8 + [ctypes.c_int, ctypes.c_float] + [vp] * 5
                                  + [ctypes.c_size_t, vp],
             "ssa_get_device_error": [vp],
@@ -81,7 +83,8 @@ def lib():
             f = getattr(L, name)
             f.argtypes = args
             f.restype = ctypes.c_int
-        for name in ("ssa_sparse_attn_bwd_workspace", "ssa_alignment_bwd_workspace"):
+        for name in ("ssa_sparse_attn_bwd_workspace", "ssa_alignment_bwd_workspace",
+                     "ssa_decode_attn_workspace"):
             getattr(L, name).argtypes = [P]
             getattr(L, name).restype = ctypes.c_size_t
         L.ssa_status_string.argtypes = [ctypes.c_int]
@@ -219,6 +222,28 @@ def ssa_alignment_bwd(p: SsaProblem, q, k, v, o_sparse, lse_sparse, o_full, lse_
           int(mode), float(alpha), _ptr(block_idx, I32, "block_idx"), _ptr(dq, BF16, "dq"),
           _ptr(dk, BF16, "dk"), _ptr(dv, BF16, "dv"), _ptr(workspace, None, "workspace"),
           int(ws_bytes), _stream(stream))
+
+
+def ssa_decode_attn_workspace(p: SsaProblem) -> int:
+    return int(lib().ssa_decode_attn_workspace(ctypes.byref(p)))
+
+
+def ssa_decode_attn(p: SsaProblem, q, k_cache, v_cache, k_pooled, lengths, o, lse, block_idx,
+                    workspace, ws_bytes: int, stream=None) -> None:
+    """One decoding step against a KV cache (p.seq_len = cache capacity); see
+    include/ssa.h.  block_idx may be None."""
+    sh = _shapes(p)
+    B, Hq, Hkv, D = p.batch, p.n_q_heads, p.n_kv_heads, p.head_dim
+    for t, s, nm in ((q, (B, Hq, D), "q"), (k_cache, sh["kv"], "k_cache"), (v_cache, sh["kv"], "v_cache"),
+                     (k_pooled, sh["pooled"], "k_pooled"), (lengths, (B,), "lengths"),
+                     (o, (B, Hq, D), "o"), (lse, (B, Hq), "lse")):
+        _numel_check(t, s, nm)
+    if block_idx is not None:
+        _numel_check(block_idx, (B, Hkv, p.top_k), "block_idx")
+    _call("ssa_decode_attn", ctypes.byref(p), _ptr(q, BF16, "q"), _ptr(k_cache, BF16, "k_cache"),
+          _ptr(v_cache, BF16, "v_cache"), _ptr(k_pooled, F32, "k_pooled"), _ptr(lengths, I32, "lengths"),
+          _ptr(o, BF16, "o"), _ptr(lse, F32, "lse"), _ptr(block_idx, I32, "block_idx"),
+          _ptr(workspace, None, "workspace"), int(ws_bytes), _stream(stream))
 
 
 def ssa_sparse_attn_bwd_noalloc(p: SsaProblem, q, k, v, o, lse, d_o, block_idx, dq, dk, dv,

@@ -18,6 +18,7 @@
 #include "attn_fwd_psmem.cuh"
 #include "attn_bwd.cuh"
 #include "align_bwd.cuh"
+#include "decode.cuh"
 
 namespace {
 
@@ -442,6 +443,59 @@ ssa_status launch_align_bwd(const Dims& d, const void* q, const void* k, const v
   return launch_result();
 }
 
+// Workspace of ssa_decode_attn: the selected blocks (unless the caller takes
+// them), then the partial softmax states.
+struct DecodeLayout {
+  size_t idx, part, total;
+};
+
+DecodeLayout decode_layout(const Dims& d) {
+  auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  const size_t rows = static_cast<size_t>(d.B) * d.Hkv * d.topk;
+  DecodeLayout L;
+  L.idx = 0;
+  L.part = al(rows * sizeof(int32_t));
+  L.total = L.part + al(rows * d.G * (d.D + 2) * sizeof(float));
+  return L;
+}
+
+template <int D>
+ssa_status launch_decode(const Dims& d, const void* q, const void* k, const void* v, const float* kbar,
+                         const int32_t* len, void* o, float* lse, int32_t* idx_out, void* workspace,
+                         cudaStream_t st) {
+  const DecodeLayout L = decode_layout(d);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  ssa::DecodeParams dp;
+  dp.B = d.B;
+  dp.S = d.S;
+  dp.Hq = d.Hq;
+  dp.Hkv = d.Hkv;
+  dp.G = d.G;
+  dp.n = d.n;
+  dp.topk = d.topk;
+  dp.scale_log2 = d.scale * 1.4426950408889634f;
+  dp.q = static_cast<const __nv_bfloat16*>(q);
+  dp.k = static_cast<const __nv_bfloat16*>(k);
+  dp.v = static_cast<const __nv_bfloat16*>(v);
+  dp.kbar = kbar;
+  dp.len = len;
+  dp.idx = idx_out != nullptr ? idx_out : reinterpret_cast<int32_t*>(ws + L.idx);
+  dp.part = reinterpret_cast<float*>(ws + L.part);
+  dp.o = static_cast<__nv_bfloat16*>(o);
+  dp.lse = lse;
+  const unsigned bh = static_cast<unsigned>(d.B) * d.Hkv;
+  ssa::decode_select_kernel<D><<<bh, ssa::kDecodeSelThreads, 4 * d.n, st>>>(dp);
+  ssa_status s = launch_result();
+  if (s != SSA_OK) return s;
+  static std::atomic<uint64_t> smem_done{0};
+  s = ensure_smem(ssa::decode_attn_kernel<D>, ssa::decode_attn_smem<D>(), &smem_done);
+  if (s != SSA_OK) return s;
+  ssa::decode_attn_kernel<D><<<bh * d.topk, 128, ssa::decode_attn_smem<D>(), st>>>(dp);
+  if ((s = launch_result()) != SSA_OK) return s;
+  ssa::decode_combine_kernel<D><<<static_cast<unsigned>(d.B) * d.Hq, D, 0, st>>>(dp);
+  return launch_result();
+}
+
 }  // namespace
 
 extern "C" {
@@ -618,6 +672,30 @@ ssa_status ssa_alignment_bwd(const ssa_problem* p, const ssa_bf16* q, const ssa_
                                              alpha, block_idx, dq, dk, dv, workspace, st);
 }
 
+size_t ssa_decode_attn_workspace(const ssa_problem* p) {
+  Dims d;
+  if (check_problem(p, &d) != SSA_OK) return 0;
+  return decode_layout(d).total;
+}
+
+ssa_status ssa_decode_attn(const ssa_problem* p, const ssa_bf16* q, const ssa_bf16* k_cache,
+                           const ssa_bf16* v_cache, const float* k_pooled, const int32_t* lengths,
+                           ssa_bf16* o, float* lse, int32_t* block_idx, void* workspace, size_t ws_bytes,
+                           ssa_stream stream) {
+  Dims d;
+  ssa_status s = check_problem(p, &d);
+  if (s != SSA_OK) return s;
+  const void* ptrs[] = {q, k_cache, v_cache, k_pooled, lengths, o, lse};
+  for (const void* ptr : ptrs)
+    if (ptr == nullptr || !aligned16(ptr)) return SSA_ERR_INVALID_ARG;
+  if (block_idx != nullptr && !aligned16(block_idx)) return SSA_ERR_INVALID_ARG;
+  if (workspace == nullptr || !aligned16(workspace) || ws_bytes < decode_layout(d).total)
+    return SSA_ERR_WORKSPACE;
+  auto st = reinterpret_cast<cudaStream_t>(stream);
+  return d.D == 64 ? launch_decode<64>(d, q, k_cache, v_cache, k_pooled, lengths, o, lse, block_idx, workspace, st)
+                   : launch_decode<128>(d, q, k_cache, v_cache, k_pooled, lengths, o, lse, block_idx, workspace, st);
+}
+
 ssa_status ssa_get_device_error(ssa_stream stream) {
   const cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
   unsigned int word = 0, zero = 0;
@@ -626,6 +704,7 @@ ssa_status ssa_get_device_error(ssa_stream stream) {
   if (word != 0 && cudaMemcpyToSymbol(ssa::g_error_word, &zero, sizeof(zero)) != cudaSuccess)
     return SSA_ERR_CUDA;
   if (word & ssa::kErrTimeout) return SSA_ERR_DEVICE_TIMEOUT;
+  if (word & ssa::kErrBadInput) return SSA_ERR_INVALID_ARG;
   return e == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;
 }
 

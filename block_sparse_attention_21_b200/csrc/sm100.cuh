@@ -14,6 +14,7 @@ namespace ssa {
 __device__ unsigned int g_error_word;
 __device__ unsigned int g_error_site;
 constexpr unsigned int kErrTimeout = 1u;
+constexpr unsigned int kErrBadInput = 2u;  // a device-side input outside its documented range
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

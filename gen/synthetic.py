@@ -180,3 +180,45 @@ def _draw(w: Workload, redraws: Sequence[Sequence[int]]) -> SynthInputs:
 
     return SynthInputs(w, _to_bf16(q), _to_bf16(k), _to_bf16(v),
                        _to_bf16(do) if do is not None else None, plants)
+
+
+@dataclasses.dataclass
+class DecodeInputs:
+    q: torch.Tensor            # [B, Hq, D] bf16: each sequence's newest token
+    k: torch.Tensor            # [B, S, Hkv, D] bf16 cache (S = capacity)
+    v: torch.Tensor            # [B, S, Hkv, D] bf16 cache
+    lengths: np.ndarray        # [B] int32 cached tokens, the newest included
+    top_k: int
+
+
+def make_decode(batch: int, capacity: int, n_q_heads: int, n_kv_heads: int, head_dim: int,
+                top_k: int, seed: int, n_plant: int = 8, plant_shift: float = 1.5,
+                lengths: Optional[Sequence[int]] = None) -> DecodeInputs:
+    """A KV cache and one new query per sequence, drawn with the recipe of the
+    module docstring: N(0, 1) values, every key block shifted by plant_shift
+    along its own unit direction u_j, and each sequence's query (all heads of a
+    KV head's group) shifted by the sum of u_j over n_plant distinct complete
+    blocks before its own.  Lengths default to uniform draws in
+    [capacity / 2, capacity]."""
+    B, S, Hq, Hkv, D = batch, capacity, n_q_heads, n_kv_heads, head_dim
+    if S % BLOCK != 0 or Hq % Hkv != 0:
+        raise ValueError("capacity must be a multiple of 64 and n_q_heads of n_kv_heads")
+    G, n = Hq // Hkv, S // BLOCK
+    rng = np.random.Generator(np.random.PCG64(seed))
+    k = rng.standard_normal((B, S, Hkv, D))
+    v = rng.standard_normal((B, S, Hkv, D))
+    u = rng.standard_normal((B, Hkv, n, D))
+    u /= np.linalg.norm(u, axis=-1, keepdims=True)
+    k.reshape(B, n, BLOCK, Hkv, D)[...] += plant_shift * u.transpose(0, 2, 1, 3)[:, :, None, :, :]
+    if lengths is None:
+        lengths = rng.integers(S // 2, S + 1, size=B)
+    lengths = np.asarray(lengths, dtype=np.int32)
+    q = rng.standard_normal((B, Hq, D))
+    for b in range(B):
+        c = (int(lengths[b]) - 1) // BLOCK
+        for h in range(Hkv):
+            m = min(n_plant, c)
+            if m > 0:
+                pick = rng.choice(c, size=m, replace=False)
+                q[b, h * G:(h + 1) * G] += u[b, h, pick].sum(axis=0)
+    return DecodeInputs(q=_to_bf16(q), k=_to_bf16(k), v=_to_bf16(v), lengths=lengths, top_k=top_k)

@@ -219,10 +219,43 @@ ssa_status ssa_sparse_attn_bwd_noalloc(const ssa_problem *p, const ssa_bf16 *q, 
                                        ssa_bf16 *dq, ssa_bf16 *dk, ssa_bf16 *dv,
                                        ssa_stream stream);
 
+/* Bytes of device workspace ssa_decode_attn needs for problem p (0 on an
+ * invalid problem). */
+size_t ssa_decode_attn_workspace(const ssa_problem *p);
+
+/* One decoding step of the sparse stream against a KV cache ([SSA-it]
+ * "Block-sparse attention e Receptive Field" applied to a single query;
+ * [SSA-es] section 4: sparse-mode inference reads only the selected blocks).
+ * p->seq_len is the cache capacity S (a multiple of 64), the other fields as
+ * for the forward.  For sequence b with lengths[b] = L cached tokens
+ * (1 <= L <= S), the query is token t = L - 1, already in the cache, with its
+ * Hq heads in q [B][Hq][D] bf16.  Its block c = t / 64 may be partial.
+ *  - Selection, per KV head h: the mean over the G heads of q is scored
+ *    against k_pooled[b][h][j] for the complete blocks j < c (fp32, the mean
+ *    keys ssa_block_pool writes, [B][Hkv][S/64][D]; rows j >= c are not
+ *    read).  The top-(k-1) scores are kept (ties: lower j) together with block
+ *    c.  If c + 1 <= k, every block 0..c is kept.
+ *  - Attention: softmax(scale q.k) over the kept blocks' tokens, causal in
+ *    block c (keys up to t), for each query head of the group.
+ * k_cache, v_cache: [B][S][Hkv][D] bf16.  Outputs: o [B][Hq][D] bf16,
+ * lse [B][Hq] fp32 (natural log), and, if block_idx is not NULL, the kept
+ * blocks [B][Hkv][k] int32, ascending, -1 padded.  `workspace`: at least
+ * ssa_decode_attn_workspace(p) bytes, 256-byte aligned.
+ * Errors: INVALID_ARG / UNSUPPORTED / WORKSPACE as for the other calls.  A
+ * length outside 1..S is found on the device; that sequence's outputs become
+ * 0 (lse -inf), and ssa_get_device_error then returns SSA_ERR_INVALID_ARG.
+ * The pages have no decode kernel of their own; this call is the sparse
+ * stream's selection and attention applied to one new token. */
+ssa_status ssa_decode_attn(const ssa_problem *p, const ssa_bf16 *q, const ssa_bf16 *k_cache,
+                           const ssa_bf16 *v_cache, const float *k_pooled, const int32_t *lengths,
+                           ssa_bf16 *o, float *lse, int32_t *block_idx, void *workspace,
+                           size_t ws_bytes, ssa_stream stream);
+
 /* Synchronises `stream`, then reports and clears the device error word of the
  * current device: SSA_ERR_DEVICE_TIMEOUT if a kernel's bounded wait ran out
- * since the last call, SSA_ERR_CUDA if the stream reported an error, else
- * SSA_OK. */
+ * since the last call, SSA_ERR_INVALID_ARG if a kernel found a device-side
+ * input outside its range (a decode length), SSA_ERR_CUDA if the stream
+ * reported an error, else SSA_OK. */
 ssa_status ssa_get_device_error(ssa_stream stream);
 
 /* Site code of the most recent bounded wait that ran out on the current

@@ -18,6 +18,8 @@ Functions (each cites the passage it follows in ssa_oracle.c):
   alignment_output_grads
                   output gradients of the alignment objective (a formula,
                   written here; pinned by finite differences with stop-gradient)
+  decode_step     one decoding step: selection for the newest token and its
+                  attention (fp64 numpy, small problems)
 """
 from __future__ import annotations
 
@@ -229,6 +231,52 @@ def alignment_output_grads(o_sparse, o_full, d_o, mode: int, alpha: float):
     else:
         raise ValueError("mode must be 0 or 1")
     return d_s, d_f
+
+
+def decode_step(q, k, v, kbar, lengths, topk: int, scale: Optional[float] = None, bs: int = BLOCK):
+    """One decoding step of the sparse stream, in fp64 ("SSA: Guida a Sparse
+    Sparse Attention per LLM", section "Block-sparse attention e Receptive
+    Field", applied to the newest token of each sequence).
+
+    q [B, Hq, D] (token t = lengths[b] - 1), k and v [B, S, Hkv, D] caches,
+    kbar [B, Hkv, n, D] mean keys.  Per KV head: the group's mean query scores
+    the complete blocks j < c = t // 64; the top k - 1 (ties: lower j) and c are
+    kept (every block 0..c when c + 1 <= k); attention over their tokens, keys
+    up to t in block c.  Returns idx [B, Hkv, k] (ascending, -1 padded), gap
+    [B, Hkv] (k-1-th minus k-th score, NaN when no boundary), o [B, Hq, D] and
+    lse [B, Hq]."""
+    q64, k64, v64 = widen(q), widen(k), widen(v)
+    kbar = np.asarray(kbar, dtype=np.float64)
+    B, Hq, D = q64.shape
+    Hkv = k64.shape[2]
+    G = Hq // Hkv
+    scale = (1.0 / np.sqrt(D)) if scale is None else float(scale)
+    idx = np.full((B, Hkv, topk), -1, dtype=np.int32)
+    gap = np.full((B, Hkv), np.nan)
+    o = np.zeros((B, Hq, D))
+    lse = np.zeros((B, Hq))
+    for b in range(B):
+        t = int(lengths[b]) - 1
+        c = t // bs
+        for h in range(Hkv):
+            if c + 1 <= topk:
+                sel = list(range(c + 1))
+            else:
+                qbar = q64[b, h * G:(h + 1) * G].mean(axis=0)
+                sc = kbar[b, h, :c] @ qbar
+                order = sorted(range(c), key=lambda j: (-sc[j], j))
+                gap[b, h] = sc[order[topk - 2]] - sc[order[topk - 1]]
+                sel = sorted(order[:topk - 1]) + [c]
+            idx[b, h, :len(sel)] = sel
+            tok = np.concatenate([np.arange(bs * j, min(bs * j + bs, t + 1)) for j in sel])
+            for g in range(G):
+                hq = h * G + g
+                logits = scale * (k64[b, tok, h] @ q64[b, hq])
+                m = logits.max()
+                w = np.exp(logits - m)
+                lse[b, hq] = m + np.log(w.sum())
+                o[b, hq] = (w / w.sum()) @ v64[b, tok, h]
+    return idx, gap, o, lse
 
 
 def sparse_forward_problem(q, k, v, topk: int, rows: Optional[np.ndarray] = None,

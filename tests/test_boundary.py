@@ -77,6 +77,8 @@ def test_bad_problem_is_rejected_by_every_entry_point(lib, kw, code):
     assert lib.ssa_sparse_attn_bwd_workspace(p) == 0
     assert lib.ssa_alignment_bwd(p, f, f, f, f, f, f, f, f, 0, 1.0, f, f, f, f, f, 1 << 30, None) == code
     assert lib.ssa_alignment_bwd_workspace(p) == 0
+    assert lib.ssa_decode_attn(p, f, f, f, f, f, f, f, None, f, 1 << 30, None) == code
+    assert lib.ssa_decode_attn_workspace(p) == 0
 
 
 def test_null_problem(lib):
@@ -118,3 +120,13 @@ def test_alignment_backward_arguments_are_checked_before_launch(lib):
     assert lib.ssa_alignment_bwd(p, f, f, f, f, f, f, f, f, 0, 1.0, f, f, f, f, f, ws - 1, None) == WORKSPACE
     assert lib.ssa_alignment_bwd(p, f, f, f, f, f, f, f, f, 0, 1.0, f, f, f, f, None, ws, None) == WORKSPACE
     assert lib.ssa_alignment_bwd(p, f, f, f, f, None, f, f, f, 0, 1.0, f, f, f, f, f, ws, None) == INVALID
+
+
+def test_decode_arguments_are_checked_before_launch(lib):
+    p = ctypes.byref(_p())
+    f = FAKE
+    ws = lib.ssa_decode_attn_workspace(p)
+    assert ws > 0
+    assert lib.ssa_decode_attn(p, f, f, f, f, f, f, f, None, f, ws - 1, None) == WORKSPACE
+    assert lib.ssa_decode_attn(p, f, f, f, f, None, f, f, None, f, ws, None) == INVALID
+    assert lib.ssa_decode_attn(p, f, f, f, f, f, f, f, f + 4, f, ws, None) == INVALID

@@ -402,3 +402,77 @@ def test_dense_table_gives_dense_causal_attention():
     np.testing.assert_allclose(o_s, o_f, atol=1e-13)
     ref = _sdpa_rows(q, k, v, lambda b, h: np.tril(np.ones((256, 256), dtype=bool)))
     np.testing.assert_allclose(o_s.transpose(0, 2, 1, 3), ref, atol=1e-12)
+
+
+# ------------------------------------------------------------------ decode
+
+def _decode_case(topk, seed, lengths, capacity=1024, Hq=4, Hkv=2, D=16):
+    x = gen.make_decode(len(lengths), capacity, Hq, Hkv, D, topk, seed=seed, n_plant=3,
+                        lengths=lengths)
+    kbar, _ = oracle.block_pool(x.k)
+    return x, kbar
+
+
+def _row_sdpa(x, b, hq, keep):
+    """torch float64 attention of one query row over the cache tokens in keep."""
+    k64, v64, q64 = oracle.widen(x.k), oracle.widen(x.v), oracle.widen(x.q)
+    G = q64.shape[1] // k64.shape[2]
+    h = hq // G
+    qt = torch.from_numpy(q64[b, hq])[None, None]
+    kt = torch.from_numpy(k64[b, :, h])[None]
+    vt = torch.from_numpy(v64[b, :, h])[None]
+    m = torch.from_numpy(keep)[None, None]
+    return F.scaled_dot_product_attention(qt, kt, vt, attn_mask=m)[0, 0].numpy()
+
+
+def test_decode_full_budget_equals_dense_causal_row():
+    lengths = [1, 64, 65, 700, 1024]
+    x, kbar = _decode_case(topk=16, seed=101, lengths=lengths)
+    idx, gap, o, lse = oracle.decode_step(x.q, x.k, x.v, kbar, x.lengths, 16)
+    for b, L in enumerate(lengths):
+        keep = np.arange(1024) < L
+        for hq in range(4):
+            np.testing.assert_allclose(o[b, hq], _row_sdpa(x, b, hq, keep), atol=1e-12)
+        assert np.all(np.isnan(gap[b]))
+
+
+def test_decode_selection_is_block_select_of_its_pooled_query():
+    lengths = [1000, 777, 1024, 513]
+    x, kbar = _decode_case(topk=4, seed=102, lengths=lengths)
+    idx, gap, _, _ = oracle.decode_step(x.q, x.k, x.v, kbar, x.lengths, 4)
+    q64 = oracle.widen(x.q)
+    B, Hkv, n, D = kbar.shape
+    G = q64.shape[1] // Hkv
+    for b, L in enumerate(lengths):
+        c = (L - 1) // 64
+        qbar = np.zeros_like(kbar)
+        for h in range(Hkv):
+            qbar[b, h, c] = q64[b, h * G:(h + 1) * G].mean(axis=0)
+        ref, rgap = oracle.block_select(qbar, kbar, 4)
+        for h in range(Hkv):
+            assert np.array_equal(idx[b, h], ref[b, h, c])
+            assert gap[b, h] == pytest.approx(rgap[b, h, c], abs=1e-12)
+        # brute force: the chosen earlier blocks maximise the summed score
+        for h in range(Hkv):
+            sc = kbar[b, h, :c] @ q64[b, h * G:(h + 1) * G].mean(axis=0)
+            best = max(itertools.combinations(range(c), 3), key=lambda s_: sum(sc[j] for j in s_))
+            assert sorted(best) == list(idx[b, h, :3])
+
+
+def test_decode_attention_is_masked_softmax_over_the_kept_tokens():
+    lengths = [1000, 641, 1024]
+    x, kbar = _decode_case(topk=3, seed=103, lengths=lengths)
+    idx, _, o, lse = oracle.decode_step(x.q, x.k, x.v, kbar, x.lengths, 3)
+    k64, q64 = oracle.widen(x.k), oracle.widen(x.q)
+    for b, L in enumerate(lengths):
+        for hq in range(4):
+            h = hq // 2
+            keep = np.zeros(1024, dtype=bool)
+            for j in idx[b, h]:
+                if j >= 0:
+                    keep[64 * j:64 * j + 64] = True
+            keep &= np.arange(1024) < L
+            np.testing.assert_allclose(o[b, hq], _row_sdpa(x, b, hq, keep), atol=1e-12)
+            logits = (k64[b, keep, h] @ q64[b, hq]) / 4.0
+            np.testing.assert_allclose(lse[b, hq], np.log(np.exp(logits - logits.max()).sum()) + logits.max(),
+                                       atol=1e-12)
