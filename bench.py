@@ -285,6 +285,8 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     assert ssa.ssa_get_device_error() == 0
 
+    decode = decode_rows(dev, timed)
+
     peaks, peak_src = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     achieved = flops / (fwd_ms * 1e-3) / 1e12
@@ -314,7 +316,8 @@ def run_ours(args, world, rank, local):
             "alignment_bwd": {
                 "ms": round(abwd_ms, 5),
                 "flops": "10 D per selected pair (sparse stream) + 10 D per causal pair (full stream)",
-                "tflops": round(2.5 * (flops + causal_flops(w)) / (abwd_ms * 1e-3) / 1e12, 2)}},
+                "tflops": round(2.5 * (flops + causal_flops(w)) / (abwd_ms * 1e-3) / 1e12, 2)},
+            "decode": decode},
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
         "pct_of_peak_step": round(100.0 * value / world / peak, 2),
@@ -335,6 +338,49 @@ def load_traffic(name):
     with open(path) as f:
         m = re.search(r"^dram_bytes_per_launch:\s*(\d+)", f.read(), re.M)
     return int(m.group(1)) if m else None
+
+
+# ------------------------------------------------------------------ decode
+
+def decode_rows(dev, timed_fn):
+    """One decoding step of the sparse stream (ssa_decode_attn) on two batch
+    shapes of the Llama-3.2-1B-like layer (Hq 32, Hkv 4, D 64, top-k 16):
+    64 sequences with 8k caches, and 8 sequences with 128k caches, the latter
+    also with top-k = every block (dense decode by the same kernels).  The
+    caches are seeded normal draws made on the device.  Algorithmic bytes: the
+    mean keys scored, the kept blocks' K and V, q and o."""
+    import block_sparse_attention_21_b200 as ssa
+    out = {}
+    for name, B, S, dense in (("decode_8k_b64", 64, 8192, False), ("decode_128k_b8", 8, 131072, False),
+                              ("decode_128k_b8_dense", 8, 131072, True)):
+        Hq, Hkv, D = 32, 4, 64
+        n = S // 64
+        topk = n if dense else 16
+        g = torch.Generator(device=dev).manual_seed(11 + S)
+        k = torch.randn(B, S, Hkv, D, generator=g, device=dev).to(torch.bfloat16)
+        v = torch.randn(B, S, Hkv, D, generator=g, device=dev).to(torch.bfloat16)
+        q = torch.randn(B, Hq, D, generator=g, device=dev).to(torch.bfloat16)
+        lengths = torch.full((B,), S, dtype=torch.int32, device=dev)
+        p = ssa.problem(B, S, Hq, Hkv, D, topk)
+        kb = torch.empty(B, Hkv, n, D, device=dev)
+        ssa.ssa_block_pool(p, k, None, kb, None)
+        o = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev)
+        lse = torch.empty(B, Hq, device=dev)
+        ws = torch.empty(max(ssa.ssa_decode_attn_workspace(p), 256), dtype=torch.uint8, device=dev)
+        ssa.ssa_decode_attn(p, q, k, v, kb, lengths, o, lse, None, ws, ws.numel())
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            ssa.ssa_decode_attn(p, q, k, v, kb, lengths, o, lse, None, ws, ws.numel())
+        reps = 50
+        ms = timed_fn(graph, reps) / reps
+        c = n - 1                                  # full caches: block n - 1 holds the query
+        kept = min(topk, c + 1)
+        nbytes = B * Hkv * ((c if kept < c + 1 else 0) * D * 4 + kept * 64 * D * 2 * 2) + 2 * B * Hq * D * 2
+        out[name] = {"ms": round(ms, 5), "batch": B, "cache_tokens": S, "top_k": topk,
+                     "gb_s": round(nbytes / (ms * 1e-3) / 1e9, 1), "bytes_per_step": int(nbytes)}
+        del k, v, kb, ws
+    out["decode_128k_sparse_vs_dense"] = round(out["decode_128k_b8_dense"]["ms"] / out["decode_128k_b8"]["ms"], 2)
+    return out
 
 
 # ----------------------------------------------------------- CPU baseline

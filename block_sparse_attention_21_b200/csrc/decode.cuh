@@ -15,9 +15,9 @@
 //                          the complete blocks, exact top-(k-1) by a radix
 //                          search on order-preserving keys (ties: lower j),
 //                          ascending table with c last.
-//   decode_attn_kernel     one CTA per (b, KV head, selected block): scores of
-//                          the G query heads against the block's 64 keys, a
-//                          partial softmax (max, sum, unnormalised output).
+//   decode_attn_kernel     one warp per (b, KV head, selected block): scores
+//                          of the G query heads against the block's 64 keys,
+//                          a partial softmax (max, sum, unnormalised output).
 //   decode_combine_kernel  one CTA per (b, query head): merges the partials.
 //
 // The work is a few rows per KV head, far below a 128-row tensor-core tile,
@@ -93,15 +93,27 @@ __global__ void __launch_bounds__(kDecodeSelThreads) decode_select_kernel(const 
     qs[d] = s / static_cast<float>(p.G);
   }
   __syncthreads();
-  // scores of the complete blocks j < c: a warp per block, lanes over D
+  // scores of the complete blocks j < c: a thread per block, its mean-key row
+  // read with 16-byte loads, eight in flight
   const float* kb = p.kbar + static_cast<size_t>(bh) * p.n * D;
-  for (int j = warp; j < c; j += kDecodeSelThreads / 32) {
-    float acc = 0.f;
+  for (int j = threadIdx.x; j < c; j += blockDim.x) {
+    const float4* row = reinterpret_cast<const float4*>(kb + static_cast<size_t>(j) * D);
+    float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-    for (int d = lane; d < D; d += 32) acc = fmaf(qs[d], kb[static_cast<size_t>(j) * D + d], acc);
+    for (int d4 = 0; d4 < D / 4; d4 += 8) {
+      float4 r[8];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) dkey[j] = dec_order_key(acc);
+      for (int x = 0; x < 8; ++x) r[x] = __ldg(row + d4 + x);
+#pragma unroll
+      for (int x = 0; x < 8; ++x) {
+        const int d = 4 * (d4 + x);
+        acc0 = fmaf(qs[d], r[x].x, acc0);
+        acc1 = fmaf(qs[d + 1], r[x].y, acc1);
+        acc0 = fmaf(qs[d + 2], r[x].z, acc0);
+        acc1 = fmaf(qs[d + 3], r[x].w, acc1);
+      }
+    }
+    dkey[j] = dec_order_key(acc0 + acc1);
   }
   __syncthreads();
   // the (k-1)-th largest key, by a 32-step radix search
@@ -137,76 +149,147 @@ __global__ void __launch_bounds__(kDecodeSelThreads) decode_select_kernel(const 
   }
 }
 
-// Dynamic shared memory of decode_attn_kernel: the block's K (rows padded by
-// one float against bank conflicts) and V in fp32, up to 16 queries, scores.
+// Warps per CTA of decode_attn_kernel, and its dynamic shared memory: per
+// warp the block's K and V (rows padded by 16 bytes, so lanes reading
+// different rows hit different banks), the G <= 16 queries and probabilities.
+constexpr int kDecodeWarps = 2;
 template <int D>
-constexpr int decode_attn_smem() {
-  return (64 * (D + 1) + 64 * D + 16 * D + 16 * 64) * 4;
+__host__ __device__ constexpr int decode_row_bytes() {
+  return D * 2 + 16;
+}
+template <int D>
+__host__ __device__ constexpr int decode_warp_smem() {
+  return 2 * 64 * decode_row_bytes<D>() + 16 * D * 4 + 16 * 64 * 4;
+}
+template <int D>
+__host__ __device__ constexpr int decode_attn_smem() {
+  return kDecodeWarps * decode_warp_smem<D>();
 }
 
-// 128 threads; G <= 16.
-template <int D>
-__global__ void __launch_bounds__(128) decode_attn_kernel(const DecodeParams p) {
-  extern __shared__ float dsm[];
-  float (*ks)[D + 1] = reinterpret_cast<float (*)[D + 1]>(dsm);
-  float (*vs)[D] = reinterpret_cast<float (*)[D]>(dsm + 64 * (D + 1));
-  float (*qs)[D] = reinterpret_cast<float (*)[D]>(dsm + 64 * (D + 1) + 64 * D);
-  float (*sc)[64] = reinterpret_cast<float (*)[64]>(dsm + 64 * (D + 1) + 64 * D + 16 * D);
-  const int slot = blockIdx.x % p.topk;
-  const int bh = blockIdx.x / p.topk, b = bh / p.Hkv, h = bh % p.Hkv;
-  const int G = p.G;
-  float* part = p.part + (static_cast<size_t>(bh) * p.topk + slot) * G * (D + 2);
+__device__ __forceinline__ void dec_cp_async16(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
+}
+
+__device__ __forceinline__ uint64_t dec_f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ uint64_t dec_f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ float dec_f2_sum(uint64_t v) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return lo + hi;
+}
+// bf16 pair (low = even element) -> packed fp32 pair
+__device__ __forceinline__ uint64_t dec_bf2(uint32_t w) {
+  return dec_f2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
+// One warp per (b, KV head, selected block), G query heads (template, so no
+// work is spent on absent heads).  The warp first copies the block's K and V
+// rows into shared memory with cp.async (one round trip for all of them);
+// lane l scores keys l and l + 32 against the G queries with packed f32x2
+// FMAs and 16-byte query loads; a per-head max and sum run over the warp; then
+// lane l accumulates its output columns of every head over the 64 keys.
+template <int D, int G>
+__global__ void __launch_bounds__(32 * kDecodeWarps) decode_attn_kernel(const DecodeParams p) {
+  constexpr int CPL = D / 32;                 // output columns per lane
+  constexpr int RB = decode_row_bytes<D>();
+  extern __shared__ __align__(16) uint8_t dsm[];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  uint8_t* ks = dsm + warp * decode_warp_smem<D>();
+  uint8_t* vs = ks + 64 * RB;
+  float (*qs)[D] = reinterpret_cast<float (*)[D]>(vs + 64 * RB);
+  float (*pr)[64] = reinterpret_cast<float (*)[64]>(vs + 64 * RB + 16 * D * 4);
+  const int item = blockIdx.x * kDecodeWarps + warp;
+  if (item >= p.B * p.Hkv * p.topk) return;
+  const int slot = item % p.topk;
+  const int bh = item / p.topk, b = bh / p.Hkv, h = bh % p.Hkv;
+  float* part = p.part + static_cast<size_t>(item) * G * (D + 2);
   const int j = p.idx[static_cast<size_t>(bh) * p.topk + slot];
   if (j < 0) {  // padding: an empty partial
-    for (int g = threadIdx.x; g < G; g += blockDim.x) {
-      part[g * (D + 2)] = -INFINITY;
-      part[g * (D + 2) + 1] = 0.f;
+    if (lane < G) {
+      part[lane * (D + 2)] = -INFINITY;
+      part[lane * (D + 2) + 1] = 0.f;
     }
     return;
   }
   const int t = p.len[b] - 1;
   const int nkeys = (j == t / 64) ? (t - 64 * j + 1) : 64;  // causal inside the query's block
-  // K and V rows of the block: 16-byte loads, D / 8 per row
-  for (int e = threadIdx.x; e < 64 * (D / 8); e += blockDim.x) {
+  // K and V rows of the block -> shared memory, 16 bytes per copy; rows past
+  // the causal end are zeroed (their probabilities are 0)
+  const size_t rstride = static_cast<size_t>(p.Hkv) * D;
+  const __nv_bfloat16* kg = p.k + ((static_cast<size_t>(b) * p.S + 64 * j) * p.Hkv + h) * D;
+  const __nv_bfloat16* vg = p.v + ((static_cast<size_t>(b) * p.S + 64 * j) * p.Hkv + h) * D;
+  for (int e = lane; e < 64 * (D / 8); e += 32) {
     const int r = e / (D / 8), c8 = e % (D / 8);
-    const size_t off = ((static_cast<size_t>(b) * p.S + 64 * j + r) * p.Hkv + h) * D + c8 * 8;
-    uint4 kk = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
     if (r < nkeys) {
-      kk = *reinterpret_cast<const uint4*>(p.k + off);
-      vv = *reinterpret_cast<const uint4*>(p.v + off);
+      dec_cp_async16(ks + r * RB + c8 * 16, kg + r * rstride + c8 * 8);
+      dec_cp_async16(vs + r * RB + c8 * 16, vg + r * rstride + c8 * 8);
+    } else {
+      *reinterpret_cast<uint4*>(ks + r * RB + c8 * 16) = make_uint4(0, 0, 0, 0);
+      *reinterpret_cast<uint4*>(vs + r * RB + c8 * 16) = make_uint4(0, 0, 0, 0);
     }
-    const uint32_t wk[4] = {kk.x, kk.y, kk.z, kk.w}, wv[4] = {vv.x, vv.y, vv.z, vv.w};
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  for (int e = lane; e < G * D; e += 32)
+    qs[e / D][e % D] = __bfloat162float(p.q[(static_cast<size_t>(b) * p.Hq + h * G) * D + e]) * p.scale_log2;
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  __syncwarp();
+  // scores of keys lane and lane + 32 against every head, 64 columns at a time
+  float sc[2][G];
 #pragma unroll
-    for (int x = 0; x < 4; ++x) {
-      ks[r][c8 * 8 + 2 * x] = __uint_as_float(wk[x] << 16);
-      ks[r][c8 * 8 + 2 * x + 1] = __uint_as_float(wk[x] & 0xFFFF0000u);
-      vs[r][c8 * 8 + 2 * x] = __uint_as_float(wv[x] << 16);
-      vs[r][c8 * 8 + 2 * x + 1] = __uint_as_float(wv[x] & 0xFFFF0000u);
+  for (int x = 0; x < 2; ++x)
+#pragma unroll
+    for (int g = 0; g < G; ++g) sc[x][g] = 0.f;
+#pragma unroll
+  for (int d0 = 0; d0 < D; d0 += 64) {
+    uint64_t kp[2][32];  // the two keys' 64 columns as fp32 pairs
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+      const uint4* krow = reinterpret_cast<const uint4*>(ks + (lane + 32 * x) * RB + 2 * d0);
+#pragma unroll
+      for (int c8 = 0; c8 < 8; ++c8) {
+        const uint4 kv = krow[c8];
+        kp[x][4 * c8] = dec_bf2(kv.x);
+        kp[x][4 * c8 + 1] = dec_bf2(kv.y);
+        kp[x][4 * c8 + 2] = dec_bf2(kv.z);
+        kp[x][4 * c8 + 3] = dec_bf2(kv.w);
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      uint64_t a0 = 0, a1 = 0;
+      const float4* qrow = reinterpret_cast<const float4*>(&qs[g][d0]);
+#pragma unroll
+      for (int c4 = 0; c4 < 16; ++c4) {
+        const float4 q4 = qrow[c4];
+        const uint64_t qa = dec_f2(q4.x, q4.y), qb = dec_f2(q4.z, q4.w);
+        a0 = dec_f2_fma(qa, kp[0][2 * c4], a0);
+        a0 = dec_f2_fma(qb, kp[0][2 * c4 + 1], a0);
+        a1 = dec_f2_fma(qa, kp[1][2 * c4], a1);
+        a1 = dec_f2_fma(qb, kp[1][2 * c4 + 1], a1);
+      }
+      sc[0][g] += dec_f2_sum(a0);
+      sc[1][g] += dec_f2_sum(a1);
     }
   }
-  for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
-    const int g = e / D, d = e % D;
-    qs[g][d] = __bfloat162float(p.q[(static_cast<size_t>(b) * p.Hq + h * G + g) * D + d]) * p.scale_log2;
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < G * 64; e += blockDim.x) {
-    const int g = e / 64, r = e % 64;
-    float acc = 0.f;
-#pragma unroll 8
-    for (int d = 0; d < D; ++d) acc = fmaf(qs[g][d], ks[r][d], acc);
-    sc[g][r] = (r < nkeys) ? acc : -INFINITY;
-  }
-  __syncthreads();
-  // per head: max and sum by one warp each (warp w takes heads w, w + 4, ...)
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  for (int g = warp; g < G; g += 4) {
-    const float a = sc[g][lane], c2 = sc[g][lane + 32];
+  // per head: max and sum over the warp, probabilities to shared memory
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const float a = lane < nkeys ? sc[0][g] : -INFINITY;
+    const float c2 = lane + 32 < nkeys ? sc[1][g] : -INFINITY;
     float m = fmaxf(a, c2);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
     const float pa = exp2f(a - m), pb = exp2f(c2 - m);
-    sc[g][lane] = pa;
-    sc[g][lane + 32] = pb;
+    pr[g][lane] = pa;
+    pr[g][lane + 32] = pb;
     float l = pa + pb;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
@@ -215,14 +298,44 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(const DecodeParams p) 
       part[g * (D + 2) + 1] = l;
     }
   }
-  __syncthreads();
-  for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
-    const int g = e / D, d = e % D;
-    float acc = 0.f;
-#pragma unroll 8
-    for (int r = 0; r < 64; ++r) acc = fmaf(sc[g][r], vs[r][d], acc);
-    part[g * (D + 2) + 2 + d] = acc;
+  __syncwarp();
+  // o[g][d] for the lane's columns d = CPL * lane .. + CPL - 1, four keys at a time
+  float acc[G][CPL];
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) acc[g][c] = 0.f;
+  for (int r0 = 0; r0 < 64; r0 += 4) {
+    float vv[4][CPL];
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      const uint8_t* vrow = vs + (r0 + x) * RB + 2 * CPL * lane;
+      if constexpr (CPL == 2) {
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(vrow);
+        vv[x][0] = __uint_as_float(w << 16);
+        vv[x][1] = __uint_as_float(w & 0xFFFF0000u);
+      } else {
+        const uint2 w = *reinterpret_cast<const uint2*>(vrow);
+        vv[x][0] = __uint_as_float(w.x << 16);
+        vv[x][1] = __uint_as_float(w.x & 0xFFFF0000u);
+        vv[x][2] = __uint_as_float(w.y << 16);
+        vv[x][3] = __uint_as_float(w.y & 0xFFFF0000u);
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float4 p4 = *reinterpret_cast<const float4*>(&pr[g][r0]);
+      const float pw[4] = {p4.x, p4.y, p4.z, p4.w};
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) acc[g][c] = fmaf(pw[x], vv[x][c], acc[g][c]);
+    }
   }
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) part[g * (D + 2) + 2 + CPL * lane + c] = acc[g][c];
 }
 
 // One CTA of D threads per (b, query head): o = sum_s 2^(m_s - M) o_s / l.

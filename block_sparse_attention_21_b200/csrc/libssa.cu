@@ -459,6 +459,17 @@ DecodeLayout decode_layout(const Dims& d) {
   return L;
 }
 
+template <int D, int G>
+ssa_status launch_decode_attn(unsigned items, const ssa::DecodeParams& dp, cudaStream_t st) {
+  static std::atomic<uint64_t> smem_done{0};
+  auto kernel = ssa::decode_attn_kernel<D, G>;
+  const ssa_status s = ensure_smem(kernel, ssa::decode_attn_smem<D>(), &smem_done);
+  if (s != SSA_OK) return s;
+  kernel<<<(items + ssa::kDecodeWarps - 1) / ssa::kDecodeWarps, 32 * ssa::kDecodeWarps, ssa::decode_attn_smem<D>(),
+           st>>>(dp);
+  return launch_result();
+}
+
 template <int D>
 ssa_status launch_decode(const Dims& d, const void* q, const void* k, const void* v, const float* kbar,
                          const int32_t* len, void* o, float* lse, int32_t* idx_out, void* workspace,
@@ -487,11 +498,14 @@ ssa_status launch_decode(const Dims& d, const void* q, const void* k, const void
   ssa::decode_select_kernel<D><<<bh, ssa::kDecodeSelThreads, 4 * d.n, st>>>(dp);
   ssa_status s = launch_result();
   if (s != SSA_OK) return s;
-  static std::atomic<uint64_t> smem_done{0};
-  s = ensure_smem(ssa::decode_attn_kernel<D>, ssa::decode_attn_smem<D>(), &smem_done);
+  const unsigned items = bh * static_cast<unsigned>(d.topk);
+  switch (d.G) {
+    case 2: s = launch_decode_attn<D, 2>(items, dp, st); break;
+    case 4: s = launch_decode_attn<D, 4>(items, dp, st); break;
+    case 8: s = launch_decode_attn<D, 8>(items, dp, st); break;
+    default: s = launch_decode_attn<D, 16>(items, dp, st); break;
+  }
   if (s != SSA_OK) return s;
-  ssa::decode_attn_kernel<D><<<bh * d.topk, 128, ssa::decode_attn_smem<D>(), st>>>(dp);
-  if ((s = launch_result()) != SSA_OK) return s;
   ssa::decode_combine_kernel<D><<<static_cast<unsigned>(d.B) * d.Hq, D, 0, st>>>(dp);
   return launch_result();
 }
