@@ -286,6 +286,25 @@ def run_ours(args, world, rank, local):
     assert ssa.ssa_get_device_error() == 0
 
     decode = decode_rows(dev, timed)
+    # the early-stop variant of the sparse forward on the same inputs and table
+    early = {}
+    n_tiles = w.batch * w.n_kv_heads * w.n_blocks * (w.n_q_heads // w.n_kv_heads // 2)
+    vis = torch.empty(n_tiles, dtype=torch.int32, device=dev)
+    g_step.replay()
+    nsel_mean = float((st.block_idx >= 0).sum(dim=-1).float().mean())
+    for tau in (0.0, 0.1, 0.2, 0.5):
+        ssa.ssa_sparse_attn_fwd_early_stop(p, q, k, v, st.q_pooled, st.k_pooled, st.block_idx, tau,
+                                           st.o, st.lse, vis.view(w.batch, w.n_kv_heads, w.n_blocks, -1))
+        g_es = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_es):
+            ssa.ssa_sparse_attn_fwd_early_stop(p, q, k, v, st.q_pooled, st.k_pooled, st.block_idx, tau,
+                                               st.o, st.lse, vis.view(w.batch, w.n_kv_heads, w.n_blocks, -1))
+        es_ms = timed(g_es, n_k) / n_k
+        torch.cuda.synchronize()
+        assert ssa.ssa_get_device_error() == 0
+        early[f"tau_{tau:g}"] = {"ms": round(es_ms, 5), "blocks_visited_mean": round(float(vis.float().mean()), 3),
+                                 "blocks_selected_mean": round(nsel_mean, 3),
+                                 "speedup_vs_sparse_fwd": round(fwd_ms / es_ms, 3)}
 
     peaks, peak_src = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
@@ -317,7 +336,8 @@ def run_ours(args, world, rank, local):
                 "ms": round(abwd_ms, 5),
                 "flops": "10 D per selected pair (sparse stream) + 10 D per causal pair (full stream)",
                 "tflops": round(2.5 * (flops + causal_flops(w)) / (abwd_ms * 1e-3) / 1e12, 2)},
-            "decode": decode},
+            "decode": decode,
+            "sparse_attn_fwd_early_stop": early},
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
         "pct_of_peak_step": round(100.0 * value / world / peak, 2),

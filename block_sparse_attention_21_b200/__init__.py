@@ -13,7 +13,7 @@ import torch
 
 from ._binding import (EXPORTED, LIB_PATH, SsaError, SsaProblem, lib, problem,
                        ssa_alignment_bwd, ssa_alignment_bwd_workspace, ssa_decode_attn,
-                       ssa_decode_attn_workspace,
+                       ssa_decode_attn_workspace, ssa_sparse_attn_fwd_early_stop,
                        ssa_block_pool, ssa_block_select, ssa_debug_exp2_poly, ssa_debug_timeout_probe,
                        ssa_full_attn_fwd_with_mass, ssa_get_device_error,
                        ssa_get_device_error_site, ssa_launch_count,
@@ -23,7 +23,7 @@ from ._binding import (EXPORTED, LIB_PATH, SsaError, SsaProblem, lib, problem,
 
 __all__ = ["EXPORTED", "LIB_PATH", "SsaError", "SsaProblem", "SparseStream", "lib", "problem",
            "ssa_alignment_bwd", "ssa_alignment_bwd_workspace", "ssa_decode_attn",
-           "ssa_decode_attn_workspace",
+           "ssa_decode_attn_workspace", "ssa_sparse_attn_fwd_early_stop",
            "ssa_block_pool", "ssa_block_select", "ssa_debug_exp2_poly", "ssa_debug_timeout_probe",
            "ssa_full_attn_fwd_with_mass", "ssa_get_device_error", "ssa_get_device_error_site",
            "ssa_launch_count",

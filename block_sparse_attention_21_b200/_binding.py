@@ -23,7 +23,7 @@ STATUS_NAMES = {0: "SSA_OK", 1: "SSA_ERR_INVALID_ARG", 2: "SSA_ERR_UNSUPPORTED",
                 3: "SSA_ERR_CUDA", 4: "SSA_ERR_DEVICE_TIMEOUT", 5: "SSA_ERR_WORKSPACE"}
 
 # every symbol include/ssa.h declares
-EXPORTED = ("ssa_block_pool", "ssa_block_select", "ssa_sparse_attn_fwd",
+EXPORTED = ("ssa_block_pool", "ssa_block_select", "ssa_sparse_attn_fwd", "ssa_sparse_attn_fwd_early_stop",
             "ssa_full_attn_fwd_with_mass", "ssa_sparse_attn_bwd_workspace",
             "ssa_sparse_attn_bwd", "ssa_sparse_attn_bwd_noalloc", "ssa_alignment_bwd_workspace",
             "ssa_alignment_bwd", "ssa_decode_attn_workspace", "ssa_decode_attn",
@@ -73,6 +73,7 @@ def lib():
             "ssa_sparse_attn_bwd": [P] + [vp] * 11 + [ctypes.c_size_t, vp],
             "ssa_sparse_attn_bwd_noalloc": [P] + [vp] * 11,
             "ssa_decode_attn": [P] + [vp] * 9 + [ctypes.c_size_t, vp],
+            "ssa_sparse_attn_fwd_early_stop": [P] + [vp] * 6 + [ctypes.c_float] + [vp] * 4,
             "ssa_alignment_bwd": [P] + [vp] * 8 + [ctypes.c_int, ctypes.c_float] + [vp] * 5
                                  + [ctypes.c_size_t, vp],
             "ssa_get_device_error": [vp],
@@ -222,6 +223,25 @@ def ssa_alignment_bwd(p: SsaProblem, q, k, v, o_sparse, lse_sparse, o_full, lse_
           int(mode), float(alpha), _ptr(block_idx, I32, "block_idx"), _ptr(dq, BF16, "dq"),
           _ptr(dk, BF16, "dk"), _ptr(dv, BF16, "dv"), _ptr(workspace, None, "workspace"),
           int(ws_bytes), _stream(stream))
+
+
+def ssa_sparse_attn_fwd_early_stop(p: SsaProblem, q, k, v, q_pooled, k_pooled, block_idx, tau: float,
+                                   o, lse, visited=None, stream=None) -> None:
+    """The sparse forward visiting the diagonal first, then the selected blocks
+    by descending pooled score, each tile stopping after the first block that
+    adds less than tau of every row's accumulated mass; see include/ssa.h."""
+    sh = _shapes(p)
+    for t, s, nm in ((q, "q", "q"), (k, "kv", "k"), (v, "kv", "v"), (q_pooled, "pooled", "q_pooled"),
+                     (k_pooled, "pooled", "k_pooled"), (block_idx, "idx", "block_idx"), (o, "q", "o"),
+                     (lse, "lse", "lse")):
+        _numel_check(t, sh[s], nm)
+    if visited is not None:
+        B, Hkv, n, _ = sh["idx"]
+        _numel_check(visited, (B, Hkv, n, p.n_q_heads // p.n_kv_heads // 2), "visited")
+    _call("ssa_sparse_attn_fwd_early_stop", ctypes.byref(p), _ptr(q, BF16, "q"), _ptr(k, BF16, "k"),
+          _ptr(v, BF16, "v"), _ptr(q_pooled, F32, "q_pooled"), _ptr(k_pooled, F32, "k_pooled"),
+          _ptr(block_idx, I32, "block_idx"), float(tau), _ptr(o, BF16, "o"), _ptr(lse, F32, "lse"),
+          _ptr(visited, I32, "visited"), _stream(stream))
 
 
 def ssa_decode_attn_workspace(p: SsaProblem) -> int:

@@ -49,7 +49,11 @@
 
 namespace ssa {
 
-template <int D, int T, bool MASS>
+// Largest top-k of the early-stop variant (its visiting order lives in the
+// 1 KB selection-bitmap area).
+constexpr int kEarlyMaxTopk = 256;
+
+template <int D, int T, bool MASS, bool EARLY = false>
 struct FwdConfig {
   static constexpr int NP = D / 64;               // 64-column panels per row
   static constexpr int QTILE = 128 * D * 2;       // bytes of one Q M-tile
@@ -64,18 +68,20 @@ struct FwdConfig {
   // shared memory: Q tiles, K ring, V ring, barriers, tmem slot, abort flag,
   // selection bitmap (up to 8192 blocks)
   static constexpr int SMEM_TILES = T * QTILE + 2 * NS * KVT;
-  static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + NBARS * 8 + 16 + 1024;
+  // EARLY: 2 KB of score scratch and 128 B of stop flags after the bitmap area
+  static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + NBARS * 8 + 16 + 1024 + (EARLY ? 2048 + 128 : 0);
   // two CTAs share an SM when both fit in TMEM (256 columns each) and in
   // shared memory: one CTA's prologue and epilogue overlap the other's loop
   static constexpr int MIN_CTAS = (TMEM_COLS <= 256 && SMEM_BYTES <= 113 * 1024) ? 2 : 1;
   static_assert(T * TSTRIDE <= 512, "TMEM budget");
 };
 
-template <int D, int T, bool MASS>
-__global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, FwdConfig<D, T, MASS>::MIN_CTAS)
+template <int D, int T, bool MASS, bool EARLY = false>
+__global__ void __launch_bounds__(FwdConfig<D, T, MASS, EARLY>::THREADS, FwdConfig<D, T, MASS, EARLY>::MIN_CTAS)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using C = FwdConfig<D, T, MASS>;
+  using C = FwdConfig<D, T, MASS, EARLY>;
+  static_assert(!(MASS && EARLY), "the early stop applies to the sparse stream only");
   constexpr int NP = C::NP, QTILE = C::QTILE, KVT = C::KVT, NS = C::NS, TSTRIDE = C::TSTRIDE;
 
   extern __shared__ uint8_t smem_raw[];
@@ -97,6 +103,13 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, FwdConfig<D, T
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_drain + C::ISS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint32_t* selbits = tmem_slot + 4;
+  // EARLY: visiting order (over the bitmap area), score scratch, stop flags
+  int32_t* ord = reinterpret_cast<int32_t*>(selbits);
+  float* esc = reinterpret_cast<float*>(selbits + 256);       // [256] scores
+  int32_t* ej = reinterpret_cast<int32_t*>(esc + 256);        // [256] their blocks
+  volatile int* all_stop = reinterpret_cast<volatile int*>(ej + 256);
+  volatile int* tile_stop = all_stop + 1;                     // [T]
+  volatile int* wflag = all_stop + 4;                         // [T][2][4]
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
@@ -142,6 +155,10 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, FwdConfig<D, T
       if (j >= 0 && j <= i) atomicOr(&selbits[j >> 5], 1u << (j & 31));
     }
   }
+  if (EARLY && threadIdx.x == 0) {
+    *all_stop = 0;
+    for (int t = 0; t < T; ++t) tile_stop[t] = 0;
+  }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
@@ -154,6 +171,14 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, FwdConfig<D, T
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    auto load_kv = [&](int st, int j) {
+      mbar_arrive_expect_tx(&bar_kfull[st], KVT);
+      for (int pn = 0; pn < NP; ++pn)
+        tma_load_4d(sK + st * KVT + pn * (64 * 128), &tm_k, &bar_kfull[st], 64 * pn, h, 64 * j, b);
+      mbar_arrive_expect_tx(&bar_vfull[st], KVT);
+      for (int pn = 0; pn < NP; ++pn)
+        tma_load_4d(sV + st * KVT + pn * (64 * 128), &tm_v, &bar_vfull[st], 64 * pn, h, 64 * j, b);
+    };
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
@@ -164,24 +189,58 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, FwdConfig<D, T
           for (int pn = 0; pn < NP; ++pn)
             tma_load_4d(sQ + t * QTILE + pn * (128 * 128) + hh * (64 * 128), &tm_q, bar_q,
                         64 * pn, hq0 + 2 * t + hh, 64 * i, b);
-      int issued = 0;
-      for (int jj = 0; jj < nblk; ++jj) {
+      if (EARLY) load_kv(0, i);  // the diagonal block is visited first
+    }
+    if (EARLY) {
+      // visiting order: the diagonal block i first, then the other selected
+      // blocks (idx_row[0 .. nsel - 2], all below i) by descending pooled score
+      // q_pooled[i] . k_pooled[j] in fp32, ties to the lower block
+      const int ne = nsel - 1;
+      const float4* qb = reinterpret_cast<const float4*>(p.qbar + ((static_cast<size_t>(b) * p.Hkv + h) * p.n + i) * D);
+      const float* kb = p.kbar + (static_cast<size_t>(b) * p.Hkv + h) * p.n * D;
+      for (int r = lane; r < ne; r += 32) {
+        const int j = idx_row[r];
+        const float4* kr = reinterpret_cast<const float4*>(kb + static_cast<size_t>(j) * D);
+        float acc = 0.f;
+        for (int d4 = 0; d4 < D / 4; ++d4) {
+          const float4 a = __ldg(qb + d4), c = __ldg(kr + d4);
+          acc = fmaf(a.x, c.x, fmaf(a.y, c.y, fmaf(a.z, c.z, fmaf(a.w, c.w, acc))));
+        }
+        esc[r] = acc;
+        ej[r] = j;
+      }
+      __syncwarp();
+      for (int r = lane; r < ne; r += 32) {
+        const float sr = esc[r];
+        const int jr = ej[r];
+        int rank = 0;
+        for (int r2 = 0; r2 < ne; ++r2) rank += (esc[r2] > sr || (esc[r2] == sr && ej[r2] < jr)) ? 1 : 0;
+        ord[1 + rank] = jr;
+      }
+      if (lane == 0) ord[0] = i;
+      __syncwarp();
+    }
+    if (lane == 0) {
+      int issued = EARLY ? 1 : 0;
+      for (int jj = issued; jj < nblk; ++jj) {
         const int st = jj % NS, use = jj / NS;
-        if (use > 0 && !mbar_wait(&bar_empty[st], (use - 1) & 1, abort_flag, tmo, 0x101)) break;
-        const int j = MASS ? jj : idx_row[jj];
-        mbar_arrive_expect_tx(&bar_kfull[st], KVT);
-        for (int pn = 0; pn < NP; ++pn)
-          tma_load_4d(sK + st * KVT + pn * (64 * 128), &tm_k, &bar_kfull[st], 64 * pn, h, 64 * j, b);
-        mbar_arrive_expect_tx(&bar_vfull[st], KVT);
-        for (int pn = 0; pn < NP; ++pn)
-          tma_load_4d(sV + st * KVT + pn * (64 * 128), &tm_v, &bar_vfull[st], 64 * pn, h, 64 * j, b);
+        if (EARLY && *all_stop) break;  // every tile stopped: no more blocks
+        // EARLY: once every tile stopped, the stage is never released; the
+        // stop flag ends the wait instead
+        if (use > 0 && !(EARLY ? mbar_wait_or(&bar_empty[st], (use - 1) & 1, abort_flag, all_stop, tmo, 0x101)
+                               : mbar_wait(&bar_empty[st], (use - 1) & 1, abort_flag, tmo, 0x101)))
+          break;
+        load_kv(st, MASS ? jj : (EARLY ? ord[jj] : idx_row[jj]));
         ++issued;
       }
-      // on abort, loads already issued are waited for (bounded) before exit
-      if (*abort_flag) {
+      // on abort or an early stop, loads already issued are waited for
+      // (bounded) before exit
+      if (*abort_flag || (EARLY && issued < nblk)) {
         volatile int never = 0;
-        for (int jj = (issued > NS ? issued - NS : 0); jj < issued; ++jj)
+        for (int jj = (issued > NS ? issued - NS : 0); jj < issued; ++jj) {
+          mbar_wait(&bar_kfull[jj % NS], (jj / NS) & 1, &never, 1000000ull, 0x1fe);
           mbar_wait(&bar_vfull[jj % NS], (jj / NS) & 1, &never, 1000000ull, 0x1ff);
+        }
       }
     }
   } else if (warp >= 1 && warp <= C::ISS) {
@@ -221,9 +280,9 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, FwdConfig<D, T
           tc_commit(&bar_sfull[t]);
         }
       }
-      bool first_sel[MT], first_uns[MT];
+      bool first_sel[MT], first_uns[MT], stopped[MT];
 #pragma unroll
-      for (int x = 0; x < MT; ++x) first_sel[x] = first_uns[x] = true;
+      for (int x = 0; x < MT; ++x) first_sel[x] = first_uns[x] = true, stopped[x] = false;
       for (int jj = 0; ok && jj < nblk; ++jj) {
         const int st = jj % NS;
         const bool more = jj + 1 < nblk;
@@ -239,7 +298,7 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, FwdConfig<D, T
 #pragma unroll
         for (int x = 0; x < MT; ++x) {
           const int t = me + x * ISS;
-          if (t >= T || !ok) continue;
+          if (t >= T || !ok || (EARLY && stopped[x])) continue;
           // keys 0..31 as soon as the first half of P is stored
           if (!mbar_wait(&bar_phalf[t], jj & 1, abort_flag, tmo, 0x205)) {
             ok = false;
@@ -261,17 +320,30 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, FwdConfig<D, T
 #pragma unroll
           for (int kk = 2; kk < 4; ++kk)
             mma_ts(o_col, base + kk * 8, v0 + ((kk * (16 * 128)) >> 4), idesc_pv, 1u);
-          if (more) {
+          // EARLY: the softmax set the tile's stop flag before it arrived on pfull
+          const bool stop_now = EARLY && tile_stop[t] != 0;
+          if (more && !stop_now) {
             issue_qk(t, st1);
             tc_commit(&bar_sfull[t]);
           } else {
             tc_commit(&bar_odone[t]);
+            if (EARLY) stopped[x] = true;
           }
           if (MASS) {
             if (is_sel) first_sel[x] = false; else first_uns[x] = false;
           }
         }
         if (ok) tc_commit(&bar_empty[st]);  // this issuer's tiles are all done with the stage
+        if (EARLY) {
+          bool all = true;
+#pragma unroll
+          for (int x = 0; x < MT; ++x)
+            if (me + x * ISS < T && !stopped[x]) all = false;
+          if (all) {  // no tile visits more blocks: the producer stops too
+            *all_stop = 1;
+            break;
+          }
+        }
       }
       if (!ok) {
         // every MMA this thread issued completes before TMEM is released
@@ -294,6 +366,7 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, FwdConfig<D, T
     const uint64_t scale2 = f2_pack(sl2, sl2);
     float m_ref = -INFINITY;  // reference maximum, scaled (log2) units
     float l_sel = 0.f, l_uns = 0.f;
+    int visited = 0;          // EARLY: blocks this tile visited
     bool ok = true;
     for (int jj = 0; jj < nblk; ++jj) {
       // waits are made warp-uniform: the tcgen05.ld/st below are .sync.aligned
@@ -302,7 +375,9 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, FwdConfig<D, T
         break;
       }
       tc_fence_after();
-      const bool diag = (jj == nblk - 1);
+      // the diagonal block comes last in the ascending table, first in the
+      // early-stop order
+      const bool diag = EARLY ? (jj == 0) : (jj == nblk - 1);
       bool is_sel = true;
       if (MASS) is_sel = (selbits[jj >> 5] >> (jj & 31)) & 1u;
       // all 64 scores with one TMEM round trip, then the raw row maximum
@@ -355,12 +430,27 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, FwdConfig<D, T
       tmem_st16(tS + 16, pk);  // P columns 16..31
       float r0, r1;
       f2_unpack(acc2, r0, r1);
+      bool stop = false;
+      if (EARLY && jj > 0 && p.tau > 0.f) {
+        // this block's mass against the mass accumulated before it (both in
+        // the current reference); the tile stops when no row gained at least
+        // tau times what it had (tau = 0 never stops: no decision is taken)
+        const bool cont_row = (r0 + r1) >= p.tau * (l_sel * alpha);
+        volatile int* wf = wflag + (t * 2 + (jj & 1)) * 4;
+        const bool wcont = __any_sync(0xffffffffu, cont_row);
+        if (lane == 0) wf[wq] = wcont ? 1 : 0;
+        named_bar_sync(1 + t, 128);
+        stop = !(wf[0] | wf[1] | wf[2] | wf[3]);
+        if (stop && r == 0) tile_stop[t] = 1;  // read by the issuer after pfull
+      }
       l_sel *= alpha;
       l_uns *= alpha;
       if (is_sel) l_sel += r0 + r1; else l_uns += r0 + r1;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bar_pfull[t]);
+      if (EARLY) visited = jj + 1;
+      if (stop) break;
     }
     // ---------------------------------------------------------- epilogue
     if (ok && __all_sync(0xffffffffu, mbar_wait(&bar_odone[t], 0, abort_flag, tmo, 0x303))) {
@@ -401,6 +491,8 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS>::THREADS, FwdConfig<D, T
       }
       constexpr float kLn2 = 0.69314718055994530942f;
       p.lse[lrow] = (m_ref + log2f(l_sel)) * kLn2;
+      if (EARLY && r == 0 && p.visited != nullptr)
+        p.visited[((static_cast<size_t>(b) * p.Hkv + h) * p.n + i) * (p.G / 2) + slice * T + t] = visited;
       if (MASS) {
         p.lse_full[lrow] = (m_ref + log2f(l_all)) * kLn2;
         p.dropped[lrow] = has_uns ? (l_uns / l_all) : 0.f;

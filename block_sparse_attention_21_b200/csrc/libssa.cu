@@ -176,13 +176,15 @@ ssa_status launch_select(const Dims& d, const ssa::SelectParams& sp, cudaStream_
                     sp);
 }
 
-template <int D, int T, bool MASS>
+// early: the early-stop variant (qbar, kbar, tau, visited are read only then)
+template <int D, int T, bool MASS, bool EARLY = false>
 ssa_status launch_fwd(const Dims& d, const void* q, const void* k, const void* v,
                       const int32_t* idx, void* o, float* lse, void* of, float* lsef,
-                      float* dropped, cudaStream_t st) {
-  using C = ssa::FwdConfig<D, T, MASS>;
+                      float* dropped, cudaStream_t st, const float* qbar = nullptr,
+                      const float* kbar = nullptr, float tau = 0.f, int32_t* visited = nullptr) {
+  using C = ssa::FwdConfig<D, T, MASS, EARLY>;
   static std::atomic<uint64_t> smem_done{0};
-  auto kernel = ssa::attn_fwd_kernel<D, T, MASS>;
+  auto kernel = ssa::attn_fwd_kernel<D, T, MASS, EARLY>;
   ssa_status s = ensure_smem(kernel, C::SMEM_BYTES, &smem_done);
   if (s != SSA_OK) return s;
   CUtensorMap mq, mk, mv;
@@ -206,6 +208,10 @@ ssa_status launch_fwd(const Dims& d, const void* q, const void* k, const void* v
   fp.lse_full = lsef;
   fp.dropped = dropped;
   fp.timeout_ns = wait_timeout_ns();
+  fp.qbar = qbar;
+  fp.kbar = kbar;
+  fp.tau = tau;
+  fp.visited = visited;
   const unsigned grid = static_cast<unsigned>(d.B) * d.Hkv * d.n * fp.slices;
   return launch_pdl(kernel, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, st, mq, mk, mv, fp);
 }
@@ -684,6 +690,31 @@ ssa_status ssa_alignment_bwd(const ssa_problem* p, const ssa_bf16* q, const ssa_
                                              alpha, block_idx, dq, dk, dv, workspace, st)
                   : launch_align_bwd<128, 1>(d, q, k, v, o_sparse, lse_sparse, o_full, lse_full, d_o, mode,
                                              alpha, block_idx, dq, dk, dv, workspace, st);
+}
+
+ssa_status ssa_sparse_attn_fwd_early_stop(const ssa_problem* p, const ssa_bf16* q, const ssa_bf16* k,
+                                          const ssa_bf16* v, const float* q_pooled, const float* k_pooled,
+                                          const int32_t* block_idx, float tau, ssa_bf16* o, float* lse,
+                                          int32_t* visited, ssa_stream stream) {
+  Dims d;
+  ssa_status s = check_problem(p, &d);
+  if (s != SSA_OK) return s;
+  const void* ptrs[] = {q, k, v, q_pooled, k_pooled, block_idx, o, lse};
+  for (const void* ptr : ptrs)
+    if (ptr == nullptr || !aligned16(ptr)) return SSA_ERR_INVALID_ARG;
+  if (visited != nullptr && !aligned16(visited)) return SSA_ERR_INVALID_ARG;
+  if (!(tau >= 0.f) || !std::isfinite(tau)) return SSA_ERR_INVALID_ARG;
+  if (d.topk > ssa::kEarlyMaxTopk) return SSA_ERR_UNSUPPORTED;
+  auto st = reinterpret_cast<cudaStream_t>(stream);
+  if (d.D == 64)
+    return d.G >= 4 ? launch_fwd<64, 2, false, true>(d, q, k, v, block_idx, o, lse, nullptr, nullptr, nullptr, st,
+                                                     q_pooled, k_pooled, tau, visited)
+                    : launch_fwd<64, 1, false, true>(d, q, k, v, block_idx, o, lse, nullptr, nullptr, nullptr, st,
+                                                     q_pooled, k_pooled, tau, visited);
+  return d.G >= 4 ? launch_fwd<128, 2, false, true>(d, q, k, v, block_idx, o, lse, nullptr, nullptr, nullptr, st,
+                                                    q_pooled, k_pooled, tau, visited)
+                  : launch_fwd<128, 1, false, true>(d, q, k, v, block_idx, o, lse, nullptr, nullptr, nullptr, st,
+                                                    q_pooled, k_pooled, tau, visited);
 }
 
 size_t ssa_decode_attn_workspace(const ssa_problem* p) {

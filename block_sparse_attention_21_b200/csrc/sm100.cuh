@@ -119,6 +119,25 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// mbar_wait that also gives up, without an error, once *release is non-zero
+// (another thread decided the phase is no longer needed).  Returns true only
+// if the phase completed.
+__device__ __forceinline__ bool mbar_wait_or(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                             volatile int* release, uint64_t timeout_ns, unsigned int site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag || *release) return false;
+    if (globaltimer_ns() - t0 > timeout_ns) {
+      *abort_flag = 1;
+      atomicOr(&g_error_word, kErrTimeout);
+      atomicExch(&g_error_site, site);
+      return false;
+    }
+  }
+}
+
 // Named barrier among `nthreads` threads (a multiple of 32) of the CTA.
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");

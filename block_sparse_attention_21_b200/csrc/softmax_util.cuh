@@ -17,6 +17,12 @@ struct FwdParams {
   float* lse_full;       // MASS
   float* dropped;        // MASS: dropped attention mass
   uint64_t timeout_ns;
+  // early stop (sparse forward only): the pooled queries and keys that order
+  // the visit, the stop threshold, and the blocks visited per M-tile
+  const float* qbar;     // [B][Hkv][n][D]
+  const float* kbar;     // [B][Hkv][n][D]
+  float tau;
+  int32_t* visited;      // [B][Hkv][n][G / 2], or null
 };
 
 __host__ __device__ constexpr int pow2_at_least(int x) {

@@ -135,6 +135,27 @@ ssa_status ssa_full_attn_fwd_with_mass(const ssa_problem *p, const ssa_bf16 *q,
                                        float *lse_sparse, ssa_bf16 *o_full, float *lse_full,
                                        float *dropped, ssa_stream stream);
 
+/* The sparse forward with an early stop ("S2O" summary, section 2, "Regla de
+ * Parada Temprana", applied to the sparse stream): each query block visits
+ * its diagonal block first, then its other selected blocks in descending
+ * pooled score q_pooled[i] . k_pooled[j] (fp32; ties: lower j), and stops
+ * after the first block that adds, for every query row of the tile, less
+ * than tau times the attention mass the row had accumulated before it (that
+ * block still counts).  A tile is one query block of one pair of query heads
+ * (2 x 64 rows) -- the unit that stops together.  tau = 0 visits every
+ * selected block (the ssa_sparse_attn_fwd result, up to summation order).
+ * q_pooled/k_pooled: the outputs of ssa_block_pool for the same q, k;
+ * block_idx: ssa_block_select's table.  Outputs o, lse as for the sparse
+ * forward, and, if visited is not NULL, the blocks each tile visited,
+ * [B][Hkv][n][G / 2] int32 (head pair p holds query heads h*G + 2p, +1).
+ * Errors: INVALID_ARG for null/misaligned pointers or tau not finite and
+ * >= 0; UNSUPPORTED for top_k > 256 and the cases of the sparse forward. */
+ssa_status ssa_sparse_attn_fwd_early_stop(const ssa_problem *p, const ssa_bf16 *q,
+                                          const ssa_bf16 *k, const ssa_bf16 *v,
+                                          const float *q_pooled, const float *k_pooled,
+                                          const int32_t *block_idx, float tau, ssa_bf16 *o,
+                                          float *lse, int32_t *visited, ssa_stream stream);
+
 /* Bytes of device workspace ssa_sparse_attn_bwd needs for problem p (0 on an
  * invalid problem). */
 size_t ssa_sparse_attn_bwd_workspace(const ssa_problem *p);

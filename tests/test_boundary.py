@@ -79,6 +79,7 @@ def test_bad_problem_is_rejected_by_every_entry_point(lib, kw, code):
     assert lib.ssa_alignment_bwd_workspace(p) == 0
     assert lib.ssa_decode_attn(p, f, f, f, f, f, f, f, None, f, 1 << 30, None) == code
     assert lib.ssa_decode_attn_workspace(p) == 0
+    assert lib.ssa_sparse_attn_fwd_early_stop(p, f, f, f, f, f, f, 0.1, f, f, None, None) == code
 
 
 def test_null_problem(lib):
@@ -130,3 +131,13 @@ def test_decode_arguments_are_checked_before_launch(lib):
     assert lib.ssa_decode_attn(p, f, f, f, f, f, f, f, None, f, ws - 1, None) == WORKSPACE
     assert lib.ssa_decode_attn(p, f, f, f, f, None, f, f, None, f, ws, None) == INVALID
     assert lib.ssa_decode_attn(p, f, f, f, f, f, f, f, f + 4, f, ws, None) == INVALID
+
+
+def test_early_stop_arguments_are_checked_before_launch(lib):
+    p = ctypes.byref(_p())
+    f = FAKE
+    assert lib.ssa_sparse_attn_fwd_early_stop(p, f, f, f, f, f, f, -0.1, f, f, None, None) == INVALID
+    assert lib.ssa_sparse_attn_fwd_early_stop(p, f, f, f, f, f, f, float("nan"), f, f, None, None) == INVALID
+    assert lib.ssa_sparse_attn_fwd_early_stop(p, f, f, f, None, f, f, 0.1, f, f, None, None) == INVALID
+    big = ctypes.byref(_p(top_k=257))
+    assert lib.ssa_sparse_attn_fwd_early_stop(big, f, f, f, f, f, f, 0.1, f, f, None, None) == UNSUPPORTED

@@ -476,3 +476,51 @@ def test_decode_attention_is_masked_softmax_over_the_kept_tokens():
             logits = (k64[b, keep, h] @ q64[b, hq]) / 4.0
             np.testing.assert_allclose(lse[b, hq], np.log(np.exp(logits - logits.max()).sum()) + logits.max(),
                                        atol=1e-12)
+
+
+# -------------------------------------------------------------- early stop
+
+def _early_case(seed):
+    q, k, v = _tiny(B=1, S=512, Hq=4, Hkv=1, D=8, seed=seed)
+    kbar, qbar = oracle.block_pool(k, q)
+    idx, _ = oracle.block_select(qbar, kbar, 5)
+    return q, k, v, qbar, kbar, idx
+
+
+def test_early_stop_with_zero_threshold_is_the_sparse_forward():
+    q, k, v, qbar, kbar, idx = _early_case(111)
+    o, lse, vis, _ = oracle.early_stop_forward(q, k, v, qbar, kbar, idx, 0.0)
+    B, S, Hq, D = q.shape
+    r = oracle.attn_rows(q, k, v, idx, oracle.all_rows(B, Hq, S), want_full=False)
+    np.testing.assert_allclose(o.transpose(0, 2, 1, 3).reshape(-1, D), r["o_sparse"], atol=1e-12)
+    np.testing.assert_allclose(lse.reshape(-1), r["lse_sparse"], atol=1e-12)
+    nsel = (idx >= 0).sum(axis=-1)
+    assert np.array_equal(vis, np.repeat(nsel[..., None], 2, axis=-1))
+
+
+def test_early_stop_with_huge_threshold_keeps_the_diagonal_and_the_best_block():
+    q, k, v, qbar, kbar, idx = _early_case(112)
+    o, _, vis, _ = oracle.early_stop_forward(q, k, v, qbar, kbar, idx, 1e30)
+    B, S, Hq, D = q.shape
+    n = S // BS
+    keep = np.zeros((n, n), dtype=bool)
+    for i in range(n):
+        keep[i, i] = True
+        earlier = [j for j in idx[0, 0, i] if 0 <= j < i]
+        if earlier:
+            keep[i, max(earlier, key=lambda j: (kbar[0, 0, j] @ qbar[0, 0, i], -j))] = True
+        assert vis[0, 0, i, 0] == (2 if earlier else 1)
+    mask = np.repeat(np.repeat(keep, BS, 0), BS, 1) & np.tril(np.ones((S, S), dtype=bool))
+    ref = _sdpa_rows(q, k, v, lambda b, h: mask)
+    np.testing.assert_allclose(o.transpose(0, 2, 1, 3), ref, atol=1e-12)
+
+
+def test_early_stop_visits_fewer_blocks_as_the_threshold_grows():
+    q, k, v, qbar, kbar, idx = _early_case(113)
+    prev = None
+    for tau in (0.0, 0.01, 0.05, 0.2, 1.0):
+        _, _, vis, _ = oracle.early_stop_forward(q, k, v, qbar, kbar, idx, tau)
+        if prev is not None:
+            assert np.all(vis <= prev)
+        prev = vis
+    assert prev.sum() < (idx >= 0).sum() * 2
