@@ -195,19 +195,39 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS, EARLY>::THREADS, FwdConf
       // visiting order: the diagonal block i first, then the other selected
       // blocks (idx_row[0 .. nsel - 2], all below i) by descending pooled score
       // q_pooled[i] . k_pooled[j] in fp32, ties to the lower block
+      // Each lane holds D/32 values of the pooled query; eight rows' dot
+      // products are in flight at once and summed across the warp.
+      constexpr int QV = D / 32;
       const int ne = nsel - 1;
-      const float4* qb = reinterpret_cast<const float4*>(p.qbar + ((static_cast<size_t>(b) * p.Hkv + h) * p.n + i) * D);
-      const float* kb = p.kbar + (static_cast<size_t>(b) * p.Hkv + h) * p.n * D;
-      for (int r = lane; r < ne; r += 32) {
-        const int j = idx_row[r];
-        const float4* kr = reinterpret_cast<const float4*>(kb + static_cast<size_t>(j) * D);
-        float acc = 0.f;
-        for (int d4 = 0; d4 < D / 4; ++d4) {
-          const float4 a = __ldg(qb + d4), c = __ldg(kr + d4);
-          acc = fmaf(a.x, c.x, fmaf(a.y, c.y, fmaf(a.z, c.z, fmaf(a.w, c.w, acc))));
+      const float* qb = p.qbar + ((static_cast<size_t>(b) * p.Hkv + h) * p.n + i) * D + lane * QV;
+      const float* kb = p.kbar + (static_cast<size_t>(b) * p.Hkv + h) * p.n * D + lane * QV;
+      float qf[QV];
+#pragma unroll
+      for (int c = 0; c < QV; ++c) qf[c] = __ldg(qb + c);
+      for (int c0 = 0; c0 < ne; c0 += 32) {
+        const int cnt = min(32, ne - c0);
+        const int jl = lane < cnt ? idx_row[c0 + lane] : 0;
+        if (lane < cnt) ej[c0 + lane] = jl;
+        for (int r = 0; r < cnt; r += 8) {  // r + 7 <= 31
+          float part[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            // clamped: a malformed table entry reads a valid row, not past the buffer
+            const int ju = min(max(__shfl_sync(0xffffffffu, jl, r + u), 0), p.n - 1);
+            const float* kr = kb + static_cast<size_t>(ju) * D;
+            float a = 0.f;
+#pragma unroll
+            for (int c = 0; c < QV; ++c) a = fmaf(qf[c], __ldg(kr + c), a);
+            part[u] = a;
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) part[u] += __shfl_xor_sync(0xffffffffu, part[u], o);
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            if (lane == u && r + u < cnt) esc[c0 + r + u] = part[u];
         }
-        esc[r] = acc;
-        ej[r] = j;
       }
       __syncwarp();
       for (int r = lane; r < ne; r += 32) {

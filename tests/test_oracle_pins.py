@@ -524,3 +524,55 @@ def test_early_stop_visits_fewer_blocks_as_the_threshold_grows():
             assert np.all(vis <= prev)
         prev = vis
     assert prev.sum() < (idx >= 0).sum() * 2
+
+
+@pytest.mark.parametrize("tau", [0.3, 0.8])
+def test_early_stop_matches_a_recomputation_from_prefix_logsumexps(tau):
+    """The stop point from whole-prefix logsumexps (one torch.logsumexp over
+    the union of the earlier blocks' keys, not a running sum) and the output
+    from masked SDPA over the visited blocks."""
+    q, k, v = _tiny(B=1, S=1024, Hq=4, Hkv=1, D=8, seed=114)
+    kbar, qbar = oracle.block_pool(k, q)
+    idx, _ = oracle.block_select(qbar, kbar, 8)
+    o, lse, vis, _ = oracle.early_stop_forward(q, k, v, qbar, kbar, idx, tau)
+    S, Hq, D = q.shape[1], q.shape[2], q.shape[3]
+    n = S // BS
+    causal = torch.tril(torch.ones(S, S, dtype=torch.bool))
+    logits = [(torch.from_numpy(q[0, :, hq]) @ torch.from_numpy(k[0, :, 0]).T) / np.sqrt(D) for hq in range(Hq)]
+    middle = 0
+    for i in range(n):
+        sel = [int(j) for j in idx[0, 0, i] if 0 <= j < i]
+        # descending pooled score, ties to the lower block (lexsort: last key first)
+        sc = np.array([kbar[0, 0, j] @ qbar[0, 0, i] for j in sel])
+        order = [i] + [sel[x] for x in np.lexsort((np.array(sel), -sc))] if sel else [i]
+        rows = slice(BS * i, BS * i + BS)
+        for hp in range(2):
+            heads = (2 * hp, 2 * hp + 1)
+            nv = len(order)
+            for jj in range(1, len(order)):
+                keys_b = torch.zeros(S, dtype=torch.bool)
+                keys_b[BS * order[jj]:BS * order[jj] + BS] = True
+                keys_p = torch.zeros(S, dtype=torch.bool)
+                for j in order[:jj]:
+                    keys_p[BS * j:BS * j + BS] = True
+                ratio = max(float((torch.logsumexp(logits[hq][rows].masked_fill(~(keys_b & causal[rows]), -np.inf), 1)
+                                   - torch.logsumexp(logits[hq][rows].masked_fill(~(keys_p & causal[rows]), -np.inf), 1)
+                                   ).max()) for hq in heads)
+                if ratio < np.log(tau):
+                    nv = jj + 1
+                    break
+            assert vis[0, 0, i, hp] == nv
+            middle += 1 < nv < len(order)
+            keep = torch.zeros(S, dtype=torch.bool)
+            for j in order[:nv]:
+                keep[BS * j:BS * j + BS] = True
+            for hq in heads:
+                m = (keep & causal[rows])[None]
+                ref = F.scaled_dot_product_attention(torch.from_numpy(q[0, rows, hq])[None],
+                                                     torch.from_numpy(k[0, :, 0])[None],
+                                                     torch.from_numpy(v[0, :, 0])[None], attn_mask=m)
+                np.testing.assert_allclose(o[0, rows, hq], ref[0].numpy(), atol=1e-12)
+                np.testing.assert_allclose(lse[0, hq, rows],
+                                           torch.logsumexp(logits[hq][rows].masked_fill(~m[0], -np.inf), 1).numpy(),
+                                           atol=1e-12)
+    assert middle > 0  # some tile stops strictly between its second and last block
