@@ -12,7 +12,7 @@ import torch
 import block_sparse_attention_21_b200 as ssa
 import gen
 import oracle
-from conftest import workload_inputs
+from conftest import oracle_table, workload_inputs
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -75,7 +75,7 @@ def test_backward_small_every_element(shape):
     x = gen.make_custom(B, S, Hq, Hkv, D, topk, seed=300 + S + D, n_plant=npl, with_do=True)
     p = ssa.problem(B, S, Hq, Hkv, D, topk)
     st, dq, dk, dv = _run(x, p, x.do)
-    _check_all(x, x.do, st.block_idx.cpu().numpy(), dq, dk, dv)
+    _check_all(x, x.do, oracle_table(x, topk, st.block_idx), dq, dk, dv)
 
 
 def test_backward_zero_gradient_for_unselected_keys():
@@ -102,7 +102,7 @@ def test_backward_training_workload_sampled_and_deterministic():
     w = x.workload
     p = ssa.problem(w.batch, w.seq_len, w.n_q_heads, w.n_kv_heads, w.head_dim, w.top_k)
     st, dq, dk, dv = _run(x, p, x.do)
-    idx = st.block_idx.cpu().numpy()
+    idx = oracle_table(x, w.top_k, st.block_idx)
     q, k, v = (t.to(DEV) for t in (x.q, x.k, x.v))
     dq2, dk2, dv2 = st.backward(q, k, v, x.do.to(DEV))
     torch.cuda.synchronize()

@@ -14,6 +14,7 @@ import torch
 import block_sparse_attention_21_b200 as ssa
 import gen
 import oracle
+from conftest import oracle_table
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -65,7 +66,7 @@ def _check(case, tau, min_clear=0.6):
     ssa.ssa_sparse_attn_fwd_early_stop(p, q, k, v, st.q_pooled, st.k_pooled, st.block_idx, tau, o, lse, vis)
     torch.cuda.synchronize()
     assert ssa.ssa_get_device_error() == 0
-    gidx = st.block_idx.cpu().numpy()
+    gidx = oracle_table(x, topk, st.block_idx)
     okb, oqb = oracle.block_pool(x.k, x.q)
     ro, rlse, rvis, margin = oracle.early_stop_forward(x.q, x.k, x.v, oqb, okb, gidx, tau)
     gvis = vis.cpu().numpy()

@@ -14,6 +14,7 @@ import torch
 import block_sparse_attention_21_b200 as ssa
 import gen
 import oracle
+from conftest import same_reverse_blocks, same_table_rows
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -70,12 +71,16 @@ def test_long_sequence_forward_and_backward(shape):
         t = np.arange(64 * blk, 64 * blk + 64)
         rows.append(np.stack([np.zeros_like(t), np.zeros_like(t), t], axis=1))
     rows = np.concatenate(rows).astype(np.int64)
-    ref = oracle.attn_rows(x.q, x.k, x.v, gidx, rows, want_full=False)
+    # the oracle works from its own table; rows whose table row differs (a
+    # near-tie at the boundary) are left out
+    same = same_table_rows(rows, gidx, oidx, Hq // Hkv)
+    assert same.mean() > 0.5
+    ref = oracle.attn_rows(x.q, x.k, x.v, oidx, rows, want_full=False)
     r = torch.as_tensor(rows, device=DEV)
     go = st.o[r[:, 0], r[:, 2], r[:, 1]].float().cpu().numpy()
     gl = st.lse[r[:, 0], r[:, 1], r[:, 2]].cpu().numpy()
-    assert np.abs(go - ref["o_sparse"]).max() <= 2e-2
-    assert np.abs(gl - ref["lse_sparse"]).max() <= 1e-3
+    assert np.abs(go - ref["o_sparse"])[same].max() <= 2e-2
+    assert np.abs(gl - ref["lse_sparse"])[same].max() <= 1e-3
 
     # sparse backward: repeatable bit for bit, sampled against the oracle
     dq, dk, dv = (t.clone() for t in st.backward(q, k, v, do))
@@ -85,12 +90,18 @@ def test_long_sequence_forward_and_backward(shape):
     for a, b_ in ((dq, dq2), (dk, dk2), (dv, dv2)):
         assert torch.equal(a.view(torch.int16), b_.view(torch.int16))
     brows = rows[:200]
-    rdq = oracle.sparse_bwd_dq_rows(x.q, x.k, x.v, x.do, gidx, brows)
+    rdq = oracle.sparse_bwd_dq_rows(x.q, x.k, x.v, x.do, oidx, brows)
     gdq = dq[r[:200, 0], r[:200, 2], r[:200, 1]].float().cpu().numpy()
-    assert np.abs(gdq - rdq).max() <= 2e-2 * max(1.0, float(np.abs(rdq).max()))
-    # key block 0 is selected by every early query block: the longest reverse list
-    blocks = np.array([[0, 0, 0], [0, Hkv - 1, n // 3], [0, 0, n - 1]], dtype=np.int64)
-    rdk, rdv = oracle.sparse_bwd_dkv_blocks(x.q, x.k, x.v, x.do, gidx, blocks)
+    bsame = same[:200]
+    assert np.abs(gdq - rdq)[bsame].max() <= 2e-2 * max(1.0, float(np.abs(rdq).max()))
+    # key block 0 is selected by every early query block: the longest reverse
+    # list; blocks whose selecting query blocks differ between the two tables
+    # are left out
+    blocks = np.array([[0, 0, 0], [0, Hkv - 1, n // 3], [0, 0, n - 1], [0, 0, n // 2], [0, 0, 1]],
+                      dtype=np.int64)
+    blocks = blocks[same_reverse_blocks(blocks, gidx, oidx)]
+    assert len(blocks) >= 2
+    rdk, rdv = oracle.sparse_bwd_dkv_blocks(x.q, x.k, x.v, x.do, oidx, blocks)
     for m, (b_, h, j) in enumerate(blocks):
         gk = dk[b_, 64 * j:64 * (j + 1), h].float().cpu().numpy()
         gv = dv[b_, 64 * j:64 * (j + 1), h].float().cpu().numpy()
