@@ -23,6 +23,12 @@ Functions (each cites the passage it follows in ssa_oracle.c):
   early_stop_forward
                   the sparse forward with the early-stop rule (fp64 numpy,
                   small problems)
+  entmax          alpha-entmax of a vector by its threshold (fp64 bisection)
+  dash_route      DashAttention chunk routing: per-head alpha-entmax over the
+                  pooled chunk logits, averaged over the GQA group, and the
+                  bit-packed support
+  dash_attention  DashAttention's prior-induced sparse softmax over the
+                  active chunks (fp64 numpy, small problems)
 """
 from __future__ import annotations
 
@@ -357,3 +363,118 @@ def sparse_forward_problem(q, k, v, topk: int, rows: Optional[np.ndarray] = None
     out = attn_rows(q, k, v, idx, rows, want_full=want_full, nthreads=nthreads)
     out.update(idx=idx, gap=gap, kbar=kbar, qbar=qbar, rows=rows)
     return out
+
+
+# ------------------------------------------------------------- DashAttention
+
+def entmax(z, alpha: float):
+    """alpha-entmax over the last axis, fp64 ("Resumen Tecnico: DashAttention",
+    stage 1: the chunk logits become a sparse probability vector whose support
+    the scores themselves decide).
+
+    alpha-entmax(z) is the maximiser over the simplex of p.z plus the Tsallis
+    alpha-entropy; its solution is p_j = [(alpha - 1) z_j - tau]_+ ^ (1/(alpha - 1))
+    with the one threshold tau that makes the p_j sum to 1.  tau is found by
+    bisection on [max x - 1, max x - m^(1 - alpha)] (x = (alpha - 1) z, m entries)
+    until the bracket stops shrinking; p is then normalised.  1 < alpha.
+    Returns (p, tau) with tau of shape z.shape[:-1]."""
+    if not alpha > 1.0:
+        raise ValueError("alpha-entmax needs alpha > 1")
+    x = (alpha - 1.0) * np.asarray(z, dtype=np.float64)
+    m = x.shape[-1]
+    xmax = x.max(axis=-1, keepdims=True)
+    lo = xmax - 1.0
+    hi = xmax - float(m) ** (1.0 - alpha)
+    inv = 1.0 / (alpha - 1.0)
+    for _ in range(2000):
+        mid = 0.5 * (lo + hi)
+        f = (np.maximum(x - mid, 0.0) ** inv).sum(axis=-1, keepdims=True) - 1.0
+        lo_new = np.where(f >= 0.0, mid, lo)
+        hi_new = np.where(f >= 0.0, hi, mid)
+        if np.array_equal(lo_new, lo) and np.array_equal(hi_new, hi):
+            break
+        lo, hi = lo_new, hi_new
+    tau = 0.5 * (lo + hi)
+    p = np.maximum(x - tau, 0.0) ** inv
+    p = p / p.sum(axis=-1, keepdims=True)
+    return p, tau[..., 0]
+
+
+def dash_route(q, kbar, alpha: float, gamma: float, scale: Optional[float] = None, bs: int = BLOCK):
+    """DashAttention chunk routing, fp64 ("Resumen Tecnico: DashAttention",
+    stage 1, with its GQA rule; chunks of 64 tokens summarised by their mean
+    key, stage 0 at its zero-initialised summary query).
+
+    Per (b, KV head h, query block i) and query head g of the group: the mean
+    query of block i, q_g, scores the complete earlier chunks j < i with
+    z_j = gamma * scale * q_g . kbar[b, h, j]; p_g = alpha-entmax(z); the group
+    shares w = mean_g p_g.  The diagonal chunk i is not routed (its own
+    branch).  Returns
+      w      [B, Hkv, n, n] fp64: w[.., i, j] for j < i, 0 elsewhere
+      mask   [B, Hkv, n, ceil(n / 32)] uint32: bit j of row i set for j < i
+             with w > 0, and bit i (the diagonal) always
+      margin [B, Hkv, n, n]: min over g of |x_gj - tau_g| (x = (alpha-1) z),
+             how far each support decision is from flipping; inf for j >= i."""
+    q64 = widen(q)
+    kbar = np.asarray(kbar, dtype=np.float64)
+    B, S, Hq, D = q64.shape
+    Hkv, n = kbar.shape[1], kbar.shape[2]
+    G = Hq // Hkv
+    scale = (1.0 / np.sqrt(D)) if scale is None else float(scale)
+    W = (n + 31) // 32
+    w = np.zeros((B, Hkv, n, n))
+    mask = np.zeros((B, Hkv, n, W), dtype=np.uint32)
+    margin = np.full((B, Hkv, n, n), np.inf)
+    qpool = q64.reshape(B, n, bs, Hq, D).mean(axis=2)          # [B, n, Hq, D]
+    for b in range(B):
+        for h in range(Hkv):
+            for i in range(n):
+                if i > 0:
+                    qg = qpool[b, i, h * G:(h + 1) * G]            # [G, D]
+                    z = gamma * scale * (qg @ kbar[b, h, :i].T)    # [G, i]
+                    p, tau = entmax(z, alpha)
+                    w[b, h, i, :i] = p.mean(axis=0)
+                    margin[b, h, i, :i] = np.abs((alpha - 1.0) * z - tau[:, None]).min(axis=0)
+                for j in [jj for jj in range(i) if w[b, h, i, jj] > 0] + [i]:
+                    mask[b, h, i, j // 32] |= np.uint32(1 << (j % 32))
+    return w, mask, margin
+
+
+def dash_attention(q, k, v, mask, w, sigma: float, scale: Optional[float] = None, bs: int = BLOCK):
+    """DashAttention's prior-induced sparse softmax, fp64 ("Resumen Tecnico:
+    DashAttention", stage 2).
+
+    The softmax's uniform reference distribution is replaced by a prior g over
+    the keys: g is uniform inside a chunk and proportional to w_j^sigma across
+    the active chunks, and 0 elsewhere, so the attention p maximising
+    z.p - KL(p || g) is p_s proportional to g_s exp(z_s).  For query t of block
+    i the active chunks are the j < i whose mask bit is set and whose w_j > 0,
+    plus the diagonal chunk i with weight 1 (its own branch); causal inside i.
+    Logits are scale * q_t . k_s + sigma * ln w_j.  Returns o [B, S, Hq, D] and
+    lse [B, Hq, S], the natural-log log-sum-exp of the biased logits."""
+    q64, k64, v64 = widen(q), widen(k), widen(v)
+    w = np.asarray(w, dtype=np.float64)
+    mask = np.asarray(mask, dtype=np.uint32)
+    B, S, Hq, D = q64.shape
+    Hkv = k64.shape[2]
+    G, n = Hq // Hkv, S // bs
+    scale = (1.0 / np.sqrt(D)) if scale is None else float(scale)
+    o = np.zeros((B, S, Hq, D))
+    lse = np.zeros((B, Hq, S))
+    tok = np.arange(bs)
+    for b in range(B):
+        for h in range(Hkv):
+            for i in range(n):
+                act = [j for j in range(i)
+                       if (int(mask[b, h, i, j // 32]) >> (j % 32)) & 1 and w[b, h, i, j] > 0]
+                keys = np.concatenate([bs * j + tok for j in act] + [bs * i + tok])
+                bias = np.concatenate([np.full(bs, sigma * np.log(w[b, h, i, j])) for j in act]
+                                      + [np.zeros(bs)])
+                for hq in range(h * G, (h + 1) * G):
+                    lg = scale * (q64[b, bs * i + tok, hq] @ k64[b, keys, h].T) + bias[None, :]
+                    lg[:, -bs:] = np.where(tok[None, :] <= tok[:, None], lg[:, -bs:], -np.inf)
+                    mx = lg.max(axis=1, keepdims=True)
+                    e = np.exp(lg - mx)
+                    lse[b, hq, bs * i + tok] = mx[:, 0] + np.log(e.sum(axis=1))
+                    o[b, bs * i + tok, hq] = (e / e.sum(axis=1, keepdims=True)) @ v64[b, keys, h]
+    return o, lse

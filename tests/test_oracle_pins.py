@@ -576,3 +576,175 @@ def test_early_stop_matches_a_recomputation_from_prefix_logsumexps(tau):
                                            torch.logsumexp(logits[hq][rows].masked_fill(~m[0], -np.inf), 1).numpy(),
                                            atol=1e-12)
     assert middle > 0  # some tile stops strictly between its second and last block
+
+
+# ------------------------------------------------------------ DashAttention
+
+def _sparsemax_by_sorting(z):
+    """Sparsemax (alpha = 2) by the sort-based closed form: the support is the
+    largest k with 1 + k z_(k) > z_(1) + ... + z_(k), tau = (that sum - 1) / k."""
+    zs = np.sort(z)[::-1]
+    cs = np.cumsum(zs)
+    k = max(kk for kk in range(1, len(z) + 1) if 1 + kk * zs[kk - 1] > cs[kk - 1])
+    tau = (cs[k - 1] - 1) / k
+    return np.maximum(z - tau, 0)
+
+
+def _entmax15_by_quadratic(z):
+    """1.5-entmax exactly: with x = z / 2 and support of size k, sum (x_j - tau)^2
+    = 1 is a quadratic in tau, tau_k = mean_k - sqrt((1 - ss_k + k mean_k^2) / k);
+    the support is the largest k with tau_k <= x_(k)."""
+    xs = np.sort(z / 2)[::-1]
+    best = None
+    for kk in range(1, len(z) + 1):
+        mean = xs[:kk].mean()
+        ss = (xs[:kk] ** 2).sum()
+        delta = (1 - ss + kk * mean ** 2) / kk
+        if delta < 0:
+            continue
+        tau = mean - np.sqrt(delta)
+        if tau <= xs[kk - 1]:
+            best = tau
+    return np.maximum(z / 2 - best, 0) ** 2
+
+
+def test_entmax_two_is_sparsemax_and_one_point_five_is_the_exact_quadratic():
+    rng = np.random.default_rng(120)
+    for _ in range(40):
+        z = rng.normal(0, rng.uniform(0.3, 4.0), size=rng.integers(2, 40))
+        np.testing.assert_allclose(oracle.entmax(z, 2.0)[0], _sparsemax_by_sorting(z), atol=1e-12)
+        np.testing.assert_allclose(oracle.entmax(z, 1.5)[0], _entmax15_by_quadratic(z), atol=1e-12)
+
+
+@pytest.mark.parametrize("alpha", [1.25, 1.5, 1.75, 2.0, 3.0])
+def test_entmax_satisfies_its_optimality_conditions(alpha):
+    # on the support p_j^(alpha-1) - (alpha-1) z_j is one constant (-tau); off
+    # it (alpha-1) z_j <= tau; the p sum to 1; shifting z changes nothing
+    rng = np.random.default_rng(121)
+    z = rng.normal(0, 2.0, size=(30, 25))
+    p, tau = oracle.entmax(z, alpha)
+    np.testing.assert_allclose(p.sum(axis=1), 1.0, atol=1e-12)
+    x = (alpha - 1) * z
+    for r in range(30):
+        s = p[r] > 0
+        np.testing.assert_allclose(p[r, s] ** (alpha - 1) - x[r, s], -tau[r], atol=1e-9)
+        assert np.all(x[r, ~s] <= tau[r] + 1e-9)
+    np.testing.assert_allclose(oracle.entmax(z + 3.7, alpha)[0], p, atol=1e-10)
+
+
+def test_entmax_tends_to_softmax_as_alpha_tends_to_one():
+    z = np.random.default_rng(122).normal(0, 1.0, size=(5, 12))
+    sm = np.exp(z) / np.exp(z).sum(axis=1, keepdims=True)
+    np.testing.assert_allclose(oracle.entmax(z, 1.0005)[0], sm, atol=2e-3)
+
+
+def _dash_case(seed, S=512, Hq=4, Hkv=2, D=16):
+    q, k, v = _tiny(B=1, S=S, Hq=Hq, Hkv=Hkv, D=D, seed=seed)
+    kbar, _ = oracle.block_pool(k, q)
+    return q, k, v, kbar
+
+
+def _bit(mask, b, h, i, j):
+    return (int(mask[b, h, i, j // 32]) >> (j % 32)) & 1
+
+
+def test_dash_route_extremes_of_gamma():
+    q, k, v, kbar = _dash_case(123)
+    B, S, Hq, D = q.shape
+    Hkv, n, G = kbar.shape[1], S // BS, Hq // kbar.shape[1]
+    # gamma -> 0: every head is uniform over the earlier chunks
+    w, mask, _ = oracle.dash_route(q, kbar, 1.5, 1e-9)
+    for h in range(Hkv):
+        for i in range(n):
+            np.testing.assert_allclose(w[0, h, i, :i], 1.0 / max(i, 1), atol=1e-9)
+            assert all(_bit(mask, 0, h, i, j) == (j <= i) for j in range(n))
+    # gamma -> inf: every head keeps only its best chunk; the group mean counts heads
+    w, mask, _ = oracle.dash_route(q, kbar, 1.5, 1e6)
+    for h in range(Hkv):
+        for i in range(1, n):
+            want = np.zeros(n)
+            for g in range(G):
+                qm = np.array([[float(x) for x in q[0, BS * i + t, h * G + g]] for t in range(BS)]).mean(axis=0)
+                want[int(np.argmax([qm @ kbar[0, h, j] for j in range(i)]))] += 1.0 / G
+            np.testing.assert_allclose(w[0, h, i], want, atol=1e-9)
+            assert all(_bit(mask, 0, h, i, j) == (want[j] > 0 or j == i) for j in range(n))
+
+
+def _dash_routing_with_oddities(n, Hkv, seed):
+    """Random support with set bits at w = 0, bits at and after the diagonal,
+    and cleared diagonal bits."""
+    rng = np.random.default_rng(seed)
+    W = (n + 31) // 32
+    w = rng.uniform(0.01, 1.0, size=(1, Hkv, n, n)) * (rng.random((1, Hkv, n, n)) < 0.7)
+    mask = np.zeros((1, Hkv, n, W), dtype=np.uint32)
+    for h in range(Hkv):
+        for i in range(n):
+            for j in range(n):
+                if rng.random() < 0.5:
+                    mask[0, h, i, j // 32] |= np.uint32(1 << (j % 32))
+    return w, mask
+
+
+def test_dash_attention_with_sigma_zero_is_masked_attention_over_the_active_chunks():
+    q, k, v, _ = _dash_case(124)
+    B, S, Hq, D = q.shape
+    Hkv, n, G = k.shape[2], S // BS, Hq // k.shape[2]
+    w, mask = _dash_routing_with_oddities(n, Hkv, 125)
+    o, lse = oracle.dash_attention(q, k, v, mask, w, 0.0)
+    q64, k64 = q.astype(np.float64), k.astype(np.float64)
+
+    def keep(b, h):
+        m = np.zeros((S, S), dtype=bool)
+        for i in range(n):
+            cols = np.zeros(S, dtype=bool)
+            for j in range(i):
+                if _bit(mask, b, h, i, j) and w[b, h, i, j] > 0:
+                    cols[BS * j:BS * j + BS] = True
+            cols[BS * i:BS * i + BS] = True
+            m[BS * i:BS * i + BS] = cols[None, :]
+        return m & np.tril(np.ones((S, S), dtype=bool))
+
+    ref = _sdpa_rows(q, k, v, keep)
+    np.testing.assert_allclose(o.transpose(0, 2, 1, 3), ref, atol=1e-12)
+    for hq in range(Hq):
+        m = torch.from_numpy(keep(0, hq // G))
+        lg = torch.from_numpy(q64[0, :, hq] @ k64[0, :, hq // G].T) / np.sqrt(D)
+        np.testing.assert_allclose(lse[0, hq], torch.logsumexp(lg.masked_fill(~m, -np.inf), 1).numpy(),
+                                   atol=1e-12)
+
+
+def test_dash_attention_maximises_score_minus_kl_to_the_prior():
+    # one-hot values read the attention rows out; each row must maximise
+    # F(p) = z.p - KL(p || g) over the simplex on g's support, with g uniform
+    # inside a chunk and proportional to w^sigma across chunks
+    S, D, sigma = 256, 256, 0.7
+    rng = np.random.default_rng(126)
+    q = rng.normal(0, 1, (1, S, 1, D)).astype(np.float32)
+    k = rng.normal(0, 1, (1, S, 1, D)).astype(np.float32)
+    v = np.eye(S, dtype=np.float32)[None, :, None, :]
+    n = S // BS
+    w, mask = _dash_routing_with_oddities(n, 1, 127)
+    o, _ = oracle.dash_attention(q, k, v, mask, w, sigma)
+    q64, k64 = q.astype(np.float64), k.astype(np.float64)
+    for t in (0, 70, 130, 200, 255):
+        i = t // BS
+        g = np.zeros(S)
+        for j in range(i):
+            if _bit(mask, 0, 0, i, j) and w[0, 0, i, j] > 0:
+                g[BS * j:BS * j + BS] = w[0, 0, i, j] ** sigma
+        g[BS * i:t + 1] = 1.0
+        g /= g.sum()
+        sup = g > 0
+        z = (q64[0, t, 0] @ k64[0, :, 0].T) / np.sqrt(D)
+        p = o[0, t, 0]
+        assert np.all(p[~sup] == 0) and abs(p.sum() - 1) < 1e-12
+
+        def F(pp):
+            return float(z[sup] @ pp[sup] - (pp[sup] * np.log(pp[sup] / g[sup])).sum())
+        best = F(p)
+        for _ in range(20):
+            d = np.zeros(S)
+            d[sup] = rng.normal(0, 1, sup.sum())
+            d[sup] -= d[sup].mean()
+            eps = 0.2 * p[sup].min() / (np.abs(d).max() + 1e-30)
+            assert F(p + eps * d) <= best + 1e-12
