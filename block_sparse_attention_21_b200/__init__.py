@@ -13,6 +13,7 @@ import torch
 
 from ._binding import (EXPORTED, LIB_PATH, SsaError, SsaProblem, lib, problem,
                        ssa_alignment_bwd, ssa_alignment_bwd_workspace, ssa_decode_attn,
+                       ssa_dash_attn_fwd, ssa_dash_route,
                        ssa_decode_attn_workspace, ssa_sparse_attn_fwd_early_stop,
                        ssa_block_pool, ssa_block_select, ssa_debug_exp2_poly, ssa_debug_timeout_probe,
                        ssa_full_attn_fwd_with_mass, ssa_get_device_error,
@@ -21,7 +22,8 @@ from ._binding import (EXPORTED, LIB_PATH, SsaError, SsaProblem, lib, problem,
                        ssa_sparse_attn_bwd_workspace,
                        ssa_sparse_attn_fwd, ssa_status_string)
 
-__all__ = ["EXPORTED", "LIB_PATH", "SsaError", "SsaProblem", "SparseStream", "lib", "problem",
+__all__ = ["EXPORTED", "LIB_PATH", "DashAttention", "SsaError", "SsaProblem", "SparseStream", "lib", "problem",
+           "ssa_dash_attn_fwd", "ssa_dash_route",
            "ssa_alignment_bwd", "ssa_alignment_bwd_workspace", "ssa_decode_attn",
            "ssa_decode_attn_workspace", "ssa_sparse_attn_fwd_early_stop",
            "ssa_block_pool", "ssa_block_select", "ssa_debug_exp2_poly", "ssa_debug_timeout_probe",
@@ -114,3 +116,32 @@ class SparseStream:
         ssa_alignment_bwd(self.p, q, k, v, self.o, self.lse, o_full, lse_full, d_o, mode, alpha,
                           self.block_idx, dq, dk, dv, workspace, workspace.numel(), stream)
         return dq, dk, dv
+
+
+class DashAttention:
+    """DashAttention's forward over buffers allocated once: the chunk summaries
+    (ssa_block_pool, keys only), the routing (ssa_dash_route) and the
+    prior-induced sparse softmax (ssa_dash_attn_fwd).  alpha: the entmax
+    exponent; gamma: the routing temperature; sigma: the prior's strength."""
+
+    def __init__(self, p: SsaProblem, alpha: float = 1.5, gamma: float = 1.0, sigma: float = 1.0,
+                 device: Optional[torch.device] = None):
+        lib()
+        self.p, self.alpha, self.gamma, self.sigma = p, float(alpha), float(gamma), float(sigma)
+        dev = device or torch.device("cuda")
+        B, S, Hq, Hkv, D = p.batch, p.seq_len, p.n_q_heads, p.n_kv_heads, p.head_dim
+        n = S // 64
+        self.k_pooled = torch.empty(B, Hkv, n, D, dtype=torch.float32, device=dev)
+        self.weights = torch.empty(B, Hkv, n, n, dtype=torch.float32, device=dev)
+        self.mask = torch.empty(B, Hkv, n, (n + 31) // 32, dtype=torch.int32, device=dev)
+        self.o = torch.empty(B, S, Hq, D, dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty(B, Hq, S, dtype=torch.float32, device=dev)
+
+    def route(self, q, k, stream=None):
+        ssa_block_pool(self.p, k, None, self.k_pooled, None, stream)
+        ssa_dash_route(self.p, q, self.k_pooled, self.alpha, self.gamma, self.weights, self.mask, stream)
+
+    def forward(self, q, k, v, stream=None):
+        self.route(q, k, stream)
+        ssa_dash_attn_fwd(self.p, q, k, v, self.weights, self.mask, self.sigma, self.o, self.lse, stream)
+        return self.o, self.lse

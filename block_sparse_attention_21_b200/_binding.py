@@ -27,6 +27,7 @@ EXPORTED = ("ssa_block_pool", "ssa_block_select", "ssa_sparse_attn_fwd", "ssa_sp
             "ssa_full_attn_fwd_with_mass", "ssa_sparse_attn_bwd_workspace",
             "ssa_sparse_attn_bwd", "ssa_sparse_attn_bwd_noalloc", "ssa_alignment_bwd_workspace",
             "ssa_alignment_bwd", "ssa_decode_attn_workspace", "ssa_decode_attn",
+            "ssa_dash_route", "ssa_dash_attn_fwd",
             "ssa_get_device_error",
             "ssa_get_device_error_site",
             "ssa_debug_timeout_probe", "ssa_debug_exp2_poly",
@@ -76,6 +77,8 @@ def lib():
             "ssa_sparse_attn_fwd_early_stop": [P] + [vp] * 6 + [ctypes.c_float] + [vp] * 4,
             "ssa_alignment_bwd": [P] + [vp] * 8 + [ctypes.c_int, ctypes.c_float] + [vp] * 5
                                  + [ctypes.c_size_t, vp],
+            "ssa_dash_route": [P, vp, vp, ctypes.c_float, ctypes.c_float, vp, vp, vp],
+            "ssa_dash_attn_fwd": [P] + [vp] * 5 + [ctypes.c_float] + [vp] * 3,
             "ssa_get_device_error": [vp],
             "ssa_debug_timeout_probe": [ctypes.c_int, vp],
             "ssa_debug_exp2_poly": [vp, vp, ctypes.c_int, vp],
@@ -242,6 +245,40 @@ def ssa_sparse_attn_fwd_early_stop(p: SsaProblem, q, k, v, q_pooled, k_pooled, b
           _ptr(v, BF16, "v"), _ptr(q_pooled, F32, "q_pooled"), _ptr(k_pooled, F32, "k_pooled"),
           _ptr(block_idx, I32, "block_idx"), float(tau), _ptr(o, BF16, "o"), _ptr(lse, F32, "lse"),
           _ptr(visited, I32, "visited"), _stream(stream))
+
+
+def _mask_ptr(t, name: str) -> int:
+    """Bit masks travel as int32 or uint32 tensors (the same 32 bits)."""
+    if t is None or t.dtype not in (I32, getattr(torch, "uint32", I32)):
+        raise ValueError(f"{name}: expected an int32 (or uint32) CUDA tensor")
+    return _ptr(t, None, name)
+
+
+def ssa_dash_route(p: SsaProblem, q, k_pooled, alpha: float, gamma: float, weights, mask,
+                   stream=None) -> None:
+    """DashAttention chunk routing: per-head alpha-entmax over the pooled chunk
+    logits, averaged over the GQA group, and the bit-packed support; see
+    include/ssa.h."""
+    sh = _shapes(p)
+    B, Hkv, n, _ = sh["idx"]
+    for t, s, nm in ((q, sh["q"], "q"), (k_pooled, sh["pooled"], "k_pooled"), (weights, (B, Hkv, n, n), "weights"),
+                     (mask, (B, Hkv, n, (n + 31) // 32), "mask")):
+        _numel_check(t, s, nm)
+    _call("ssa_dash_route", ctypes.byref(p), _ptr(q, BF16, "q"), _ptr(k_pooled, F32, "k_pooled"), float(alpha),
+          float(gamma), _ptr(weights, F32, "weights"), _mask_ptr(mask, "mask"), _stream(stream))
+
+
+def ssa_dash_attn_fwd(p: SsaProblem, q, k, v, weights, mask, sigma: float, o, lse, stream=None) -> None:
+    """DashAttention's prior-induced sparse softmax over the routed chunks and
+    the diagonal; see include/ssa.h."""
+    sh = _shapes(p)
+    B, Hkv, n, _ = sh["idx"]
+    for t, s, nm in ((q, sh["q"], "q"), (k, sh["kv"], "k"), (v, sh["kv"], "v"), (weights, (B, Hkv, n, n), "weights"),
+                     (mask, (B, Hkv, n, (n + 31) // 32), "mask"), (o, sh["q"], "o"), (lse, sh["lse"], "lse")):
+        _numel_check(t, s, nm)
+    _call("ssa_dash_attn_fwd", ctypes.byref(p), _ptr(q, BF16, "q"), _ptr(k, BF16, "k"), _ptr(v, BF16, "v"),
+          _ptr(weights, F32, "weights"), _mask_ptr(mask, "mask"), float(sigma), _ptr(o, BF16, "o"),
+          _ptr(lse, F32, "lse"), _stream(stream))
 
 
 def ssa_decode_attn_workspace(p: SsaProblem) -> int:

@@ -53,7 +53,7 @@ namespace ssa {
 // 1 KB selection-bitmap area).
 constexpr int kEarlyMaxTopk = 256;
 
-template <int D, int T, bool MASS, bool EARLY = false>
+template <int D, int T, bool MASS, bool EARLY = false, bool DASH = false>
 struct FwdConfig {
   static constexpr int NP = D / 64;               // 64-column panels per row
   static constexpr int QTILE = 128 * D * 2;       // bytes of one Q M-tile
@@ -68,20 +68,24 @@ struct FwdConfig {
   // shared memory: Q tiles, K ring, V ring, barriers, tmem slot, abort flag,
   // selection bitmap (up to 8192 blocks)
   static constexpr int SMEM_TILES = T * QTILE + 2 * NS * KVT;
-  // EARLY: 2 KB of score scratch and 128 B of stop flags after the bitmap area
-  static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + NBARS * 8 + 16 + 1024 + (EARLY ? 2048 + 128 : 0);
+  // EARLY: 2 KB of score scratch and 128 B of stop flags after the bitmap area;
+  // DASH: the routed chunk list and its biases (kDashMaxN each) and the count
+  static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + NBARS * 8 + 16 + 1024 + (EARLY ? 2048 + 128 : 0) +
+                                    (DASH ? 8 * kDashMaxN + 16 : 0);
   // two CTAs share an SM when both fit in TMEM (256 columns each) and in
   // shared memory: one CTA's prologue and epilogue overlap the other's loop
   static constexpr int MIN_CTAS = (TMEM_COLS <= 256 && SMEM_BYTES <= 113 * 1024) ? 2 : 1;
   static_assert(T * TSTRIDE <= 512, "TMEM budget");
 };
 
-template <int D, int T, bool MASS, bool EARLY = false>
-__global__ void __launch_bounds__(FwdConfig<D, T, MASS, EARLY>::THREADS, FwdConfig<D, T, MASS, EARLY>::MIN_CTAS)
+template <int D, int T, bool MASS, bool EARLY = false, bool DASH = false>
+__global__ void __launch_bounds__(FwdConfig<D, T, MASS, EARLY, DASH>::THREADS,
+                                  FwdConfig<D, T, MASS, EARLY, DASH>::MIN_CTAS)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using C = FwdConfig<D, T, MASS, EARLY>;
+  using C = FwdConfig<D, T, MASS, EARLY, DASH>;
   static_assert(!(MASS && EARLY), "the early stop applies to the sparse stream only");
+  static_assert(!(DASH && (MASS || EARLY)), "the routed softmax is a mode of its own");
   constexpr int NP = C::NP, QTILE = C::QTILE, KVT = C::KVT, NS = C::NS, TSTRIDE = C::TSTRIDE;
 
   extern __shared__ uint8_t smem_raw[];
@@ -110,6 +114,11 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS, EARLY>::THREADS, FwdConf
   volatile int* all_stop = reinterpret_cast<volatile int*>(ej + 256);
   volatile int* tile_stop = all_stop + 1;                     // [T]
   volatile int* wflag = all_stop + 4;                         // [T][2][4]
+  // DASH: routed chunks in ascending order then the diagonal, their biases
+  // (sigma * log2 w, in the exp2 domain of the scores), and their count
+  int32_t* dord = reinterpret_cast<int32_t*>(selbits + 256);
+  float* dbias = reinterpret_cast<float*>(dord + kDashMaxN);
+  int* dcount = reinterpret_cast<int*>(dbias + kDashMaxN);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
@@ -123,7 +132,7 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS, EARLY>::THREADS, FwdConf
   const int b = rem / p.Hkv;
   const int hq0 = h * p.G + slice * 2 * T;
   const int nsel = min(p.topk, i + 1);
-  const int nblk = MASS ? (i + 1) : nsel;
+  int nblk = MASS ? (i + 1) : nsel;  // DASH: the routed count, known after the prologue
   const int32_t* idx_row = p.idx + ((static_cast<size_t>(b) * p.Hkv + h) * p.n + i) * p.topk;
 
   if (threadIdx.x == 0) {
@@ -155,6 +164,7 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS, EARLY>::THREADS, FwdConf
       if (j >= 0 && j <= i) atomicOr(&selbits[j >> 5], 1u << (j & 31));
     }
   }
+  if (DASH && warp == 0) dash_build_list(p, b, h, i, lane, dord, dbias, dcount);
   if (EARLY && threadIdx.x == 0) {
     *all_stop = 0;
     for (int t = 0; t < T; ++t) tile_stop[t] = 0;
@@ -168,6 +178,7 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS, EARLY>::THREADS, FwdConf
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint64_t tmo = p.timeout_ns;
+  if (DASH) nblk = *dcount;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -250,7 +261,7 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS, EARLY>::THREADS, FwdConf
         if (use > 0 && !(EARLY ? mbar_wait_or(&bar_empty[st], (use - 1) & 1, abort_flag, all_stop, tmo, 0x101)
                                : mbar_wait(&bar_empty[st], (use - 1) & 1, abort_flag, tmo, 0x101)))
           break;
-        load_kv(st, MASS ? jj : (EARLY ? ord[jj] : idx_row[jj]));
+        load_kv(st, MASS ? jj : (EARLY ? ord[jj] : (DASH ? dord[jj] : idx_row[jj])));
         ++issued;
       }
       // on abort or an early stop, loads already issued are waited for
@@ -406,14 +417,16 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS, EARLY>::THREADS, FwdConf
       float mx = diag ? row_max32<true>(sv + 32, 32, tq, -INFINITY)
                       : row_max32<false>(sv + 32, 32, tq, -INFINITY);
       mx = diag ? row_max32<true>(sv, 0, tq, mx) : row_max32<false>(sv, 0, tq, mx);
-      const float mx_s = mx * sl2;
+      // DASH: the chunk's prior adds sigma * log2 w_j to every score of the block
+      const float bias = DASH ? dbias[jj] : 0.f;
+      const float mx_s = mx * sl2 + bias;
       float alpha = 1.f;
       const bool moved = mx_s > m_ref + 8.f;
       if (moved) {
         alpha = ex2(m_ref - mx_s);
         m_ref = mx_s;
       }
-      const uint64_t negm2 = f2_pack(-m_ref, -m_ref);
+      const uint64_t negm2 = f2_pack(bias - m_ref, bias - m_ref);
       uint64_t acc2 = f2_pack(0.f, 0.f);
       uint32_t pk[16];
       if (diag) exp_pack32<true>(sv, 0, tq, scale2, negm2, acc2, pk);

@@ -46,7 +46,7 @@
 
 namespace ssa {
 
-template <int D, int T, bool MASS>
+template <int D, int T, bool MASS, bool DASH = false>
 struct PsFwdConfig {
   static constexpr int NP = D / 64;               // 64-column panels per row
   static constexpr int QTILE = 128 * D * 2;       // bytes of one Q M-tile
@@ -62,9 +62,10 @@ struct PsFwdConfig {
   // barriers: q, kfull/vfull/empty[NS], sfull/sfree/pfull/pvdone/odone/drain[T]
   static constexpr int NBARS = 1 + 3 * NS + 7 * T;
   // shared memory: Q tiles, K ring, V ring, P tiles, barriers, tmem slot,
-  // abort flag, selection bitmap (up to 8192 blocks)
+  // abort flag, selection bitmap (up to 8192 blocks); DASH: the routed chunk
+  // list and its biases (kDashMaxN each) and the count
   static constexpr int SMEM_TILES = T * QTILE + 2 * NS * KVT + T * PTILE;
-  static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + NBARS * 8 + 16 + 1024;
+  static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + NBARS * 8 + 16 + 1024 + (DASH ? 8 * kDashMaxN + 16 : 0);
   static_assert(T * TSTRIDE <= 512, "TMEM budget");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
@@ -75,11 +76,12 @@ __device__ __forceinline__ int ps_issuer_warp(int t) {
   return t < 3 ? 1 + t : 4 + 4 * T;
 }
 
-template <int D, int T, bool MASS>
-__global__ void __launch_bounds__(PsFwdConfig<D, T, MASS>::THREADS, 1)
+template <int D, int T, bool MASS, bool DASH = false>
+__global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH>::THREADS, 1)
     attn_fwd_psmem_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using C = PsFwdConfig<D, T, MASS>;
+  using C = PsFwdConfig<D, T, MASS, DASH>;
+  static_assert(!(MASS && DASH), "the routed softmax is a mode of its own");
   constexpr int NP = C::NP, QTILE = C::QTILE, KVT = C::KVT, PTILE = C::PTILE, NS = C::NS,
                 TSTRIDE = C::TSTRIDE;
 
@@ -105,6 +107,11 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS>::THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_turn + T);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint32_t* selbits = tmem_slot + 4;
+  // DASH: routed chunks in ascending order then the diagonal, their biases
+  // (sigma * log2 w, in the exp2 domain of the scores), and their count
+  int32_t* dord = reinterpret_cast<int32_t*>(selbits + 256);
+  float* dbias = reinterpret_cast<float*>(dord + kDashMaxN);
+  int* dcount = reinterpret_cast<int*>(dbias + kDashMaxN);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
@@ -118,7 +125,7 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS>::THREADS, 1)
   const int b = rem / p.Hkv;
   const int hq0 = h * p.G + slice * 2 * T;
   const int nsel = min(p.topk, i + 1);
-  const int nblk = MASS ? (i + 1) : nsel;
+  int nblk = MASS ? (i + 1) : nsel;  // DASH: the routed count, known after the prologue
   const int32_t* idx_row = p.idx + ((static_cast<size_t>(b) * p.Hkv + h) * p.n + i) * p.topk;
 
   if (threadIdx.x == 0) {
@@ -152,6 +159,7 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS>::THREADS, 1)
       if (j >= 0 && j <= i) atomicOr(&selbits[j >> 5], 1u << (j & 31));
     }
   }
+  if (DASH && warp == 2) dash_build_list(p, b, h, i, lane, dord, dbias, dcount);
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
@@ -161,6 +169,7 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS>::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint64_t tmo = p.timeout_ns;
+  if (DASH) nblk = *dcount;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -178,7 +187,7 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS>::THREADS, 1)
       for (int jj = 0; jj < nblk; ++jj) {
         const int st = jj % NS, use = jj / NS;
         if (use > 0 && !mbar_wait(&bar_empty[st], (use - 1) & 1, abort_flag, tmo, 0x101)) break;
-        const int j = MASS ? jj : idx_row[jj];
+        const int j = MASS ? jj : (DASH ? dord[jj] : idx_row[jj]);
         mbar_arrive_expect_tx(&bar_kfull[st], KVT);
         for (int pn = 0; pn < NP; ++pn)
           tma_load_4d(sK + st * KVT + pn * (64 * 128), &tm_k, &bar_kfull[st], 64 * pn, h, 64 * j, b);
@@ -313,14 +322,16 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS>::THREADS, 1)
       }
       float mx = diag ? row_max32<true>(sB, 32, tq, -INFINITY) : row_max32<false>(sB, 32, tq, -INFINITY);
       mx = diag ? row_max32<true>(sA, 0, tq, mx) : row_max32<false>(sA, 0, tq, mx);
-      const float mx_s = mx * sl2;
+      // DASH: the chunk's prior adds sigma * log2 w_j to every score of the block
+      const float bias = DASH ? dbias[jj] : 0.f;
+      const float mx_s = mx * sl2 + bias;
       float alpha = 1.f;
       const bool moved = mx_s > m_ref + 8.f;
       if (moved) {
         alpha = ex2(m_ref - mx_s);
         m_ref = mx_s;
       }
-      const uint64_t negm2 = f2_pack(-m_ref, -m_ref);
+      const uint64_t negm2 = f2_pack(bias - m_ref, bias - m_ref);
       uint64_t acc2 = f2_pack(0.f, 0.f);
       uint32_t pk[32];
       if (diag) {

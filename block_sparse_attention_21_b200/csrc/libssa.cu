@@ -19,6 +19,7 @@
 #include "attn_bwd.cuh"
 #include "align_bwd.cuh"
 #include "decode.cuh"
+#include "dash.cuh"
 
 namespace {
 
@@ -176,15 +177,24 @@ ssa_status launch_select(const Dims& d, const ssa::SelectParams& sp, cudaStream_
                     sp);
 }
 
-// early: the early-stop variant (qbar, kbar, tau, visited are read only then)
-template <int D, int T, bool MASS, bool EARLY = false>
+// Inputs of the routed (DashAttention) mode of the forward kernels.
+struct DashIn {
+  const uint32_t* mask = nullptr;
+  const float* w = nullptr;
+  float sigma = 0.f;
+};
+
+// EARLY: the early-stop variant (qbar, kbar, tau, visited are read only then);
+// DASH: the routed softmax (dash is read only then)
+template <int D, int T, bool MASS, bool EARLY = false, bool DASH = false>
 ssa_status launch_fwd(const Dims& d, const void* q, const void* k, const void* v,
                       const int32_t* idx, void* o, float* lse, void* of, float* lsef,
                       float* dropped, cudaStream_t st, const float* qbar = nullptr,
-                      const float* kbar = nullptr, float tau = 0.f, int32_t* visited = nullptr) {
-  using C = ssa::FwdConfig<D, T, MASS, EARLY>;
+                      const float* kbar = nullptr, float tau = 0.f, int32_t* visited = nullptr,
+                      DashIn dash = DashIn()) {
+  using C = ssa::FwdConfig<D, T, MASS, EARLY, DASH>;
   static std::atomic<uint64_t> smem_done{0};
-  auto kernel = ssa::attn_fwd_kernel<D, T, MASS, EARLY>;
+  auto kernel = ssa::attn_fwd_kernel<D, T, MASS, EARLY, DASH>;
   ssa_status s = ensure_smem(kernel, C::SMEM_BYTES, &smem_done);
   if (s != SSA_OK) return s;
   CUtensorMap mq, mk, mv;
@@ -212,18 +222,21 @@ ssa_status launch_fwd(const Dims& d, const void* q, const void* k, const void* v
   fp.kbar = kbar;
   fp.tau = tau;
   fp.visited = visited;
+  fp.dmask = dash.mask;
+  fp.dw = dash.w;
+  fp.sigma = dash.sigma;
   const unsigned grid = static_cast<unsigned>(d.B) * d.Hkv * d.n * fp.slices;
   return launch_pdl(kernel, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, st, mq, mk, mv, fp);
 }
 
 // The same launch for the kernel that stages P in shared memory.
-template <int D, int T, bool MASS>
+template <int D, int T, bool MASS, bool DASH = false>
 ssa_status launch_psfwd(const Dims& d, const void* q, const void* k, const void* v,
                       const int32_t* idx, void* o, float* lse, void* of, float* lsef,
-                      float* dropped, cudaStream_t st) {
-  using C = ssa::PsFwdConfig<D, T, MASS>;
+                      float* dropped, cudaStream_t st, DashIn dash = DashIn()) {
+  using C = ssa::PsFwdConfig<D, T, MASS, DASH>;
   static std::atomic<uint64_t> smem_done{0};
-  auto kernel = ssa::attn_fwd_psmem_kernel<D, T, MASS>;
+  auto kernel = ssa::attn_fwd_psmem_kernel<D, T, MASS, DASH>;
   ssa_status s = ensure_smem(kernel, C::SMEM_BYTES, &smem_done);
   if (s != SSA_OK) return s;
   CUtensorMap mq, mk, mv;
@@ -247,8 +260,44 @@ ssa_status launch_psfwd(const Dims& d, const void* q, const void* k, const void*
   fp.lse_full = lsef;
   fp.dropped = dropped;
   fp.timeout_ns = wait_timeout_ns();
+  fp.qbar = nullptr;
+  fp.kbar = nullptr;
+  fp.tau = 0.f;
+  fp.visited = nullptr;
+  fp.dmask = dash.mask;
+  fp.dw = dash.w;
+  fp.sigma = dash.sigma;
   const unsigned grid = static_cast<unsigned>(d.B) * d.Hkv * d.n * fp.slices;
   return launch_pdl(kernel, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, st, mq, mk, mv, fp);
+}
+
+// ------------------------------------------------------- DashAttention route
+
+template <int D>
+ssa_status launch_dash_route(const Dims& d, const void* q, const float* kbar, float alpha, float gamma,
+                             float* w, uint32_t* mask, cudaStream_t st) {
+  static std::atomic<uint64_t> done{0};
+  auto kernel = ssa::dash_route_kernel<D>;
+  const ssa_status s =
+      ensure_smem(kernel, static_cast<int>(ssa::dash_route_smem(ssa::kDashMaxG, 128, ssa::kDashMaxN)), &done);
+  if (s != SSA_OK) return s;
+  ssa::DashRouteParams rp;
+  rp.B = d.B;
+  rp.S = d.S;
+  rp.Hq = d.Hq;
+  rp.Hkv = d.Hkv;
+  rp.G = d.G;
+  rp.n = d.n;
+  rp.W = (d.n + 31) / 32;
+  rp.am1 = alpha - 1.f;
+  rp.inv_am1 = 1.f / (alpha - 1.f);
+  rp.pw_mode = alpha == 1.5f ? 0 : (alpha == 2.f ? 1 : 2);
+  rp.zscale = gamma * d.scale;
+  rp.q = static_cast<const __nv_bfloat16*>(q);
+  rp.kbar = kbar;
+  rp.w = w;
+  rp.mask = mask;
+  return launch_pdl(kernel, dim3(d.n, d.Hkv, d.B), dim3(256), ssa::dash_route_smem(d.G, D, d.n), st, rp);
 }
 
 // ---------------------------------------------------------------- backward
@@ -739,6 +788,50 @@ ssa_status ssa_decode_attn(const ssa_problem* p, const ssa_bf16* q, const ssa_bf
   auto st = reinterpret_cast<cudaStream_t>(stream);
   return d.D == 64 ? launch_decode<64>(d, q, k_cache, v_cache, k_pooled, lengths, o, lse, block_idx, workspace, st)
                    : launch_decode<128>(d, q, k_cache, v_cache, k_pooled, lengths, o, lse, block_idx, workspace, st);
+}
+
+// ------------------------------------------------------------ DashAttention
+
+ssa_status ssa_dash_route(const ssa_problem* p, const ssa_bf16* q, const float* k_pooled, float alpha,
+                          float gamma, float* weights, uint32_t* mask, ssa_stream stream) {
+  Dims d;
+  ssa_status s = check_problem(p, &d);
+  if (s != SSA_OK) return s;
+  const void* ptrs[] = {q, k_pooled, weights, mask};
+  for (const void* ptr : ptrs)
+    if (ptr == nullptr || !aligned16(ptr)) return SSA_ERR_INVALID_ARG;
+  if (!(alpha > 1.f) || !(alpha <= 4.f)) return SSA_ERR_INVALID_ARG;
+  if (!(gamma > 0.f) || !std::isfinite(gamma)) return SSA_ERR_INVALID_ARG;
+  if (d.n > ssa::kDashMaxN) return SSA_ERR_UNSUPPORTED;
+  auto st = reinterpret_cast<cudaStream_t>(stream);
+  return d.D == 64 ? launch_dash_route<64>(d, q, k_pooled, alpha, gamma, weights, mask, st)
+                   : launch_dash_route<128>(d, q, k_pooled, alpha, gamma, weights, mask, st);
+}
+
+ssa_status ssa_dash_attn_fwd(const ssa_problem* p, const ssa_bf16* q, const ssa_bf16* k, const ssa_bf16* v,
+                             const float* weights, const uint32_t* mask, float sigma, ssa_bf16* o, float* lse,
+                             ssa_stream stream) {
+  Dims d;
+  ssa_status s = check_problem(p, &d);
+  if (s != SSA_OK) return s;
+  const void* ptrs[] = {q, k, v, weights, mask, o, lse};
+  for (const void* ptr : ptrs)
+    if (ptr == nullptr || !aligned16(ptr)) return SSA_ERR_INVALID_ARG;
+  if (!(sigma >= 0.f) || !std::isfinite(sigma)) return SSA_ERR_INVALID_ARG;
+  if (d.n > ssa::kDashMaxN) return SSA_ERR_UNSUPPORTED;
+  auto st = reinterpret_cast<cudaStream_t>(stream);
+  DashIn dash;
+  dash.mask = mask;
+  dash.w = weights;
+  dash.sigma = sigma;
+  if (d.D == 64)
+    return d.G >= 4 ? launch_fwd<64, 2, false, false, true>(d, q, k, v, nullptr, o, lse, nullptr, nullptr, nullptr,
+                                                            st, nullptr, nullptr, 0.f, nullptr, dash)
+                    : launch_fwd<64, 1, false, false, true>(d, q, k, v, nullptr, o, lse, nullptr, nullptr, nullptr,
+                                                            st, nullptr, nullptr, 0.f, nullptr, dash);
+  return d.G >= 4
+             ? launch_psfwd<128, 2, false, true>(d, q, k, v, nullptr, o, lse, nullptr, nullptr, nullptr, st, dash)
+             : launch_psfwd<128, 1, false, true>(d, q, k, v, nullptr, o, lse, nullptr, nullptr, nullptr, st, dash);
 }
 
 ssa_status ssa_get_device_error(ssa_stream stream) {

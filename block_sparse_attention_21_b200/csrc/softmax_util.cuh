@@ -7,6 +7,11 @@
 
 namespace ssa {
 
+// Limits of the DashAttention path: chunks per sequence (the routed list of a
+// query block lives in shared memory) and query heads per KV head.
+constexpr int kDashMaxN = 1024;
+constexpr int kDashMaxG = 16;
+
 struct FwdParams {
   int B, S, Hq, Hkv, G, n, topk, slices;
   float scale_log2;  // softmax scale * log2(e)
@@ -23,10 +28,59 @@ struct FwdParams {
   const float* kbar;     // [B][Hkv][n][D]
   float tau;
   int32_t* visited;      // [B][Hkv][n][G / 2], or null
+  // DashAttention (prior-induced softmax): the routed chunks of each query
+  // block as a bit mask, their group weights, and the prior strength
+  const uint32_t* dmask; // [B][Hkv][n][ceil(n / 32)]
+  const float* dw;       // [B][Hkv][n][n]
+  float sigma;
 };
 
 __host__ __device__ constexpr int pow2_at_least(int x) {
   return x <= 32 ? 32 : x <= 64 ? 64 : x <= 128 ? 128 : x <= 256 ? 256 : 512;
+}
+
+// DashAttention: warp-wide decode of query block i's routed chunks (KV head
+// h, batch b) into an ascending list with per-chunk biases sigma * log2 w_j,
+// followed by the diagonal chunk i with bias 0; *count receives the length.
+__device__ __forceinline__ void dash_build_list(const FwdParams& p, int b, int h, int i, int lane,
+                                                int32_t* dord, float* dbias, int* dcount) {
+  // only chunks before the diagonal whose bit is set and whose weight is
+  // positive are visited, in ascending order, and the diagonal chunk last
+  // (its own branch, bias 0) whatever its bit says.  Lane l holds mask word
+  // l (n <= 32 * 32); the weights are read eight words at a time, coalesced,
+  // and each word's chunks are placed with a ballot.
+  const int W = (p.n + 31) / 32;
+  const size_t rowid = (static_cast<size_t>(b) * p.Hkv + h) * p.n + i;
+  const float* wrow = p.dw + rowid * p.n;
+  const uint32_t myword = lane < W ? p.dmask[rowid * W + lane] : 0u;
+  int base = 0;
+  for (int w0 = 0; w0 * 32 < i; w0 += 8) {
+    float wv[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int j = (w0 + u) * 32 + lane;
+      wv[u] = j < i ? wrow[j] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int wd = w0 + u;
+      const uint32_t word = __shfl_sync(0xffffffffu, myword, wd & 31);
+      const int j = wd * 32 + lane;
+      const bool on = j < i && ((word >> lane) & 1u) != 0u && wv[u] > 0.f && wv[u] < INFINITY;
+      const uint32_t bal = __ballot_sync(0xffffffffu, on);
+      if (on) {
+        const int pos = base + __popc(bal & ((1u << lane) - 1u));
+        dord[pos] = j;
+        dbias[pos] = p.sigma * log2f(wv[u]);
+      }
+      base += __popc(bal);
+    }
+  }
+  if (lane == 0) {
+    dord[base] = i;
+    dbias[base] = 0.f;
+    *dcount = base + 1;
+  }
 }
 
 // Packed fp32 pair helpers (Blackwell f32x2 FMA-pipe instructions).

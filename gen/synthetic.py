@@ -222,3 +222,31 @@ def make_decode(batch: int, capacity: int, n_q_heads: int, n_kv_heads: int, head
                 pick = rng.choice(c, size=m, replace=False)
                 q[b, h * G:(h + 1) * G] += u[b, h, pick].sum(axis=0)
     return DecodeInputs(q=_to_bf16(q), k=_to_bf16(k), v=_to_bf16(v), lengths=lengths, top_k=top_k)
+
+
+@dataclasses.dataclass
+class DashRouting:
+    """A synthetic DashAttention routing: group weights and a bit mask."""
+    weights: np.ndarray   # [B, Hkv, n, n] float32
+    mask: np.ndarray      # [B, Hkv, n, ceil(n / 32)] uint32
+
+
+def make_dash_routing(batch: int, n_kv_heads: int, n_blocks: int, seed: int, density: float = 0.5,
+                      zero_frac: float = 0.3) -> DashRouting:
+    """Random routing inputs for the prior-induced softmax, independent of any
+    scores: each mask bit is set with probability `density` (bits at and after
+    the diagonal and the diagonal bit itself included, so the rule that ignores
+    the former and always keeps the diagonal is exercised), and each weight is
+    uniform in [0.01, 1) except a `zero_frac` share that is exactly 0 (set bits
+    with zero weight must be skipped)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    n = n_blocks
+    shape = (batch, n_kv_heads, n, n)
+    w = rng.uniform(0.01, 1.0, size=shape) * (rng.random(shape) >= zero_frac)
+    bits = rng.random(shape) < density
+    words = (n + 31) // 32
+    padded = np.zeros((batch, n_kv_heads, n, words * 32), dtype=bool)
+    padded[..., :n] = bits
+    weights_of_bits = (1 << np.arange(32, dtype=np.uint64)).astype(np.uint64)
+    mask = (padded.reshape(batch, n_kv_heads, n, words, 32).astype(np.uint64) * weights_of_bits).sum(axis=-1)
+    return DashRouting(weights=w.astype(np.float32), mask=mask.astype(np.uint32))

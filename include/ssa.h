@@ -156,6 +156,49 @@ ssa_status ssa_sparse_attn_fwd_early_stop(const ssa_problem *p, const ssa_bf16 *
                                           const int32_t *block_idx, float tau, ssa_bf16 *o,
                                           float *lse, int32_t *visited, ssa_stream stream);
 
+/* DashAttention chunk routing ("Resumen Tecnico: DashAttention", stage 1 and
+ * its GQA rule; chunks are the 64-token blocks, summarised by their mean key
+ * -- stage 0 with its summary query at its zero initialisation).  For query
+ * block i of KV head h, each query head g of the group scores the complete
+ * earlier chunks j < i:
+ *   z_gj = gamma * scale * qmean_g(i) . k_pooled[b][h][j]
+ * (qmean_g(i): the mean of head g's 64 queries of block i; scale: the
+ * problem's softmax scale), p_g = alpha-entmax(z_g), the distribution
+ *   p_gj = [(alpha - 1) z_gj - tau_g]_+ ^ (1 / (alpha - 1)),  sum_j p_gj = 1,
+ * and the group shares w_j = mean_g p_gj.  tau_g is found in fp32 by
+ * bisection until its bracket stops shrinking; p_g is then normalised.
+ *   q         [B][S][Hq][D] bf16
+ *   k_pooled  [B][Hkv][n][D] fp32, ssa_block_pool's mean keys
+ *   weights   [B][Hkv][n][n] fp32 out: row i holds w_j for j < i, 0 elsewhere
+ *   mask      [B][Hkv][n][ceil(n / 32)] uint32 out: bit j of row i (word
+ *             j / 32, bit j % 32) is set for j < i with w_j > 0, and bit i
+ *             (the diagonal chunk, which is not routed) always.
+ * top_k of the problem is not used.  Errors: INVALID_ARG for null/misaligned
+ * pointers, alpha outside (1, 4] or gamma not finite and > 0; UNSUPPORTED for
+ * more than 1024 chunks (n = S / 64). */
+ssa_status ssa_dash_route(const ssa_problem *p, const ssa_bf16 *q, const float *k_pooled, float alpha,
+                          float gamma, float *weights, uint32_t *mask, ssa_stream stream);
+
+/* DashAttention's prior-induced sparse softmax ("Resumen Tecnico:
+ * DashAttention", stage 2): softmax attention whose reference distribution
+ * is a prior g over the keys instead of the uniform one, i.e. attention
+ * weights proportional to g_s exp(z_s).  g is uniform inside a chunk and
+ * proportional to w_j^sigma across the active chunks (sigma: the prior's
+ * strength; 0 gives plain attention over the support), and 0 elsewhere.  For
+ * query t of block i the active chunks are the j < i whose mask bit is set and
+ * whose weight is finite and > 0, plus the diagonal chunk i (its own branch,
+ * weight 1, causal), so the logits are
+ *   scale * q_t . k_s + sigma * ln w_j(s)   over the active keys s <= t.
+ * weights/mask: as written by ssa_dash_route (any values are accepted; bits
+ * at or after the diagonal are ignored).  Outputs o [B][S][Hq][D] bf16 and lse
+ * [B][Hq][S] fp32, the natural-log log-sum-exp of the biased logits.
+ * top_k of the problem is not used.  Errors: INVALID_ARG for null/misaligned
+ * pointers or sigma not finite and >= 0; UNSUPPORTED for more than 1024
+ * chunks. */
+ssa_status ssa_dash_attn_fwd(const ssa_problem *p, const ssa_bf16 *q, const ssa_bf16 *k, const ssa_bf16 *v,
+                             const float *weights, const uint32_t *mask, float sigma, ssa_bf16 *o, float *lse,
+                             ssa_stream stream);
+
 /* Bytes of device workspace ssa_sparse_attn_bwd needs for problem p (0 on an
  * invalid problem). */
 size_t ssa_sparse_attn_bwd_workspace(const ssa_problem *p);

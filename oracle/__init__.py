@@ -440,7 +440,8 @@ def dash_route(q, kbar, alpha: float, gamma: float, scale: Optional[float] = Non
     return w, mask, margin
 
 
-def dash_attention(q, k, v, mask, w, sigma: float, scale: Optional[float] = None, bs: int = BLOCK):
+def dash_attention(q, k, v, mask, w, sigma: float, scale: Optional[float] = None, bs: int = BLOCK,
+                   blocks=None):
     """DashAttention's prior-induced sparse softmax, fp64 ("Resumen Tecnico:
     DashAttention", stage 2).
 
@@ -448,10 +449,13 @@ def dash_attention(q, k, v, mask, w, sigma: float, scale: Optional[float] = None
     the keys: g is uniform inside a chunk and proportional to w_j^sigma across
     the active chunks, and 0 elsewhere, so the attention p maximising
     z.p - KL(p || g) is p_s proportional to g_s exp(z_s).  For query t of block
-    i the active chunks are the j < i whose mask bit is set and whose w_j > 0,
-    plus the diagonal chunk i with weight 1 (its own branch); causal inside i.
+    i the active chunks are the j < i whose mask bit is set and whose w_j is
+    finite and > 0, plus the diagonal chunk i with weight 1 (its own branch);
+    causal inside i.
     Logits are scale * q_t . k_s + sigma * ln w_j.  Returns o [B, S, Hq, D] and
-    lse [B, Hq, S], the natural-log log-sum-exp of the biased logits."""
+    lse [B, Hq, S], the natural-log log-sum-exp of the biased logits; with
+    `blocks` (rows of (b, KV head, query block)) only those are computed and
+    the rest is left 0."""
     q64, k64, v64 = widen(q), widen(k), widen(v)
     w = np.asarray(w, dtype=np.float64)
     mask = np.asarray(mask, dtype=np.uint32)
@@ -462,19 +466,19 @@ def dash_attention(q, k, v, mask, w, sigma: float, scale: Optional[float] = None
     o = np.zeros((B, S, Hq, D))
     lse = np.zeros((B, Hq, S))
     tok = np.arange(bs)
-    for b in range(B):
-        for h in range(Hkv):
-            for i in range(n):
-                act = [j for j in range(i)
-                       if (int(mask[b, h, i, j // 32]) >> (j % 32)) & 1 and w[b, h, i, j] > 0]
-                keys = np.concatenate([bs * j + tok for j in act] + [bs * i + tok])
-                bias = np.concatenate([np.full(bs, sigma * np.log(w[b, h, i, j])) for j in act]
-                                      + [np.zeros(bs)])
-                for hq in range(h * G, (h + 1) * G):
-                    lg = scale * (q64[b, bs * i + tok, hq] @ k64[b, keys, h].T) + bias[None, :]
-                    lg[:, -bs:] = np.where(tok[None, :] <= tok[:, None], lg[:, -bs:], -np.inf)
-                    mx = lg.max(axis=1, keepdims=True)
-                    e = np.exp(lg - mx)
-                    lse[b, hq, bs * i + tok] = mx[:, 0] + np.log(e.sum(axis=1))
-                    o[b, bs * i + tok, hq] = (e / e.sum(axis=1, keepdims=True)) @ v64[b, keys, h]
+    if blocks is None:
+        blocks = [(b, h, i) for b in range(B) for h in range(Hkv) for i in range(n)]
+    for b, h, i in blocks:
+        act = [j for j in range(i)
+               if (int(mask[b, h, i, j // 32]) >> (j % 32)) & 1 and 0 < w[b, h, i, j] < np.inf]
+        keys = np.concatenate([bs * j + tok for j in act] + [bs * i + tok])
+        bias = np.concatenate([np.full(bs, sigma * np.log(w[b, h, i, j])) for j in act]
+                              + [np.zeros(bs)])
+        for hq in range(h * G, (h + 1) * G):
+            lg = scale * (q64[b, bs * i + tok, hq] @ k64[b, keys, h].T) + bias[None, :]
+            lg[:, -bs:] = np.where(tok[None, :] <= tok[:, None], lg[:, -bs:], -np.inf)
+            mx = lg.max(axis=1, keepdims=True)
+            e = np.exp(lg - mx)
+            lse[b, hq, bs * i + tok] = mx[:, 0] + np.log(e.sum(axis=1))
+            o[b, bs * i + tok, hq] = (e / e.sum(axis=1, keepdims=True)) @ v64[b, keys, h]
     return o, lse

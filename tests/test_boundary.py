@@ -80,6 +80,8 @@ def test_bad_problem_is_rejected_by_every_entry_point(lib, kw, code):
     assert lib.ssa_decode_attn(p, f, f, f, f, f, f, f, None, f, 1 << 30, None) == code
     assert lib.ssa_decode_attn_workspace(p) == 0
     assert lib.ssa_sparse_attn_fwd_early_stop(p, f, f, f, f, f, f, 0.1, f, f, None, None) == code
+    assert lib.ssa_dash_route(p, f, f, 1.5, 1.0, f, f, None) == code
+    assert lib.ssa_dash_attn_fwd(p, f, f, f, f, f, 1.0, f, f, None) == code
 
 
 def test_null_problem(lib):
@@ -141,3 +143,21 @@ def test_early_stop_arguments_are_checked_before_launch(lib):
     assert lib.ssa_sparse_attn_fwd_early_stop(p, f, f, f, None, f, f, 0.1, f, f, None, None) == INVALID
     big = ctypes.byref(_p(top_k=257))
     assert lib.ssa_sparse_attn_fwd_early_stop(big, f, f, f, f, f, f, 0.1, f, f, None, None) == UNSUPPORTED
+
+
+def test_dash_arguments_are_checked_before_launch(lib):
+    p = ctypes.byref(_p())
+    f = FAKE
+    for alpha in (1.0, 0.5, 4.5, float("nan"), float("inf")):
+        assert lib.ssa_dash_route(p, f, f, alpha, 1.0, f, f, None) == INVALID
+    for gamma in (0.0, -1.0, float("nan"), float("inf")):
+        assert lib.ssa_dash_route(p, f, f, 1.5, gamma, f, f, None) == INVALID
+    assert lib.ssa_dash_route(p, None, f, 1.5, 1.0, f, f, None) == INVALID
+    assert lib.ssa_dash_route(p, f, f, 1.5, 1.0, f, f + 4, None) == INVALID
+    for sigma in (-0.1, float("nan"), float("inf")):
+        assert lib.ssa_dash_attn_fwd(p, f, f, f, f, f, sigma, f, f, None) == INVALID
+    assert lib.ssa_dash_attn_fwd(p, f, f, f, None, f, 1.0, f, f, None) == INVALID
+    # more than 1024 chunks: the routed list of a query block no longer fits
+    big = ctypes.byref(_p(seq_len=65536 + 64))
+    assert lib.ssa_dash_route(big, f, f, 1.5, 1.0, f, f, None) == UNSUPPORTED
+    assert lib.ssa_dash_attn_fwd(big, f, f, f, f, f, 1.0, f, f, None) == UNSUPPORTED
