@@ -286,6 +286,7 @@ def run_ours(args, world, rank, local):
     assert ssa.ssa_get_device_error() == 0
 
     decode = decode_rows(dev, timed)
+    dash = dash_rows(p, w, q, k, v, timed, n_k)
     # the early-stop variant of the sparse forward on the same inputs and table
     early = {}
     n_tiles = w.batch * w.n_kv_heads * w.n_blocks * (w.n_q_heads // w.n_kv_heads // 2)
@@ -337,7 +338,8 @@ def run_ours(args, world, rank, local):
                 "flops": "10 D per selected pair (sparse stream) + 10 D per causal pair (full stream)",
                 "tflops": round(2.5 * (flops + causal_flops(w)) / (abwd_ms * 1e-3) / 1e12, 2)},
             "decode": decode,
-            "sparse_attn_fwd_early_stop": early},
+            "sparse_attn_fwd_early_stop": early,
+            "dash_attention": dash},
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
         "pct_of_peak_step": round(100.0 * value / world / peak, 2),
@@ -361,6 +363,38 @@ def load_traffic(name):
 
 
 # ------------------------------------------------------------------ decode
+
+def dash_rows(p, w, q, k, v, timed_fn, n_k, alpha=1.5, gamma=8.0, sigma=1.0):
+    """DashAttention on the bench workload: the routing (keys-only pooling then
+    ssa_dash_route) and the prior-induced softmax (ssa_dash_attn_fwd), each
+    timed alone.  gamma = 8 routes about as many chunks as the sparse stream's
+    top-k = 16 on these inputs.  FLOPs: 4 D per unmasked (query, key) pair of
+    the routed chunks and the diagonal, counted from the mask and weights the
+    routing wrote."""
+    import block_sparse_attention_21_b200 as ssa
+    da = ssa.DashAttention(p, alpha=alpha, gamma=gamma, sigma=sigma)
+    da.forward(q, k, v)
+    g_route, g_attn = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_route):
+        da.route(q, k)
+    with torch.cuda.graph(g_attn):
+        ssa.ssa_dash_attn_fwd(p, q, k, v, da.weights, da.mask, sigma, da.o, da.lse)
+    route_ms = timed_fn(g_route, n_k) / n_k
+    attn_ms = timed_fn(g_attn, n_k) / n_k
+    torch.cuda.synchronize()
+    assert ssa.ssa_get_device_error() == 0
+    n = w.n_blocks
+    bits = np.unpackbits(da.mask.cpu().numpy().view(np.uint8), axis=-1, bitorder="little")[..., :n].astype(bool)
+    earlier = np.tril(np.ones((n, n), dtype=bool), -1)
+    routed = (bits & earlier & (da.weights.cpu().numpy() > 0)).sum(axis=-1)     # [B, Hkv, n]
+    pairs = float((routed * 64 * 64 + 64 * 65 // 2).sum()) * (w.n_q_heads // w.n_kv_heads)
+    flops = 4.0 * w.head_dim * pairs
+    return {"alpha": alpha, "gamma": gamma, "sigma": sigma,
+            "chunks_routed_mean": round(float(routed.mean()) + 1.0, 3),
+            "route_ms": round(route_ms, 5), "attn_ms": round(attn_ms, 5),
+            "attn_tflops": round(flops / (attn_ms * 1e-3) / 1e12, 2),
+            "flops": "4 D per unmasked (query, key) pair of the routed chunks and the diagonal"}
+
 
 def decode_rows(dev, timed_fn):
     """One decoding step of the sparse stream (ssa_decode_attn) on two batch
