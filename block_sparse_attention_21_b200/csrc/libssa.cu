@@ -10,6 +10,7 @@
 #include <cmath>
 #include <cstdlib>
 #include <mutex>
+#include <type_traits>
 
 #include "ssa.h"
 #include "sm100.cuh"
@@ -273,11 +274,11 @@ ssa_status launch_psfwd(const Dims& d, const void* q, const void* k, const void*
 
 // ------------------------------------------------------- DashAttention route
 
-template <int D>
+template <int D, int G>
 ssa_status launch_dash_route(const Dims& d, const void* q, const float* kbar, float alpha, float gamma,
                              float* w, uint32_t* mask, cudaStream_t st) {
   static std::atomic<uint64_t> done{0};
-  auto kernel = ssa::dash_route_kernel<D>;
+  auto kernel = ssa::dash_route_kernel<D, G>;
   const ssa_status s =
       ensure_smem(kernel, static_cast<int>(ssa::dash_route_smem(ssa::kDashMaxG, 128, ssa::kDashMaxN)), &done);
   if (s != SSA_OK) return s;
@@ -292,6 +293,7 @@ ssa_status launch_dash_route(const Dims& d, const void* q, const float* kbar, fl
   rp.am1 = alpha - 1.f;
   rp.inv_am1 = 1.f / (alpha - 1.f);
   rp.pw_mode = alpha == 1.5f ? 0 : (alpha == 2.f ? 1 : 2);
+  rp.newton = alpha <= 2.f ? 1 : 0;
   rp.zscale = gamma * d.scale;
   rp.q = static_cast<const __nv_bfloat16*>(q);
   rp.kbar = kbar;
@@ -804,8 +806,22 @@ ssa_status ssa_dash_route(const ssa_problem* p, const ssa_bf16* q, const float* 
   if (!(gamma > 0.f) || !std::isfinite(gamma)) return SSA_ERR_INVALID_ARG;
   if (d.n > ssa::kDashMaxN) return SSA_ERR_UNSUPPORTED;
   auto st = reinterpret_cast<cudaStream_t>(stream);
-  return d.D == 64 ? launch_dash_route<64>(d, q, k_pooled, alpha, gamma, weights, mask, st)
-                   : launch_dash_route<128>(d, q, k_pooled, alpha, gamma, weights, mask, st);
+  auto route = [&](auto dd, auto gg) {
+    return launch_dash_route<decltype(dd)::value, decltype(gg)::value>(d, q, k_pooled, alpha, gamma, weights,
+                                                                       mask, st);
+  };
+  using I64 = std::integral_constant<int, 64>;
+  using I128 = std::integral_constant<int, 128>;
+  switch (d.G) {
+    case 2: return d.D == 64 ? route(I64(), std::integral_constant<int, 2>())
+                             : route(I128(), std::integral_constant<int, 2>());
+    case 4: return d.D == 64 ? route(I64(), std::integral_constant<int, 4>())
+                             : route(I128(), std::integral_constant<int, 4>());
+    case 8: return d.D == 64 ? route(I64(), std::integral_constant<int, 8>())
+                             : route(I128(), std::integral_constant<int, 8>());
+    default: return d.D == 64 ? route(I64(), std::integral_constant<int, 16>())
+                              : route(I128(), std::integral_constant<int, 16>());
+  }
 }
 
 ssa_status ssa_dash_attn_fwd(const ssa_problem* p, const ssa_bf16* q, const ssa_bf16* k, const ssa_bf16* v,
