@@ -18,7 +18,8 @@
 //   decode_attn_kernel     one warp per (b, KV head, selected block): scores
 //                          of the G query heads against the block's 64 keys,
 //                          a partial softmax (max, sum, unnormalised output).
-//   decode_combine_kernel  one CTA per (b, query head): merges the partials.
+//   decode_combine_kernel  one CTA per (b, query head): merges the partials
+//                          (row groups of threads over the partials).
 //
 // The work is a few rows per KV head, far below a 128-row tensor-core tile,
 // and it is bound by the HBM reads of K-bar and of the selected K/V blocks;
@@ -338,26 +339,91 @@ __global__ void __launch_bounds__(32 * kDecodeWarps) decode_attn_kernel(const De
     for (int c = 0; c < CPL; ++c) part[g * (D + 2) + 2 + CPL * lane + c] = acc[g][c];
 }
 
-// One CTA of D threads per (b, query head): o = sum_s 2^(m_s - M) o_s / l.
-template <int D>
-__global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeParams p) {
+// One CTA of NT threads per (b, query head): o = sum_s 2^(m_s - M) o_s / l
+// over the partials s.  M first (a strided max), then the threads split into
+// D/4 float4 columns x R row groups; each row group walks every R-th partial
+// with eight loads in flight, and the row groups' sums are added in a fixed
+// order in shared memory.  NT = 256 for many partials, 64 for a few.
+template <int D, int NT>
+__global__ void __launch_bounds__(NT) decode_combine_kernel(const DecodeParams p) {
+  constexpr int C4 = D / 4;                  // float4 columns
+  constexpr int R = NT / C4;                 // row groups
+  constexpr int U = 8;
+  static_assert(R >= 1 && NT % 32 == 0, "combine layout");
+  __shared__ float red[NT / 32];
+  __shared__ float4 osum[R][C4];
+  __shared__ float lsum[R];
   const int bq = blockIdx.x, b = bq / p.Hq, hq = bq % p.Hq;
   const int h = hq / p.G, g = hq % p.G;
-  const float* base = p.part + (static_cast<size_t>(b) * p.Hkv + h) * p.topk * p.G * (D + 2);
-  float M = -INFINITY;
-  for (int s = 0; s < p.topk; ++s) M = fmaxf(M, base[(s * p.G + g) * (D + 2)]);
-  float l = 0.f, acc = 0.f;
-  for (int s = 0; s < p.topk; ++s) {
-    const float* ps = base + (s * p.G + g) * (D + 2);
-    const float m = ps[0];
-    if (m == -INFINITY) continue;
-    const float w = exp2f(m - M);
-    l = fmaf(w, ps[1], l);
-    acc = fmaf(w, ps[2 + threadIdx.x], acc);
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const size_t stride = static_cast<size_t>(p.G) * (D + 2);   // floats between partials
+  const float* base = p.part + (static_cast<size_t>(b) * p.Hkv + h) * p.topk * stride + g * (D + 2);
+
+  float mx = -INFINITY;
+  for (int s = tid; s < p.topk; s += NT) mx = fmaxf(mx, base[s * stride]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if (lane == 0) red[warp] = mx;
+  __syncthreads();
+  float M = red[0];
+#pragma unroll
+  for (int w = 1; w < NT / 32; ++w) M = fmaxf(M, red[w]);
+
+  const int c = tid % C4, r = tid / C4;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float l = 0.f;
+  if (M != -INFINITY) {
+    for (int s0 = r; s0 < p.topk; s0 += R * U) {
+      float m[U], ls[U];
+      float4 ov[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int s = s0 + u * R;
+        if (s < p.topk) {
+          const float* ps = base + s * stride;
+          m[u] = ps[0];
+          ls[u] = ps[1];
+          ov[u] = make_float4(ps[2 + 4 * c], ps[3 + 4 * c], ps[4 + 4 * c], ps[5 + 4 * c]);
+        } else {
+          m[u] = -INFINITY;
+          ls[u] = 0.f;
+          ov[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const float w = m[u] == -INFINITY ? 0.f : exp2f(m[u] - M);
+        l = fmaf(w, ls[u], l);
+        acc.x = fmaf(w, ov[u].x, acc.x);
+        acc.y = fmaf(w, ov[u].y, acc.y);
+        acc.z = fmaf(w, ov[u].z, acc.z);
+        acc.w = fmaf(w, ov[u].w, acc.w);
+      }
+    }
   }
-  // l == 0 only for a length the selection rejected: zeros and -inf
-  p.o[static_cast<size_t>(bq) * D + threadIdx.x] = __float2bfloat16_rn(l > 0.f ? acc / l : 0.f);
-  if (threadIdx.x == 0) p.lse[bq] = l > 0.f ? (M + log2f(l)) * 0.69314718055994530942f : -INFINITY;
+  osum[r][c] = acc;
+  if (c == 0) lsum[r] = l;
+  __syncthreads();
+  if (tid < C4) {
+    float4 o = osum[0][tid];
+    float lt = lsum[0];
+    for (int rr = 1; rr < R; ++rr) {
+      const float4 v = osum[rr][tid];
+      o.x += v.x;
+      o.y += v.y;
+      o.z += v.z;
+      o.w += v.w;
+      lt += lsum[rr];
+    }
+    // l == 0 only for a length the selection rejected: zeros and -inf
+    const float inv = lt > 0.f ? 1.f / lt : 0.f;
+    __nv_bfloat16* out = p.o + static_cast<size_t>(bq) * D + 4 * tid;
+    out[0] = __float2bfloat16_rn(o.x * inv);
+    out[1] = __float2bfloat16_rn(o.y * inv);
+    out[2] = __float2bfloat16_rn(o.z * inv);
+    out[3] = __float2bfloat16_rn(o.w * inv);
+    if (tid == 0) p.lse[bq] = lt > 0.f ? (M + log2f(lt)) * 0.69314718055994530942f : -INFINITY;
+  }
 }
 
 }  // namespace ssa

@@ -563,7 +563,11 @@ ssa_status launch_decode(const Dims& d, const void* q, const void* k, const void
     default: s = launch_decode_attn<D, 16>(items, dp, st); break;
   }
   if (s != SSA_OK) return s;
-  ssa::decode_combine_kernel<D><<<static_cast<unsigned>(d.B) * d.Hq, D, 0, st>>>(dp);
+  const unsigned rows = static_cast<unsigned>(d.B) * d.Hq;
+  if (d.topk >= 64)
+    ssa::decode_combine_kernel<D, 256><<<rows, 256, 0, st>>>(dp);
+  else
+    ssa::decode_combine_kernel<D, 64><<<rows, 64, 0, st>>>(dp);
   return launch_result();
 }
 
