@@ -15,7 +15,7 @@
 //                          the complete blocks, exact top-(k-1) by a radix
 //                          search on order-preserving keys (ties: lower j),
 //                          ascending table with c last.
-//   decode_attn_kernel     one warp per (b, KV head, selected block): scores
+//   decode_attn_kernel     one CTA per (b, KV head, selected block): scores
 //                          of the G query heads against the block's 64 keys,
 //                          a partial softmax (max, sum, unnormalised output).
 //   decode_combine_kernel  one CTA per (b, query head): merges the partials
@@ -150,21 +150,17 @@ __global__ void __launch_bounds__(kDecodeSelThreads) decode_select_kernel(const 
   }
 }
 
-// Warps per CTA of decode_attn_kernel, and its dynamic shared memory: per
-// warp the block's K and V (rows padded by 16 bytes, so lanes reading
-// different rows hit different banks), the G <= 16 queries and probabilities.
-constexpr int kDecodeWarps = 2;
+// decode_attn_kernel: one CTA of kDecodeThreads threads per kept block.
+constexpr int kDecodeThreads = 128;
 template <int D>
 __host__ __device__ constexpr int decode_row_bytes() {
-  return D * 2 + 16;
+  return D * 2 + 16;  // a K or V row padded by 16 B: lane-per-row reads spread over the banks
 }
-template <int D>
-__host__ __device__ constexpr int decode_warp_smem() {
-  return 2 * 64 * decode_row_bytes<D>() + 16 * D * 4 + 16 * 64 * 4;
-}
-template <int D>
+// K and V rows, the G scaled queries, the G x 64 probabilities, and the
+// per-warp maxima and sums of the two key warps
+template <int D, int G>
 __host__ __device__ constexpr int decode_attn_smem() {
-  return kDecodeWarps * decode_warp_smem<D>();
+  return 2 * 64 * decode_row_bytes<D>() + G * D * 4 + G * 64 * 4 + 2 * 2 * G * 4;
 }
 
 __device__ __forceinline__ void dec_cp_async16(void* smem, const void* gmem) {
@@ -191,32 +187,38 @@ __device__ __forceinline__ uint64_t dec_bf2(uint32_t w) {
   return dec_f2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
 
-// One warp per (b, KV head, selected block), G query heads (template, so no
-// work is spent on absent heads).  The warp first copies the block's K and V
-// rows into shared memory with cp.async (one round trip for all of them);
-// lane l scores keys l and l + 32 against the G queries with packed f32x2
-// FMAs and 16-byte query loads; a per-head max and sum run over the warp; then
-// lane l accumulates its output columns of every head over the 64 keys.
+// One CTA of 128 threads per (b, KV head, selected block), G query heads
+// (template, so no work is spent on absent heads).  The CTA copies the
+// block's K and V rows into shared memory with cp.async (one round trip), then
+//   scores: thread (key tid % 64, heads of half tid / 64) dots its key row with
+//           the scaled queries using packed f32x2 FMAs;
+//   softmax: per head, max and sum over the 64 keys (two warps, combined in
+//           shared memory), probabilities to shared memory;
+//   P V:     thread (column pair, head group) accumulates over the 64 keys.
+// A partial (m, l, o) per head goes to the workspace for the combine.
 template <int D, int G>
-__global__ void __launch_bounds__(32 * kDecodeWarps) decode_attn_kernel(const DecodeParams p) {
-  constexpr int CPL = D / 32;                 // output columns per lane
+__global__ void __launch_bounds__(kDecodeThreads) decode_attn_kernel(const DecodeParams p) {
   constexpr int RB = decode_row_bytes<D>();
+  constexpr int GH = G / 2;                      // heads per score thread (G >= 2)
+  constexpr int CP = D / 2;                      // output column pairs
+  constexpr int HG = kDecodeThreads / CP;        // head groups in P V
+  constexpr int GPH = (G + HG - 1) / HG;         // heads per P V thread
   extern __shared__ __align__(16) uint8_t dsm[];
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  uint8_t* ks = dsm + warp * decode_warp_smem<D>();
+  uint8_t* ks = dsm;
   uint8_t* vs = ks + 64 * RB;
-  float (*qs)[D] = reinterpret_cast<float (*)[D]>(vs + 64 * RB);
-  float (*pr)[64] = reinterpret_cast<float (*)[64]>(vs + 64 * RB + 16 * D * 4);
-  const int item = blockIdx.x * kDecodeWarps + warp;
-  if (item >= p.B * p.Hkv * p.topk) return;
+  float* qs = reinterpret_cast<float*>(vs + 64 * RB);   // [G][D]
+  float* ps = qs + G * D;                               // [G][64]
+  float* red = ps + G * 64;                             // [2 warps][G] max, then [2][G] sum
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int item = blockIdx.x;
   const int slot = item % p.topk;
   const int bh = item / p.topk, b = bh / p.Hkv, h = bh % p.Hkv;
   float* part = p.part + static_cast<size_t>(item) * G * (D + 2);
   const int j = p.idx[static_cast<size_t>(bh) * p.topk + slot];
   if (j < 0) {  // padding: an empty partial
-    if (lane < G) {
-      part[lane * (D + 2)] = -INFINITY;
-      part[lane * (D + 2) + 1] = 0.f;
+    if (tid < G) {
+      part[tid * (D + 2)] = -INFINITY;
+      part[tid * (D + 2) + 1] = 0.f;
     }
     return;
   }
@@ -227,7 +229,7 @@ __global__ void __launch_bounds__(32 * kDecodeWarps) decode_attn_kernel(const De
   const size_t rstride = static_cast<size_t>(p.Hkv) * D;
   const __nv_bfloat16* kg = p.k + ((static_cast<size_t>(b) * p.S + 64 * j) * p.Hkv + h) * D;
   const __nv_bfloat16* vg = p.v + ((static_cast<size_t>(b) * p.S + 64 * j) * p.Hkv + h) * D;
-  for (int e = lane; e < 64 * (D / 8); e += 32) {
+  for (int e = tid; e < 64 * (D / 8); e += kDecodeThreads) {
     const int r = e / (D / 8), c8 = e % (D / 8);
     if (r < nkeys) {
       dec_cp_async16(ks + r * RB + c8 * 16, kg + r * rstride + c8 * 8);
@@ -238,105 +240,85 @@ __global__ void __launch_bounds__(32 * kDecodeWarps) decode_attn_kernel(const De
     }
   }
   asm volatile("cp.async.commit_group;" ::: "memory");
-  for (int e = lane; e < G * D; e += 32)
-    qs[e / D][e % D] = __bfloat162float(p.q[(static_cast<size_t>(b) * p.Hq + h * G) * D + e]) * p.scale_log2;
+  for (int e = tid; e < G * D; e += kDecodeThreads)
+    qs[e] = __bfloat162float(p.q[(static_cast<size_t>(b) * p.Hq + h * G) * D + e]) * p.scale_log2;
   asm volatile("cp.async.wait_group 0;" ::: "memory");
-  __syncwarp();
-  // scores of keys lane and lane + 32 against every head, 64 columns at a time
-  float sc[2][G];
+  __syncthreads();
+
+  // scores of key k against heads g0 .. g0 + GH - 1
+  const int k = tid & 63, g0 = (tid >> 6) * GH;
+  uint64_t a2[GH];
 #pragma unroll
-  for (int x = 0; x < 2; ++x)
+  for (int x = 0; x < GH; ++x) a2[x] = 0;
+  const uint4* krow = reinterpret_cast<const uint4*>(ks + k * RB);
+#pragma unroll 4
+  for (int c8 = 0; c8 < D / 8; ++c8) {
+    const uint4 kv = krow[c8];
+    const uint64_t k0 = dec_bf2(kv.x), k1 = dec_bf2(kv.y), k2 = dec_bf2(kv.z), k3 = dec_bf2(kv.w);
 #pragma unroll
-    for (int g = 0; g < G; ++g) sc[x][g] = 0.f;
-#pragma unroll
-  for (int d0 = 0; d0 < D; d0 += 64) {
-    uint64_t kp[2][32];  // the two keys' 64 columns as fp32 pairs
-#pragma unroll
-    for (int x = 0; x < 2; ++x) {
-      const uint4* krow = reinterpret_cast<const uint4*>(ks + (lane + 32 * x) * RB + 2 * d0);
-#pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
-        const uint4 kv = krow[c8];
-        kp[x][4 * c8] = dec_bf2(kv.x);
-        kp[x][4 * c8 + 1] = dec_bf2(kv.y);
-        kp[x][4 * c8 + 2] = dec_bf2(kv.z);
-        kp[x][4 * c8 + 3] = dec_bf2(kv.w);
-      }
-    }
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      uint64_t a0 = 0, a1 = 0;
-      const float4* qrow = reinterpret_cast<const float4*>(&qs[g][d0]);
-#pragma unroll
-      for (int c4 = 0; c4 < 16; ++c4) {
-        const float4 q4 = qrow[c4];
-        const uint64_t qa = dec_f2(q4.x, q4.y), qb = dec_f2(q4.z, q4.w);
-        a0 = dec_f2_fma(qa, kp[0][2 * c4], a0);
-        a0 = dec_f2_fma(qb, kp[0][2 * c4 + 1], a0);
-        a1 = dec_f2_fma(qa, kp[1][2 * c4], a1);
-        a1 = dec_f2_fma(qb, kp[1][2 * c4 + 1], a1);
-      }
-      sc[0][g] += dec_f2_sum(a0);
-      sc[1][g] += dec_f2_sum(a1);
+    for (int x = 0; x < GH; ++x) {
+      const float4* q4 = reinterpret_cast<const float4*>(qs + (g0 + x) * D + c8 * 8);
+      const float4 qa = q4[0], qb = q4[1];
+      a2[x] = dec_f2_fma(dec_f2(qa.x, qa.y), k0, a2[x]);
+      a2[x] = dec_f2_fma(dec_f2(qa.z, qa.w), k1, a2[x]);
+      a2[x] = dec_f2_fma(dec_f2(qb.x, qb.y), k2, a2[x]);
+      a2[x] = dec_f2_fma(dec_f2(qb.z, qb.w), k3, a2[x]);
     }
   }
-  // per head: max and sum over the warp, probabilities to shared memory
+  // per head: max and sum over the 64 keys, held by warps (tid >> 5) and its pair
+  float sc[GH];
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const float a = lane < nkeys ? sc[0][g] : -INFINITY;
-    const float c2 = lane + 32 < nkeys ? sc[1][g] : -INFINITY;
-    float m = fmaxf(a, c2);
+  for (int x = 0; x < GH; ++x) {
+    sc[x] = k < nkeys ? dec_f2_sum(a2[x]) : -INFINITY;
+    float m = sc[x];
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-    const float pa = exp2f(a - m), pb = exp2f(c2 - m);
-    pr[g][lane] = pa;
-    pr[g][lane + 32] = pb;
-    float l = pa + pb;
+    if (lane == 0) red[(warp & 1) * G + g0 + x] = m;
+  }
+  __syncthreads();
+  float* red_l = red + 2 * G;
+#pragma unroll
+  for (int x = 0; x < GH; ++x) {
+    const float m = fmaxf(red[g0 + x], red[G + g0 + x]);
+    const float pk = exp2f(sc[x] - m);  // 0 for keys past the causal end
+    ps[(g0 + x) * 64 + k] = pk;
+    float l = pk;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
-    if (lane == 0) {
-      part[g * (D + 2)] = m;
-      part[g * (D + 2) + 1] = l;
-    }
+    if (lane == 0) red_l[(warp & 1) * G + g0 + x] = l;
   }
-  __syncwarp();
-  // o[g][d] for the lane's columns d = CPL * lane .. + CPL - 1, four keys at a time
-  float acc[G][CPL];
+  __syncthreads();
+  if (tid < G) {
+    part[tid * (D + 2)] = fmaxf(red[tid], red[G + tid]);
+    part[tid * (D + 2) + 1] = red_l[tid] + red_l[G + tid];
+  }
+
+  // o[g][2c .. 2c + 1] over the 64 keys for the heads of this thread's group
+  const int cp = tid % CP, hg = tid / CP;
+  uint64_t acc[GPH];
 #pragma unroll
-  for (int g = 0; g < G; ++g)
+  for (int x = 0; x < GPH; ++x) acc[x] = 0;
+#pragma unroll 8
+  for (int r = 0; r < 64; ++r) {
+    const uint64_t v2 = dec_bf2(*reinterpret_cast<const uint32_t*>(vs + r * RB + 4 * cp));
 #pragma unroll
-    for (int c = 0; c < CPL; ++c) acc[g][c] = 0.f;
-  for (int r0 = 0; r0 < 64; r0 += 4) {
-    float vv[4][CPL];
-#pragma unroll
-    for (int x = 0; x < 4; ++x) {
-      const uint8_t* vrow = vs + (r0 + x) * RB + 2 * CPL * lane;
-      if constexpr (CPL == 2) {
-        const uint32_t w = *reinterpret_cast<const uint32_t*>(vrow);
-        vv[x][0] = __uint_as_float(w << 16);
-        vv[x][1] = __uint_as_float(w & 0xFFFF0000u);
-      } else {
-        const uint2 w = *reinterpret_cast<const uint2*>(vrow);
-        vv[x][0] = __uint_as_float(w.x << 16);
-        vv[x][1] = __uint_as_float(w.x & 0xFFFF0000u);
-        vv[x][2] = __uint_as_float(w.y << 16);
-        vv[x][3] = __uint_as_float(w.y & 0xFFFF0000u);
+    for (int x = 0; x < GPH; ++x) {
+      const int g = hg * GPH + x;
+      if (g < G) {
+        const float pr = ps[g * 64 + r];
+        acc[x] = dec_f2_fma(dec_f2(pr, pr), v2, acc[x]);
       }
     }
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float4 p4 = *reinterpret_cast<const float4*>(&pr[g][r0]);
-      const float pw[4] = {p4.x, p4.y, p4.z, p4.w};
-#pragma unroll
-      for (int x = 0; x < 4; ++x)
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) acc[g][c] = fmaf(pw[x], vv[x][c], acc[g][c]);
-    }
   }
 #pragma unroll
-  for (int g = 0; g < G; ++g)
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) part[g * (D + 2) + 2 + CPL * lane + c] = acc[g][c];
+  for (int x = 0; x < GPH; ++x) {
+    const int g = hg * GPH + x;
+    if (g < G) {
+      float lo, hi;
+      asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(acc[x]));
+      *reinterpret_cast<float2*>(part + g * (D + 2) + 2 + 2 * cp) = make_float2(lo, hi);
+    }
+  }
 }
 
 // One CTA of NT threads per (b, query head): o = sum_s 2^(m_s - M) o_s / l

@@ -520,10 +520,10 @@ template <int D, int G>
 ssa_status launch_decode_attn(unsigned items, const ssa::DecodeParams& dp, cudaStream_t st) {
   static std::atomic<uint64_t> smem_done{0};
   auto kernel = ssa::decode_attn_kernel<D, G>;
-  const ssa_status s = ensure_smem(kernel, ssa::decode_attn_smem<D>(), &smem_done);
+  constexpr int smem = ssa::decode_attn_smem<D, G>();
+  const ssa_status s = ensure_smem(kernel, smem, &smem_done);
   if (s != SSA_OK) return s;
-  kernel<<<(items + ssa::kDecodeWarps - 1) / ssa::kDecodeWarps, 32 * ssa::kDecodeWarps, ssa::decode_attn_smem<D>(),
-           st>>>(dp);
+  kernel<<<items, ssa::kDecodeThreads, smem, st>>>(dp);
   return launch_result();
 }
 
