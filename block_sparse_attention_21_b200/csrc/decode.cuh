@@ -11,6 +11,7 @@
 // those tokens only ("Resumen Tecnico: SSA", section 4: inference in the
 // sparse mode reads only the selected blocks).
 //
+//   decode_score_kernel    long caches only: the block scores over many CTAs.
 //   decode_select_kernel   one CTA per (b, KV head): pooled query, scores of
 //                          the complete blocks, exact top-(k-1) by a radix
 //                          search on order-preserving keys (ties: lower j),
@@ -40,6 +41,7 @@ struct DecodeParams {
   const int32_t* len;             // [B] cached tokens per sequence, 1..S
   int32_t* idx;                   // [B][Hkv][topk] selected blocks, ascending, -1 padded
   float* part;                    // [B][Hkv][topk][G][D + 2]: m, l, o (log2 units)
+  uint32_t* keys;                 // [B][Hkv][n] order keys of the scores, or null (scored in the selection)
   __nv_bfloat16* o;               // [B][Hq][D]
   float* lse;                     // [B][Hq] natural log
 };
@@ -62,6 +64,59 @@ __device__ __forceinline__ unsigned cta_sum(unsigned x, unsigned* red) {
 #pragma unroll
   for (int w = 0; w < kDecodeSelThreads / 32; ++w) s += red[w];
   return s;
+}
+
+// The group-mean query of (b, h) into qs[D] (a CTA-wide loop; the caller
+// synchronises before reading it).
+template <int D>
+__device__ __forceinline__ void decode_group_query(const DecodeParams& p, int b, int h, float* qs) {
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    float s = 0.f;
+    for (int g = 0; g < p.G; ++g)
+      s += __bfloat162float(p.q[(static_cast<size_t>(b) * p.Hq + h * p.G + g) * D + d]);
+    qs[d] = s / static_cast<float>(p.G);
+  }
+}
+
+// Order key of block j's score against the group-mean query: its mean-key
+// row read with 16-byte loads, eight in flight.
+template <int D>
+__device__ __forceinline__ uint32_t decode_score_key(const float* kb, int j, const float* qs) {
+  const float4* row = reinterpret_cast<const float4*>(kb + static_cast<size_t>(j) * D);
+  float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+  for (int d4 = 0; d4 < D / 4; d4 += 8) {
+    float4 r[8];
+#pragma unroll
+    for (int x = 0; x < 8; ++x) r[x] = __ldg(row + d4 + x);
+#pragma unroll
+    for (int x = 0; x < 8; ++x) {
+      const int d = 4 * (d4 + x);
+      acc0 = fmaf(qs[d], r[x].x, acc0);
+      acc1 = fmaf(qs[d + 1], r[x].y, acc1);
+      acc0 = fmaf(qs[d + 2], r[x].z, acc0);
+      acc1 = fmaf(qs[d + 3], r[x].w, acc1);
+    }
+  }
+  return dec_order_key(acc0 + acc1);
+}
+
+// Long caches: the scores of the complete blocks spread over many CTAs (a
+// thread per block), written as order keys for the selection kernel.
+// grid (ceil((n - 1) / kDecodeSelThreads), B * Hkv).
+template <int D>
+__global__ void __launch_bounds__(kDecodeSelThreads) decode_score_kernel(const DecodeParams p) {
+  __shared__ float qs[D];
+  const int bh = blockIdx.y, b = bh / p.Hkv, h = bh % p.Hkv;
+  const int L = p.len[b];
+  if (L < 1 || L > p.S) return;  // reported by the selection kernel
+  const int c = (L - 1) / 64;   // complete blocks before the query's own
+  const int j0 = blockIdx.x * kDecodeSelThreads;
+  if (j0 >= c) return;           // the whole CTA: nothing to score here
+  decode_group_query<D>(p, b, h, qs);
+  __syncthreads();
+  const int j = j0 + threadIdx.x;
+  if (j < c) p.keys[static_cast<size_t>(bh) * p.n + j] = decode_score_key<D>(p.kbar + static_cast<size_t>(bh) * p.n * D, j, qs);
 }
 
 // dynamic shared memory: 4 * n bytes of keys
@@ -87,34 +142,16 @@ __global__ void __launch_bounds__(kDecodeSelThreads) decode_select_kernel(const 
     for (int r = threadIdx.x; r < p.topk; r += blockDim.x) out[r] = (r <= c) ? r : -1;
     return;
   }
-  for (int d = threadIdx.x; d < D; d += blockDim.x) {
-    float s = 0.f;
-    for (int g = 0; g < p.G; ++g)
-      s += __bfloat162float(p.q[(static_cast<size_t>(b) * p.Hq + h * p.G + g) * D + d]);
-    qs[d] = s / static_cast<float>(p.G);
-  }
-  __syncthreads();
-  // scores of the complete blocks j < c: a thread per block, its mean-key row
-  // read with 16-byte loads, eight in flight
-  const float* kb = p.kbar + static_cast<size_t>(bh) * p.n * D;
-  for (int j = threadIdx.x; j < c; j += blockDim.x) {
-    const float4* row = reinterpret_cast<const float4*>(kb + static_cast<size_t>(j) * D);
-    float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll
-    for (int d4 = 0; d4 < D / 4; d4 += 8) {
-      float4 r[8];
-#pragma unroll
-      for (int x = 0; x < 8; ++x) r[x] = __ldg(row + d4 + x);
-#pragma unroll
-      for (int x = 0; x < 8; ++x) {
-        const int d = 4 * (d4 + x);
-        acc0 = fmaf(qs[d], r[x].x, acc0);
-        acc1 = fmaf(qs[d + 1], r[x].y, acc1);
-        acc0 = fmaf(qs[d + 2], r[x].z, acc0);
-        acc1 = fmaf(qs[d + 3], r[x].w, acc1);
-      }
-    }
-    dkey[j] = dec_order_key(acc0 + acc1);
+  if (p.keys != nullptr) {
+    // scored by decode_score_kernel
+    const uint32_t* kin = p.keys + static_cast<size_t>(bh) * p.n;
+    for (int j = threadIdx.x; j < c; j += blockDim.x) dkey[j] = kin[j];
+  } else {
+    decode_group_query<D>(p, b, h, qs);
+    __syncthreads();
+    // scores of the complete blocks j < c: a thread per block
+    const float* kb = p.kbar + static_cast<size_t>(bh) * p.n * D;
+    for (int j = threadIdx.x; j < c; j += blockDim.x) dkey[j] = decode_score_key<D>(kb, j, qs);
   }
   __syncthreads();
   // the (k-1)-th largest key, by a 32-step radix search

@@ -502,8 +502,12 @@ ssa_status launch_align_bwd(const Dims& d, const void* q, const void* k, const v
 
 // Workspace of ssa_decode_attn: the selected blocks (unless the caller takes
 // them), then the partial softmax states.
+// From this many blocks per sequence on, decode scores the blocks in a grid
+// of its own (many CTAs) before the per-(b, KV head) selection.
+constexpr int kDecodeSplitBlocks = 1024;
+
 struct DecodeLayout {
-  size_t idx, part, total;
+  size_t idx, part, keys, total;
 };
 
 DecodeLayout decode_layout(const Dims& d) {
@@ -512,7 +516,9 @@ DecodeLayout decode_layout(const Dims& d) {
   DecodeLayout L;
   L.idx = 0;
   L.part = al(rows * sizeof(int32_t));
-  L.total = L.part + al(rows * d.G * (d.D + 2) * sizeof(float));
+  L.keys = L.part + al(rows * d.G * (d.D + 2) * sizeof(float));
+  const size_t keys = d.n >= kDecodeSplitBlocks ? static_cast<size_t>(d.B) * d.Hkv * d.n * sizeof(uint32_t) : 0;
+  L.total = L.keys + al(keys);
   return L;
 }
 
@@ -552,6 +558,14 @@ ssa_status launch_decode(const Dims& d, const void* q, const void* k, const void
   dp.o = static_cast<__nv_bfloat16*>(o);
   dp.lse = lse;
   const unsigned bh = static_cast<unsigned>(d.B) * d.Hkv;
+  dp.keys = nullptr;
+  if (d.n >= kDecodeSplitBlocks) {
+    dp.keys = reinterpret_cast<uint32_t*>(ws + L.keys);
+    const dim3 grid((d.n - 1 + ssa::kDecodeSelThreads - 1) / ssa::kDecodeSelThreads, bh);
+    ssa::decode_score_kernel<D><<<grid, ssa::kDecodeSelThreads, 0, st>>>(dp);
+    const ssa_status s0 = launch_result();
+    if (s0 != SSA_OK) return s0;
+  }
   ssa::decode_select_kernel<D><<<bh, ssa::kDecodeSelThreads, 4 * d.n, st>>>(dp);
   ssa_status s = launch_result();
   if (s != SSA_OK) return s;
