@@ -14,7 +14,8 @@
 //   decode_score_kernel    long caches only: the block scores over many CTAs.
 //   decode_select_kernel   one CTA per (b, KV head): pooled query, scores of
 //                          the complete blocks, exact top-(k-1) by a radix
-//                          search on order-preserving keys (ties: lower j),
+//                          search (8-bit digits) on order-preserving keys
+//                          (ties: lower j),
 //                          ascending table with c last.
 //   decode_attn_kernel     one CTA per (b, KV head, selected block): scores
 //                          of the G query heads against the block's 64 keys,
@@ -125,6 +126,8 @@ __global__ void __launch_bounds__(kDecodeSelThreads) decode_select_kernel(const 
   extern __shared__ uint32_t dkey[];
   __shared__ float qs[D];
   __shared__ unsigned red[kDecodeSelThreads / 32];
+  __shared__ unsigned hist[256];
+  __shared__ unsigned sel_digit[2];
   const int bh = blockIdx.x, b = bh / p.Hkv, h = bh % p.Hkv;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int L = p.len[b];
@@ -154,14 +157,57 @@ __global__ void __launch_bounds__(kDecodeSelThreads) decode_select_kernel(const 
     for (int j = threadIdx.x; j < c; j += blockDim.x) dkey[j] = decode_score_key<D>(kb, j, qs);
   }
   __syncthreads();
-  // the (k-1)-th largest key, by a 32-step radix search
+  // the (k-1)-th largest key, by a radix search over 8-bit digits (most
+  // significant first): a histogram of the keys that match the digits found so
+  // far, then warp 0 finds the digit holding the wanted rank
   const unsigned need = static_cast<unsigned>(p.topk - 1);
-  uint32_t T = 0;
-  for (int bit = 31; bit >= 0; --bit) {
-    const uint32_t cand = T | (1u << bit);
-    unsigned cnt = 0;
-    for (int j = threadIdx.x; j < c; j += blockDim.x) cnt += (dkey[j] >= cand) ? 1u : 0u;
-    if (cta_sum(cnt, red) >= need) T = cand;
+  // top-k 1 keeps only the query's own block: no key is chosen (T above all)
+  uint32_t T = need == 0 ? 0xFFFFFFFFu : 0u, tmask = 0;
+  unsigned rank = need;  // wanted rank among the keys matching T on tmask
+  for (int shift = 24; shift >= 0 && need > 0; shift -= 8) {
+    for (int x = threadIdx.x; x < 256; x += blockDim.x) hist[x] = 0u;
+    __syncthreads();
+    for (int j = threadIdx.x; j < c; j += blockDim.x) {
+      const uint32_t kj = dkey[j];
+      if ((kj & tmask) == T) atomicAdd(&hist[(kj >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // lane l holds digits 255 - 8 l down to 248 - 8 l (descending)
+      unsigned cnt[8], local = 0;
+#pragma unroll
+      for (int x = 0; x < 8; ++x) {
+        cnt[x] = hist[255 - 8 * lane - x];
+        local += cnt[x];
+      }
+      unsigned incl = local;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const unsigned excl = incl - local;
+      if (excl < rank && rank <= incl) {  // exactly one lane
+        unsigned acc = excl, left = 0;
+        int digit = 0;
+#pragma unroll
+        for (int x = 0; x < 8; ++x) {
+          if (acc + cnt[x] >= rank) {
+            digit = 255 - 8 * lane - x;
+            left = rank - acc;
+            break;
+          }
+          acc += cnt[x];
+        }
+        sel_digit[0] = static_cast<unsigned>(digit);
+        sel_digit[1] = left;
+      }
+    }
+    __syncthreads();
+    T |= sel_digit[0] << shift;
+    tmask |= 255u << shift;
+    rank = sel_digit[1];
+    __syncthreads();  // sel_digit and hist are rewritten by the next pass
   }
   unsigned above = 0;
   for (int j = threadIdx.x; j < c; j += blockDim.x) above += (dkey[j] > T) ? 1u : 0u;

@@ -45,6 +45,9 @@ CASES = [
     (3, 1024, 4, 2, 128, 3, [1000, 129, 1024]),
     (2, 4096, 16, 1, 64, 8, [4096, 3333]),
     (2, 131072, 8, 1, 64, 16, [131072, 100001]),   # 2048 blocks to score
+    (2, 2048, 4, 2, 64, 1, [2048, 700]),            # top-k 1: the query's own block only
+    (1, 65536, 4, 1, 128, 32, [65536]),             # 1024 blocks: scored by a grid of their own
+    (2, 4096, 8, 2, 64, 16, [1024, 1025]),          # 16 blocks: all kept; 17: the search
 ]
 
 
