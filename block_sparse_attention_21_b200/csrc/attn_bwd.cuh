@@ -77,6 +77,8 @@ __host__ __device__ inline BwdWorkspace bwd_workspace_layout(int B, int S, int H
 
 // Index-table entries the reverse-index CTAs stage in shared memory at a time.
 constexpr int kRevStage = 2048;
+// Tokens of one (b, query head) per D_t CTA of bwd_prep_kernel.
+constexpr int kDtRows = 256;
 
 // Dynamic shared memory of bwd_prep_kernel for n key blocks.
 __host__ __device__ inline size_t bwd_prep_smem(int n) {
@@ -91,8 +93,9 @@ __host__ __device__ inline size_t bwd_prep_smem(int n) {
 //    each of its blocks.  A row's blocks are distinct, so the lanes of one row
 //    never touch the same list, and the lists come out in ascending order
 //    without sorting: deterministic.
-//  - D_t: each row's D elements are read by D / 8 lanes (16 B each) and
-//    reduced with shuffles; every lane group has four rows' loads in flight.
+//  - D_t: kDtRows tokens of one (b, query head) per CTA; each row's D
+//    elements are read by D / 8 lanes (16 B each) and reduced with shuffles;
+//    every lane group has four rows' loads in flight.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p, int rev_blocks) {
   if (static_cast<int>(blockIdx.x) < rev_blocks) {
@@ -156,32 +159,40 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p, int re
     }
     return;
   }
-  // ---- D_t: four rows per lane group in flight
+  // ---- D_t: CTA c covers kDtRows consecutive tokens of one (b, query head),
+  //      so the D_t writes are coalesced and no per-row index division is
+  //      needed; each row's D elements are read by D / 8 lanes (16 B each) and
+  //      reduced with shuffles, four steps' loads in flight.
   constexpr int LPR = D / 8;            // lanes per row
-  constexpr int RPW = 32 / LPR;         // rows per warp per iteration
-  constexpr int U = 4;                  // iterations whose loads are in flight together
-  const int dt_blocks = static_cast<int>(gridDim.x) - rev_blocks;
-  const int warp_global = ((blockIdx.x - rev_blocks) * blockDim.x + threadIdx.x) / 32;
-  const int nwarps = dt_blocks * (blockDim.x / 32);
-  const int lane = threadIdx.x % 32;
+  constexpr int RPW = 32 / LPR;         // rows per warp per step
+  constexpr int RPC = RPW * 8;          // rows per CTA per step (256 threads)
+  constexpr int U = 4;                  // steps whose loads are in flight together
+  const int c = static_cast<int>(blockIdx.x) - rev_blocks;
+  const int tiles = (p.S + kDtRows - 1) / kDtRows;
+  const int bhq = c / tiles;
+  const int t0 = (c % tiles) * kDtRows;
+  const int b = bhq / p.Hq, hq = bhq % p.Hq;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int sub = lane / LPR, part = lane % LPR;
-  const long long rows = static_cast<long long>(p.B) * p.S * p.Hq;  // (b, t, hq) row-major
-  const long long stride = static_cast<long long>(nwarps) * RPW;
-  for (long long r0 = static_cast<long long>(warp_global) * RPW; r0 < rows; r0 += U * stride) {
+  const size_t rstride = static_cast<size_t>(p.Hq) * D;
+  const __nv_bfloat16* ob = p.o + (static_cast<size_t>(b) * p.S * p.Hq + hq) * D + part * 8;
+  const __nv_bfloat16* gb = p.d_o + (static_cast<size_t>(b) * p.S * p.Hq + hq) * D + part * 8;
+  float* dtrow = p.dt + static_cast<size_t>(bhq) * p.S;
+  for (int s0 = 0; s0 < kDtRows; s0 += U * RPC) {
     uint4 a[U], g[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const long long r = r0 + u * stride + sub;
-      if (r < rows) {
-        a[u] = *reinterpret_cast<const uint4*>(p.o + r * D + part * 8);
-        g[u] = *reinterpret_cast<const uint4*>(p.d_o + r * D + part * 8);
+      const int t = t0 + s0 + u * RPC + warp * RPW + sub;
+      if (t < p.S) {
+        a[u] = *reinterpret_cast<const uint4*>(ob + static_cast<size_t>(t) * rstride);
+        g[u] = *reinterpret_cast<const uint4*>(gb + static_cast<size_t>(t) * rstride);
       }
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const long long r = r0 + u * stride + sub;
+      const int t = t0 + s0 + u * RPC + warp * RPW + sub;
       float acc = 0.f;
-      if (r < rows) {
+      if (t < p.S) {
         const uint32_t wa[4] = {a[u].x, a[u].y, a[u].z, a[u].w}, wg[4] = {g[u].x, g[u].y, g[u].z, g[u].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -191,12 +202,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p, int re
       }
 #pragma unroll
       for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-      if (r < rows && part == 0) {
-        const int hq = static_cast<int>(r % p.Hq);
-        const long long bt = r / p.Hq;
-        const int t = static_cast<int>(bt % p.S), b = static_cast<int>(bt / p.S);
-        p.dt[(static_cast<size_t>(b) * p.Hq + hq) * p.S + t] = acc;
-      }
+      if (t < p.S && part == 0) dtrow[t] = acc;
     }
   }
 }
@@ -533,6 +539,9 @@ struct DqConfig {
   static constexpr int THREADS = 128 * (T + 1);
   static constexpr int NBARS = 1 + 3 * NS + 3 * T + 1;
   static constexpr int SMEM_BYTES = 1024 + 2 * T * QTILE + 2 * NS * KVT + NBARS * 8 + 16;
+  // two CTAs share an SM when both fit in TMEM and shared memory: one CTA's
+  // prologue and epilogue overlap the other's main loop
+  static constexpr int MIN_CTAS = (TMEM_COLS <= 256 && SMEM_BYTES + 1024 <= 116736) ? 2 : 1;
   static_assert(T * TSTRIDE <= 512, "TMEM budget");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
@@ -546,7 +555,7 @@ struct DqConfig {
 // dS(jj) is overwritten by S(jj+1) only after the dQ MMA read it (the tensor
 // pipe runs one thread's MMAs in issue order).
 template <int D, int T_>
-__global__ void __launch_bounds__(DqConfig<D, T_>::THREADS, 1)
+__global__ void __launch_bounds__(DqConfig<D, T_>::THREADS, DqConfig<D, T_>::MIN_CTAS)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                        const BwdParams p) {

@@ -354,10 +354,7 @@ ssa_status launch_bwd(const Dims& d, const void* q, const void* k, const void* v
     return SSA_ERR_CUDA;
 
   // 1. D_t and the reverse index
-  const long long rows = static_cast<long long>(d.B) * d.S * d.Hq;
-  const int rows_per_block = 8 * (32 / (D / 8));
-  long long dt_blocks_ll = (rows + rows_per_block - 1) / rows_per_block;
-  const int dt_blocks = static_cast<int>(dt_blocks_ll < 4096 ? dt_blocks_ll : 4096);
+  const int dt_blocks = d.B * d.Hq * ((d.S + ssa::kDtRows - 1) / ssa::kDtRows);
   // the reverse-index CTAs first (they run longest), then the D_t CTAs; the
   // shared-memory attribute is set once, for the largest supported n
   static std::atomic<uint64_t> prep_done{0};
@@ -701,8 +698,7 @@ ssa_status ssa_sparse_attn_bwd(const ssa_problem* p, const ssa_bf16* q, const ss
   auto st = reinterpret_cast<cudaStream_t>(stream);
   // dQ kernel: two head pairs per CTA when the group has them
   if (d.D == 64)
-    return d.G >= 4 ? launch_bwd<64, 2>(d, q, k, v, o, lse, d_o, block_idx, dq, dk, dv, workspace, st)
-                    : launch_bwd<64, 1>(d, q, k, v, o, lse, d_o, block_idx, dq, dk, dv, workspace, st);
+    return launch_bwd<64, 1>(d, q, k, v, o, lse, d_o, block_idx, dq, dk, dv, workspace, st);
   return d.G >= 4 ? launch_bwd<128, 2>(d, q, k, v, o, lse, d_o, block_idx, dq, dk, dv, workspace, st)
                   : launch_bwd<128, 1>(d, q, k, v, o, lse, d_o, block_idx, dq, dk, dv, workspace, st);
 }
@@ -722,8 +718,7 @@ ssa_status ssa_sparse_attn_bwd_noalloc(const ssa_problem* p, const ssa_bf16* q, 
   if (scratch == nullptr) return SSA_ERR_CUDA;
   auto st = reinterpret_cast<cudaStream_t>(stream);
   if (d.D == 64)
-    return d.G >= 4 ? launch_bwd<64, 2>(d, q, k, v, o, lse, d_o, block_idx, dq, dk, dv, scratch, st)
-                    : launch_bwd<64, 1>(d, q, k, v, o, lse, d_o, block_idx, dq, dk, dv, scratch, st);
+    return launch_bwd<64, 1>(d, q, k, v, o, lse, d_o, block_idx, dq, dk, dv, scratch, st);
   return d.G >= 4 ? launch_bwd<128, 2>(d, q, k, v, o, lse, d_o, block_idx, dq, dk, dv, scratch, st)
                   : launch_bwd<128, 1>(d, q, k, v, o, lse, d_o, block_idx, dq, dk, dv, scratch, st);
 }
@@ -751,10 +746,8 @@ ssa_status ssa_alignment_bwd(const ssa_problem* p, const ssa_bf16* q, const ssa_
     return SSA_ERR_WORKSPACE;
   auto st = reinterpret_cast<cudaStream_t>(stream);
   if (d.D == 64)
-    return d.G >= 4 ? launch_align_bwd<64, 2>(d, q, k, v, o_sparse, lse_sparse, o_full, lse_full, d_o, mode,
-                                              alpha, block_idx, dq, dk, dv, workspace, st)
-                    : launch_align_bwd<64, 1>(d, q, k, v, o_sparse, lse_sparse, o_full, lse_full, d_o, mode,
-                                              alpha, block_idx, dq, dk, dv, workspace, st);
+    return launch_align_bwd<64, 1>(d, q, k, v, o_sparse, lse_sparse, o_full, lse_full, d_o, mode, alpha,
+                                   block_idx, dq, dk, dv, workspace, st);
   return d.G >= 4 ? launch_align_bwd<128, 2>(d, q, k, v, o_sparse, lse_sparse, o_full, lse_full, d_o, mode,
                                              alpha, block_idx, dq, dk, dv, workspace, st)
                   : launch_align_bwd<128, 1>(d, q, k, v, o_sparse, lse_sparse, o_full, lse_full, d_o, mode,
