@@ -46,7 +46,7 @@
 
 namespace ssa {
 
-template <int D, int T, bool MASS, bool DASH = false>
+template <int D, int T, bool MASS, bool DASH = false, bool EARLY = false>
 struct PsFwdConfig {
   static constexpr int NP = D / 64;               // 64-column panels per row
   static constexpr int QTILE = 128 * D * 2;       // bytes of one Q M-tile
@@ -65,7 +65,9 @@ struct PsFwdConfig {
   // abort flag, selection bitmap (up to 8192 blocks); DASH: the routed chunk
   // list and its biases (kDashMaxN each) and the count
   static constexpr int SMEM_TILES = T * QTILE + 2 * NS * KVT + T * PTILE;
-  static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + NBARS * 8 + 16 + 1024 + (DASH ? 8 * kDashMaxN + 16 : 0);
+  // EARLY: 2 KB of visiting-order scratch and 128 B of stop flags
+  static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + NBARS * 8 + 16 + 1024 + (DASH ? 8 * kDashMaxN + 16 : 0) +
+                                    (EARLY ? 2048 + 128 : 0);
   static_assert(T * TSTRIDE <= 512, "TMEM budget");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
@@ -76,12 +78,13 @@ __device__ __forceinline__ int ps_issuer_warp(int t) {
   return t < 3 ? 1 + t : 4 + 4 * T;
 }
 
-template <int D, int T, bool MASS, bool DASH = false>
-__global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH>::THREADS, 1)
+template <int D, int T, bool MASS, bool DASH = false, bool EARLY = false>
+__global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH, EARLY>::THREADS, 1)
     attn_fwd_psmem_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using C = PsFwdConfig<D, T, MASS, DASH>;
+  using C = PsFwdConfig<D, T, MASS, DASH, EARLY>;
   static_assert(!(MASS && DASH), "the routed softmax is a mode of its own");
+  static_assert(!(EARLY && (MASS || DASH)), "the early stop applies to the sparse stream only");
   constexpr int NP = C::NP, QTILE = C::QTILE, KVT = C::KVT, PTILE = C::PTILE, NS = C::NS,
                 TSTRIDE = C::TSTRIDE;
 
@@ -112,6 +115,14 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH>::THREADS, 1)
   int32_t* dord = reinterpret_cast<int32_t*>(selbits + 256);
   float* dbias = reinterpret_cast<float*>(dord + kDashMaxN);
   int* dcount = reinterpret_cast<int*>(dbias + kDashMaxN);
+  // EARLY: visiting order (over the bitmap area), score scratch, stop flags
+  int32_t* ord = reinterpret_cast<int32_t*>(selbits);
+  float* esc = reinterpret_cast<float*>(selbits + 256);       // [256] scores
+  int32_t* ej = reinterpret_cast<int32_t*>(esc + 256);        // [256] their blocks
+  volatile int* all_stop = reinterpret_cast<volatile int*>(ej + 256);
+  volatile int* tile_stop = all_stop + 1;                     // [T]
+  volatile int* wflag = all_stop + 4;                         // [T][2][4]
+  int* nstopped = const_cast<int*>(all_stop) + 24;            // tiles stopped so far
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
@@ -160,6 +171,11 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH>::THREADS, 1)
     }
   }
   if (DASH && warp == 2) dash_build_list(p, b, h, i, lane, dord, dbias, dcount);
+  if (EARLY && threadIdx.x == 0) {
+    *all_stop = 0;
+    *nstopped = 0;
+    for (int t = 0; t < T; ++t) tile_stop[t] = 0;
+  }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
@@ -173,6 +189,14 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH>::THREADS, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    auto load_kv = [&](int st, int j) {
+      mbar_arrive_expect_tx(&bar_kfull[st], KVT);
+      for (int pn = 0; pn < NP; ++pn)
+        tma_load_4d(sK + st * KVT + pn * (64 * 128), &tm_k, &bar_kfull[st], 64 * pn, h, 64 * j, b);
+      mbar_arrive_expect_tx(&bar_vfull[st], KVT);
+      for (int pn = 0; pn < NP; ++pn)
+        tma_load_4d(sV + st * KVT + pn * (64 * 128), &tm_v, &bar_vfull[st], 64 * pn, h, 64 * j, b);
+    };
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
@@ -183,24 +207,30 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH>::THREADS, 1)
           for (int pn = 0; pn < NP; ++pn)
             tma_load_4d(sQ + t * QTILE + pn * (128 * 128) + hh * (64 * 128), &tm_q, bar_q,
                         64 * pn, hq0 + 2 * t + hh, 64 * i, b);
-      int issued = 0;
-      for (int jj = 0; jj < nblk; ++jj) {
+      if (EARLY) load_kv(0, i);  // the diagonal block is visited first
+    }
+    if (EARLY) early_visit_order<D>(p, b, h, i, nsel, idx_row, lane, ord, esc, ej);
+    if (lane == 0) {
+      int issued = EARLY ? 1 : 0;
+      for (int jj = issued; jj < nblk; ++jj) {
         const int st = jj % NS, use = jj / NS;
-        if (use > 0 && !mbar_wait(&bar_empty[st], (use - 1) & 1, abort_flag, tmo, 0x101)) break;
-        const int j = MASS ? jj : (DASH ? dord[jj] : idx_row[jj]);
-        mbar_arrive_expect_tx(&bar_kfull[st], KVT);
-        for (int pn = 0; pn < NP; ++pn)
-          tma_load_4d(sK + st * KVT + pn * (64 * 128), &tm_k, &bar_kfull[st], 64 * pn, h, 64 * j, b);
-        mbar_arrive_expect_tx(&bar_vfull[st], KVT);
-        for (int pn = 0; pn < NP; ++pn)
-          tma_load_4d(sV + st * KVT + pn * (64 * 128), &tm_v, &bar_vfull[st], 64 * pn, h, 64 * j, b);
+        if (EARLY && *all_stop) break;  // every tile stopped: no more blocks
+        // EARLY: once every tile stopped, the stage may never be released;
+        // the stop flag ends the wait instead
+        if (use > 0 && !(EARLY ? mbar_wait_or(&bar_empty[st], (use - 1) & 1, abort_flag, all_stop, tmo, 0x101)
+                               : mbar_wait(&bar_empty[st], (use - 1) & 1, abort_flag, tmo, 0x101)))
+          break;
+        load_kv(st, MASS ? jj : (DASH ? dord[jj] : (EARLY ? ord[jj] : idx_row[jj])));
         ++issued;
       }
-      // on abort, loads already issued are waited for (bounded) before exit
-      if (*abort_flag) {
+      // on abort or an early stop, loads already issued are waited for
+      // (bounded) before exit
+      if (*abort_flag || (EARLY && issued < nblk)) {
         volatile int never = 0;
-        for (int jj = (issued > NS ? issued - NS : 0); jj < issued; ++jj)
+        for (int jj = (issued > NS ? issued - NS : 0); jj < issued; ++jj) {
+          mbar_wait(&bar_kfull[jj % NS], (jj / NS) & 1, &never, 1000000ull, 0x1fe);
           mbar_wait(&bar_vfull[jj % NS], (jj / NS) & 1, &never, 1000000ull, 0x1ff);
+        }
       }
     }
   } else if (warp != 0 && (warp < 4 || warp >= 4 + 4 * T)) {
@@ -265,10 +295,24 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH>::THREADS, 1)
           mma_ss(o_col, a, bd, idesc_pv, (first && kk == 0) ? 0u : 1u);
         }
         tc_commit(&bar_pvdone[t]);
-        if (s + 1 == nblk) tc_commit(&bar_odone[t]);
+        // EARLY: the softmax set the tile's stop flag before it arrived on pfull
+        const bool stop_now = EARLY && tile_stop[t] != 0;
+        if (s + 1 == nblk || stop_now) tc_commit(&bar_odone[t]);
         tc_commit(&bar_empty[st]);
         if (MASS) {
           if (is_sel) first_sel = false; else first_uns = false;
+        }
+        if (EARLY && stop_now) {
+          // the other tiles still need every stage released by this tile too:
+          // release each remaining block's stage once it is loaded, until the
+          // last block or until every tile has stopped (the producer then
+          // loads nothing more)
+          if (atomicAdd(nstopped, 1) + 1 == T) *all_stop = 1;
+          for (int s2 = s + 1; s2 < nblk; ++s2) {
+            if (!mbar_wait_or(&bar_vfull[s2 % NS], (s2 / NS) & 1, abort_flag, all_stop, tmo, 0x207)) break;
+            tc_commit(&bar_empty[s2 % NS]);
+          }
+          break;
         }
       }
       if (!ok) {
@@ -294,6 +338,7 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH>::THREADS, 1)
     const uint64_t scale2 = f2_pack(sl2, sl2);
     float m_ref = -INFINITY;  // reference maximum, scaled (log2) units
     float l_sel = 0.f, l_uns = 0.f;
+    int visited = 0;          // EARLY: blocks this tile visited
     bool ok = true;
     for (int jj = 0; jj < nblk; ++jj) {
       // waits are made warp-uniform: the tcgen05.ld/st below are .sync.aligned
@@ -308,13 +353,16 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH>::THREADS, 1)
       // the scores are in registers: the issuer may overwrite S with the next block's
       tc_fence_before();
       mbar_arrive(&bar_sfree[t]);
-      const bool diag = (jj == nblk - 1);
+      // the diagonal block comes last in the ascending table, first in the
+      // early-stop order
+      const bool diag = EARLY ? (jj == 0) : (jj == nblk - 1);
       bool is_sel = true;
       if (MASS) is_sel = (selbits[jj >> 5] >> (jj & 31)) & 1u;
       // with two tiles, their exponential phases alternate: tile 1's block jj
       // follows tile 0's block jj, tile 0's block jj + 1 follows tile 1's
-      // block jj, so one tile's MMAs run while the other exponentiates
-      if (T == 2 && (t == 1 || jj > 0) &&
+      // block jj, so one tile's MMAs run while the other exponentiates (not
+      // with the early stop, where one tile may stop before the other)
+      if (T == 2 && !EARLY && (t == 1 || jj > 0) &&
           !__all_sync(0xffffffffu, mbar_wait(&bar_turn[t], (t == 1 ? jj : jj - 1) & 1, abort_flag, tmo,
                                              0x305))) {
         ok = false;
@@ -341,9 +389,22 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH>::THREADS, 1)
         exp_pack32<false, C::POLY>(sA, 0, tq, scale2, negm2, acc2, pk);
         exp_pack32<false, C::POLY>(sB, 32, tq, scale2, negm2, acc2, pk + 16);
       }
-      if (T == 2) mbar_arrive(&bar_turn[1 - t]);
+      if (T == 2 && !EARLY) mbar_arrive(&bar_turn[1 - t]);
       float r0, r1;
       f2_unpack(acc2, r0, r1);
+      bool stop = false;
+      if (EARLY && jj > 0 && p.tau > 0.f) {
+        // this block's mass against the mass accumulated before it (both in
+        // the current reference); the tile stops when no row gained at least
+        // tau times what it had (tau = 0 never stops: no decision is taken)
+        const bool cont_row = (r0 + r1) >= p.tau * (l_sel * alpha);
+        volatile int* wf = wflag + (t * 2 + (jj & 1)) * 4;
+        const bool wcont = __any_sync(0xffffffffu, cont_row);
+        if (lane == 0) wf[wq] = wcont ? 1 : 0;
+        named_bar_sync(1 + t, 128);
+        stop = !(wf[0] | wf[1] | wf[2] | wf[3]);
+        if (stop && r == 0) tile_stop[t] = 1;  // read by the issuer after pfull
+      }
       l_sel *= alpha;
       l_uns *= alpha;
       if (is_sel) l_sel += r0 + r1; else l_uns += r0 + r1;
@@ -384,6 +445,8 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH>::THREADS, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bar_pfull[t]);
+      if (EARLY) visited = jj + 1;
+      if (stop) break;
     }
     // ---------------------------------------------------------- epilogue
     if (ok && __all_sync(0xffffffffu, mbar_wait(&bar_odone[t], 0, abort_flag, tmo, 0x303))) {
@@ -424,6 +487,8 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH>::THREADS, 1)
       }
       constexpr float kLn2 = 0.69314718055994530942f;
       p.lse[lrow] = (m_ref + log2f(l_sel)) * kLn2;
+      if (EARLY && r == 0 && p.visited != nullptr)
+        p.visited[((static_cast<size_t>(b) * p.Hkv + h) * p.n + i) * (p.G / 2) + slice * T + t] = visited;
       if (MASS) {
         p.lse_full[lrow] = (m_ref + log2f(l_all)) * kLn2;
         p.dropped[lrow] = has_uns ? (l_uns / l_all) : 0.f;

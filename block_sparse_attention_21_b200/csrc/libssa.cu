@@ -231,13 +231,14 @@ ssa_status launch_fwd(const Dims& d, const void* q, const void* k, const void* v
 }
 
 // The same launch for the kernel that stages P in shared memory.
-template <int D, int T, bool MASS, bool DASH = false>
+template <int D, int T, bool MASS, bool DASH = false, bool EARLY = false>
 ssa_status launch_psfwd(const Dims& d, const void* q, const void* k, const void* v,
                       const int32_t* idx, void* o, float* lse, void* of, float* lsef,
-                      float* dropped, cudaStream_t st, DashIn dash = DashIn()) {
-  using C = ssa::PsFwdConfig<D, T, MASS, DASH>;
+                      float* dropped, cudaStream_t st, DashIn dash = DashIn(), const float* qbar = nullptr,
+                      const float* kbar = nullptr, float tau = 0.f, int32_t* visited = nullptr) {
+  using C = ssa::PsFwdConfig<D, T, MASS, DASH, EARLY>;
   static std::atomic<uint64_t> smem_done{0};
-  auto kernel = ssa::attn_fwd_psmem_kernel<D, T, MASS, DASH>;
+  auto kernel = ssa::attn_fwd_psmem_kernel<D, T, MASS, DASH, EARLY>;
   ssa_status s = ensure_smem(kernel, C::SMEM_BYTES, &smem_done);
   if (s != SSA_OK) return s;
   CUtensorMap mq, mk, mv;
@@ -261,10 +262,10 @@ ssa_status launch_psfwd(const Dims& d, const void* q, const void* k, const void*
   fp.lse_full = lsef;
   fp.dropped = dropped;
   fp.timeout_ns = wait_timeout_ns();
-  fp.qbar = nullptr;
-  fp.kbar = nullptr;
-  fp.tau = 0.f;
-  fp.visited = nullptr;
+  fp.qbar = qbar;
+  fp.kbar = kbar;
+  fp.tau = tau;
+  fp.visited = visited;
   fp.dmask = dash.mask;
   fp.dw = dash.w;
   fp.sigma = dash.sigma;
@@ -773,10 +774,10 @@ ssa_status ssa_sparse_attn_fwd_early_stop(const ssa_problem* p, const ssa_bf16* 
                                                      q_pooled, k_pooled, tau, visited)
                     : launch_fwd<64, 1, false, true>(d, q, k, v, block_idx, o, lse, nullptr, nullptr, nullptr, st,
                                                      q_pooled, k_pooled, tau, visited);
-  return d.G >= 4 ? launch_fwd<128, 2, false, true>(d, q, k, v, block_idx, o, lse, nullptr, nullptr, nullptr, st,
-                                                    q_pooled, k_pooled, tau, visited)
-                  : launch_fwd<128, 1, false, true>(d, q, k, v, block_idx, o, lse, nullptr, nullptr, nullptr, st,
-                                                    q_pooled, k_pooled, tau, visited);
+  return d.G >= 4 ? launch_psfwd<128, 2, false, false, true>(d, q, k, v, block_idx, o, lse, nullptr, nullptr,
+                                                             nullptr, st, DashIn(), q_pooled, k_pooled, tau, visited)
+                  : launch_psfwd<128, 1, false, false, true>(d, q, k, v, block_idx, o, lse, nullptr, nullptr,
+                                                             nullptr, st, DashIn(), q_pooled, k_pooled, tau, visited);
 }
 
 size_t ssa_decode_attn_workspace(const ssa_problem* p) {

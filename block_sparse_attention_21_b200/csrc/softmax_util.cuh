@@ -83,6 +83,64 @@ __device__ __forceinline__ void dash_build_list(const FwdParams& p, int b, int h
   }
 }
 
+// Early stop: the visiting order of query block i (KV head h, batch b) into
+// ord[0 .. nsel - 1], by the whole warp: the diagonal block i first, then the
+// other selected blocks (idx_row[0 .. nsel - 2], all below i) by descending
+// pooled score q_pooled[i] . k_pooled[j] in fp32, ties to the lower block.
+// esc and ej are scratch of nsel - 1 entries.
+template <int D>
+__device__ __forceinline__ void early_visit_order(const FwdParams& p, int b, int h, int i, int nsel,
+                                                  const int32_t* idx_row, int lane, int32_t* ord, float* esc,
+                                                  int32_t* ej) {
+  // visiting order: the diagonal block i first, then the other selected
+  // blocks (idx_row[0 .. nsel - 2], all below i) by descending pooled score
+  // q_pooled[i] . k_pooled[j] in fp32, ties to the lower block
+  // Each lane holds D/32 values of the pooled query; eight rows' dot
+  // products are in flight at once and summed across the warp.
+  constexpr int QV = D / 32;
+  const int ne = nsel - 1;
+  const float* qb = p.qbar + ((static_cast<size_t>(b) * p.Hkv + h) * p.n + i) * D + lane * QV;
+  const float* kb = p.kbar + (static_cast<size_t>(b) * p.Hkv + h) * p.n * D + lane * QV;
+  float qf[QV];
+#pragma unroll
+  for (int c = 0; c < QV; ++c) qf[c] = __ldg(qb + c);
+  for (int c0 = 0; c0 < ne; c0 += 32) {
+    const int cnt = min(32, ne - c0);
+    const int jl = lane < cnt ? idx_row[c0 + lane] : 0;
+    if (lane < cnt) ej[c0 + lane] = jl;
+    for (int r = 0; r < cnt; r += 8) {  // r + 7 <= 31
+      float part[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        // clamped: a malformed table entry reads a valid row, not past the buffer
+        const int ju = min(max(__shfl_sync(0xffffffffu, jl, r + u), 0), p.n - 1);
+        const float* kr = kb + static_cast<size_t>(ju) * D;
+        float a = 0.f;
+#pragma unroll
+        for (int c = 0; c < QV; ++c) a = fmaf(qf[c], __ldg(kr + c), a);
+        part[u] = a;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) part[u] += __shfl_xor_sync(0xffffffffu, part[u], o);
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (lane == u && r + u < cnt) esc[c0 + r + u] = part[u];
+    }
+  }
+  __syncwarp();
+  for (int r = lane; r < ne; r += 32) {
+    const float sr = esc[r];
+    const int jr = ej[r];
+    int rank = 0;
+    for (int r2 = 0; r2 < ne; ++r2) rank += (esc[r2] > sr || (esc[r2] == sr && ej[r2] < jr)) ? 1 : 0;
+    ord[1 + rank] = jr;
+  }
+  if (lane == 0) ord[0] = i;
+  __syncwarp();
+}
+
 // Packed fp32 pair helpers (Blackwell f32x2 FMA-pipe instructions).
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
   uint64_t r;

@@ -34,6 +34,7 @@ CASES = [
     (1, 1024, 8, 2, 64, 6, 4),
     (1, 768, 4, 2, 128, 5, 3),
     (1, 2048, 16, 2, 64, 8, 6),
+    (1, 1536, 8, 2, 128, 6, 4),     # two M-tiles per CTA at head_dim 128
 ]
 
 
@@ -44,7 +45,8 @@ def test_early_stop_matches_oracle(case, tau):
 
 
 @pytest.mark.parametrize("tau", [0.3, 1.0])
-@pytest.mark.parametrize("case", [(1, 4096, 8, 2, 64, 40, 8), (1, 4096, 4, 2, 128, 40, 8)],
+@pytest.mark.parametrize("case", [(1, 4096, 8, 2, 64, 40, 8), (1, 4096, 4, 2, 128, 40, 8),
+                                  (1, 4096, 8, 2, 128, 40, 8)],
                          ids=lambda c: "x".join(map(str, c)))
 def test_early_stop_well_before_the_last_block(case, tau):
     vis, nsel = _check(case, tau, min_clear=0.5)
