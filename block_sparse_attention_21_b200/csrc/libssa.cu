@@ -673,7 +673,7 @@ ssa_status ssa_full_attn_fwd_with_mass(const ssa_problem* p, const ssa_bf16* q, 
     return d.G >= 4
                ? launch_fwd<64, 2, true>(d, q, k, v, block_idx, o_sparse, lse_sparse, o_full, lse_full, dropped, st)
                : launch_fwd<64, 1, true>(d, q, k, v, block_idx, o_sparse, lse_sparse, o_full, lse_full, dropped, st);
-  return launch_fwd<128, 1, true>(d, q, k, v, block_idx, o_sparse, lse_sparse, o_full, lse_full, dropped, st);
+  return launch_psfwd<128, 1, true>(d, q, k, v, block_idx, o_sparse, lse_sparse, o_full, lse_full, dropped, st);
 }
 
 size_t ssa_sparse_attn_bwd_workspace(const ssa_problem* p) {
