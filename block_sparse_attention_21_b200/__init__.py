@@ -13,7 +13,8 @@ import torch
 
 from ._binding import (EXPORTED, LIB_PATH, SsaError, SsaProblem, lib, problem,
                        ssa_alignment_bwd, ssa_alignment_bwd_workspace, ssa_decode_attn,
-                       ssa_dash_attn_fwd, ssa_dash_route,
+                       ssa_dash_attn_fwd, ssa_dash_route, ssa_sparse_attn_fwd_host,
+                       ssa_sparse_attn_fwd_host_workspace,
                        ssa_decode_attn_workspace, ssa_sparse_attn_fwd_early_stop,
                        ssa_block_pool, ssa_block_select, ssa_debug_exp2_poly, ssa_debug_timeout_probe,
                        ssa_full_attn_fwd_with_mass, ssa_get_device_error,
@@ -23,7 +24,8 @@ from ._binding import (EXPORTED, LIB_PATH, SsaError, SsaProblem, lib, problem,
                        ssa_sparse_attn_fwd, ssa_status_string)
 
 __all__ = ["EXPORTED", "LIB_PATH", "DashAttention", "SsaError", "SsaProblem", "SparseStream", "lib", "problem",
-           "ssa_dash_attn_fwd", "ssa_dash_route",
+           "ssa_dash_attn_fwd", "ssa_dash_route", "ssa_sparse_attn_fwd_host",
+           "ssa_sparse_attn_fwd_host_workspace",
            "ssa_alignment_bwd", "ssa_alignment_bwd_workspace", "ssa_decode_attn",
            "ssa_decode_attn_workspace", "ssa_sparse_attn_fwd_early_stop",
            "ssa_block_pool", "ssa_block_select", "ssa_debug_exp2_poly", "ssa_debug_timeout_probe",
@@ -66,6 +68,15 @@ class SparseStream:
         self.select(q, k, stream)
         ssa_sparse_attn_fwd(self.p, q, k, v, self.block_idx, self.o, self.lse, stream)
         return self.o
+
+    def forward_host(self, q, k, v, o, lse, stream=None):
+        """The forward on host tensors (page-locked for overlap): q, k, v in,
+        o and lse out, pipelined by (batch, KV head) inside the library."""
+        if getattr(self, "_host_ws", None) is None:
+            n = ssa_sparse_attn_fwd_host_workspace(self.p)
+            self._host_ws = torch.empty(n, dtype=torch.uint8, device=self.o.device)
+        ssa_sparse_attn_fwd_host(self.p, q, k, v, o, lse, self._host_ws, self._host_ws.numel(), stream)
+        return o
 
     def alignment(self, q, k, v, stream=None):
         if self._full is None:

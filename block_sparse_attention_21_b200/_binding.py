@@ -27,7 +27,8 @@ EXPORTED = ("ssa_block_pool", "ssa_block_select", "ssa_sparse_attn_fwd", "ssa_sp
             "ssa_full_attn_fwd_with_mass", "ssa_sparse_attn_bwd_workspace",
             "ssa_sparse_attn_bwd", "ssa_sparse_attn_bwd_noalloc", "ssa_alignment_bwd_workspace",
             "ssa_alignment_bwd", "ssa_decode_attn_workspace", "ssa_decode_attn",
-            "ssa_dash_route", "ssa_dash_attn_fwd",
+            "ssa_dash_route", "ssa_dash_attn_fwd", "ssa_sparse_attn_fwd_host_workspace",
+            "ssa_sparse_attn_fwd_host",
             "ssa_get_device_error",
             "ssa_get_device_error_site",
             "ssa_debug_timeout_probe", "ssa_debug_exp2_poly",
@@ -78,6 +79,7 @@ def lib():
             "ssa_alignment_bwd": [P] + [vp] * 8 + [ctypes.c_int, ctypes.c_float] + [vp] * 5
                                  + [ctypes.c_size_t, vp],
             "ssa_dash_route": [P, vp, vp, ctypes.c_float, ctypes.c_float, vp, vp, vp],
+            "ssa_sparse_attn_fwd_host": [P] + [vp] * 6 + [ctypes.c_size_t, vp],
             "ssa_dash_attn_fwd": [P] + [vp] * 5 + [ctypes.c_float] + [vp] * 3,
             "ssa_get_device_error": [vp],
             "ssa_debug_timeout_probe": [ctypes.c_int, vp],
@@ -88,7 +90,7 @@ def lib():
             f.argtypes = args
             f.restype = ctypes.c_int
         for name in ("ssa_sparse_attn_bwd_workspace", "ssa_alignment_bwd_workspace",
-                     "ssa_decode_attn_workspace"):
+                     "ssa_decode_attn_workspace", "ssa_sparse_attn_fwd_host_workspace"):
             getattr(L, name).argtypes = [P]
             getattr(L, name).restype = ctypes.c_size_t
         L.ssa_status_string.argtypes = [ctypes.c_int]
@@ -279,6 +281,33 @@ def ssa_dash_attn_fwd(p: SsaProblem, q, k, v, weights, mask, sigma: float, o, ls
     _call("ssa_dash_attn_fwd", ctypes.byref(p), _ptr(q, BF16, "q"), _ptr(k, BF16, "k"), _ptr(v, BF16, "v"),
           _ptr(weights, F32, "weights"), _mask_ptr(mask, "mask"), float(sigma), _ptr(o, BF16, "o"),
           _ptr(lse, F32, "lse"), _stream(stream))
+
+
+def _host_ptr(t, dtype, name: str) -> int:
+    if t is None or t.is_cuda:
+        raise ValueError(f"{name}: expected a host (CPU) tensor, page-locked for overlap")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: expected {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def ssa_sparse_attn_fwd_host_workspace(p: SsaProblem) -> int:
+    return int(lib().ssa_sparse_attn_fwd_host_workspace(ctypes.byref(p)))
+
+
+def ssa_sparse_attn_fwd_host(p: SsaProblem, q, k, v, o, lse, workspace, ws_bytes: int, stream=None) -> None:
+    """Pool, select and the sparse forward on host buffers, pipelined by
+    (batch, KV head) so copies in, kernels and copies out overlap; see
+    include/ssa.h."""
+    sh = _shapes(p)
+    for t, s, nm in ((q, sh["q"], "q"), (k, sh["kv"], "k"), (v, sh["kv"], "v"), (o, sh["q"], "o"),
+                     (lse, sh["lse"], "lse")):
+        _numel_check(t, s, nm)
+    _call("ssa_sparse_attn_fwd_host", ctypes.byref(p), _host_ptr(q, BF16, "q"), _host_ptr(k, BF16, "k"),
+          _host_ptr(v, BF16, "v"), _host_ptr(o, BF16, "o"), _host_ptr(lse, F32, "lse"),
+          _ptr(workspace, None, "workspace"), int(ws_bytes), _stream(stream))
 
 
 def ssa_decode_attn_workspace(p: SsaProblem) -> int:

@@ -583,6 +583,56 @@ ssa_status launch_decode(const Dims& d, const void* q, const void* k, const void
   return launch_result();
 }
 
+// ------------------------------------------------------------ host buffers
+// ssa_sparse_attn_fwd_host: per (batch, KV head) unit, the unit's Q, K, V in
+// one of two device buffer sets, its pooled keys and queries, table, O, LSE.
+// K and V are copied whole first (contiguous, at full PCIe speed; their
+// per-unit rows of D values would be short strided copies) and each unit's
+// slice is taken from there on the device.
+struct HostLayout {
+  size_t kall, vall, sets, q, k, v, kb, qb, idx, o, lse, set, total;
+};
+
+HostLayout host_layout(const Dims& d) {
+  auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  const size_t S = d.S, G = d.G, D = d.D, n = d.n, k = d.topk;
+  const size_t kv_all = static_cast<size_t>(d.B) * S * d.Hkv * D * 2;
+  HostLayout L;
+  L.kall = 0;
+  L.vall = al(kv_all);
+  L.sets = L.vall + al(kv_all);
+  L.q = 0;
+  L.k = al(S * G * D * 2);
+  L.v = L.k + al(S * D * 2);
+  L.kb = L.v + al(S * D * 2);
+  L.qb = L.kb + al(n * D * 4);
+  L.idx = L.qb + al(n * D * 4);
+  L.o = L.idx + al(n * k * 4);
+  L.lse = L.o + al(S * G * D * 2);
+  L.set = L.lse + al(G * S * 4);
+  L.total = L.sets + 2 * L.set;
+  return L;
+}
+
+// The copy-in and copy-out streams of the host-buffer path, one pair per
+// device, created on first use and kept for the life of the process.
+std::mutex g_pipe_mutex;
+cudaStream_t g_pipe_in[kMaxDevices], g_pipe_out[kMaxDevices];
+
+ssa_status pipe_streams(cudaStream_t* in, cudaStream_t* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return SSA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_pipe_mutex);
+  if (g_pipe_in[dev] == nullptr) {
+    if (cudaStreamCreateWithFlags(&g_pipe_in[dev], cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&g_pipe_out[dev], cudaStreamNonBlocking) != cudaSuccess)
+      return SSA_ERR_CUDA;
+  }
+  *in = g_pipe_in[dev];
+  *out = g_pipe_out[dev];
+  return SSA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -656,6 +706,94 @@ ssa_status ssa_sparse_attn_fwd(const ssa_problem* p, const ssa_bf16* q, const ss
   return d.G >= 4
              ? launch_psfwd<128, 2, false>(d, q, k, v, block_idx, o, lse, nullptr, nullptr, nullptr, st)
              : launch_psfwd<128, 1, false>(d, q, k, v, block_idx, o, lse, nullptr, nullptr, nullptr, st);
+}
+
+size_t ssa_sparse_attn_fwd_host_workspace(const ssa_problem* p) {
+  Dims d;
+  if (check_problem(p, &d) != SSA_OK) return 0;
+  return host_layout(d).total;
+}
+
+ssa_status ssa_sparse_attn_fwd_host(const ssa_problem* p, const ssa_bf16* q, const ssa_bf16* k, const ssa_bf16* v,
+                                    ssa_bf16* o, float* lse, void* workspace, size_t ws_bytes, ssa_stream stream) {
+  Dims d;
+  ssa_status s = check_problem(p, &d);
+  if (s != SSA_OK) return s;
+  const void* ptrs[] = {q, k, v, o, lse};
+  for (const void* ptr : ptrs)
+    if (ptr == nullptr) return SSA_ERR_INVALID_ARG;
+  const HostLayout L = host_layout(d);
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || ws_bytes < L.total)
+    return SSA_ERR_WORKSPACE;
+  auto sc = reinterpret_cast<cudaStream_t>(stream);
+  cudaStream_t sin = nullptr, sout = nullptr;
+  s = pipe_streams(&sin, &sout);
+  if (s != SSA_OK) return s;
+  // one unit = one batch entry and one KV head: its G query heads, its K and V
+  ssa_problem unit = *p;
+  unit.batch = 1;
+  unit.n_q_heads = d.G;
+  unit.n_kv_heads = 1;
+  cudaEvent_t ev[8];
+  for (auto& e : ev)
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return SSA_ERR_CUDA;
+  cudaEvent_t ev_start = ev[0], ev_end = ev[1], in_done[2] = {ev[2], ev[3]}, comp_done[2] = {ev[4], ev[5]},
+              out_done[2] = {ev[6], ev[7]};
+  const size_t S = d.S, D = d.D, G = d.G, Hq = d.Hq, Hkv = d.Hkv;
+  const size_t qrow = G * D * 2, krow = D * 2;  // bytes of a unit's token row
+  bool ok = cudaEventRecord(ev_start, sc) == cudaSuccess && cudaStreamWaitEvent(sin, ev_start, 0) == cudaSuccess &&
+            cudaStreamWaitEvent(sout, ev_start, 0) == cudaSuccess;
+  // K and V whole, ahead of the first unit's Q
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t kv_all = static_cast<size_t>(d.B) * S * Hkv * D * 2;
+  ok = ok && cudaMemcpyAsync(ws + L.kall, k, kv_all, cudaMemcpyHostToDevice, sin) == cudaSuccess &&
+       cudaMemcpyAsync(ws + L.vall, v, kv_all, cudaMemcpyHostToDevice, sin) == cudaSuccess;
+  const int units = d.B * d.Hkv;
+  for (int u = 0; ok && u < units; ++u) {
+    const int set = u & 1;
+    const size_t b = u / d.Hkv, h = u % d.Hkv;
+    uint8_t* base = ws + L.sets + set * L.set;
+    auto* uq = reinterpret_cast<ssa_bf16*>(base + L.q);
+    auto* uk = reinterpret_cast<ssa_bf16*>(base + L.k);
+    auto* uv = reinterpret_cast<ssa_bf16*>(base + L.v);
+    auto* ukb = reinterpret_cast<float*>(base + L.kb);
+    auto* uqb = reinterpret_cast<float*>(base + L.qb);
+    auto* uidx = reinterpret_cast<int32_t*>(base + L.idx);
+    auto* uo = reinterpret_cast<ssa_bf16*>(base + L.o);
+    auto* ulse = reinterpret_cast<float*>(base + L.lse);
+    // copy in, once unit u - 2's compute no longer reads this buffer set
+    const auto* hq_src = reinterpret_cast<const uint8_t*>(q) + ((b * S) * Hq + h * G) * D * 2;
+    const uint8_t* dk_src = ws + L.kall + ((b * S) * Hkv + h) * D * 2;
+    const uint8_t* dv_src = ws + L.vall + ((b * S) * Hkv + h) * D * 2;
+    ok = (u < 2 || cudaStreamWaitEvent(sin, comp_done[set], 0) == cudaSuccess) &&
+         cudaMemcpy2DAsync(uq, qrow, hq_src, Hq * D * 2, qrow, S, cudaMemcpyHostToDevice, sin) == cudaSuccess &&
+         cudaEventRecord(in_done[set], sin) == cudaSuccess;
+    // compute on the caller's stream, once the inputs landed (K and V whole
+    // came first on the same stream) and unit u - 2's outputs left this
+    // buffer set; the unit's K and V rows are gathered on the device
+    ok = ok && cudaStreamWaitEvent(sc, in_done[set], 0) == cudaSuccess &&
+         (u < 2 || cudaStreamWaitEvent(sc, out_done[set], 0) == cudaSuccess) &&
+         cudaMemcpy2DAsync(uk, krow, dk_src, Hkv * D * 2, krow, S, cudaMemcpyDeviceToDevice, sc) == cudaSuccess &&
+         cudaMemcpy2DAsync(uv, krow, dv_src, Hkv * D * 2, krow, S, cudaMemcpyDeviceToDevice, sc) == cudaSuccess;
+    if (ok) s = ssa_block_pool(&unit, uk, uq, ukb, uqb, stream);
+    if (ok && s == SSA_OK) s = ssa_block_select(&unit, uqb, ukb, uidx, stream);
+    if (ok && s == SSA_OK) s = ssa_sparse_attn_fwd(&unit, uq, uk, uv, uidx, uo, ulse, stream);
+    ok = ok && s == SSA_OK && cudaEventRecord(comp_done[set], sc) == cudaSuccess;
+    // copy out
+    auto* ho_dst = reinterpret_cast<uint8_t*>(o) + ((b * S) * Hq + h * G) * D * 2;
+    float* hl_dst = lse + (b * Hq + h * G) * S;
+    ok = ok && cudaStreamWaitEvent(sout, comp_done[set], 0) == cudaSuccess &&
+         cudaMemcpy2DAsync(ho_dst, Hq * D * 2, uo, qrow, qrow, S, cudaMemcpyDeviceToHost, sout) == cudaSuccess &&
+         cudaMemcpyAsync(hl_dst, ulse, G * S * 4, cudaMemcpyDeviceToHost, sout) == cudaSuccess &&
+         cudaEventRecord(out_done[set], sout) == cudaSuccess;
+  }
+  // the caller's stream continues after the last copies; copy-in waits too, so
+  // a later call cannot overwrite buffers still being read
+  ok = ok && cudaEventRecord(ev_end, sout) == cudaSuccess && cudaStreamWaitEvent(sc, ev_end, 0) == cudaSuccess &&
+       cudaStreamWaitEvent(sin, ev_end, 0) == cudaSuccess;
+  for (auto& e : ev) cudaEventDestroy(e);  // released once the streams are past them
+  if (s != SSA_OK) return s;
+  return ok ? SSA_OK : SSA_ERR_CUDA;
 }
 
 ssa_status ssa_full_attn_fwd_with_mass(const ssa_problem* p, const ssa_bf16* q, const ssa_bf16* k,

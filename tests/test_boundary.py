@@ -82,6 +82,8 @@ def test_bad_problem_is_rejected_by_every_entry_point(lib, kw, code):
     assert lib.ssa_sparse_attn_fwd_early_stop(p, f, f, f, f, f, f, 0.1, f, f, None, None) == code
     assert lib.ssa_dash_route(p, f, f, 1.5, 1.0, f, f, None) == code
     assert lib.ssa_dash_attn_fwd(p, f, f, f, f, f, 1.0, f, f, None) == code
+    assert lib.ssa_sparse_attn_fwd_host(p, f, f, f, f, f, f, 1 << 30, None) == code
+    assert lib.ssa_sparse_attn_fwd_host_workspace(p) == 0
 
 
 def test_null_problem(lib):
@@ -161,3 +163,15 @@ def test_dash_arguments_are_checked_before_launch(lib):
     big = ctypes.byref(_p(seq_len=65536 + 64))
     assert lib.ssa_dash_route(big, f, f, 1.5, 1.0, f, f, None) == UNSUPPORTED
     assert lib.ssa_dash_attn_fwd(big, f, f, f, f, f, 1.0, f, f, None) == UNSUPPORTED
+
+
+def test_host_buffer_forward_checks_pointers_and_workspace_before_any_copy(lib):
+    p = ctypes.byref(_p())
+    f = FAKE
+    need = lib.ssa_sparse_attn_fwd_host_workspace(p)
+    assert need > 0
+    assert lib.ssa_sparse_attn_fwd_host(p, None, f, f, f, f, f, need, None) == INVALID
+    assert lib.ssa_sparse_attn_fwd_host(p, f, f, f, f, None, f, need, None) == INVALID
+    assert lib.ssa_sparse_attn_fwd_host(p, f, f, f, f, f, None, need, None) == WORKSPACE
+    assert lib.ssa_sparse_attn_fwd_host(p, f, f, f, f, f, f, need - 1, None) == WORKSPACE
+    assert lib.ssa_sparse_attn_fwd_host(p, f, f, f, f, f, f + 16, need, None) == WORKSPACE   # not 256-aligned
