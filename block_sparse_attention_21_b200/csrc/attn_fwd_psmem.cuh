@@ -13,6 +13,15 @@
 // one pass ("Resumen Tecnico: SSA", section 2, "Alineacion Bidireccional",
 // and section 1 on the dropped mass).
 //
+// Two more modes reuse the pipeline:
+//   DASH   the routed chunks of a DashAttention mask, each block's scores
+//          offset by sigma * log2 w_j ("Resumen Tecnico: DashAttention",
+//          stage 2, prior-induced softmax); see dash_build_list.
+//   EARLY  the selected blocks in descending pooled score after the diagonal,
+//          each M-tile stopping once a block adds less than tau times the
+//          mass gathered before it (the "S2O" summary, section 2); see
+//          early_visit_order.
+//
 // Pipeline per M-tile t and visited block jj:
 //   S_t(jj) = Q_t K(jj)^T          tensor core, fp32 in TMEM
 //   softmax warps load S_t(jj) into registers and release it at once, so the
