@@ -112,6 +112,7 @@ __global__ void __launch_bounds__(kDecodeSelThreads) decode_score_kernel(const D
   const int L = p.len[b];
   if (L < 1 || L > p.S) return;  // reported by the selection kernel
   const int c = (L - 1) / 64;   // complete blocks before the query's own
+  if (c + 1 <= p.topk) return;   // every causal block is kept: no ranking
   const int j0 = blockIdx.x * kDecodeSelThreads;
   if (j0 >= c) return;           // the whole CTA: nothing to score here
   decode_group_query<D>(p, b, h, qs);
@@ -167,9 +168,15 @@ __global__ void __launch_bounds__(kDecodeSelThreads) decode_select_kernel(const 
   for (int shift = 24; shift >= 0 && need > 0; shift -= 8) {
     for (int x = threadIdx.x; x < 256; x += blockDim.x) hist[x] = 0u;
     __syncthreads();
-    for (int j = threadIdx.x; j < c; j += blockDim.x) {
-      const uint32_t kj = dkey[j];
-      if ((kj & tmask) == T) atomicAdd(&hist[(kj >> shift) & 255u], 1u);
+    // lanes with the same digit add once per warp (scores of similar size
+    // share their leading digits, so a plain atomic per key would serialise)
+    for (int j0 = 0; j0 < c; j0 += blockDim.x) {
+      const int j = j0 + static_cast<int>(threadIdx.x);
+      const uint32_t kj = j < c ? dkey[j] : 0u;
+      const bool in = j < c && (kj & tmask) == T;
+      const unsigned digit = in ? (kj >> shift) & 255u : 256u;  // 256: not counted
+      const unsigned peers = __match_any_sync(0xffffffffu, digit);
+      if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], static_cast<unsigned>(__popc(peers)));
     }
     __syncthreads();
     if (warp == 0) {
