@@ -388,15 +388,22 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_attn_kernel(const Decod
   uint64_t acc[GPH];
 #pragma unroll
   for (int x = 0; x < GPH; ++x) acc[x] = 0;
-#pragma unroll 8
-  for (int r = 0; r < 64; ++r) {
-    const uint64_t v2 = dec_bf2(*reinterpret_cast<const uint32_t*>(vs + r * RB + 4 * cp));
+  // four keys at a time: their V pairs, then each head's four probabilities
+  // with one 16-byte load
+#pragma unroll 2
+  for (int r0 = 0; r0 < 64; r0 += 4) {
+    uint64_t v2[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v2[u] = dec_bf2(*reinterpret_cast<const uint32_t*>(vs + (r0 + u) * RB + 4 * cp));
 #pragma unroll
     for (int x = 0; x < GPH; ++x) {
       const int g = hg * GPH + x;
       if (g < G) {
-        const float pr = ps[g * 64 + r];
-        acc[x] = dec_f2_fma(dec_f2(pr, pr), v2, acc[x]);
+        const float4 p4 = *reinterpret_cast<const float4*>(ps + g * 64 + r0);
+        acc[x] = dec_f2_fma(dec_f2(p4.x, p4.x), v2[0], acc[x]);
+        acc[x] = dec_f2_fma(dec_f2(p4.y, p4.y), v2[1], acc[x]);
+        acc[x] = dec_f2_fma(dec_f2(p4.z, p4.z), v2[2], acc[x]);
+        acc[x] = dec_f2_fma(dec_f2(p4.w, p4.w), v2[3], acc[x]);
       }
     }
   }
