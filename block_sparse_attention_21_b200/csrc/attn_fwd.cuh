@@ -72,7 +72,7 @@ struct FwdConfig {
   static constexpr int TMEM_COLS = pow2_at_least(T * TSTRIDE);
   static constexpr int THREADS = 64 + 128 * T;
   static constexpr int ISS = 1;                   // MMA issuer warps (warp 1)
-  static constexpr int POLY = (D == 128) ? 3 : 0; // exp2 pairs of 8 on the FMA pipe
+  static constexpr int POLY = (D == 128) ? 3 : (MASS ? 0 : 1);  // exp2 pairs of 8 on the FMA pipe
   static constexpr int NBARS = 1 + ISS + 3 * NS + 4 * T;
   // shared memory: Q tiles, K ring, V ring, barriers, tmem slot, abort flag,
   // selection bitmap (up to 8192 blocks)
