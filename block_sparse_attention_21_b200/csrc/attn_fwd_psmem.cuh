@@ -64,7 +64,7 @@ struct PsFwdConfig {
   static constexpr int NS = (D == 64) ? 4 : 3;    // K/V ring stages
   static constexpr int TSTRIDE = 64 + (MASS ? 2 : 1) * D;  // TMEM columns per M-tile
   static constexpr int TMEM_COLS = pow2_at_least(T * TSTRIDE);
-  static constexpr int POLY = 3;                  // exp2 pairs of 8 on the FMA pipe
+  static constexpr int POLY = 4;                  // exp2 pairs of 8 on the FMA pipe
   // warps: 0 producer, 1..3 issuers, 4.. softmax (4 per tile), then the
   // issuer of a fourth tile
   static constexpr int THREADS = 128 * (T + 1) + (T > 3 ? 32 : 0);
