@@ -48,6 +48,19 @@
 //
 // TMEM per M-tile t (stride 64 + D, or 64 + 2D with MASS): S at +0 (64 fp32
 // columns), O (O_selected with MASS) at +64, O_unselected at +64 + D.
+//
+// Persistent CTAs (plain sparse stream).  One CTA per SM takes the work units
+// blockIdx.x, blockIdx.x + gridDim.x, ... (heaviest query blocks first) and
+// every barrier keeps counting across units: the K/V ring, the score, P and
+// P.V barriers by the CTA's running block count, the Q and output barriers by
+// its running unit count.  So the producer loads the next unit's first K/V
+// block, and its Q as soon as both tiles' last score MMA has read the old Q
+// (bar_qfree); each issuer starts the next unit's first score MMA while the
+// softmax warps still write the previous unit's output; and the next unit's
+// first P.V (which overwrites O) waits on P, which the softmax warps store only
+// after their epilogue has read O.  With one CTA per SM, a new CTA per unit
+// would leave the SM idle for the unit's prologue and epilogue.  The other
+// modes run one unit per CTA through the same code.
 #pragma once
 
 #include "sm100.cuh"
@@ -68,8 +81,8 @@ struct PsFwdConfig {
   // warps: 0 producer, 1..3 issuers, 4.. softmax (4 per tile), then the
   // issuer of a fourth tile
   static constexpr int THREADS = 128 * (T + 1) + (T > 3 ? 32 : 0);
-  // barriers: q, kfull/vfull/empty[NS], sfull/sfree/pfull/pvdone/odone/drain[T]
-  static constexpr int NBARS = 1 + 3 * NS + 7 * T;
+  // barriers: q, kfull/vfull/empty[NS], sfull/sfree/pfull/pvdone/odone/drain/turn[T], qfree
+  static constexpr int NBARS = 1 + 3 * NS + 7 * T + 1;
   // shared memory: Q tiles, K ring, V ring, P tiles, barriers, tmem slot,
   // abort flag, selection bitmap (up to 8192 blocks); DASH: the routed chunk
   // list and its biases (kDashMaxN each) and the count
@@ -116,7 +129,8 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH, EARLY>::THREADS,
   uint64_t* bar_odone = bar_pvdone + T;         // [T] last P.V completed
   uint64_t* bar_drain = bar_odone + T;          // [T] issuer's MMAs drained (abort)
   uint64_t* bar_turn = bar_drain + T;           // [T] tile t may exponentiate (T = 2)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_turn + T);
+  uint64_t* bar_qfree = bar_turn + T;           // every tile's last score MMA of a unit read Q
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_qfree + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint32_t* selbits = tmem_slot + 4;
   // DASH: routed chunks in ascending order then the diagonal, their biases
@@ -135,18 +149,33 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH, EARLY>::THREADS,
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
-  // work unit, heaviest query blocks first
+  // work units, heaviest query blocks first; the plain sparse stream runs
+  // persistent CTAs over units blockIdx.x, blockIdx.x + gridDim.x, ..., the
+  // other modes one unit per CTA
+  constexpr bool PERSIST = !MASS && !DASH && !EARLY;
   const int per_i = p.B * p.Hkv * p.slices;
-  const int i = p.n - 1 - static_cast<int>(blockIdx.x) / per_i;
-  int rem = static_cast<int>(blockIdx.x) % per_i;
-  const int slice = rem % p.slices;
-  rem /= p.slices;
-  const int h = rem % p.Hkv;
-  const int b = rem / p.Hkv;
-  const int hq0 = h * p.G + slice * 2 * T;
-  const int nsel = min(p.topk, i + 1);
+  const int n_units = PERSIST ? p.n * per_i : static_cast<int>(blockIdx.x) + 1;
+  struct Unit {
+    int i, b, h, slice, hq0, nsel;
+    const int32_t* idx_row;
+  };
+  auto unit_of = [&](int u) {
+    Unit w;
+    w.i = p.n - 1 - u / per_i;
+    int rem = u % per_i;
+    w.slice = rem % p.slices;
+    rem /= p.slices;
+    w.h = rem % p.Hkv;
+    w.b = rem / p.Hkv;
+    w.hq0 = w.h * p.G + w.slice * 2 * T;
+    w.nsel = min(p.topk, w.i + 1);
+    w.idx_row = p.idx + ((static_cast<size_t>(w.b) * p.Hkv + w.h) * p.n + w.i) * p.topk;
+    return w;
+  };
+  const Unit u0 = unit_of(static_cast<int>(blockIdx.x));
+  const int i = u0.i, b = u0.b, h = u0.h, slice = u0.slice, hq0 = u0.hq0, nsel = u0.nsel;
   int nblk = MASS ? (i + 1) : nsel;  // DASH: the routed count, known after the prologue
-  const int32_t* idx_row = p.idx + ((static_cast<size_t>(b) * p.Hkv + h) * p.n + i) * p.topk;
+  const int32_t* idx_row = u0.idx_row;
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
@@ -164,6 +193,7 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH, EARLY>::THREADS,
       mbar_init(&bar_drain[t], 1);
       mbar_init(&bar_turn[t], 128);
     }
+    mbar_init(bar_qfree, T);  // one commit per tile's issuer and unit
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -206,46 +236,97 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH, EARLY>::THREADS,
       for (int pn = 0; pn < NP; ++pn)
         tma_load_4d(sV + st * KVT + pn * (64 * 128), &tm_v, &bar_vfull[st], 64 * pn, h, 64 * j, b);
     };
-    if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(bar_q, T * QTILE);
-      for (int t = 0; t < T; ++t)
-        for (int hh = 0; hh < 2; ++hh)
-          for (int pn = 0; pn < NP; ++pn)
-            tma_load_4d(sQ + t * QTILE + pn * (128 * 128) + hh * (64 * 128), &tm_q, bar_q,
-                        64 * pn, hq0 + 2 * t + hh, 64 * i, b);
-      if (EARLY) load_kv(0, i);  // the diagonal block is visited first
-    }
-    if (EARLY) early_visit_order<D>(p, b, h, i, nsel, idx_row, lane, ord, esc, ej);
-    if (lane == 0) {
-      int issued = EARLY ? 1 : 0;
-      for (int jj = issued; jj < nblk; ++jj) {
-        const int st = jj % NS, use = jj / NS;
-        if (EARLY && *all_stop) break;  // every tile stopped: no more blocks
-        // EARLY: once every tile stopped, the stage may never be released;
-        // the stop flag ends the wait instead
-        if (use > 0 && !(EARLY ? mbar_wait_or(&bar_empty[st], (use - 1) & 1, abort_flag, all_stop, tmo, 0x101)
-                               : mbar_wait(&bar_empty[st], (use - 1) & 1, abort_flag, tmo, 0x101)))
-          break;
-        load_kv(st, MASS ? jj : (DASH ? dord[jj] : (EARLY ? ord[jj] : idx_row[jj])));
-        ++issued;
-      }
-      // on abort or an early stop, loads already issued are waited for
-      // (bounded) before exit
-      if (*abort_flag || (EARLY && issued < nblk)) {
-        volatile int never = 0;
-        for (int jj = (issued > NS ? issued - NS : 0); jj < issued; ++jj) {
-          mbar_wait(&bar_kfull[jj % NS], (jj / NS) & 1, &never, 1000000ull, 0x1fe);
-          mbar_wait(&bar_vfull[jj % NS], (jj / NS) & 1, &never, 1000000ull, 0x1ff);
+    if (PERSIST) {
+      if (lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        // per unit: its first K/V block, then its Q once both tiles' last
+        // score MMA of the previous unit has read the old Q, then the rest
+        int g = 0, k = 0;  // K/V blocks and units loaded so far
+        int qk = -1;       // the last unit whose Q was loaded
+        bool alive = true;
+        for (int u = static_cast<int>(blockIdx.x); alive && u < n_units; u += gridDim.x, ++k) {
+          const Unit w = unit_of(u);
+          for (int s = 0; s < w.nsel; ++s) {
+            const int st = g % NS, use = g / NS;
+            if (use > 0 && !mbar_wait(&bar_empty[st], (use - 1) & 1, abort_flag, tmo, 0x101)) {
+              alive = false;
+              break;
+            }
+            const int j = w.idx_row[s];
+            mbar_arrive_expect_tx(&bar_kfull[st], KVT);
+            for (int pn = 0; pn < NP; ++pn)
+              tma_load_4d(sK + st * KVT + pn * (64 * 128), &tm_k, &bar_kfull[st], 64 * pn, w.h, 64 * j, w.b);
+            mbar_arrive_expect_tx(&bar_vfull[st], KVT);
+            for (int pn = 0; pn < NP; ++pn)
+              tma_load_4d(sV + st * KVT + pn * (64 * 128), &tm_v, &bar_vfull[st], 64 * pn, w.h, 64 * j, w.b);
+            ++g;
+            if (s == 0) {
+              if (k > 0 && !mbar_wait(bar_qfree, (k - 1) & 1, abort_flag, tmo, 0x102)) {
+                alive = false;
+                break;
+              }
+              mbar_arrive_expect_tx(bar_q, T * QTILE);
+              for (int t = 0; t < T; ++t)
+                for (int hh = 0; hh < 2; ++hh)
+                  for (int pn = 0; pn < NP; ++pn)
+                    tma_load_4d(sQ + t * QTILE + pn * (128 * 128) + hh * (64 * 128), &tm_q, bar_q,
+                                64 * pn, w.hq0 + 2 * t + hh, 64 * w.i, w.b);
+              qk = k;
+            }
+          }
+        }
+        // on abort, the loads already issued are waited for (bounded) before exit
+        if (*abort_flag) {
+          volatile int never = 0;
+          for (int gj = (g > NS ? g - NS : 0); gj < g; ++gj) {
+            mbar_wait(&bar_kfull[gj % NS], (gj / NS) & 1, &never, 1000000ull, 0x1fe);
+            mbar_wait(&bar_vfull[gj % NS], (gj / NS) & 1, &never, 1000000ull, 0x1ff);
+          }
+          if (qk >= 0) mbar_wait(bar_q, qk & 1, &never, 1000000ull, 0x1fd);
         }
       }
-    }
+    } else {
+      if (lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        mbar_arrive_expect_tx(bar_q, T * QTILE);
+        for (int t = 0; t < T; ++t)
+          for (int hh = 0; hh < 2; ++hh)
+            for (int pn = 0; pn < NP; ++pn)
+              tma_load_4d(sQ + t * QTILE + pn * (128 * 128) + hh * (64 * 128), &tm_q, bar_q,
+                          64 * pn, hq0 + 2 * t + hh, 64 * i, b);
+        if (EARLY) load_kv(0, i);  // the diagonal block is visited first
+      }
+      if (EARLY) early_visit_order<D>(p, b, h, i, nsel, idx_row, lane, ord, esc, ej);
+      if (lane == 0) {
+        int issued = EARLY ? 1 : 0;
+        for (int jj = issued; jj < nblk; ++jj) {
+          const int st = jj % NS, use = jj / NS;
+          if (EARLY && *all_stop) break;  // every tile stopped: no more blocks
+          // EARLY: once every tile stopped, the stage may never be released;
+          // the stop flag ends the wait instead
+          if (use > 0 && !(EARLY ? mbar_wait_or(&bar_empty[st], (use - 1) & 1, abort_flag, all_stop, tmo, 0x101)
+                                 : mbar_wait(&bar_empty[st], (use - 1) & 1, abort_flag, tmo, 0x101)))
+            break;
+          load_kv(st, MASS ? jj : (DASH ? dord[jj] : (EARLY ? ord[jj] : idx_row[jj])));
+          ++issued;
+        }
+        // on abort or an early stop, loads already issued are waited for
+        // (bounded) before exit
+        if (*abort_flag || (EARLY && issued < nblk)) {
+          volatile int never = 0;
+          for (int jj = (issued > NS ? issued - NS : 0); jj < issued; ++jj) {
+            mbar_wait(&bar_kfull[jj % NS], (jj / NS) & 1, &never, 1000000ull, 0x1fe);
+            mbar_wait(&bar_vfull[jj % NS], (jj / NS) & 1, &never, 1000000ull, 0x1ff);
+          }
+        }
+      }
+    }  // one unit
   } else if (warp != 0 && (warp < 4 || warp >= 4 + 4 * T)) {
     // ------------------------------------------------------------ MMA issuers
-    // The issuer of tile t walks  S(0);  then for s = 0, 1, ...:
-    //   [S(s) read]  S(s+1);   [P(s) in shared memory]  O += P(s) V(s)
     int t = -1;
 #pragma unroll
     for (int x = 0; x < T; ++x)
@@ -264,65 +345,78 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH, EARLY>::THREADS,
           mma_ss(s_tmem, a, bd, idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(bar_q, 0, abort_flag, tmo, 0x201) &&
-                mbar_wait(&bar_kfull[0], 0, abort_flag, tmo, 0x202);
-      if (ok) {
+      // Per unit: S(0) once its Q and first K/V block landed and the softmax
+      // read the previous unit's last scores; then for s = 0, 1, ...:
+      //   [S(s) read]  S(s+1);   [P(s) in shared memory]  O += P(s) V(s)
+      // Parities count the CTA's blocks (g + s) and units (k).
+      bool ok = true;
+      int g = 0, k = 0;
+      for (int u = static_cast<int>(blockIdx.x); ok && u < n_units; u += gridDim.x, ++k) {
+        const int nb = PERSIST ? unit_of(u).nsel : nblk;
+        ok = mbar_wait(bar_q, k & 1, abort_flag, tmo, 0x201) &&
+             mbar_wait(&bar_kfull[g % NS], (g / NS) & 1, abort_flag, tmo, 0x202) &&
+             (g == 0 || mbar_wait(&bar_sfree[t], (g - 1) & 1, abort_flag, tmo, 0x203));
+        if (!ok) break;
         tc_fence_after();
-        issue_qk(0);
+        issue_qk(g % NS);
         tc_commit(&bar_sfull[t]);
-      }
-      bool first_sel = true, first_uns = true;
-      for (int s = 0; ok && s < nblk; ++s) {
-        if (s + 1 < nblk) {
-          // S(s+1) as soon as the softmax has read S(s)
-          const int st1 = (s + 1) % NS;
-          if (!mbar_wait(&bar_sfree[t], s & 1, abort_flag, tmo, 0x203) ||
-              !mbar_wait(&bar_kfull[st1], ((s + 1) / NS) & 1, abort_flag, tmo, 0x204)) {
+        if (PERSIST && nb == 1) tc_commit(bar_qfree);  // the unit's last score MMA read Q
+        bool first_sel = true, first_uns = true;
+        for (int s = 0; ok && s < nb; ++s) {
+          const int gs = g + s;
+          if (s + 1 < nb) {
+            // S(s+1) as soon as the softmax has read S(s)
+            const int st1 = (gs + 1) % NS;
+            if (!mbar_wait(&bar_sfree[t], gs & 1, abort_flag, tmo, 0x203) ||
+                !mbar_wait(&bar_kfull[st1], ((gs + 1) / NS) & 1, abort_flag, tmo, 0x204)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_qk(st1);
+            tc_commit(&bar_sfull[t]);
+            if (PERSIST && s + 2 == nb) tc_commit(bar_qfree);
+          }
+          // P(s).V once P(s) is in shared memory
+          const int st = gs % NS;
+          if (!mbar_wait(&bar_pfull[t], gs & 1, abort_flag, tmo, 0x205) ||
+              !mbar_wait(&bar_vfull[st], (gs / NS) & 1, abort_flag, tmo, 0x206)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          issue_qk(st1);
-          tc_commit(&bar_sfull[t]);
-        }
-        // P(s).V once P(s) is in shared memory
-        const int st = s % NS;
-        if (!mbar_wait(&bar_pfull[t], s & 1, abort_flag, tmo, 0x205) ||
-            !mbar_wait(&bar_vfull[st], (s / NS) & 1, abort_flag, tmo, 0x206)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        bool is_sel = true;
-        if (MASS) is_sel = (selbits[s >> 5] >> (s & 31)) & 1u;
-        const bool first = MASS ? (is_sel ? first_sel : first_uns) : (s == 0);
-        const uint32_t o_col = s_tmem + 64 + ((MASS && !is_sel) ? D : 0);
+          bool is_sel = true;
+          if (MASS) is_sel = (selbits[s >> 5] >> (s & 31)) & 1u;
+          const bool first = MASS ? (is_sel ? first_sel : first_uns) : (s == 0);
+          const uint32_t o_col = s_tmem + 64 + ((MASS && !is_sel) ? D : 0);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t a = sdesc_sw128(sPa + t * PTILE + kk * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(sVa + st * KVT + kk * (16 * 128), 64 * 128, 1024);
-          mma_ss(o_col, a, bd, idesc_pv, (first && kk == 0) ? 0u : 1u);
-        }
-        tc_commit(&bar_pvdone[t]);
-        // EARLY: the softmax set the tile's stop flag before it arrived on pfull
-        const bool stop_now = EARLY && tile_stop[t] != 0;
-        if (s + 1 == nblk || stop_now) tc_commit(&bar_odone[t]);
-        tc_commit(&bar_empty[st]);
-        if (MASS) {
-          if (is_sel) first_sel = false; else first_uns = false;
-        }
-        if (EARLY && stop_now) {
-          // the other tiles still need every stage released by this tile too:
-          // release each remaining block's stage once it is loaded, until the
-          // last block or until every tile has stopped (the producer then
-          // loads nothing more)
-          if (atomicAdd(nstopped, 1) + 1 == T) *all_stop = 1;
-          for (int s2 = s + 1; s2 < nblk; ++s2) {
-            if (!mbar_wait_or(&bar_vfull[s2 % NS], (s2 / NS) & 1, abort_flag, all_stop, tmo, 0x207)) break;
-            tc_commit(&bar_empty[s2 % NS]);
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t a = sdesc_sw128(sPa + t * PTILE + kk * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(sVa + st * KVT + kk * (16 * 128), 64 * 128, 1024);
+            mma_ss(o_col, a, bd, idesc_pv, (first && kk == 0) ? 0u : 1u);
           }
-          break;
+          tc_commit(&bar_pvdone[t]);
+          // EARLY: the softmax set the tile's stop flag before it arrived on pfull
+          const bool stop_now = EARLY && tile_stop[t] != 0;
+          if (s + 1 == nb || stop_now) tc_commit(&bar_odone[t]);
+          tc_commit(&bar_empty[st]);
+          if (MASS) {
+            if (is_sel) first_sel = false; else first_uns = false;
+          }
+          if (EARLY && stop_now) {
+            // the other tiles still need every stage released by this tile too:
+            // release each remaining block's stage once it is loaded, until the
+            // last block or until every tile has stopped (the producer then
+            // loads nothing more)
+            if (atomicAdd(nstopped, 1) + 1 == T) *all_stop = 1;
+            for (int s2 = g + s + 1; s2 < g + nb; ++s2) {
+              if (!mbar_wait_or(&bar_vfull[s2 % NS], (s2 / NS) & 1, abort_flag, all_stop, tmo, 0x207)) break;
+              tc_commit(&bar_empty[s2 % NS]);
+            }
+            break;
+          }
         }
+        g += nb;
       }
       if (!ok) {
         // every MMA this thread issued completes before TMEM is released
@@ -337,7 +431,6 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH, EARLY>::THREADS,
     const int wq = warp % 4;
     const int r = wq * 32 + lane;
     const int hh = r / 64, tq = r % 64;
-    const int hq = hq0 + 2 * t + hh;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16) + t * TSTRIDE;
     const uint32_t tS = lane_base, tO = lane_base + 64;
     const uint32_t tOu = tO + D;
@@ -345,164 +438,178 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH, EARLY>::THREADS,
     uint8_t* prow = sP + t * PTILE + r * 128;
     const float sl2 = p.scale_log2;
     const uint64_t scale2 = f2_pack(sl2, sl2);
-    float m_ref = -INFINITY;  // reference maximum, scaled (log2) units
-    float l_sel = 0.f, l_uns = 0.f;
-    int visited = 0;          // EARLY: blocks this tile visited
     bool ok = true;
-    for (int jj = 0; jj < nblk; ++jj) {
-      // waits are made warp-uniform: the tcgen05.ld/st below are .sync.aligned
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar_sfull[t], jj & 1, abort_flag, tmo, 0x301))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      float sA[32], sB[32];
-      tmem_ld32(tS, sA);
-      tmem_ld32(tS + 32, sB);
-      // the scores are in registers: the issuer may overwrite S with the next block's
-      tc_fence_before();
-      mbar_arrive(&bar_sfree[t]);
-      // the diagonal block comes last in the ascending table, first in the
-      // early-stop order
-      const bool diag = EARLY ? (jj == 0) : (jj == nblk - 1);
-      bool is_sel = true;
-      if (MASS) is_sel = (selbits[jj >> 5] >> (jj & 31)) & 1u;
-      // with two tiles, their exponential phases alternate: tile 1's block jj
-      // follows tile 0's block jj, tile 0's block jj + 1 follows tile 1's
-      // block jj, so one tile's MMAs run while the other exponentiates (not
-      // with the early stop, where one tile may stop before the other)
-      if (T == 2 && !EARLY && (t == 1 || jj > 0) &&
-          !__all_sync(0xffffffffu, mbar_wait(&bar_turn[t], (t == 1 ? jj : jj - 1) & 1, abort_flag, tmo,
-                                             0x305))) {
-        ok = false;
-        break;
-      }
-      float mx = diag ? row_max32<true>(sB, 32, tq, -INFINITY) : row_max32<false>(sB, 32, tq, -INFINITY);
-      mx = diag ? row_max32<true>(sA, 0, tq, mx) : row_max32<false>(sA, 0, tq, mx);
-      // DASH: the chunk's prior adds sigma * log2 w_j to every score of the block
-      const float bias = DASH ? dbias[jj] : 0.f;
-      const float mx_s = mx * sl2 + bias;
-      float alpha = 1.f;
-      const bool moved = mx_s > m_ref + 8.f;
-      if (moved) {
-        alpha = ex2(m_ref - mx_s);
-        m_ref = mx_s;
-      }
-      const uint64_t negm2 = f2_pack(bias - m_ref, bias - m_ref);
-      uint64_t acc2 = f2_pack(0.f, 0.f);
-      uint32_t pk[32];
-      if (diag) {
-        exp_pack32<true>(sA, 0, tq, scale2, negm2, acc2, pk);
-        exp_pack32<true>(sB, 32, tq, scale2, negm2, acc2, pk + 16);
-      } else {
-        exp_pack32<false, C::POLY>(sA, 0, tq, scale2, negm2, acc2, pk);
-        exp_pack32<false, C::POLY>(sB, 32, tq, scale2, negm2, acc2, pk + 16);
-      }
-      if (T == 2 && !EARLY) mbar_arrive(&bar_turn[1 - t]);
-      float r0, r1;
-      f2_unpack(acc2, r0, r1);
-      bool stop = false;
-      if (EARLY && jj > 0 && p.tau > 0.f) {
-        // this block's mass against the mass accumulated before it (both in
-        // the current reference); the tile stops when no row gained at least
-        // tau times what it had (tau = 0 never stops: no decision is taken)
-        const bool cont_row = (r0 + r1) >= p.tau * (l_sel * alpha);
-        volatile int* wf = wflag + (t * 2 + (jj & 1)) * 4;
-        const bool wcont = __any_sync(0xffffffffu, cont_row);
-        if (lane == 0) wf[wq] = wcont ? 1 : 0;
-        named_bar_sync(1 + t, 128);
-        stop = !(wf[0] | wf[1] | wf[2] | wf[3]);
-        if (stop && r == 0) tile_stop[t] = 1;  // read by the issuer after pfull
-      }
-      l_sel *= alpha;
-      l_uns *= alpha;
-      if (is_sel) l_sel += r0 + r1; else l_uns += r0 + r1;
-      if (jj > 0) {
-        // P(jj-1).V has finished: the P tile may be overwritten and O is stable
-        if (!__all_sync(0xffffffffu, mbar_wait(&bar_pvdone[t], (jj - 1) & 1, abort_flag, tmo, 0x302))) {
+    // parities count the CTA's blocks (g + jj) and units (k)
+    int g = 0, k = 0;
+    for (int u = static_cast<int>(blockIdx.x); ok && u < n_units; u += gridDim.x, ++k) {
+      const Unit w = PERSIST ? unit_of(u) : u0;
+      const int nb = PERSIST ? w.nsel : nblk;
+      const int hq = w.hq0 + 2 * t + hh;
+      float m_ref = -INFINITY;  // reference maximum, scaled (log2) units
+      float l_sel = 0.f, l_uns = 0.f;
+      int visited = 0;          // EARLY: blocks this tile visited
+      for (int jj = 0; jj < nb; ++jj) {
+        const int gj = g + jj;
+        // waits are made warp-uniform: the tcgen05.ld/st below are .sync.aligned
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar_sfull[t], gj & 1, abort_flag, tmo, 0x301))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, moved)) {
-          const uint64_t a2 = f2_pack(alpha, alpha);
-#pragma unroll
-          for (int acc = 0; acc < (MASS ? 2 : 1); ++acc) {
-            const uint32_t base = acc ? tOu : tO;
-#pragma unroll
-            for (int ch = 0; ch < D / 16; ++ch) {
-              float o[16];
-              uint32_t w[16];
-              tmem_ld16(base + ch * 16, o);
-#pragma unroll
-              for (int c = 0; c < 16; c += 2) {
-                float lo, hi;
-                f2_unpack(f2_mul(f2_pack(o[c], o[c + 1]), a2), lo, hi);
-                w[c] = __float_as_uint(lo);
-                w[c + 1] = __float_as_uint(hi);
-              }
-              tmem_st16(base + ch * 16, w);
-            }
-          }
-          tmem_wait_st();
+        float sA[32], sB[32];
+        tmem_ld32(tS, sA);
+        tmem_ld32(tS + 32, sB);
+        // the scores are in registers: the issuer may overwrite S with the next block's
+        tc_fence_before();
+        mbar_arrive(&bar_sfree[t]);
+        // the diagonal block comes last in the ascending table, first in the
+        // early-stop order
+        const bool diag = EARLY ? (jj == 0) : (jj == nb - 1);
+        bool is_sel = true;
+        if (MASS) is_sel = (selbits[jj >> 5] >> (jj & 31)) & 1u;
+        // with two tiles, their exponential phases alternate: tile 1's block jj
+        // follows tile 0's block jj, tile 0's block jj + 1 follows tile 1's
+        // block jj, so one tile's MMAs run while the other exponentiates (not
+        // with the early stop, where one tile may stop before the other); the
+        // order runs on across units
+        if (T == 2 && !EARLY && (t == 1 || gj > 0) &&
+            !__all_sync(0xffffffffu, mbar_wait(&bar_turn[t], (t == 1 ? gj : gj - 1) & 1, abort_flag, tmo,
+                                               0x305))) {
+          ok = false;
+          break;
         }
-      }
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) =
-            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(&bar_pfull[t]);
-      if (EARLY) visited = jj + 1;
-      if (stop) break;
-    }
-    // ---------------------------------------------------------- epilogue
-    if (ok && __all_sync(0xffffffffu, mbar_wait(&bar_odone[t], 0, abort_flag, tmo, 0x303))) {
-      tc_fence_after();
-      const int tok = 64 * i + tq;
-      const size_t orow = ((static_cast<size_t>(b) * p.S + tok) * p.Hq + hq) * D;
-      const size_t lrow = (static_cast<size_t>(b) * p.Hq + hq) * p.S + tok;
-      const bool has_uns = MASS && (nblk > nsel);
-      const float inv_sel = 1.f / l_sel;
-      const float l_all = l_sel + (has_uns ? l_uns : 0.f);
-      const float inv_all = 1.f / l_all;
-#pragma unroll
-      for (int ch = 0; ch < D / 32; ++ch) {
-        float o[32];
-        tmem_ld32(tO + ch * 32, o);
-        uint32_t w[16];
-#pragma unroll
-        for (int c = 0; c < 16; ++c) w[c] = pack_bf16x2(o[2 * c] * inv_sel, o[2 * c + 1] * inv_sel);
-        uint4* dst = reinterpret_cast<uint4*>(p.o + orow + ch * 32);
-#pragma unroll
-        for (int v4 = 0; v4 < 4; ++v4)
-          dst[v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
-        if (MASS) {
-          if (has_uns) {
-            float ou[32];
-            tmem_ld32(tOu + ch * 32, ou);
-#pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] += ou[c];
+        float mx = diag ? row_max32<true>(sB, 32, tq, -INFINITY) : row_max32<false>(sB, 32, tq, -INFINITY);
+        mx = diag ? row_max32<true>(sA, 0, tq, mx) : row_max32<false>(sA, 0, tq, mx);
+        // DASH: the chunk's prior adds sigma * log2 w_j to every score of the block
+        const float bias = DASH ? dbias[jj] : 0.f;
+        const float mx_s = mx * sl2 + bias;
+        float alpha = 1.f;
+        const bool moved = mx_s > m_ref + 8.f;
+        if (moved) {
+          alpha = ex2(m_ref - mx_s);
+          m_ref = mx_s;
+        }
+        const uint64_t negm2 = f2_pack(bias - m_ref, bias - m_ref);
+        uint64_t acc2 = f2_pack(0.f, 0.f);
+        uint32_t pk[32];
+        if (diag) {
+          exp_pack32<true>(sA, 0, tq, scale2, negm2, acc2, pk);
+          exp_pack32<true>(sB, 32, tq, scale2, negm2, acc2, pk + 16);
+        } else {
+          exp_pack32<false, C::POLY>(sA, 0, tq, scale2, negm2, acc2, pk);
+          exp_pack32<false, C::POLY>(sB, 32, tq, scale2, negm2, acc2, pk + 16);
+        }
+        if (T == 2 && !EARLY) mbar_arrive(&bar_turn[1 - t]);
+        float r0, r1;
+        f2_unpack(acc2, r0, r1);
+        bool stop = false;
+        if (EARLY && jj > 0 && p.tau > 0.f) {
+          // this block's mass against the mass accumulated before it (both in
+          // the current reference); the tile stops when no row gained at least
+          // tau times what it had (tau = 0 never stops: no decision is taken)
+          const bool cont_row = (r0 + r1) >= p.tau * (l_sel * alpha);
+          volatile int* wf = wflag + (t * 2 + (jj & 1)) * 4;
+          const bool wcont = __any_sync(0xffffffffu, cont_row);
+          if (lane == 0) wf[wq] = wcont ? 1 : 0;
+          named_bar_sync(1 + t, 128);
+          stop = !(wf[0] | wf[1] | wf[2] | wf[3]);
+          if (stop && r == 0) tile_stop[t] = 1;  // read by the issuer after pfull
+        }
+        l_sel *= alpha;
+        l_uns *= alpha;
+        if (is_sel) l_sel += r0 + r1; else l_uns += r0 + r1;
+        if (jj > 0) {
+          // P(jj-1).V has finished: the P tile may be overwritten and O is stable
+          // (for jj = 0 the previous unit's epilogue waited for its last P.V)
+          if (!__all_sync(0xffffffffu, mbar_wait(&bar_pvdone[t], (gj - 1) & 1, abort_flag, tmo, 0x302))) {
+            ok = false;
+            break;
           }
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, moved)) {
+            const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
-          for (int c = 0; c < 16; ++c)
-            w[c] = pack_bf16x2(o[2 * c] * inv_all, o[2 * c + 1] * inv_all);
-          uint4* dstf = reinterpret_cast<uint4*>(p.o_full + orow + ch * 32);
+            for (int acc = 0; acc < (MASS ? 2 : 1); ++acc) {
+              const uint32_t base = acc ? tOu : tO;
+#pragma unroll
+              for (int ch = 0; ch < D / 16; ++ch) {
+                float o[16];
+                uint32_t w[16];
+                tmem_ld16(base + ch * 16, o);
+#pragma unroll
+                for (int c = 0; c < 16; c += 2) {
+                  float lo, hi;
+                  f2_unpack(f2_mul(f2_pack(o[c], o[c + 1]), a2), lo, hi);
+                  w[c] = __float_as_uint(lo);
+                  w[c + 1] = __float_as_uint(hi);
+                }
+                tmem_st16(base + ch * 16, w);
+              }
+            }
+            tmem_wait_st();
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) =
+              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&bar_pfull[t]);
+        if (EARLY) visited = jj + 1;
+        if (stop) break;
+      }
+      // ---------------------------------------------------------- epilogue
+      // (O is read here before this tile's next P store, which the next unit's
+      // first P.V waits for: so that P.V never overwrites O still being read)
+      if (ok && !__all_sync(0xffffffffu, mbar_wait(&bar_odone[t], k & 1, abort_flag, tmo, 0x303))) ok = false;
+      if (ok) {
+        tc_fence_after();
+        const int tok = 64 * w.i + tq;
+        const size_t orow = ((static_cast<size_t>(w.b) * p.S + tok) * p.Hq + hq) * D;
+        const size_t lrow = (static_cast<size_t>(w.b) * p.Hq + hq) * p.S + tok;
+        const bool has_uns = MASS && (nb > w.nsel);
+        const float inv_sel = 1.f / l_sel;
+        const float l_all = l_sel + (has_uns ? l_uns : 0.f);
+        const float inv_all = 1.f / l_all;
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) {
+          float o[32];
+          tmem_ld32(tO + ch * 32, o);
+          uint32_t w[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) w[c] = pack_bf16x2(o[2 * c] * inv_sel, o[2 * c + 1] * inv_sel);
+          uint4* dst = reinterpret_cast<uint4*>(p.o + orow + ch * 32);
 #pragma unroll
           for (int v4 = 0; v4 < 4; ++v4)
-            dstf[v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+            dst[v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+          if (MASS) {
+            if (has_uns) {
+              float ou[32];
+              tmem_ld32(tOu + ch * 32, ou);
+#pragma unroll
+              for (int c = 0; c < 32; ++c) o[c] += ou[c];
+            }
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+              w[c] = pack_bf16x2(o[2 * c] * inv_all, o[2 * c + 1] * inv_all);
+            uint4* dstf = reinterpret_cast<uint4*>(p.o_full + orow + ch * 32);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              dstf[v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+          }
+        }
+        constexpr float kLn2 = 0.69314718055994530942f;
+        p.lse[lrow] = (m_ref + log2f(l_sel)) * kLn2;
+        if (EARLY && r == 0 && p.visited != nullptr)
+          p.visited[((static_cast<size_t>(w.b) * p.Hkv + w.h) * p.n + w.i) * (p.G / 2) + w.slice * T + t] = visited;
+        if (MASS) {
+          p.lse_full[lrow] = (m_ref + log2f(l_all)) * kLn2;
+          p.dropped[lrow] = has_uns ? (l_uns / l_all) : 0.f;
         }
       }
-      constexpr float kLn2 = 0.69314718055994530942f;
-      p.lse[lrow] = (m_ref + log2f(l_sel)) * kLn2;
-      if (EARLY && r == 0 && p.visited != nullptr)
-        p.visited[((static_cast<size_t>(b) * p.Hkv + h) * p.n + i) * (p.G / 2) + slice * T + t] = visited;
-      if (MASS) {
-        p.lse_full[lrow] = (m_ref + log2f(l_all)) * kLn2;
-        p.dropped[lrow] = has_uns ? (l_uns / l_all) : 0.f;
-      }
-    }
+      g += nb;
+    }  // units
   }
 
   tc_fence_before();

@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdlib>
@@ -118,6 +119,19 @@ ssa_status ensure_smem(K kernel, int bytes, std::atomic<uint64_t>* done_mask) {
     return SSA_ERR_CUDA;
   done_mask->fetch_or(bit);
   return SSA_OK;
+}
+
+// Streaming multiprocessors of the current device (cached per device).
+int sm_count() {
+  static std::atomic<int> cached[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return 0;
+  int c = cached[dev].load();
+  if (c == 0) {
+    if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cached[dev].store(c);
+  }
+  return c;
 }
 
 ssa_status launch_result() {
@@ -269,7 +283,13 @@ ssa_status launch_psfwd(const Dims& d, const void* q, const void* k, const void*
   fp.dmask = dash.mask;
   fp.dw = dash.w;
   fp.sigma = dash.sigma;
-  const unsigned grid = static_cast<unsigned>(d.B) * d.Hkv * d.n * fp.slices;
+  // the plain sparse stream runs persistent CTAs, one per SM, over the units;
+  // the other modes one CTA per unit
+  const unsigned units = static_cast<unsigned>(d.B) * d.Hkv * d.n * fp.slices;
+  const unsigned sms = static_cast<unsigned>(sm_count());
+  const bool persist = !MASS && !DASH && !EARLY;
+  if (persist && sms == 0) return SSA_ERR_CUDA;
+  const unsigned grid = persist ? std::min(units, sms) : units;
   return launch_pdl(kernel, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, st, mq, mk, mv, fp);
 }
 
