@@ -24,6 +24,19 @@
 // Two CTAs share an SM when T = 2 (256 TMEM columns each), so one CTA's
 // prologue and epilogue overlap the other's main loop.
 //
+// Persistent CTAs (plain sparse stream): as many CTAs as fit on the GPU take
+// the work units blockIdx.x, blockIdx.x + gridDim.x, ... (heaviest query
+// blocks first), and every barrier keeps counting across units (the K/V ring,
+// score and P barriers by the CTA's running block count, the Q and output
+// barriers by its running unit count).  The producer loads the next unit's
+// first K/V block, and its Q once the last score MMAs of the previous unit
+// have read the old Q (bar_qfree); the issuer starts the next unit's score
+// MMAs right after the previous unit's last P.V (one thread's MMAs execute in
+// order, so S never overwrites a P still being read); and the next unit's
+// first P.V, which overwrites O, waits for P, which the softmax warps store
+// only after their epilogue has read O.  The other modes run one unit per CTA
+// through the same code.
+//
 // Warp roles (64 + 128 * T threads):
 //   warp 0      builds the selection bitmap (MASS), then is the TMA producer:
 //               the Q tiles once, then K and V of each visited block through
@@ -73,7 +86,7 @@ struct FwdConfig {
   static constexpr int THREADS = 64 + 128 * T;
   static constexpr int ISS = 1;                   // MMA issuer warps (warp 1)
   static constexpr int POLY = (D == 128) ? 3 : (MASS ? 0 : 1);  // exp2 pairs of 8 on the FMA pipe
-  static constexpr int NBARS = 1 + ISS + 3 * NS + 4 * T;
+  static constexpr int NBARS = 1 + ISS + 3 * NS + 4 * T + 1;
   // shared memory: Q tiles, K ring, V ring, barriers, tmem slot, abort flag,
   // selection bitmap (up to 8192 blocks)
   static constexpr int SMEM_TILES = T * QTILE + 2 * NS * KVT;
@@ -113,7 +126,8 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS, EARLY, DASH>::THREADS,
   uint64_t* bar_pfull = bar_phalf + T;  // all of P stored
   uint64_t* bar_odone = bar_pfull + T;
   uint64_t* bar_drain = bar_odone + T;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_drain + C::ISS);
+  uint64_t* bar_qfree = bar_drain + C::ISS;  // the last score MMAs of a unit read Q
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_qfree + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint32_t* selbits = tmem_slot + 4;
   // EARLY: visiting order (over the bitmap area), score scratch, stop flags
@@ -131,18 +145,33 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS, EARLY, DASH>::THREADS,
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
-  // work unit, heaviest query blocks first
+  // work units, heaviest query blocks first; the plain sparse stream runs
+  // persistent CTAs over units blockIdx.x, blockIdx.x + gridDim.x, ..., the
+  // other modes one unit per CTA
+  constexpr bool PERSIST = !MASS && !EARLY && !DASH;
   const int per_i = p.B * p.Hkv * p.slices;
-  const int i = p.n - 1 - static_cast<int>(blockIdx.x) / per_i;
-  int rem = static_cast<int>(blockIdx.x) % per_i;
-  const int slice = rem % p.slices;
-  rem /= p.slices;
-  const int h = rem % p.Hkv;
-  const int b = rem / p.Hkv;
-  const int hq0 = h * p.G + slice * 2 * T;
-  const int nsel = min(p.topk, i + 1);
+  const int n_units = PERSIST ? p.n * per_i : static_cast<int>(blockIdx.x) + 1;
+  struct Unit {
+    int i, b, h, slice, hq0, nsel;
+    const int32_t* idx_row;
+  };
+  auto unit_of = [&](int u) {
+    Unit w;
+    w.i = p.n - 1 - u / per_i;
+    int rem = u % per_i;
+    w.slice = rem % p.slices;
+    rem /= p.slices;
+    w.h = rem % p.Hkv;
+    w.b = rem / p.Hkv;
+    w.hq0 = w.h * p.G + w.slice * 2 * T;
+    w.nsel = min(p.topk, w.i + 1);
+    w.idx_row = p.idx + ((static_cast<size_t>(w.b) * p.Hkv + w.h) * p.n + w.i) * p.topk;
+    return w;
+  };
+  const Unit u0 = unit_of(static_cast<int>(blockIdx.x));
+  const int i = u0.i, b = u0.b, h = u0.h, hq0 = u0.hq0, nsel = u0.nsel;
   int nblk = MASS ? (i + 1) : nsel;  // DASH: the routed count, known after the prologue
-  const int32_t* idx_row = p.idx + ((static_cast<size_t>(b) * p.Hkv + h) * p.n + i) * p.topk;
+  const int32_t* idx_row = u0.idx_row;
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
@@ -158,6 +187,7 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS, EARLY, DASH>::THREADS,
       mbar_init(&bar_odone[t], 1);
     }
     for (int x = 0; x < C::ISS; ++x) mbar_init(&bar_drain[x], 1);
+    mbar_init(bar_qfree, C::ISS);  // one commit per issuer and unit
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -199,42 +229,95 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS, EARLY, DASH>::THREADS,
       for (int pn = 0; pn < NP; ++pn)
         tma_load_4d(sV + st * KVT + pn * (64 * 128), &tm_v, &bar_vfull[st], 64 * pn, h, 64 * j, b);
     };
-    if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(bar_q, T * QTILE);
-      for (int t = 0; t < T; ++t)
-        for (int hh = 0; hh < 2; ++hh)
-          for (int pn = 0; pn < NP; ++pn)
-            tma_load_4d(sQ + t * QTILE + pn * (128 * 128) + hh * (64 * 128), &tm_q, bar_q,
-                        64 * pn, hq0 + 2 * t + hh, 64 * i, b);
-      if (EARLY) load_kv(0, i);  // the diagonal block is visited first
-    }
-    if (EARLY) early_visit_order<D>(p, b, h, i, nsel, idx_row, lane, ord, esc, ej);
-    if (lane == 0) {
-      int issued = EARLY ? 1 : 0;
-      for (int jj = issued; jj < nblk; ++jj) {
-        const int st = jj % NS, use = jj / NS;
-        if (EARLY && *all_stop) break;  // every tile stopped: no more blocks
-        // EARLY: once every tile stopped, the stage is never released; the
-        // stop flag ends the wait instead
-        if (use > 0 && !(EARLY ? mbar_wait_or(&bar_empty[st], (use - 1) & 1, abort_flag, all_stop, tmo, 0x101)
-                               : mbar_wait(&bar_empty[st], (use - 1) & 1, abort_flag, tmo, 0x101)))
-          break;
-        load_kv(st, MASS ? jj : (EARLY ? ord[jj] : (DASH ? dord[jj] : idx_row[jj])));
-        ++issued;
-      }
-      // on abort or an early stop, loads already issued are waited for
-      // (bounded) before exit
-      if (*abort_flag || (EARLY && issued < nblk)) {
-        volatile int never = 0;
-        for (int jj = (issued > NS ? issued - NS : 0); jj < issued; ++jj) {
-          mbar_wait(&bar_kfull[jj % NS], (jj / NS) & 1, &never, 1000000ull, 0x1fe);
-          mbar_wait(&bar_vfull[jj % NS], (jj / NS) & 1, &never, 1000000ull, 0x1ff);
+    if (PERSIST) {
+      if (lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        // per unit: its first K/V block, then its Q once the previous unit's
+        // last score MMAs have read the old Q, then the rest of its blocks
+        int g = 0, k = 0;  // K/V blocks and units loaded so far
+        int qk = -1;       // the last unit whose Q was loaded
+        bool alive = true;
+        for (int u = static_cast<int>(blockIdx.x); alive && u < n_units; u += gridDim.x, ++k) {
+          const Unit w = unit_of(u);
+          for (int s = 0; s < w.nsel; ++s) {
+            const int st = g % NS, use = g / NS;
+            if (use > 0 && !mbar_wait(&bar_empty[st], (use - 1) & 1, abort_flag, tmo, 0x101)) {
+              alive = false;
+              break;
+            }
+            const int j = w.idx_row[s];
+            mbar_arrive_expect_tx(&bar_kfull[st], KVT);
+            for (int pn = 0; pn < NP; ++pn)
+              tma_load_4d(sK + st * KVT + pn * (64 * 128), &tm_k, &bar_kfull[st], 64 * pn, w.h, 64 * j, w.b);
+            mbar_arrive_expect_tx(&bar_vfull[st], KVT);
+            for (int pn = 0; pn < NP; ++pn)
+              tma_load_4d(sV + st * KVT + pn * (64 * 128), &tm_v, &bar_vfull[st], 64 * pn, w.h, 64 * j, w.b);
+            ++g;
+            if (s == 0) {
+              if (k > 0 && !mbar_wait(bar_qfree, (k - 1) & 1, abort_flag, tmo, 0x102)) {
+                alive = false;
+                break;
+              }
+              mbar_arrive_expect_tx(bar_q, T * QTILE);
+              for (int t = 0; t < T; ++t)
+                for (int hh = 0; hh < 2; ++hh)
+                  for (int pn = 0; pn < NP; ++pn)
+                    tma_load_4d(sQ + t * QTILE + pn * (128 * 128) + hh * (64 * 128), &tm_q, bar_q,
+                                64 * pn, w.hq0 + 2 * t + hh, 64 * w.i, w.b);
+              qk = k;
+            }
+          }
+        }
+        // on abort, the loads already issued are waited for (bounded) before exit
+        if (*abort_flag) {
+          volatile int never = 0;
+          for (int gj = (g > NS ? g - NS : 0); gj < g; ++gj) {
+            mbar_wait(&bar_kfull[gj % NS], (gj / NS) & 1, &never, 1000000ull, 0x1fe);
+            mbar_wait(&bar_vfull[gj % NS], (gj / NS) & 1, &never, 1000000ull, 0x1ff);
+          }
+          if (qk >= 0) mbar_wait(bar_q, qk & 1, &never, 1000000ull, 0x1fd);
         }
       }
-    }
+    } else {
+      if (lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        mbar_arrive_expect_tx(bar_q, T * QTILE);
+        for (int t = 0; t < T; ++t)
+          for (int hh = 0; hh < 2; ++hh)
+            for (int pn = 0; pn < NP; ++pn)
+              tma_load_4d(sQ + t * QTILE + pn * (128 * 128) + hh * (64 * 128), &tm_q, bar_q,
+                          64 * pn, hq0 + 2 * t + hh, 64 * i, b);
+        if (EARLY) load_kv(0, i);  // the diagonal block is visited first
+      }
+      if (EARLY) early_visit_order<D>(p, b, h, i, nsel, idx_row, lane, ord, esc, ej);
+      if (lane == 0) {
+        int issued = EARLY ? 1 : 0;
+        for (int jj = issued; jj < nblk; ++jj) {
+          const int st = jj % NS, use = jj / NS;
+          if (EARLY && *all_stop) break;  // every tile stopped: no more blocks
+          // EARLY: once every tile stopped, the stage is never released; the
+          // stop flag ends the wait instead
+          if (use > 0 && !(EARLY ? mbar_wait_or(&bar_empty[st], (use - 1) & 1, abort_flag, all_stop, tmo, 0x101)
+                                 : mbar_wait(&bar_empty[st], (use - 1) & 1, abort_flag, tmo, 0x101)))
+            break;
+          load_kv(st, MASS ? jj : (EARLY ? ord[jj] : (DASH ? dord[jj] : idx_row[jj])));
+          ++issued;
+        }
+        // on abort or an early stop, loads already issued are waited for
+        // (bounded) before exit
+        if (*abort_flag || (EARLY && issued < nblk)) {
+          volatile int never = 0;
+          for (int jj = (issued > NS ? issued - NS : 0); jj < issued; ++jj) {
+            mbar_wait(&bar_kfull[jj % NS], (jj / NS) & 1, &never, 1000000ull, 0x1fe);
+            mbar_wait(&bar_vfull[jj % NS], (jj / NS) & 1, &never, 1000000ull, 0x1ff);
+          }
+        }
+      }
+    }  // one unit
   } else if (warp >= 1 && warp <= C::ISS) {
     // ------------------------------------------------------------ MMA issuers
     // Issuer warp w owns M-tiles t = w - 1, w - 1 + ISS, ...  Every tile
@@ -263,79 +346,91 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS, EARLY, DASH>::THREADS,
           mma_ss(d, a0 + oa, b0 + ob, idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(bar_q, 0, abort_flag, tmo, 0x201) &&
-                mbar_wait(&bar_kfull[0], 0, abort_flag, tmo, 0x202);
-      if (ok) {
+      // Per unit: the score MMAs of its first block once its Q and first K/V
+      // block landed (S and P of every tile are free: this thread issued the
+      // previous unit's last P.V before them), then block by block as above.
+      // Parities count the CTA's blocks (g + jj) and units (k).
+      bool ok = true;
+      int g = 0, k = 0;
+      for (int u = static_cast<int>(blockIdx.x); ok && u < n_units; u += gridDim.x, ++k) {
+        const int nb = PERSIST ? unit_of(u).nsel : nblk;
+        ok = mbar_wait(bar_q, k & 1, abort_flag, tmo, 0x201) &&
+             mbar_wait(&bar_kfull[g % NS], (g / NS) & 1, abort_flag, tmo, 0x202);
+        if (!ok) break;
         tc_fence_after();
         for (int t = me; t < T; t += ISS) {
-          issue_qk(t, 0);
+          issue_qk(t, g % NS);
           tc_commit(&bar_sfull[t]);
         }
-      }
-      bool first_sel[MT], first_uns[MT], stopped[MT];
+        if (PERSIST && nb == 1) tc_commit(bar_qfree);  // the unit's last score MMAs read Q
+        bool first_sel[MT], first_uns[MT], stopped[MT];
 #pragma unroll
-      for (int x = 0; x < MT; ++x) first_sel[x] = first_uns[x] = true, stopped[x] = false;
-      for (int jj = 0; ok && jj < nblk; ++jj) {
-        const int st = jj % NS;
-        const bool more = jj + 1 < nblk;
-        const int st1 = (jj + 1) % NS;
-        if (!mbar_wait(&bar_vfull[st], (jj / NS) & 1, abort_flag, tmo, 0x203) ||
-            (more && !mbar_wait(&bar_kfull[st1], ((jj + 1) / NS) & 1, abort_flag, tmo, 0x204))) {
-          ok = false;
-          break;
-        }
-        bool is_sel = true;
-        if (MASS) is_sel = (selbits[jj >> 5] >> (jj & 31)) & 1u;
-        const uint64_t v0 = dV + ((st * KVT) >> 4);
-#pragma unroll
-        for (int x = 0; x < MT; ++x) {
-          const int t = me + x * ISS;
-          if (t >= T || !ok || (EARLY && stopped[x])) continue;
-          // keys 0..31 as soon as the first half of P is stored
-          if (!mbar_wait(&bar_phalf[t], jj & 1, abort_flag, tmo, 0x205)) {
+        for (int x = 0; x < MT; ++x) first_sel[x] = first_uns[x] = true, stopped[x] = false;
+        for (int jj = 0; ok && jj < nb; ++jj) {
+          const int gj = g + jj;
+          const int st = gj % NS;
+          const bool more = jj + 1 < nb;
+          const int st1 = (gj + 1) % NS;
+          if (!mbar_wait(&bar_vfull[st], (gj / NS) & 1, abort_flag, tmo, 0x203) ||
+              (more && !mbar_wait(&bar_kfull[st1], ((gj + 1) / NS) & 1, abort_flag, tmo, 0x204))) {
             ok = false;
-            continue;
-          }
-          tc_fence_after();
-          const bool first = MASS ? (is_sel ? first_sel[x] : first_uns[x]) : (jj == 0);
-          const uint32_t base = tmem + t * TSTRIDE;
-          const uint32_t o_col = base + 64 + ((MASS && !is_sel) ? D : 0);
-#pragma unroll
-          for (int kk = 0; kk < 2; ++kk)  // 16 keys per MMA: 16 rows of 128 B
-            mma_ts(o_col, base + kk * 8, v0 + ((kk * (16 * 128)) >> 4), idesc_pv,
-                   (first && kk == 0) ? 0u : 1u);
-          if (!mbar_wait(&bar_pfull[t], jj & 1, abort_flag, tmo, 0x206)) {
-            ok = false;
-            continue;
-          }
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 2; kk < 4; ++kk)
-            mma_ts(o_col, base + kk * 8, v0 + ((kk * (16 * 128)) >> 4), idesc_pv, 1u);
-          // EARLY: the softmax set the tile's stop flag before it arrived on pfull
-          const bool stop_now = EARLY && tile_stop[t] != 0;
-          if (more && !stop_now) {
-            issue_qk(t, st1);
-            tc_commit(&bar_sfull[t]);
-          } else {
-            tc_commit(&bar_odone[t]);
-            if (EARLY) stopped[x] = true;
-          }
-          if (MASS) {
-            if (is_sel) first_sel[x] = false; else first_uns[x] = false;
-          }
-        }
-        if (ok) tc_commit(&bar_empty[st]);  // this issuer's tiles are all done with the stage
-        if (EARLY) {
-          bool all = true;
-#pragma unroll
-          for (int x = 0; x < MT; ++x)
-            if (me + x * ISS < T && !stopped[x]) all = false;
-          if (all) {  // no tile visits more blocks: the producer stops too
-            *all_stop = 1;
             break;
           }
+          bool is_sel = true;
+          if (MASS) is_sel = (selbits[jj >> 5] >> (jj & 31)) & 1u;
+          const uint64_t v0 = dV + ((st * KVT) >> 4);
+#pragma unroll
+          for (int x = 0; x < MT; ++x) {
+            const int t = me + x * ISS;
+            if (t >= T || !ok || (EARLY && stopped[x])) continue;
+            // keys 0..31 as soon as the first half of P is stored
+            if (!mbar_wait(&bar_phalf[t], gj & 1, abort_flag, tmo, 0x205)) {
+              ok = false;
+              continue;
+            }
+            tc_fence_after();
+            const bool first = MASS ? (is_sel ? first_sel[x] : first_uns[x]) : (jj == 0);
+            const uint32_t base = tmem + t * TSTRIDE;
+            const uint32_t o_col = base + 64 + ((MASS && !is_sel) ? D : 0);
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk)  // 16 keys per MMA: 16 rows of 128 B
+              mma_ts(o_col, base + kk * 8, v0 + ((kk * (16 * 128)) >> 4), idesc_pv,
+                     (first && kk == 0) ? 0u : 1u);
+            if (!mbar_wait(&bar_pfull[t], gj & 1, abort_flag, tmo, 0x206)) {
+              ok = false;
+              continue;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 2; kk < 4; ++kk)
+              mma_ts(o_col, base + kk * 8, v0 + ((kk * (16 * 128)) >> 4), idesc_pv, 1u);
+            // EARLY: the softmax set the tile's stop flag before it arrived on pfull
+            const bool stop_now = EARLY && tile_stop[t] != 0;
+            if (more && !stop_now) {
+              issue_qk(t, st1);
+              tc_commit(&bar_sfull[t]);
+            } else {
+              tc_commit(&bar_odone[t]);
+              if (EARLY) stopped[x] = true;
+            }
+            if (MASS) {
+              if (is_sel) first_sel[x] = false; else first_uns[x] = false;
+            }
+          }
+          if (PERSIST && ok && jj + 2 == nb) tc_commit(bar_qfree);  // every tile's last S issued
+          if (ok) tc_commit(&bar_empty[st]);  // this issuer's tiles are all done with the stage
+          if (EARLY) {
+            bool all = true;
+#pragma unroll
+            for (int x = 0; x < MT; ++x)
+              if (me + x * ISS < T && !stopped[x]) all = false;
+            if (all) {  // no tile visits more blocks: the producer stops too
+              *all_stop = 1;
+              break;
+            }
+          }
         }
+        g += nb;
       }
       if (!ok) {
         // every MMA this thread issued completes before TMEM is released
@@ -350,148 +445,159 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS, EARLY, DASH>::THREADS,
     const int wq = warp % 4;
     const int r = wq * 32 + lane;
     const int hh = r / 64, tq = r % 64;
-    const int hq = hq0 + 2 * t + hh;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16) + t * TSTRIDE;
     const uint32_t tS = lane_base, tO = lane_base + 64;
     const uint32_t tOu = tO + D;
     const float sl2 = p.scale_log2;
     const uint64_t scale2 = f2_pack(sl2, sl2);
-    float m_ref = -INFINITY;  // reference maximum, scaled (log2) units
-    float l_sel = 0.f, l_uns = 0.f;
-    int visited = 0;          // EARLY: blocks this tile visited
     bool ok = true;
-    for (int jj = 0; jj < nblk; ++jj) {
-      // waits are made warp-uniform: the tcgen05.ld/st below are .sync.aligned
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar_sfull[t], jj & 1, abort_flag, tmo, 0x301))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      // the diagonal block comes last in the ascending table, first in the
-      // early-stop order
-      const bool diag = EARLY ? (jj == 0) : (jj == nblk - 1);
-      bool is_sel = true;
-      if (MASS) is_sel = (selbits[jj >> 5] >> (jj & 31)) & 1u;
-      // all 64 scores with one TMEM round trip, then the raw row maximum
-      float sv[64];
-      tmem_ld64(tS, sv);
-      float mx = diag ? row_max32<true>(sv + 32, 32, tq, -INFINITY)
-                      : row_max32<false>(sv + 32, 32, tq, -INFINITY);
-      mx = diag ? row_max32<true>(sv, 0, tq, mx) : row_max32<false>(sv, 0, tq, mx);
-      // DASH: the chunk's prior adds sigma * log2 w_j to every score of the block
-      const float bias = DASH ? dbias[jj] : 0.f;
-      const float mx_s = mx * sl2 + bias;
-      float alpha = 1.f;
-      const bool moved = mx_s > m_ref + 8.f;
-      if (moved) {
-        alpha = ex2(m_ref - mx_s);
-        m_ref = mx_s;
-      }
-      const uint64_t negm2 = f2_pack(bias - m_ref, bias - m_ref);
-      uint64_t acc2 = f2_pack(0.f, 0.f);
-      uint32_t pk[16];
-      if (diag) exp_pack32<true>(sv, 0, tq, scale2, negm2, acc2, pk);
-      else exp_pack32<false, C::POLY>(sv, 0, tq, scale2, negm2, acc2, pk);
-      // O is stable here (S(jj) was committed after P(jj-1).V) and is read by
-      // the tensor core only after phalf: rescale it when the maximum moved
-      if (jj > 0 && __any_sync(0xffffffffu, moved)) {
-        const uint64_t a2 = f2_pack(alpha, alpha);
+    // parities count the CTA's blocks (g + jj) and units (k)
+    int g = 0, k = 0;
+    for (int u = static_cast<int>(blockIdx.x); ok && u < n_units; u += gridDim.x, ++k) {
+      const int nb = PERSIST ? min(p.topk, p.n - u / per_i) : nblk;
+      float m_ref = -INFINITY;  // reference maximum, scaled (log2) units
+      float l_sel = 0.f, l_uns = 0.f;
+      int visited = 0;          // EARLY: blocks this tile visited
+      for (int jj = 0; jj < nb; ++jj) {
+        const int gj = g + jj;
+        // waits are made warp-uniform: the tcgen05.ld/st below are .sync.aligned
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar_sfull[t], gj & 1, abort_flag, tmo, 0x301))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // the diagonal block comes last in the ascending table, first in the
+        // early-stop order
+        const bool diag = EARLY ? (jj == 0) : (jj == nb - 1);
+        bool is_sel = true;
+        if (MASS) is_sel = (selbits[jj >> 5] >> (jj & 31)) & 1u;
+        // all 64 scores with one TMEM round trip, then the raw row maximum
+        float sv[64];
+        tmem_ld64(tS, sv);
+        float mx = diag ? row_max32<true>(sv + 32, 32, tq, -INFINITY)
+                        : row_max32<false>(sv + 32, 32, tq, -INFINITY);
+        mx = diag ? row_max32<true>(sv, 0, tq, mx) : row_max32<false>(sv, 0, tq, mx);
+        // DASH: the chunk's prior adds sigma * log2 w_j to every score of the block
+        const float bias = DASH ? dbias[jj] : 0.f;
+        const float mx_s = mx * sl2 + bias;
+        float alpha = 1.f;
+        const bool moved = mx_s > m_ref + 8.f;
+        if (moved) {
+          alpha = ex2(m_ref - mx_s);
+          m_ref = mx_s;
+        }
+        const uint64_t negm2 = f2_pack(bias - m_ref, bias - m_ref);
+        uint64_t acc2 = f2_pack(0.f, 0.f);
+        uint32_t pk[16];
+        if (diag) exp_pack32<true>(sv, 0, tq, scale2, negm2, acc2, pk);
+        else exp_pack32<false, C::POLY>(sv, 0, tq, scale2, negm2, acc2, pk);
+        // O is stable here (S(jj) was committed after P(jj-1).V) and is read by
+        // the tensor core only after phalf: rescale it when the maximum moved
+        if (jj > 0 && __any_sync(0xffffffffu, moved)) {
+          const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
-        for (int acc = 0; acc < (MASS ? 2 : 1); ++acc) {
-          const uint32_t base = acc ? tOu : tO;
+          for (int acc = 0; acc < (MASS ? 2 : 1); ++acc) {
+            const uint32_t base = acc ? tOu : tO;
 #pragma unroll
-          for (int ch = 0; ch < D / 16; ++ch) {
-            float o[16];
-            uint32_t w[16];
-            tmem_ld16(base + ch * 16, o);
+            for (int ch = 0; ch < D / 16; ++ch) {
+              float o[16];
+              uint32_t w[16];
+              tmem_ld16(base + ch * 16, o);
 #pragma unroll
-            for (int c = 0; c < 16; c += 2) {
-              float lo, hi;
-              f2_unpack(f2_mul(f2_pack(o[c], o[c + 1]), a2), lo, hi);
-              w[c] = __float_as_uint(lo);
-              w[c + 1] = __float_as_uint(hi);
+              for (int c = 0; c < 16; c += 2) {
+                float lo, hi;
+                f2_unpack(f2_mul(f2_pack(o[c], o[c + 1]), a2), lo, hi);
+                w[c] = __float_as_uint(lo);
+                w[c + 1] = __float_as_uint(hi);
+              }
+              tmem_st16(base + ch * 16, w);
             }
-            tmem_st16(base + ch * 16, w);
           }
         }
+        tmem_st16(tS, pk);  // P columns 0..15 over S columns 0..15 (already read)
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bar_phalf[t]);
+        if (diag) exp_pack32<true>(sv + 32, 32, tq, scale2, negm2, acc2, pk);
+        else exp_pack32<false, C::POLY>(sv + 32, 32, tq, scale2, negm2, acc2, pk);
+        tmem_st16(tS + 16, pk);  // P columns 16..31
+        float r0, r1;
+        f2_unpack(acc2, r0, r1);
+        bool stop = false;
+        if (EARLY && jj > 0 && p.tau > 0.f) {
+          // this block's mass against the mass accumulated before it (both in
+          // the current reference); the tile stops when no row gained at least
+          // tau times what it had (tau = 0 never stops: no decision is taken)
+          const bool cont_row = (r0 + r1) >= p.tau * (l_sel * alpha);
+          volatile int* wf = wflag + (t * 2 + (jj & 1)) * 4;
+          const bool wcont = __any_sync(0xffffffffu, cont_row);
+          if (lane == 0) wf[wq] = wcont ? 1 : 0;
+          named_bar_sync(1 + t, 128);
+          stop = !(wf[0] | wf[1] | wf[2] | wf[3]);
+          if (stop && r == 0) tile_stop[t] = 1;  // read by the issuer after pfull
+        }
+        l_sel *= alpha;
+        l_uns *= alpha;
+        if (is_sel) l_sel += r0 + r1; else l_uns += r0 + r1;
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bar_pfull[t]);
+        if (EARLY) visited = jj + 1;
+        if (stop) break;
       }
-      tmem_st16(tS, pk);  // P columns 0..15 over S columns 0..15 (already read)
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&bar_phalf[t]);
-      if (diag) exp_pack32<true>(sv + 32, 32, tq, scale2, negm2, acc2, pk);
-      else exp_pack32<false, C::POLY>(sv + 32, 32, tq, scale2, negm2, acc2, pk);
-      tmem_st16(tS + 16, pk);  // P columns 16..31
-      float r0, r1;
-      f2_unpack(acc2, r0, r1);
-      bool stop = false;
-      if (EARLY && jj > 0 && p.tau > 0.f) {
-        // this block's mass against the mass accumulated before it (both in
-        // the current reference); the tile stops when no row gained at least
-        // tau times what it had (tau = 0 never stops: no decision is taken)
-        const bool cont_row = (r0 + r1) >= p.tau * (l_sel * alpha);
-        volatile int* wf = wflag + (t * 2 + (jj & 1)) * 4;
-        const bool wcont = __any_sync(0xffffffffu, cont_row);
-        if (lane == 0) wf[wq] = wcont ? 1 : 0;
-        named_bar_sync(1 + t, 128);
-        stop = !(wf[0] | wf[1] | wf[2] | wf[3]);
-        if (stop && r == 0) tile_stop[t] = 1;  // read by the issuer after pfull
-      }
-      l_sel *= alpha;
-      l_uns *= alpha;
-      if (is_sel) l_sel += r0 + r1; else l_uns += r0 + r1;
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&bar_pfull[t]);
-      if (EARLY) visited = jj + 1;
-      if (stop) break;
-    }
-    // ---------------------------------------------------------- epilogue
-    if (ok && __all_sync(0xffffffffu, mbar_wait(&bar_odone[t], 0, abort_flag, tmo, 0x303))) {
-      tc_fence_after();
-      const int tok = 64 * i + tq;
-      const size_t orow = ((static_cast<size_t>(b) * p.S + tok) * p.Hq + hq) * D;
-      const size_t lrow = (static_cast<size_t>(b) * p.Hq + hq) * p.S + tok;
-      const bool has_uns = MASS && (nblk > nsel);
-      const float inv_sel = 1.f / l_sel;
-      const float l_all = l_sel + (has_uns ? l_uns : 0.f);
-      const float inv_all = 1.f / l_all;
+      // ---------------------------------------------------------- epilogue
+      // (O is read here before this tile's next P store, which the next unit's
+      // first P.V waits for: so that P.V never overwrites O still being read)
+      if (ok && !__all_sync(0xffffffffu, mbar_wait(&bar_odone[t], k & 1, abort_flag, tmo, 0x303))) ok = false;
+      if (ok) {
+        tc_fence_after();
+        const Unit w = PERSIST ? unit_of(u) : u0;  // this unit's rows
+        const int hq = w.hq0 + 2 * t + hh;
+        const int tok = 64 * w.i + tq;
+        const size_t orow = ((static_cast<size_t>(w.b) * p.S + tok) * p.Hq + hq) * D;
+        const size_t lrow = (static_cast<size_t>(w.b) * p.Hq + hq) * p.S + tok;
+        const bool has_uns = MASS && (nb > w.nsel);
+        const float inv_sel = 1.f / l_sel;
+        const float l_all = l_sel + (has_uns ? l_uns : 0.f);
+        const float inv_all = 1.f / l_all;
 #pragma unroll
-      for (int ch = 0; ch < D / 32; ++ch) {
-        float o[32];
-        tmem_ld32(tO + ch * 32, o);
-        uint32_t w[16];
+        for (int ch = 0; ch < D / 32; ++ch) {
+          float o[32];
+          tmem_ld32(tO + ch * 32, o);
+          uint32_t w[16];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) w[c] = pack_bf16x2(o[2 * c] * inv_sel, o[2 * c + 1] * inv_sel);
-        uint4* dst = reinterpret_cast<uint4*>(p.o + orow + ch * 32);
-#pragma unroll
-        for (int v4 = 0; v4 < 4; ++v4)
-          dst[v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
-        if (MASS) {
-          if (has_uns) {
-            float ou[32];
-            tmem_ld32(tOu + ch * 32, ou);
-#pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] += ou[c];
-          }
-#pragma unroll
-          for (int c = 0; c < 16; ++c)
-            w[c] = pack_bf16x2(o[2 * c] * inv_all, o[2 * c + 1] * inv_all);
-          uint4* dstf = reinterpret_cast<uint4*>(p.o_full + orow + ch * 32);
+          for (int c = 0; c < 16; ++c) w[c] = pack_bf16x2(o[2 * c] * inv_sel, o[2 * c + 1] * inv_sel);
+          uint4* dst = reinterpret_cast<uint4*>(p.o + orow + ch * 32);
 #pragma unroll
           for (int v4 = 0; v4 < 4; ++v4)
-            dstf[v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+            dst[v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+          if (MASS) {
+            if (has_uns) {
+              float ou[32];
+              tmem_ld32(tOu + ch * 32, ou);
+#pragma unroll
+              for (int c = 0; c < 32; ++c) o[c] += ou[c];
+            }
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+              w[c] = pack_bf16x2(o[2 * c] * inv_all, o[2 * c + 1] * inv_all);
+            uint4* dstf = reinterpret_cast<uint4*>(p.o_full + orow + ch * 32);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              dstf[v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+          }
+        }
+        constexpr float kLn2 = 0.69314718055994530942f;
+        p.lse[lrow] = (m_ref + log2f(l_sel)) * kLn2;
+        if (EARLY && r == 0 && p.visited != nullptr)
+          p.visited[((static_cast<size_t>(w.b) * p.Hkv + w.h) * p.n + w.i) * (p.G / 2) + w.slice * T + t] = visited;
+        if (MASS) {
+          p.lse_full[lrow] = (m_ref + log2f(l_all)) * kLn2;
+          p.dropped[lrow] = has_uns ? (l_uns / l_all) : 0.f;
         }
       }
-      constexpr float kLn2 = 0.69314718055994530942f;
-      p.lse[lrow] = (m_ref + log2f(l_sel)) * kLn2;
-      if (EARLY && r == 0 && p.visited != nullptr)
-        p.visited[((static_cast<size_t>(b) * p.Hkv + h) * p.n + i) * (p.G / 2) + slice * T + t] = visited;
-      if (MASS) {
-        p.lse_full[lrow] = (m_ref + log2f(l_all)) * kLn2;
-        p.dropped[lrow] = has_uns ? (l_uns / l_all) : 0.f;
-      }
-    }
+      g += nb;
+    }  // units
   }
 
   tc_fence_before();

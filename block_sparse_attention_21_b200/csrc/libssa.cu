@@ -240,7 +240,13 @@ ssa_status launch_fwd(const Dims& d, const void* q, const void* k, const void* v
   fp.dmask = dash.mask;
   fp.dw = dash.w;
   fp.sigma = dash.sigma;
-  const unsigned grid = static_cast<unsigned>(d.B) * d.Hkv * d.n * fp.slices;
+  // the plain sparse stream runs persistent CTAs, as many as are resident at
+  // once, over the units; the other modes one CTA per unit
+  const unsigned units = static_cast<unsigned>(d.B) * d.Hkv * d.n * fp.slices;
+  const unsigned slots = static_cast<unsigned>(sm_count()) * C::MIN_CTAS;
+  const bool persist = !MASS && !EARLY && !DASH;
+  if (persist && slots == 0) return SSA_ERR_CUDA;
+  const unsigned grid = persist ? std::min(units, slots) : units;
   return launch_pdl(kernel, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, st, mq, mk, mv, fp);
 }
 
