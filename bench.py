@@ -154,6 +154,16 @@ def dist_barrier(world: int):
         dist.barrier()
 
 
+def check_device(where: str) -> None:
+    """Raise if a kernel reported a device-side error (a bounded wait that
+    expired), naming the wait site the library recorded."""
+    import block_sparse_attention_21_b200 as ssa
+    err = ssa.ssa_get_device_error()
+    if err != 0:
+        raise RuntimeError(f"device error {err} after the {where}, wait site "
+                           f"{hex(ssa.ssa_get_device_error_site())}")
+
+
 def config_of(w, l2: str):
     return {"workload": w.name, "batch": w.batch, "seq_len": w.seq_len, "n_q_heads": w.n_q_heads,
             "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim, "block_size": 64,
@@ -280,7 +290,7 @@ def run_ours(args, world, rank, local):
     bwd_ms = timed(g_bwd, n_k) / n_k
     abwd_ms = timed(g_abwd, n_k) / n_k
     torch.cuda.synchronize()
-    assert ssa.ssa_get_device_error() == 0
+    check_device("timed rows")
 
     decode = decode_rows(dev, timed)
     dash = dash_rows(p, w, q, k, v, timed, n_k)
@@ -299,7 +309,7 @@ def run_ours(args, world, rank, local):
                                                st.o, st.lse, vis.view(w.batch, w.n_kv_heads, w.n_blocks, -1))
         es_ms = timed(g_es, n_k) / n_k
         torch.cuda.synchronize()
-        assert ssa.ssa_get_device_error() == 0
+        check_device("early-stop rows")
         early[f"tau_{tau:g}"] = {"ms": round(es_ms, 5), "blocks_visited_mean": round(float(vis.float().mean()), 3),
                                  "blocks_selected_mean": round(nsel_mean, 3),
                                  "speedup_vs_sparse_fwd": round(fwd_ms / es_ms, 3)}
@@ -379,7 +389,7 @@ def dash_rows(p, w, q, k, v, timed_fn, n_k, alpha=1.5, gamma=8.0, sigma=1.0):
     route_ms = timed_fn(g_route, n_k) / n_k
     attn_ms = timed_fn(g_attn, n_k) / n_k
     torch.cuda.synchronize()
-    assert ssa.ssa_get_device_error() == 0
+    check_device("decode and routing rows")
     n = w.n_blocks
     bits = np.unpackbits(da.mask.cpu().numpy().view(np.uint8), axis=-1, bitorder="little")[..., :n].astype(bool)
     earlier = np.tril(np.ones((n, n), dtype=bool), -1)

@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH, EARLY>::THREADS,
     return w;
   };
   const Unit u0 = unit_of(static_cast<int>(blockIdx.x));
-  const int i = u0.i, b = u0.b, h = u0.h, slice = u0.slice, hq0 = u0.hq0, nsel = u0.nsel;
+  const int i = u0.i, b = u0.b, h = u0.h, hq0 = u0.hq0, nsel = u0.nsel;
   int nblk = MASS ? (i + 1) : nsel;  // DASH: the routed count, known after the prologue
   const int32_t* idx_row = u0.idx_row;
 
