@@ -1,9 +1,10 @@
 // attn_fwd_psmem.cuh -- block-sparse causal attention forward on tcgen05 tensor
 // cores, with P staged in shared memory (the variant used at head_dim 128).
 //
-// One CTA handles one query block i (64 tokens) of one batch entry for 2*T
-// query heads that share KV head h.  Its rows form T M-tiles of 128 rows
-// (2 heads x 64 tokens).  The KV blocks it visits are either the selected
+// A work unit is one query block i (64 tokens) of one batch entry for 2*T
+// query heads that share KV head h; a CTA takes one unit, or in the plain
+// sparse stream a sequence of them (persistent CTAs, below).  A unit's rows
+// form T M-tiles of 128 rows (2 heads x 64 tokens).  The KV blocks it visits are either the selected
 // blocks of the index table (sparse stream: "SSA: Guida a Sparse Sparse
 // Attention per LLM", section "Block-sparse attention e Receptive Field",
 // attention computed only over the tokens of the selected blocks) or, with
