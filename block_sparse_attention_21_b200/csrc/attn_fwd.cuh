@@ -405,8 +405,10 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS, EARLY, DASH>::THREADS,
 #pragma unroll
             for (int kk = 2; kk < 4; ++kk)
               mma_ts(o_col, base + kk * 8, v0 + ((kk * (16 * 128)) >> 4), idesc_pv, 1u);
-            // EARLY: the softmax set the tile's stop flag before it arrived on pfull
-            const bool stop_now = EARLY && tile_stop[t] != 0;
+            // EARLY: the softmax records the position of the block it stops at
+            // before it arrives on that block's pfull (the same rule as the
+            // head_dim-128 kernel, where the next S is issued before this read)
+            const bool stop_now = EARLY && tile_stop[t] == jj + 1;
             if (more && !stop_now) {
               issue_qk(t, st1);
               tc_commit(&bar_sfull[t]);
@@ -535,7 +537,7 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS, EARLY, DASH>::THREADS,
           if (lane == 0) wf[wq] = wcont ? 1 : 0;
           named_bar_sync(1 + t, 128);
           stop = !(wf[0] | wf[1] | wf[2] | wf[3]);
-          if (stop && r == 0) tile_stop[t] = 1;  // read by the issuer after pfull
+          if (stop && r == 0) tile_stop[t] = jj + 1;  // read by the issuer after pfull
         }
         l_sel *= alpha;
         l_uns *= alpha;

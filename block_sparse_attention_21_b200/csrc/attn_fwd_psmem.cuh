@@ -397,8 +397,11 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH, EARLY>::THREADS,
             mma_ss(o_col, a, bd, idesc_pv, (first && kk == 0) ? 0u : 1u);
           }
           tc_commit(&bar_pvdone[t]);
-          // EARLY: the softmax set the tile's stop flag before it arrived on pfull
-          const bool stop_now = EARLY && tile_stop[t] != 0;
+          // EARLY: the softmax records the position of the block it stops at
+          // before it arrives on that block's pfull.  The issuer compares with
+          // its own position: S(s+1) is already issued here, so the softmax
+          // may have decided a stop at s+1 before this thread reads the flag.
+          const bool stop_now = EARLY && tile_stop[t] == s + 1;
           if (s + 1 == nb || stop_now) tc_commit(&bar_odone[t]);
           tc_commit(&bar_empty[st]);
           if (MASS) {
@@ -514,7 +517,7 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH, EARLY>::THREADS,
           if (lane == 0) wf[wq] = wcont ? 1 : 0;
           named_bar_sync(1 + t, 128);
           stop = !(wf[0] | wf[1] | wf[2] | wf[3]);
-          if (stop && r == 0) tile_stop[t] = 1;  // read by the issuer after pfull
+          if (stop && r == 0) tile_stop[t] = jj + 1;  // read by the issuer after pfull
         }
         l_sel *= alpha;
         l_uns *= alpha;
