@@ -97,35 +97,3 @@ def _check(case, tau, min_clear=0.6):
         assert np.array_equal(gvis, np.repeat(nsel[..., None], G // 2, axis=-1))
         assert (o.float() - st.o.float()).abs().max().item() <= 2e-2
     return gvis, nsel
-
-
-@pytest.mark.parametrize("D", [64, 128])
-def test_early_stop_repeats_bit_for_bit(D):
-    # Each tile's visiting order, stop point and arithmetic are fixed, so
-    # repeated launches must agree bit for bit.  At head_dim 128 the next
-    # block's scores are issued before the issuer reads the tile's stop
-    # record; a stop decided one block ahead once made the issuer drop the
-    # stop block's P.V.  Many launches of a case whose tiles stop early give
-    # that ordering many chances to show.
-    B, S, Hq, Hkv, topk, npl = 1, 4096, 8, 2, 40, 8
-    x = gen.make_custom(B, S, Hq, Hkv, D, topk, seed=800 + S + D, n_plant=npl)
-    p = ssa.problem(B, S, Hq, Hkv, D, topk)
-    q, k, v = (t.to(DEV) for t in (x.q, x.k, x.v))
-    st = ssa.SparseStream(p)
-    st.forward(q, k, v)
-    n, G = S // 64, Hq // Hkv
-    runs = []
-    for _ in range(40):
-        o = torch.empty_like(st.o)
-        lse = torch.empty_like(st.lse)
-        vis = torch.empty(B, Hkv, n, G // 2, dtype=torch.int32, device=DEV)
-        ssa.ssa_sparse_attn_fwd_early_stop(p, q, k, v, st.q_pooled, st.k_pooled, st.block_idx, 0.3, o, lse, vis)
-        runs.append((o, lse, vis))
-    torch.cuda.synchronize()
-    assert ssa.ssa_get_device_error() == 0
-    o0, l0, v0 = runs[0]
-    nsel = np.minimum(topk, np.arange(n) + 1)
-    assert np.mean(nsel[None, :, None] - v0.cpu().numpy() >= 8) > 0.5  # most tiles stop early
-    for o, lse, vis in runs[1:]:
-        assert torch.equal(vis, v0)
-        assert torch.equal(o.view(torch.int16), o0.view(torch.int16)) and torch.equal(lse, l0)
