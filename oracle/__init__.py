@@ -21,8 +21,9 @@ Functions (each cites the passage it follows in ssa_oracle.c):
   decode_step     one decoding step: selection for the newest token and its
                   attention (fp64 numpy, small problems)
   early_stop_forward
-                  the sparse forward with the early-stop rule (fp64 numpy,
-                  small problems)
+                  the sparse forward with the early-stop rule, each query
+                  segment of one head stopping on its own (fp64 numpy, small
+                  problems)
   entmax          alpha-entmax of a vector by its threshold (fp64 bisection)
   dash_route      DashAttention chunk routing: per-head alpha-entmax over the
                   pooled chunk logits, averaged over the GQA group, and the
@@ -293,15 +294,18 @@ def early_stop_forward(q, k, v, qbar, kbar, idx: np.ndarray, tau: float,
     """The sparse forward with an early stop, in fp64 ("S2O" summary, section 2,
     "Regla de Parada Temprana", applied to the sparse stream; small problems).
 
-    Per tile (b, KV head h, query block i, head pair hp: query heads
-    h*G + 2hp and + 1, the 64 tokens of block i) the blocks are visited in the
-    order: i first, then the other selected blocks of idx by descending pooled
-    score qbar[b,h,i] . kbar[b,h,j] (ties: lower j).  After each block after the
-    first, the tile stops if every row's mass in that block is below tau times
-    the row's mass in the blocks before it (the block itself counts).
-    Returns o [B,S,Hq,D], lse [B,Hq,S], visited [B,Hkv,n,G/2] and margin
-    [B,Hkv,n,G/2]: the smallest |ln(max row ratio) - ln tau| over the tile's
-    decisions (inf when tau = 0 or no decision was taken)."""
+    The unit that stops is one query segment of one attention head: query
+    head hq, query block i, the 64 tokens of block i (b fixed).  Its blocks are
+    visited in the order: i first (the segment's own causal window), then the
+    other selected blocks of idx by descending pooled score
+    qbar[b,h,i] . kbar[b,h,j] (ties: lower j), h the KV head of hq; this is
+    the score the selection ranks by, shared by the heads of the group.  After
+    each block after the first, the segment stops if every one of its rows
+    gained less than tau times the mass it had in the blocks before it (the
+    block itself still counts).  tau = 0 never stops.
+    Returns o [B,S,Hq,D], lse [B,Hq,S], visited [B,Hq,n] (blocks each segment
+    used) and margin [B,Hq,n]: the smallest |ln(max row ratio) - ln tau| over
+    the segment's decisions (inf when tau = 0 or no decision was taken)."""
     q64, k64, v64 = widen(q), widen(k), widen(v)
     qbar = np.asarray(qbar, dtype=np.float64)
     kbar = np.asarray(kbar, dtype=np.float64)
@@ -311,8 +315,8 @@ def early_stop_forward(q, k, v, qbar, kbar, idx: np.ndarray, tau: float,
     scale = (1.0 / np.sqrt(D)) if scale is None else float(scale)
     o = np.zeros((B, S, Hq, D))
     lse = np.zeros((B, Hq, S))
-    visited = np.zeros((B, Hkv, n, G // 2), dtype=np.int32)
-    margin = np.full((B, Hkv, n, G // 2), np.inf)
+    visited = np.zeros((B, Hq, n), dtype=np.int32)
+    margin = np.full((B, Hq, n), np.inf)
     tok = np.arange(bs)
     for b in range(B):
         for h in range(Hkv):
@@ -320,35 +324,32 @@ def early_stop_forward(q, k, v, qbar, kbar, idx: np.ndarray, tau: float,
                 sel = [int(j) for j in idx[b, h, i] if 0 <= j < i]
                 sc = {j: float(kbar[b, h, j] @ qbar[b, h, i]) for j in sel}
                 order = [i] + sorted(sel, key=lambda j: (-sc[j], j))
-                for hp in range(G // 2):
-                    heads = (h * G + 2 * hp, h * G + 2 * hp + 1)
-                    # per row and block: the block's logits (causal in block i)
-                    lg = {}
-                    for hq in heads:
-                        qrows = q64[b, bs * i + tok, hq]                  # [64, D]
-                        for j in order:
-                            l_ = scale * (qrows @ k64[b, bs * j + tok, h].T)  # [64 rows, 64 keys]
-                            if j == i:
-                                l_ = np.where(tok[None, :] <= tok[:, None], l_, -np.inf)
-                            lg[hq, j] = l_
-                    blk = np.array([[np.logaddexp.reduce(lg[hq, j], axis=1) for j in order] for hq in heads])
+                for hq in range(h * G, (h + 1) * G):
+                    qrows = q64[b, bs * i + tok, hq]                          # [64, D]
+                    # per block: the logits of the segment's rows (causal in block i)
+                    lg = []
+                    for j in order:
+                        l_ = scale * (qrows @ k64[b, bs * j + tok, h].T)      # [64 rows, 64 keys]
+                        if j == i:
+                            l_ = np.where(tok[None, :] <= tok[:, None], l_, -np.inf)
+                        lg.append(l_)
+                    blk = np.array([np.logaddexp.reduce(l_, axis=1) for l_ in lg])   # [blocks, 64]
                     nv = len(order)
                     for jj in range(1, len(order)):
-                        before = np.logaddexp.reduce(blk[:, :jj], axis=1)          # [2, 64]
-                        lr = float(np.max(blk[:, jj] - before))                    # ln max ratio
+                        before = np.logaddexp.reduce(blk[:jj], axis=0)              # [64]
+                        lr = float(np.max(blk[jj] - before))                        # ln max row ratio
                         if tau > 0:
-                            margin[b, h, i, hp] = min(margin[b, h, i, hp], abs(lr - np.log(tau)))
+                            margin[b, hq, i] = min(margin[b, hq, i], abs(lr - np.log(tau)))
                         if tau > 0 and lr < np.log(tau):
                             nv = jj + 1
                             break
-                    visited[b, h, i, hp] = nv
-                    for a, hq in enumerate(heads):
-                        logits = np.concatenate([lg[hq, j] for j in order[:nv]], axis=1)
-                        vals = np.concatenate([v64[b, bs * j + tok, h] for j in order[:nv]], axis=0)
-                        m = logits.max(axis=1, keepdims=True)
-                        w = np.exp(logits - m)
-                        lse[b, hq, bs * i + tok] = m[:, 0] + np.log(w.sum(axis=1))
-                        o[b, bs * i + tok, hq] = (w / w.sum(axis=1, keepdims=True)) @ vals
+                    visited[b, hq, i] = nv
+                    logits = np.concatenate(lg[:nv], axis=1)
+                    vals = np.concatenate([v64[b, bs * j + tok, h] for j in order[:nv]], axis=0)
+                    m = logits.max(axis=1, keepdims=True)
+                    w = np.exp(logits - m)
+                    lse[b, hq, bs * i + tok] = m[:, 0] + np.log(w.sum(axis=1))
+                    o[b, bs * i + tok, hq] = (w / w.sum(axis=1, keepdims=True)) @ vals
     return o, lse, visited, margin
 
 

@@ -494,8 +494,8 @@ def test_early_stop_with_zero_threshold_is_the_sparse_forward():
     r = oracle.attn_rows(q, k, v, idx, oracle.all_rows(B, Hq, S), want_full=False)
     np.testing.assert_allclose(o.transpose(0, 2, 1, 3).reshape(-1, D), r["o_sparse"], atol=1e-12)
     np.testing.assert_allclose(lse.reshape(-1), r["lse_sparse"], atol=1e-12)
-    nsel = (idx >= 0).sum(axis=-1)
-    assert np.array_equal(vis, np.repeat(nsel[..., None], 2, axis=-1))
+    nsel = (idx >= 0).sum(axis=-1)                      # [B, Hkv, n]
+    assert np.array_equal(vis, np.repeat(nsel, Hq // k.shape[2], axis=1))
 
 
 def test_early_stop_with_huge_threshold_keeps_the_diagonal_and_the_best_block():
@@ -509,7 +509,7 @@ def test_early_stop_with_huge_threshold_keeps_the_diagonal_and_the_best_block():
         earlier = [j for j in idx[0, 0, i] if 0 <= j < i]
         if earlier:
             keep[i, max(earlier, key=lambda j: (kbar[0, 0, j] @ qbar[0, 0, i], -j))] = True
-        assert vis[0, 0, i, 0] == (2 if earlier else 1)
+        assert np.all(vis[0, :, i] == (2 if earlier else 1))
     mask = np.repeat(np.repeat(keep, BS, 0), BS, 1) & np.tril(np.ones((S, S), dtype=bool))
     ref = _sdpa_rows(q, k, v, lambda b, h: mask)
     np.testing.assert_allclose(o.transpose(0, 2, 1, 3), ref, atol=1e-12)
@@ -523,14 +523,16 @@ def test_early_stop_visits_fewer_blocks_as_the_threshold_grows():
         if prev is not None:
             assert np.all(vis <= prev)
         prev = vis
-    assert prev.sum() < (idx >= 0).sum() * 2
+    assert prev.sum() < (idx >= 0).sum() * q.shape[2]
 
 
 @pytest.mark.parametrize("tau", [0.3, 0.8])
 def test_early_stop_matches_a_recomputation_from_prefix_logsumexps(tau):
-    """The stop point from whole-prefix logsumexps (one torch.logsumexp over
-    the union of the earlier blocks' keys, not a running sum) and the output
-    from masked SDPA over the visited blocks."""
+    """The stop point of each head's query segment from whole-prefix
+    logsumexps (one torch.logsumexp over the union of the earlier blocks'
+    keys, not a running sum) and the output from masked SDPA over the visited
+    blocks.  Heads of one group share the visiting order but stop on their own
+    rows only: some pair of heads of the same query block must stop apart."""
     q, k, v = _tiny(B=1, S=1024, Hq=4, Hkv=1, D=8, seed=114)
     kbar, qbar = oracle.block_pool(k, q)
     idx, _ = oracle.block_select(qbar, kbar, 8)
@@ -539,15 +541,14 @@ def test_early_stop_matches_a_recomputation_from_prefix_logsumexps(tau):
     n = S // BS
     causal = torch.tril(torch.ones(S, S, dtype=torch.bool))
     logits = [(torch.from_numpy(q[0, :, hq]) @ torch.from_numpy(k[0, :, 0]).T) / np.sqrt(D) for hq in range(Hq)]
-    middle = 0
+    middle = apart = 0
     for i in range(n):
         sel = [int(j) for j in idx[0, 0, i] if 0 <= j < i]
         # descending pooled score, ties to the lower block (lexsort: last key first)
         sc = np.array([kbar[0, 0, j] @ qbar[0, 0, i] for j in sel])
         order = [i] + [sel[x] for x in np.lexsort((np.array(sel), -sc))] if sel else [i]
         rows = slice(BS * i, BS * i + BS)
-        for hp in range(2):
-            heads = (2 * hp, 2 * hp + 1)
+        for hq in range(Hq):
             nv = len(order)
             for jj in range(1, len(order)):
                 keys_b = torch.zeros(S, dtype=torch.bool)
@@ -555,27 +556,28 @@ def test_early_stop_matches_a_recomputation_from_prefix_logsumexps(tau):
                 keys_p = torch.zeros(S, dtype=torch.bool)
                 for j in order[:jj]:
                     keys_p[BS * j:BS * j + BS] = True
-                ratio = max(float((torch.logsumexp(logits[hq][rows].masked_fill(~(keys_b & causal[rows]), -np.inf), 1)
-                                   - torch.logsumexp(logits[hq][rows].masked_fill(~(keys_p & causal[rows]), -np.inf), 1)
-                                   ).max()) for hq in heads)
+                ratio = float((torch.logsumexp(logits[hq][rows].masked_fill(~(keys_b & causal[rows]), -np.inf), 1)
+                               - torch.logsumexp(logits[hq][rows].masked_fill(~(keys_p & causal[rows]), -np.inf), 1)
+                               ).max())
                 if ratio < np.log(tau):
                     nv = jj + 1
                     break
-            assert vis[0, 0, i, hp] == nv
+            assert vis[0, hq, i] == nv
             middle += 1 < nv < len(order)
             keep = torch.zeros(S, dtype=torch.bool)
             for j in order[:nv]:
                 keep[BS * j:BS * j + BS] = True
-            for hq in heads:
-                m = (keep & causal[rows])[None]
-                ref = F.scaled_dot_product_attention(torch.from_numpy(q[0, rows, hq])[None],
-                                                     torch.from_numpy(k[0, :, 0])[None],
-                                                     torch.from_numpy(v[0, :, 0])[None], attn_mask=m)
-                np.testing.assert_allclose(o[0, rows, hq], ref[0].numpy(), atol=1e-12)
-                np.testing.assert_allclose(lse[0, hq, rows],
-                                           torch.logsumexp(logits[hq][rows].masked_fill(~m[0], -np.inf), 1).numpy(),
-                                           atol=1e-12)
-    assert middle > 0  # some tile stops strictly between its second and last block
+            m = (keep & causal[rows])[None]
+            ref = F.scaled_dot_product_attention(torch.from_numpy(q[0, rows, hq])[None],
+                                                 torch.from_numpy(k[0, :, 0])[None],
+                                                 torch.from_numpy(v[0, :, 0])[None], attn_mask=m)
+            np.testing.assert_allclose(o[0, rows, hq], ref[0].numpy(), atol=1e-12)
+            np.testing.assert_allclose(lse[0, hq, rows],
+                                       torch.logsumexp(logits[hq][rows].masked_fill(~m[0], -np.inf), 1).numpy(),
+                                       atol=1e-12)
+        apart += len(set(int(x) for x in vis[0, :, i])) > 1
+    assert middle > 0  # some segment stops strictly between its second and last block
+    assert apart > 0   # the heads of a group do not stop together
 
 
 # ------------------------------------------------------------ DashAttention
