@@ -233,8 +233,9 @@ def ssa_alignment_bwd(p: SsaProblem, q, k, v, o_sparse, lse_sparse, o_full, lse_
 def ssa_sparse_attn_fwd_early_stop(p: SsaProblem, q, k, v, q_pooled, k_pooled, block_idx, tau: float,
                                    o, lse, visited=None, stream=None) -> None:
     """The sparse forward visiting the diagonal first, then the selected blocks
-    by descending pooled score, each tile stopping after the first block that
-    adds less than tau of every row's accumulated mass; see include/ssa.h."""
+    by descending pooled score, each head's query segment stopping after the
+    first block that adds less than tau of every row's accumulated mass;
+    visited is [B, Hq, n]; see include/ssa.h."""
     sh = _shapes(p)
     for t, s, nm in ((q, "q", "q"), (k, "kv", "k"), (v, "kv", "v"), (q_pooled, "pooled", "q_pooled"),
                      (k_pooled, "pooled", "k_pooled"), (block_idx, "idx", "block_idx"), (o, "q", "o"),
@@ -242,7 +243,7 @@ def ssa_sparse_attn_fwd_early_stop(p: SsaProblem, q, k, v, q_pooled, k_pooled, b
         _numel_check(t, sh[s], nm)
     if visited is not None:
         B, Hkv, n, _ = sh["idx"]
-        _numel_check(visited, (B, Hkv, n, p.n_q_heads // p.n_kv_heads // 2), "visited")
+        _numel_check(visited, (B, p.n_q_heads, n), "visited")
     _call("ssa_sparse_attn_fwd_early_stop", ctypes.byref(p), _ptr(q, BF16, "q"), _ptr(k, BF16, "k"),
           _ptr(v, BF16, "v"), _ptr(q_pooled, F32, "q_pooled"), _ptr(k_pooled, F32, "k_pooled"),
           _ptr(block_idx, I32, "block_idx"), float(tau), _ptr(o, BF16, "o"), _ptr(lse, F32, "lse"),

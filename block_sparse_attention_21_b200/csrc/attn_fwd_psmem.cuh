@@ -19,8 +19,11 @@
 //          offset by sigma * log2 w_j ("Resumen Tecnico: DashAttention",
 //          stage 2, prior-induced softmax); see dash_build_list.
 //   EARLY  the selected blocks in descending pooled score after the diagonal,
-//          each M-tile stopping once a block adds less than tau times the
-//          mass gathered before it (the "S2O" summary, section 2); see
+//          each head's query segment (the 64 rows of one head in a tile)
+//          stopping once a block adds less than tau times the mass gathered
+//          before it to every one of its rows (the "S2O" summary, section 2);
+//          a stopped head's P is zero from then on, and the tile ends its
+//          block loop once both of its heads have stopped; see
 //          early_visit_order.
 //
 // Pipeline per M-tile t and visited block jj:
@@ -451,7 +454,11 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH, EARLY>::THREADS,
       const int hq = w.hq0 + 2 * t + hh;
       float m_ref = -INFINITY;  // reference maximum, scaled (log2) units
       float l_sel = 0.f, l_uns = 0.f;
-      int visited = 0;          // EARLY: blocks this tile visited
+      // EARLY: each head of the tile (64-row half: warps wq 0-1 and 2-3)
+      // stops on its own; a stopped head's P is stored as zeros, so P.V adds
+      // nothing to its rows and its maximum, mass and O stay as they were
+      bool hstop = false;       // this thread's head has stopped
+      int hvis = 0;             // blocks this thread's head visited
       for (int jj = 0; jj < nb; ++jj) {
         const int gj = g + jj;
         // waits are made warp-uniform: the tcgen05.ld/st below are .sync.aligned
@@ -460,9 +467,13 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH, EARLY>::THREADS,
           break;
         }
         tc_fence_after();
+        // warp-uniform: both warps of a head stop together
+        const bool live = !EARLY || !hstop;
         float sA[32], sB[32];
-        tmem_ld32(tS, sA);
-        tmem_ld32(tS + 32, sB);
+        if (live) {
+          tmem_ld32(tS, sA);
+          tmem_ld32(tS + 32, sB);
+        }
         // the scores are in registers: the issuer may overwrite S with the next block's
         tc_fence_before();
         mbar_arrive(&bar_sfree[t]);
@@ -482,26 +493,32 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH, EARLY>::THREADS,
           ok = false;
           break;
         }
-        float mx = diag ? row_max32<true>(sB, 32, tq, -INFINITY) : row_max32<false>(sB, 32, tq, -INFINITY);
-        mx = diag ? row_max32<true>(sA, 0, tq, mx) : row_max32<false>(sA, 0, tq, mx);
-        // DASH: the chunk's prior adds sigma * log2 w_j to every score of the block
-        const float bias = DASH ? dbias[jj] : 0.f;
-        const float mx_s = mx * sl2 + bias;
         float alpha = 1.f;
-        const bool moved = mx_s > m_ref + 8.f;
-        if (moved) {
-          alpha = ex2(m_ref - mx_s);
-          m_ref = mx_s;
-        }
-        const uint64_t negm2 = f2_pack(bias - m_ref, bias - m_ref);
+        bool moved = false;
         uint64_t acc2 = f2_pack(0.f, 0.f);
         uint32_t pk[32];
-        if (diag) {
-          exp_pack32<true>(sA, 0, tq, scale2, negm2, acc2, pk);
-          exp_pack32<true>(sB, 32, tq, scale2, negm2, acc2, pk + 16);
+        if (live) {
+          float mx = diag ? row_max32<true>(sB, 32, tq, -INFINITY) : row_max32<false>(sB, 32, tq, -INFINITY);
+          mx = diag ? row_max32<true>(sA, 0, tq, mx) : row_max32<false>(sA, 0, tq, mx);
+          // DASH: the chunk's prior adds sigma * log2 w_j to every score of the block
+          const float bias = DASH ? dbias[jj] : 0.f;
+          const float mx_s = mx * sl2 + bias;
+          moved = mx_s > m_ref + 8.f;
+          if (moved) {
+            alpha = ex2(m_ref - mx_s);
+            m_ref = mx_s;
+          }
+          const uint64_t negm2 = f2_pack(bias - m_ref, bias - m_ref);
+          if (diag) {
+            exp_pack32<true>(sA, 0, tq, scale2, negm2, acc2, pk);
+            exp_pack32<true>(sB, 32, tq, scale2, negm2, acc2, pk + 16);
+          } else {
+            exp_pack32<false, C::POLY>(sA, 0, tq, scale2, negm2, acc2, pk);
+            exp_pack32<false, C::POLY>(sB, 32, tq, scale2, negm2, acc2, pk + 16);
+          }
         } else {
-          exp_pack32<false, C::POLY>(sA, 0, tq, scale2, negm2, acc2, pk);
-          exp_pack32<false, C::POLY>(sB, 32, tq, scale2, negm2, acc2, pk + 16);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) pk[c] = 0u;
         }
         if (T == 2 && !EARLY) mbar_arrive(&bar_turn[1 - t]);
         float r0, r1;
@@ -509,15 +526,19 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH, EARLY>::THREADS,
         bool stop = false;
         if (EARLY && jj > 0 && p.tau > 0.f) {
           // this block's mass against the mass accumulated before it (both in
-          // the current reference); the tile stops when no row gained at least
-          // tau times what it had (tau = 0 never stops: no decision is taken)
-          const bool cont_row = (r0 + r1) >= p.tau * (l_sel * alpha);
+          // the current reference); a head stops when none of its rows gained
+          // at least tau times what it had, the tile when both heads have
+          // stopped (tau = 0 never stops: no decision is taken).  A stopped
+          // head votes 0.
+          const bool cont_row = live && (r0 + r1) >= p.tau * (l_sel * alpha);
           volatile int* wf = wflag + (t * 2 + (jj & 1)) * 4;
           const bool wcont = __any_sync(0xffffffffu, cont_row);
           if (lane == 0) wf[wq] = wcont ? 1 : 0;
           named_bar_sync(1 + t, 128);
+          const bool head_stop = !(wf[2 * hh] | wf[2 * hh + 1]);
           stop = !(wf[0] | wf[1] | wf[2] | wf[3]);
           if (stop && r == 0) tile_stop[t] = jj + 1;  // read by the issuer after pfull
+          if (live && head_stop) hstop = true;       // this block is the head's last
         }
         l_sel *= alpha;
         l_uns *= alpha;
@@ -560,7 +581,7 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH, EARLY>::THREADS,
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&bar_pfull[t]);
-        if (EARLY) visited = jj + 1;
+        if (EARLY && live) hvis = jj + 1;
         if (stop) break;
       }
       // ---------------------------------------------------------- epilogue
@@ -605,8 +626,8 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH, EARLY>::THREADS,
         }
         constexpr float kLn2 = 0.69314718055994530942f;
         p.lse[lrow] = (m_ref + log2f(l_sel)) * kLn2;
-        if (EARLY && r == 0 && p.visited != nullptr)
-          p.visited[((static_cast<size_t>(w.b) * p.Hkv + w.h) * p.n + w.i) * (p.G / 2) + w.slice * T + t] = visited;
+        if (EARLY && tq == 0 && p.visited != nullptr)
+          p.visited[(static_cast<size_t>(w.b) * p.Hq + hq) * p.n + w.i] = hvis;
         if (MASS) {
           p.lse_full[lrow] = (m_ref + log2f(l_all)) * kLn2;
           p.dropped[lrow] = has_uns ? (l_uns / l_all) : 0.f;

@@ -161,16 +161,17 @@ ssa_status ssa_full_attn_fwd_with_mass(const ssa_problem *p, const ssa_bf16 *q,
 /* The sparse forward with an early stop ("S2O" summary, section 2, "Regla de
  * Parada Temprana", applied to the sparse stream): each query block visits
  * its diagonal block first, then its other selected blocks in descending
- * pooled score q_pooled[i] . k_pooled[j] (fp32; ties: lower j), and stops
- * after the first block that adds, for every query row of the tile, less
- * than tau times the attention mass the row had accumulated before it (that
- * block still counts).  A tile is one query block of one pair of query heads
- * (2 x 64 rows) -- the unit that stops together.  tau = 0 visits every
- * selected block (the ssa_sparse_attn_fwd result, up to summation order).
+ * pooled score q_pooled[i] . k_pooled[j] (fp32; ties: lower j).  The unit
+ * that stops is one query segment of one head: query head hq, the 64 tokens
+ * of query block i.  It stops after the first block that adds, for every one
+ * of its rows, less than tau times the attention mass the row had
+ * accumulated before it (that block still counts); the heads of a KV group
+ * share the order and stop on their own.  tau = 0 visits every selected
+ * block (the ssa_sparse_attn_fwd result, up to summation order).
  * q_pooled/k_pooled: the outputs of ssa_block_pool for the same q, k;
  * block_idx: ssa_block_select's table.  Outputs o, lse as for the sparse
- * forward, and, if visited is not NULL, the blocks each tile visited,
- * [B][Hkv][n][G / 2] int32 (head pair p holds query heads h*G + 2p, +1).
+ * forward, and, if visited is not NULL, the blocks each segment visited,
+ * [B][Hq][n] int32.
  * Errors: INVALID_ARG for null/misaligned pointers or tau not finite and
  * >= 0; UNSUPPORTED for top_k > 256 and the cases of the sparse forward. */
 ssa_status ssa_sparse_attn_fwd_early_stop(const ssa_problem *p, const ssa_bf16 *q,
@@ -293,9 +294,11 @@ ssa_status ssa_alignment_bwd(const ssa_problem *p, const ssa_bf16 *q, const ssa_
  *    SSA_NOALLOC_SCRATCH_BYTES is rejected with SSA_ERR_WORKSPACE before
  *    anything is launched.
  *  - The first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture on the device.  A failed look-up returns
- *    SSA_ERR_CUDA.
+ *    (cudaGetSymbolAddress) with that device current, once, and keeps it.
+ *    Make that first call before any stream capture on the device: the
+ *    look-up may load the library's device code onto the device, which is
+ *    not allowed while a stream is being captured.  A failed look-up
+ *    returns SSA_ERR_CUDA.
  *  - Every call on a device shares the one array and leaves its contents
  *    behind; nothing in it has to start at zero.  Calls whose kernels
  *    overlap on the GPU (on different streams, or from several threads)

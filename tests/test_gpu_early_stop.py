@@ -1,12 +1,15 @@
 """GPU parity of the early-stop sparse forward (ssa_sparse_attn_fwd_early_stop)
-against the fp64 oracle.  A tile's stop decision compares a mass ratio with
-tau, and its visiting order compares pooled scores; tiles where either is
+against the fp64 oracle.  The unit that stops is one head's query segment
+(query head, query block).  Its stop decision compares a mass ratio with tau,
+and its visiting order compares pooled scores; segments where either is
 within rounding of flipping (stop margin under 0.05 in log ratio, or two of
 the scores it reaches closer than 1e-3) are left out of the exact comparison.
-Elsewhere: the blocks visited per tile are equal, outputs max-abs <= 2e-2,
-LSE <= 1e-3; and tau = 0 reproduces ssa_sparse_attn_fwd.  A large top-k with a
-high tau makes every tile of a CTA stop while the loader is still several
-blocks ahead, which must end without a timed-out wait."""
+Elsewhere: the blocks visited per segment are equal, outputs max-abs <= 2e-2,
+LSE <= 1e-3; and tau = 0 reproduces ssa_sparse_attn_fwd.  The kernel packs two
+heads into one 128-row tile, so the cases must include tiles whose two heads
+stop at different blocks.  A large top-k with a high tau makes every tile of a
+CTA stop while the loader is still several blocks ahead, which must end
+without a timed-out wait."""
 import numpy as np
 import pytest
 import torch
@@ -49,9 +52,11 @@ def test_early_stop_matches_oracle(case, tau):
                                   (1, 4096, 8, 2, 128, 40, 8)],
                          ids=lambda c: "x".join(map(str, c)))
 def test_early_stop_well_before_the_last_block(case, tau):
-    vis, nsel = _check(case, tau, min_clear=0.5)
-    # most tiles stop with more than a pipeline's depth of blocks left
-    assert np.mean(nsel[..., None] - vis >= 8) > 0.5
+    vis, nsel, apart = _check(case, tau, min_clear=0.5)
+    # most segments stop with more than a pipeline's depth of blocks left
+    assert np.mean(nsel - vis >= 8) > 0.5
+    # and in some tile the two heads stop at different blocks
+    assert apart > 0
 
 
 def _check(case, tau, min_clear=0.6):
@@ -64,36 +69,39 @@ def _check(case, tau, min_clear=0.6):
     n, G = S // 64, Hq // Hkv
     o = torch.empty_like(st.o)
     lse = torch.empty_like(st.lse)
-    vis = torch.empty(B, Hkv, n, G // 2, dtype=torch.int32, device=DEV)
+    vis = torch.empty(B, Hq, n, dtype=torch.int32, device=DEV)
     ssa.ssa_sparse_attn_fwd_early_stop(p, q, k, v, st.q_pooled, st.k_pooled, st.block_idx, tau, o, lse, vis)
     torch.cuda.synchronize()
     assert ssa.ssa_get_device_error() == 0
     gidx = oracle_table(x, topk, st.block_idx)
     okb, oqb = oracle.block_pool(x.k, x.q)
     ro, rlse, rvis, margin = oracle.early_stop_forward(x.q, x.k, x.v, oqb, okb, gidx, tau)
-    gvis = vis.cpu().numpy()
-    nsel = (gidx >= 0).sum(axis=-1)
-    assert np.all(gvis >= 1) and np.all(gvis <= nsel[..., None])
-    # tiles whose order or stop decision could flip between fp32 and fp64
+    gvis = vis.cpu().numpy()                                   # [B, Hq, n]
+    nsel = np.repeat((gidx >= 0).sum(axis=-1), G, axis=1)      # [B, Hq, n]
+    assert np.all(gvis >= 1) and np.all(gvis <= nsel)
+    # segments whose order or stop decision could flip between fp32 and fp64
     clear = margin > 0.05
     for b in range(B):
-        for h in range(Hkv):
+        for hq in range(Hq):
+            h = hq // G
             for i in range(n):
                 sel = [j for j in gidx[b, h, i] if 0 <= j < i]
-                # only the order of the blocks a tile reaches (and of the next
-                # one) can change its result
-                sc = np.sort([okb[b, h, j] @ oqb[b, h, i] for j in sel])[::-1][: rvis[b, h, i].max() + 1]
+                # only the order of the blocks a segment reaches (and of the
+                # next one) can change its result
+                sc = np.sort([okb[b, h, j] @ oqb[b, h, i] for j in sel])[::-1][: rvis[b, hq, i] + 1]
                 if len(sc) > 1 and np.min(np.abs(np.diff(sc))) < 1e-3:
-                    clear[b, h, i, :] = False
+                    clear[b, hq, i] = False
     assert clear.mean() > min_clear
     assert np.array_equal(gvis[clear], rvis[clear])
     go, gl = o.float().cpu().numpy(), lse.cpu().numpy()
-    for b, h, i, hp in zip(*np.nonzero(clear)):
-        heads = [h * G + 2 * hp, h * G + 2 * hp + 1]
+    for b, hq, i in zip(*np.nonzero(clear)):
         rows = slice(64 * i, 64 * i + 64)
-        assert np.abs(go[b, rows][:, heads] - ro[b, rows][:, heads]).max() <= 2e-2
-        assert np.abs(gl[b, heads][:, rows] - rlse[b, heads][:, rows]).max() <= 1e-3
+        assert np.abs(go[b, rows, hq] - ro[b, rows, hq]).max() <= 2e-2
+        assert np.abs(gl[b, hq, rows] - rlse[b, hq, rows]).max() <= 1e-3
+    # tiles (head pairs 2p, 2p + 1 of one query block) whose heads stop apart
+    pair = clear[:, 0::2] & clear[:, 1::2]
+    apart = int(np.sum(pair & (gvis[:, 0::2] != gvis[:, 1::2])))
     if tau == 0.0:
-        assert np.array_equal(gvis, np.repeat(nsel[..., None], G // 2, axis=-1))
+        assert np.array_equal(gvis, nsel)
         assert (o.float() - st.o.float()).abs().max().item() <= 2e-2
-    return gvis, nsel
+    return gvis, nsel, apart

@@ -1,13 +1,18 @@
 """Repeated launches of the early-stop sparse forward
-(ssa_sparse_attn_fwd_early_stop) on a case whose tiles stop well before the
-end of their tables must agree bit for bit.  Collected after the other GPU
-parity tests, so a run that stops at the first failure has run those."""
+(ssa_sparse_attn_fwd_early_stop) on a case whose segments stop well before
+the end of their tables must agree bit for bit, and the first launch must
+match the fp64 oracle on the segments whose decisions are clear (a result
+that is wrong the same way every time would otherwise pass).  Collected after
+the other GPU parity tests, so a run that stops at the first failure has run
+those."""
 import numpy as np
 import pytest
 import torch
 
 import block_sparse_attention_21_b200 as ssa
 import gen
+import oracle
+from conftest import oracle_table
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -41,14 +46,34 @@ def test_early_stop_repeats_bit_for_bit(D):
     for _ in range(40):
         o = torch.empty_like(st.o)
         lse = torch.empty_like(st.lse)
-        vis = torch.empty(B, Hkv, n, G // 2, dtype=torch.int32, device=DEV)
+        vis = torch.empty(B, Hq, n, dtype=torch.int32, device=DEV)
         ssa.ssa_sparse_attn_fwd_early_stop(p, q, k, v, st.q_pooled, st.k_pooled, st.block_idx, 0.3, o, lse, vis)
         runs.append((o, lse, vis))
     torch.cuda.synchronize()
     assert ssa.ssa_get_device_error() == 0
     o0, l0, v0 = runs[0]
     nsel = np.minimum(topk, np.arange(n) + 1)
-    assert np.mean(nsel[None, :, None] - v0.cpu().numpy() >= 8) > 0.5  # most tiles stop early
+    assert np.mean(nsel[None, None, :] - v0.cpu().numpy() >= 8) > 0.5  # most segments stop early
     for o, lse, vis in runs[1:]:
         assert torch.equal(vis, v0)
         assert torch.equal(o.view(torch.int16), o0.view(torch.int16)) and torch.equal(lse, l0)
+    # the first launch against the oracle, on the segments whose visiting
+    # order and stop decision are clear of rounding (as in test_gpu_early_stop)
+    gidx = oracle_table(x, topk, st.block_idx)
+    okb, oqb = oracle.block_pool(x.k, x.q)
+    ro, rlse, rvis, margin = oracle.early_stop_forward(x.q, x.k, x.v, oqb, okb, gidx, 0.3)
+    clear = margin > 0.05
+    for hq in range(Hq):
+        h = hq // G
+        for i in range(n):
+            sc = np.sort([okb[0, h, j] @ oqb[0, h, i] for j in gidx[0, h, i] if 0 <= j < i])[::-1]
+            sc = sc[: rvis[0, hq, i] + 1]
+            if len(sc) > 1 and np.min(np.abs(np.diff(sc))) < 1e-3:
+                clear[0, hq, i] = False
+    assert clear.mean() > 0.5
+    gv, go, gl = v0.cpu().numpy(), o0.float().cpu().numpy(), l0.cpu().numpy()
+    assert np.array_equal(gv[clear], rvis[clear])
+    for _, hq, i in zip(*np.nonzero(clear)):
+        rows = slice(64 * i, 64 * i + 64)
+        assert np.abs(go[0, rows, hq] - ro[0, rows, hq]).max() <= 2e-2
+        assert np.abs(gl[0, hq, rows] - rlse[0, hq, rows]).max() <= 1e-3
