@@ -227,8 +227,16 @@ struct DkdvConfig {
 
 // kDkdvSplit CTAs per (batch b, KV head h, key block j), CTA sp taking tiles
 // sp, sp + kDkdvSplit, ... of j's list.  TMEM: S at +0 and dP at +64
-// (128 lanes x 64 fp32 each), dV at +128 and dK at +128 + D (M = 64
-// accumulators: key row r sits in lane (r % 16) + 32 * (r / 16)).
+// (128 lanes x 64 fp32 each), then one M = 128, N = 2D accumulator at +128:
+// dV and dK come from a single MMA per K-step with the operands stacked,
+//   A = [P^T ; dS^T]  (128 x 16: the P tile then the dS tile, MN-major)
+//   B = [Q | dO]      (16 x 2D: the Q tile then the dO tile, MN-major)
+// so lanes 0..63 hold P^T Q | P^T dO and lanes 64..127 dS^T Q | dS^T dO:
+// dV = P^T dO sits in lanes 0..63, columns D..2D-1, and dK = dS^T Q in lanes
+// 64..127, columns 0..D-1 (the other two quadrants are discarded).  One
+// M = 128 MMA in place of two M = 64 ones halves the instructions of this
+// step, which is bound by their issue, at the cost of tensor work that is
+// not used.  Key row r of dV is lane r, of dK lane 64 + r.
 template <int D>
 __global__ void __launch_bounds__(256, DkdvConfig<D>::MIN_CTAS)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -247,9 +255,11 @@ __global__ void __launch_bounds__(256, DkdvConfig<D>::MIN_CTAS)
   uint8_t* smem = smem_raw;
   uint8_t* sK = smem;
   uint8_t* sV = sK + KVT;
-  uint8_t* sQ = sV + KVT;              // [NQ][QTILE]
-  uint8_t* sdO = sQ + NQ * QTILE;      // [NQ][QTILE]
-  uint8_t* sP = sdO + NQ * QTILE;      // P tile, then dS tile
+  // stage qs holds its Q tile, then its dO tile: the B operand [Q | dO] of
+  // the dV/dK MMA steps through the 64-column panels of both at one stride
+  uint8_t* sQ = sV + KVT;              // [NQ][Q tile, dO tile]
+  uint8_t* sdO = sQ + QTILE;
+  uint8_t* sP = sQ + NQ * 2 * QTILE;   // P tile, then dS tile
   uint8_t* sdS = sP + PTILE;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sdS + PTILE);
   uint64_t* kv_full = bars;
@@ -323,9 +333,9 @@ __global__ void __launch_bounds__(256, DkdvConfig<D>::MIN_CTAS)
         mbar_arrive_expect_tx(&q_full[qs], 2 * QTILE);
         for (int hh = 0; hh < 2; ++hh)
           for (int pn = 0; pn < NP; ++pn) {
-            tma_load_4d(sQ + qs * QTILE + pn * (128 * 128) + hh * (64 * 128), &tm_q, &q_full[qs],
+            tma_load_4d(sQ + qs * 2 * QTILE + pn * (128 * 128) + hh * (64 * 128), &tm_q, &q_full[qs],
                         64 * pn, hq0 + hh, 64 * i, b);
-            tma_load_4d(sdO + qs * QTILE + pn * (128 * 128) + hh * (64 * 128), &tm_do, &q_full[qs],
+            tma_load_4d(sdO + qs * 2 * QTILE + pn * (128 * 128) + hh * (64 * 128), &tm_do, &q_full[qs],
                         64 * pn, hq0 + hh, 64 * i, b);
           }
         ++issued;
@@ -341,25 +351,26 @@ __global__ void __launch_bounds__(256, DkdvConfig<D>::MIN_CTAS)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && ntiles > 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, false);
-      // M = 64 keys, N = D, both operands MN-major (bit 15: A, bit 16: B)
-      constexpr uint32_t idesc_kv = idesc_bf16_f32(64, D, true) | (1u << 15);
+      // M = 128 (P^T over dS^T), N = 2D (Q then dO), both operands MN-major
+      // (bit 15: A, bit 16: B)
+      constexpr uint32_t idesc_kv = idesc_bf16_f32(128, 2 * D, true) | (1u << 15);
       const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), adO = smem_u32(sdO),
-                     aP = smem_u32(sP), adS = smem_u32(sdS);
-      const uint32_t tS = tmem, tdP = tmem + 64, tdV = tmem + 128, tdK = tmem + 128 + D;
+                     aP = smem_u32(sP);
+      const uint32_t tS = tmem, tdP = tmem + 64, tKV = tmem + 128;
       auto issue_scores = [&](int x) {
         const int qs = x % NQ;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t o = (kk / 4) * (128 * 128) + (kk % 4) * 32;
           const uint32_t ok_ = (kk / 4) * (64 * 128) + (kk % 4) * 32;
-          mma_ss(tS, sdesc_sw128(aQ + qs * QTILE + o, 16, 1024), sdesc_sw128(aK + ok_, 16, 1024),
+          mma_ss(tS, sdesc_sw128(aQ + qs * 2 * QTILE + o, 16, 1024), sdesc_sw128(aK + ok_, 16, 1024),
                  idesc_s, kk > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t o = (kk / 4) * (128 * 128) + (kk % 4) * 32;
           const uint32_t ok_ = (kk / 4) * (64 * 128) + (kk % 4) * 32;
-          mma_ss(tdP, sdesc_sw128(adO + qs * QTILE + o, 16, 1024), sdesc_sw128(aV + ok_, 16, 1024),
+          mma_ss(tdP, sdesc_sw128(adO + qs * 2 * QTILE + o, 16, 1024), sdesc_sw128(aV + ok_, 16, 1024),
                  idesc_s, kk > 0 ? 1u : 0u);
         }
         tc_commit(s_full);
@@ -387,14 +398,14 @@ __global__ void __launch_bounds__(256, DkdvConfig<D>::MIN_CTAS)
           break;
         }
         tc_fence_after();
-        // dV += P^T dO and dK += dS^T Q over the tile's 128 rows (8 K-steps)
+        // [P^T ; dS^T] [Q | dO] over the tile's 128 rows (8 K-steps of 16
+        // rows = 2048 B): A's second 64-row chunk (dS) sits PTILE after the
+        // first (P), B's 64-column panels (Q, then dO) are 128 x 128 B apart
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t acc = (x > 0 || kk > 0) ? 1u : 0u;
-          mma_ss(tdV, sdesc_sw128(aP + kk * 2048, PTILE, 1024),
-                 sdesc_sw128(adO + qs * QTILE + kk * 2048, 128 * 128, 1024), idesc_kv, acc);
-          mma_ss(tdK, sdesc_sw128(adS + kk * 2048, PTILE, 1024),
-                 sdesc_sw128(aQ + qs * QTILE + kk * 2048, 128 * 128, 1024), idesc_kv, acc);
+          mma_ss(tKV, sdesc_sw128(aP + kk * 2048, PTILE, 1024),
+                 sdesc_sw128(aQ + qs * 2 * QTILE + kk * 2048, 128 * 128, 1024), idesc_kv, acc);
         }
         tc_commit(p_done);
         tc_commit(&q_empty[qs]);
@@ -463,31 +474,27 @@ __global__ void __launch_bounds__(256, DkdvConfig<D>::MIN_CTAS)
       mbar_arrive(p_full);
     }
     // ---------------------------------------------------------- epilogue
-    // key row kr = 16 * wq + lane (lanes 0..15 of each quadrant hold the M = 64
-    // rows); this CTA's fp32 partial sums of dV and dK (dK not yet scaled)
-    const int kr = 16 * wq + lane;
+    // lanes 0..63 (warps wq 0, 1) hold dV's key rows in columns D..2D-1,
+    // lanes 64..127 (wq 2, 3) dK's in columns 0..D-1: this CTA's fp32 partial
+    // sums of dV and dK (dK not yet scaled)
+    const int which = wq / 2;                  // 0: dV, 1: dK
+    const int kr = 32 * (wq % 2) + lane;       // key row
     float* part = p.part + (static_cast<size_t>(bhn) * kDkdvSplit + sp) * 2 * 64 * D;
+    float* out_row = part + (which * 64 + kr) * D;
     if (ntiles == 0) {
-      if (lane < 16)
-        for (int which = 0; which < 2; ++which)
-          for (int d = 0; d < D; d += 4)
-            *reinterpret_cast<float4*>(part + (which * 64 + kr) * D + d) = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int d = 0; d < D; d += 4)
+        *reinterpret_cast<float4*>(out_row + d) = make_float4(0.f, 0.f, 0.f, 0.f);
     } else if (ok && __all_sync(0xffffffffu, mbar_wait(o_done, 0, abort_flag, tmo, 0xa03))) {
       tc_fence_after();
+      const uint32_t base = row + 128 + (which == 0 ? D : 0);
 #pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        const uint32_t base = row + 128 + which * D;
+      for (int ch = 0; ch < D / 32; ++ch) {
+        float o[32];
+        tmem_ld32(base + ch * 32, o);
+        float4* out = reinterpret_cast<float4*>(out_row + ch * 32);
 #pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
-          float o[32];
-          tmem_ld32(base + ch * 32, o);
-          if (lane < 16) {
-            float4* out = reinterpret_cast<float4*>(part + (which * 64 + kr) * D + ch * 32);
-#pragma unroll
-            for (int v4 = 0; v4 < 8; ++v4)
-              out[v4] = make_float4(o[4 * v4], o[4 * v4 + 1], o[4 * v4 + 2], o[4 * v4 + 3]);
-          }
-        }
+        for (int v4 = 0; v4 < 8; ++v4)
+          out[v4] = make_float4(o[4 * v4], o[4 * v4 + 1], o[4 * v4 + 2], o[4 * v4 + 3]);
       }
     }
   }
