@@ -215,7 +215,7 @@ struct DkdvConfig {
   static constexpr int PTILE = 128 * 64 * 2;   // P or dS tile
   static constexpr int NQ = 2;                 // Q/dO ring stages
   static constexpr int TMEM_COLS = pow2_at_least(128 + 2 * D);
-  static constexpr int THREADS = 256;          // warp 0 producer, 1 issuer, 4..7 elementwise
+  static constexpr int THREADS = 256;          // warp 0 producer, 1-2 issuers, 4..7 elementwise
   static constexpr int NBARS = 1 + 2 * NQ + 7;
   // no alignment slack: the dynamic shared memory of a kernel without static
   // shared memory starts 1024-byte aligned (the kernel checks it), which lets
@@ -294,14 +294,15 @@ __global__ void __launch_bounds__(256, DkdvConfig<D>::MIN_CTAS)
     mbar_init(kv_full, 1);
     for (int s = 0; s < NQ; ++s) {
       mbar_init(&q_full[s], 1);
-      mbar_init(&q_empty[s], 1);
+      mbar_init(&q_empty[s], 2);  // released by both issuers
     }
     mbar_init(s_full, 1);
     mbar_init(s_free, 128);
     mbar_init(p_full, 128);
     mbar_init(p_done, 1);
     mbar_init(o_done, 1);
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -347,43 +348,48 @@ __global__ void __launch_bounds__(256, DkdvConfig<D>::MIN_CTAS)
           mbar_wait(&q_full[x % NQ], (x / NQ) & 1, &never, 1000000ull, 0x8ff);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == 2) {
+    // ------------------------------------------------------------ MMA issuers
+    // Two issuing threads, so that the issue cost of one tile's dV/dK MMAs
+    // overlaps that of the next tile's S and dP (each thread's tcgen05.mma
+    // issue, not the tensor pipe, bounds this kernel):
+    //   warp 1  S(x+1) = Q K^T and dP(x+1) = dO V^T once the elementwise
+    //           warps hold tile x's (they write TMEM columns 0..127 only)
+    //   warp 2  the dV/dK MMAs of tile x once P(x) and dS(x) are in shared
+    //           memory (they write the accumulator at column 128 only)
+    // Each releases a Q/dO stage once its own MMAs on it have completed.
     if (lane == 0 && ntiles > 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, false);
-      // M = 128 (P^T over dS^T), N = 2D (Q then dO), both operands MN-major
-      // (bit 15: A, bit 16: B)
-      constexpr uint32_t idesc_kv = idesc_bf16_f32(128, 2 * D, true) | (1u << 15);
       const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), adO = smem_u32(sdO),
                      aP = smem_u32(sP);
-      const uint32_t tS = tmem, tdP = tmem + 64, tKV = tmem + 128;
-      auto issue_scores = [&](int x) {
-        const int qs = x % NQ;
+      bool ok = true;
+      if (warp == 1) {
+        constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, false);
+        const uint32_t tS = tmem, tdP = tmem + 64;
+        auto issue_scores = [&](int x) {
+          const int qs = x % NQ;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t o = (kk / 4) * (128 * 128) + (kk % 4) * 32;
-          const uint32_t ok_ = (kk / 4) * (64 * 128) + (kk % 4) * 32;
-          mma_ss(tS, sdesc_sw128(aQ + qs * 2 * QTILE + o, 16, 1024), sdesc_sw128(aK + ok_, 16, 1024),
-                 idesc_s, kk > 0 ? 1u : 0u);
-        }
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t o = (kk / 4) * (128 * 128) + (kk % 4) * 32;
+            const uint32_t ok_ = (kk / 4) * (64 * 128) + (kk % 4) * 32;
+            mma_ss(tS, sdesc_sw128(aQ + qs * 2 * QTILE + o, 16, 1024), sdesc_sw128(aK + ok_, 16, 1024),
+                   idesc_s, kk > 0 ? 1u : 0u);
+          }
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t o = (kk / 4) * (128 * 128) + (kk % 4) * 32;
-          const uint32_t ok_ = (kk / 4) * (64 * 128) + (kk % 4) * 32;
-          mma_ss(tdP, sdesc_sw128(adO + qs * 2 * QTILE + o, 16, 1024), sdesc_sw128(aV + ok_, 16, 1024),
-                 idesc_s, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t o = (kk / 4) * (128 * 128) + (kk % 4) * 32;
+            const uint32_t ok_ = (kk / 4) * (64 * 128) + (kk % 4) * 32;
+            mma_ss(tdP, sdesc_sw128(adO + qs * 2 * QTILE + o, 16, 1024), sdesc_sw128(aV + ok_, 16, 1024),
+                   idesc_s, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(s_full);
+          tc_commit(&q_empty[qs]);  // this thread's reads of the stage
+        };
+        ok = mbar_wait(kv_full, 0, abort_flag, tmo, 0x901) && mbar_wait(&q_full[0], 0, abort_flag, tmo, 0x902);
+        if (ok) {
+          tc_fence_after();
+          issue_scores(0);
         }
-        tc_commit(s_full);
-      };
-      bool ok = mbar_wait(kv_full, 0, abort_flag, tmo, 0x901) &&
-                mbar_wait(&q_full[0], 0, abort_flag, tmo, 0x902);
-      if (ok) {
-        tc_fence_after();
-        issue_scores(0);
-      }
-      for (int x = 0; ok && x < ntiles; ++x) {
-        const int qs = x % NQ;
-        if (x + 1 < ntiles) {
+        for (int x = 0; ok && x + 1 < ntiles; ++x) {
           // the next tile's S and dP once the elementwise warps hold this one's
           if (!mbar_wait(s_free, x & 1, abort_flag, tmo, 0x903) ||
               !mbar_wait(&q_full[(x + 1) % NQ], ((x + 1) / NQ) & 1, abort_flag, tmo, 0x904)) {
@@ -393,29 +399,39 @@ __global__ void __launch_bounds__(256, DkdvConfig<D>::MIN_CTAS)
           tc_fence_after();
           issue_scores(x + 1);
         }
-        if (!mbar_wait(p_full, x & 1, abort_flag, tmo, 0x905)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        // [P^T ; dS^T] [Q | dO] over the tile's 128 rows (8 K-steps of 16
-        // rows = 2048 B): A's second 64-row chunk (dS) sits PTILE after the
-        // first (P), B's 64-column panels (Q, then dO) are 128 x 128 B apart
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t acc = (x > 0 || kk > 0) ? 1u : 0u;
-          mma_ss(tKV, sdesc_sw128(aP + kk * 2048, PTILE, 1024),
-                 sdesc_sw128(aQ + qs * 2 * QTILE + kk * 2048, 128 * 128, 1024), idesc_kv, acc);
-        }
-        tc_commit(p_done);
-        tc_commit(&q_empty[qs]);
-      }
-      if (ok) {
-        tc_commit(o_done);
       } else {
-        tc_commit(drain);
+        // M = 128 (P^T over dS^T), N = 2D (Q then dO), both operands MN-major
+        // (bit 15: A, bit 16: B)
+        constexpr uint32_t idesc_kv = idesc_bf16_f32(128, 2 * D, true) | (1u << 15);
+        const uint32_t tKV = tmem + 128;
+        for (int x = 0; ok && x < ntiles; ++x) {
+          const int qs = x % NQ;
+          if (!mbar_wait(p_full, x & 1, abort_flag, tmo, 0x905) ||
+              !mbar_wait(&q_full[qs], (x / NQ) & 1, abort_flag, tmo, 0x906)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          // [P^T ; dS^T] [Q | dO] over the tile's 128 rows (8 K-steps of 16
+          // rows = 2048 B): A's second 64-row chunk (dS) sits PTILE after the
+          // first (P), B's 64-column panels (Q, then dO) are 128 x 128 B apart
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t acc = (x > 0 || kk > 0) ? 1u : 0u;
+            mma_ss(tKV, sdesc_sw128(aP + kk * 2048, PTILE, 1024),
+                   sdesc_sw128(aQ + qs * 2 * QTILE + kk * 2048, 128 * 128, 1024), idesc_kv, acc);
+          }
+          tc_commit(p_done);
+          tc_commit(&q_empty[qs]);
+        }
+        if (ok) tc_commit(o_done);
+      }
+      if (!ok) {
+        // every MMA this thread issued completes before TMEM is released
+        uint64_t* dr = &drain[warp - 1];
+        tc_commit(dr);
         volatile int never = 0;
-        mbar_wait(drain, 0, &never, tmo, 0x9ff);
+        mbar_wait(dr, 0, &never, tmo, 0x9ff);
       }
     }
   } else if (warp >= 4) {
