@@ -102,13 +102,17 @@ __device__ __forceinline__ void report_timeout(volatile int* abort_flag, unsigne
 // Waits for the phase with the given parity to complete.  Gives up when the
 // CTA's abort flag is raised by another thread, or after timeout_ns of
 // %globaltimer, in which case it raises the abort flag and records the site in
-// the device error word.  Returns true only if the phase completed.
+// the device error word.  Returns true only if the phase completed.  The flag
+// and the clock are read once per 16 try_wait attempts, so a waiting warp
+// takes few issue slots from the warps that work.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           uint64_t timeout_ns, unsigned int site) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+#pragma unroll 1
+    for (int i = 0; i < 16; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
     if (globaltimer_ns() - t0 > timeout_ns) {
       *abort_flag = 1;
@@ -129,6 +133,26 @@ __device__ __forceinline__ bool mbar_wait_or(uint64_t* bar, uint32_t parity, vol
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag || *release) return false;
+    if (globaltimer_ns() - t0 > timeout_ns) {
+      *abort_flag = 1;
+      atomicOr(&g_error_word, kErrTimeout);
+      atomicExch(&g_error_site, site);
+      return false;
+    }
+  }
+}
+
+// mbar_wait that also gives up, without an error, once *flag == value
+// (another thread decided the phase is no longer needed).  Returns true only
+// if the phase completed.
+__device__ __forceinline__ bool mbar_wait_until(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                volatile int* flag, int value, uint64_t timeout_ns,
+                                                unsigned int site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag || *flag == value) return false;
     if (globaltimer_ns() - t0 > timeout_ns) {
       *abort_flag = 1;
       atomicOr(&g_error_word, kErrTimeout);

@@ -27,7 +27,7 @@ struct FwdParams {
   const float* qbar;     // [B][Hkv][n][D]
   const float* kbar;     // [B][Hkv][n][D]
   float tau;
-  int32_t* visited;      // [B][Hkv][n][G / 2], or null
+  int32_t* visited;      // [B][Hq][n], or null
   // DashAttention (prior-induced softmax): the routed chunks of each query
   // block as a bit mask, their group weights, and the prior strength
   const uint32_t* dmask; // [B][Hkv][n][ceil(n / 32)]

@@ -48,6 +48,8 @@ CASES = [
     (2, 2048, 4, 2, 64, 1, [2048, 700]),            # top-k 1: the query's own block only
     (1, 65536, 4, 1, 128, 32, [65536]),             # 1024 blocks: scored by a grid of their own
     (2, 4096, 8, 2, 64, 16, [1024, 1025]),          # 16 blocks: all kept; 17: the search
+    (2, 8192, 8, 2, 64, 64, [4096, 8192]),          # 64 blocks: all kept; 128: the search
+    (1, 16384, 8, 2, 64, 96, [16384]),              # a budget of 96 blocks: 96 partials per row
 ]
 
 

@@ -125,6 +125,9 @@ SMALL = [
     # O and statistics buffers are reused (two O buffers at D = 64, one at 128)
     (1, 8192, 16, 2, 64, 2, 2),
     (1, 4096, 16, 2, 128, 3, 2),
+    # 400 units at D = 64 on 296 persistent CTAs: some CTAs walk one unit,
+    # some two, of block counts from 1 to 8 (B = 2, G = 4)
+    (2, 6400, 8, 2, 64, 8, 3),
 ]
 
 
