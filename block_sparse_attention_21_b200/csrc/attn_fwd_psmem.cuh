@@ -1,5 +1,6 @@
 // attn_fwd_psmem.cuh -- block-sparse causal attention forward on tcgen05 tensor
-// cores, with P staged in shared memory (the variant used at head_dim 128).
+// cores, with P in TMEM columns of its own, so each tile's next scores are
+// computed while it exponentiates (the variant used at head_dim 128).
 //
 // A work unit is one query block i (64 tokens) of one batch entry for 2*T
 // query heads that share KV head h; a CTA takes one unit, or in the plain
@@ -30,8 +31,8 @@
 //   S_t(jj) = Q_t K(jj)^T          tensor core, fp32 in TMEM
 //   softmax warps load S_t(jj) into registers and release it at once, so the
 //   issuer can start S_t(jj+1) while they exponentiate
-//   P_t(jj) (bf16) -> shared memory, 128-byte swizzled like Q
-//   O_t += P_t(jj) V(jj)           tensor core, A and B from shared memory
+//   P_t(jj) (bf16 pairs) -> TMEM columns of its own
+//   O_t += P_t(jj) V(jj)           tensor core, A from TMEM, B from shared memory
 // so the score MMA of the next block and the P.V of this block both overlap
 // the softmax.  O is rescaled in TMEM (lazily, see below) after the previous
 // P.V has completed.
@@ -50,8 +51,12 @@
 //               reference maximum only moves when the row maximum exceeds it
 //               by more than 8, i.e. a factor 256), and the epilogue.
 //
-// TMEM per M-tile t (stride 64 + D, or 64 + 2D with MASS): S at +0 (64 fp32
-// columns), O (O_selected with MASS) at +64, O_unselected at +64 + D.
+// TMEM per M-tile t (stride 96 + D, or 96 + 2D with MASS): S at +0 (64 fp32
+// columns), P at +64 (64 keys as 32 columns of bf16 pairs), O (O_selected
+// with MASS) at +96, O_unselected at +96 + D.  Two tiles take 448 of the 512
+// columns at head_dim 128.  Keeping P out of shared memory leaves the shared
+// memory bandwidth to the operand reads of the MMAs (P was written and then
+// read again as the P.V MMA's A operand: 32 KB per tile and block).
 //
 // Persistent CTAs (plain sparse stream).  One CTA per SM takes the work units
 // blockIdx.x, blockIdx.x + gridDim.x, ... (heaviest query blocks first) and
@@ -77,9 +82,10 @@ struct PsFwdConfig {
   static constexpr int NP = D / 64;               // 64-column panels per row
   static constexpr int QTILE = 128 * D * 2;       // bytes of one Q M-tile
   static constexpr int KVT = 64 * D * 2;          // bytes of one K (or V) block
-  static constexpr int PTILE = 128 * 64 * 2;      // bytes of one P tile (128 rows x 64 keys)
-  static constexpr int NS = (D == 64) ? 4 : 3;    // K/V ring stages
-  static constexpr int TSTRIDE = 64 + (MASS ? 2 : 1) * D;  // TMEM columns per M-tile
+  static constexpr int NS = 4;                    // K/V ring stages
+  // TMEM columns per M-tile: S (64 fp32), P (32: 64 keys as bf16 pairs), O
+  // (O_selected with MASS), O_unselected (MASS)
+  static constexpr int TSTRIDE = 96 + (MASS ? 2 : 1) * D;
   static constexpr int TMEM_COLS = pow2_at_least(T * TSTRIDE);
   static constexpr int POLY = 4;                  // exp2 pairs of 8 on the FMA pipe
   // warps: 0 producer, 1..3 issuers, 4.. softmax (4 per tile), then the
@@ -87,10 +93,10 @@ struct PsFwdConfig {
   static constexpr int THREADS = 128 * (T + 1) + (T > 3 ? 32 : 0);
   // barriers: q, kfull/vfull/empty[NS], sfull/sfree/pfull/pvdone/odone/drain/turn[T], qfree
   static constexpr int NBARS = 1 + 3 * NS + 7 * T + 1;
-  // shared memory: Q tiles, K ring, V ring, P tiles, barriers, tmem slot,
+  // shared memory: Q tiles, K ring, V ring, barriers, tmem slot,
   // abort flag, selection bitmap (up to 8192 blocks); DASH: the routed chunk
   // list and its biases (kDashMaxN each) and the count
-  static constexpr int SMEM_TILES = T * QTILE + 2 * NS * KVT + T * PTILE;
+  static constexpr int SMEM_TILES = T * QTILE + 2 * NS * KVT;
   // EARLY: 2 KB of visiting-order scratch and 128 B of stop flags
   static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + NBARS * 8 + 16 + 1024 + (DASH ? 8 * kDashMaxN + 16 : 0) +
                                     (EARLY ? 2048 + 128 : 0);
@@ -111,8 +117,7 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH, EARLY>::THREADS,
   using C = PsFwdConfig<D, T, MASS, DASH, EARLY>;
   static_assert(!(MASS && DASH), "the routed softmax is a mode of its own");
   static_assert(!(EARLY && (MASS || DASH)), "the early stop applies to the sparse stream only");
-  constexpr int NP = C::NP, QTILE = C::QTILE, KVT = C::KVT, PTILE = C::PTILE, NS = C::NS,
-                TSTRIDE = C::TSTRIDE;
+  constexpr int NP = C::NP, QTILE = C::QTILE, KVT = C::KVT, NS = C::NS, TSTRIDE = C::TSTRIDE;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -120,15 +125,14 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH, EARLY>::THREADS,
   uint8_t* sQ = smem;                 // [T][QTILE]
   uint8_t* sK = sQ + T * QTILE;       // [NS][KVT]
   uint8_t* sV = sK + NS * KVT;        // [NS][KVT]
-  uint8_t* sP = sV + NS * KVT;        // [T][PTILE]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + T * PTILE);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + NS * KVT);
   uint64_t* bar_q = bars;
   uint64_t* bar_kfull = bar_q + 1;              // [NS]
   uint64_t* bar_vfull = bar_kfull + NS;
   uint64_t* bar_empty = bar_vfull + NS;
   uint64_t* bar_sfull = bar_empty + NS;         // [T] scores in TMEM
   uint64_t* bar_sfree = bar_sfull + T;          // [T] scores read by the softmax
-  uint64_t* bar_pfull = bar_sfree + T;          // [T] P in shared memory (O rescaled)
+  uint64_t* bar_pfull = bar_sfree + T;          // [T] P stored in TMEM (O rescaled)
   uint64_t* bar_pvdone = bar_pfull + T;         // [T] P.V completed
   uint64_t* bar_odone = bar_pvdone + T;         // [T] last P.V completed
   uint64_t* bar_drain = bar_odone + T;          // [T] issuer's MMAs drained (abort)
@@ -338,7 +342,7 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH, EARLY>::THREADS,
     if (lane == 0 && t >= 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 64, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
-      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV), sPa = smem_u32(sP);
+      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
       const uint32_t s_tmem = tmem + t * TSTRIDE;
       auto issue_qk = [&](int st) {
 #pragma unroll
@@ -351,7 +355,7 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH, EARLY>::THREADS,
       };
       // Per unit: S(0) once its Q and first K/V block landed and the softmax
       // read the previous unit's last scores; then for s = 0, 1, ...:
-      //   [S(s) read]  S(s+1);   [P(s) in shared memory]  O += P(s) V(s)
+      //   [S(s) read]  S(s+1);   [P(s) stored]  O += P(s) V(s)
       // Parities count the CTA's blocks (g + s) and units (k).
       bool ok = true;
       int g = 0, k = 0;
@@ -381,7 +385,7 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH, EARLY>::THREADS,
             tc_commit(&bar_sfull[t]);
             if (PERSIST && s + 2 == nb) tc_commit(bar_qfree);
           }
-          // P(s).V once P(s) is in shared memory
+          // P(s).V once P(s) is stored
           const int st = gs % NS;
           if (!mbar_wait(&bar_pfull[t], gs & 1, abort_flag, tmo, 0x205) ||
               !mbar_wait(&bar_vfull[st], (gs / NS) & 1, abort_flag, tmo, 0x206)) {
@@ -392,12 +396,11 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH, EARLY>::THREADS,
           bool is_sel = true;
           if (MASS) is_sel = (selbits[s >> 5] >> (s & 31)) & 1u;
           const bool first = MASS ? (is_sel ? first_sel : first_uns) : (s == 0);
-          const uint32_t o_col = s_tmem + 64 + ((MASS && !is_sel) ? D : 0);
+          const uint32_t o_col = s_tmem + 96 + ((MASS && !is_sel) ? D : 0);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t a = sdesc_sw128(sPa + t * PTILE + kk * 32, 16, 1024);
+          for (int kk = 0; kk < 4; ++kk) {  // 16 keys of P (8 TMEM columns) per MMA
             const uint64_t bd = sdesc_sw128(sVa + st * KVT + kk * (16 * 128), 64 * 128, 1024);
-            mma_ss(o_col, a, bd, idesc_pv, (first && kk == 0) ? 0u : 1u);
+            mma_ts(o_col, s_tmem + 64 + kk * 8, bd, idesc_pv, (first && kk == 0) ? 0u : 1u);
           }
           tc_commit(&bar_pvdone[t]);
           // EARLY: the softmax records the position of the block it stops at
@@ -439,10 +442,8 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH, EARLY>::THREADS,
     const int r = wq * 32 + lane;
     const int hh = r / 64, tq = r % 64;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16) + t * TSTRIDE;
-    const uint32_t tS = lane_base, tO = lane_base + 64;
+    const uint32_t tS = lane_base, tP = lane_base + 64, tO = lane_base + 96;
     const uint32_t tOu = tO + D;
-    // this row of the P tile: 8 chunks of 16 B (8 keys each), 128-byte swizzle
-    uint8_t* prow = sP + t * PTILE + r * 128;
     const float sl2 = p.scale_log2;
     const uint64_t scale2 = f2_pack(sl2, sl2);
     bool ok = true;
@@ -574,11 +575,9 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH, EARLY>::THREADS,
             tmem_wait_st();
           }
         }
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) =
-              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        fence_proxy_async_smem();
+        tmem_st16(tP, pk);       // keys 0..31
+        tmem_st16(tP + 16, pk + 16);  // keys 32..63
+        tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bar_pfull[t]);
         if (EARLY && live) hvis = jj + 1;
