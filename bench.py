@@ -719,6 +719,35 @@ def run_reference(args, world, rank):
                     "d2h_bytes_per_step": 0}}
 
 
+def decode_only():
+    """The decode rows alone, timed as in run_ours (L2 flushed by a write and a
+    read-back of 256 MiB before each step, CUDA events around each replay)."""
+    import torch
+    import block_sparse_attention_21_b200 as ssa
+    dev = torch.device("cuda", 0)
+    check_device("decode rows")
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    sink = torch.empty((), dtype=torch.int64, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def timed(graph, n):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n)]
+        for s in range(n):
+            flush.fill_(s & 0xFF)
+            torch.sum(flush.view(torch.int64), dim=0, out=sink)
+            evs[s][0].record(stream)
+            graph.replay()
+            evs[s][1].record(stream)
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in evs)
+
+    n0 = ssa.ssa_launch_count()
+    rows = decode_rows(dev, timed)
+    rows["gpu_launches_total"] = int(ssa.ssa_launch_count() - n0)
+    return {"decode": rows}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -729,9 +758,14 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-other-workloads", action="store_true",
                     help="skip the 32k, batch-2 alignment and batch-4 training workloads")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="time only the decode rows (one GPU) and print them; for profiling")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.decode_only:
+        print(json.dumps(decode_only()), flush=True)
+        return
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":

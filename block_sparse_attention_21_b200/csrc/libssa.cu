@@ -524,45 +524,71 @@ ssa_status launch_align_bwd(const Dims& d, const void* q, const void* k, const v
   return launch_result();
 }
 
-// Workspace of ssa_decode_attn: the selected blocks (unless the caller takes
-// them), then the partial softmax states.
-// From this many blocks per sequence on, decode scores the blocks in a grid
-// of its own (many CTAs) before the per-(b, KV head) selection.
-constexpr int kDecodeSplitBlocks = 1024;
-
-struct DecodeLayout {
-  size_t idx, part, keys, total;
+// ssa_decode_attn: one launch of decode_kernel<D, G>, a cluster of ns CTAs per
+// (b, KV head).  ns fills the resident CTA slots once (up to 8, and no more
+// than the blocks a row keeps); the CTAs of a cluster split the scoring and
+// the kept blocks between them.
+struct DecodeLaunch {
+  int ns, slice_cap, cand_cap, smem;
 };
 
-DecodeLayout decode_layout(const Dims& d) {
-  auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
-  const size_t rows = static_cast<size_t>(d.B) * d.Hkv * d.topk;
-  DecodeLayout L;
-  L.idx = 0;
-  L.part = al(rows * sizeof(int32_t));
-  L.keys = L.part + al(rows * d.G * (d.D + 2) * sizeof(float));
-  const size_t keys = d.n >= kDecodeSplitBlocks ? static_cast<size_t>(d.B) * d.Hkv * d.n * sizeof(uint32_t) : 0;
-  L.total = L.keys + al(keys);
-  return L;
+template <int D, int G>
+DecodeLaunch decode_launch_shape(const Dims& d) {
+  const int need = d.topk - 1;
+  const bool can_search = d.topk < d.n;  // else every causal block is kept
+  auto shape = [&](int ns) {
+    DecodeLaunch s;
+    s.ns = ns;
+    s.slice_cap = can_search ? (d.n - 1 + ns - 1) / ns : 0;
+    s.cand_cap = can_search ? std::min(d.n - 1, ns * std::min(need, s.slice_cap)) : 0;
+    s.smem = ssa::decode_smem<D, G>(d.n, d.topk, s.slice_cap, s.cand_cap).total;
+    return s;
+  };
+  const DecodeLaunch one = shape(1);
+  const int per_sm = std::max(1, std::min(2048 / ssa::kDecodeThreads, (228 * 1024) / (one.smem + 1024)));
+  const int slots = std::max(1, sm_count()) * per_sm;
+  const int units = d.B * d.Hkv;
+  int ns = std::max(1, std::min(ssa::kDecodeMaxCluster, slots / units));
+  ns = std::min(ns, std::max(1, std::min(d.topk, d.n)));
+  return shape(ns);
 }
 
 template <int D, int G>
-ssa_status launch_decode_attn(unsigned items, const ssa::DecodeParams& dp, cudaStream_t st) {
+ssa_status launch_decode_g(const Dims& d, ssa::DecodeParams dp, cudaStream_t st) {
   static std::atomic<uint64_t> smem_done{0};
-  auto kernel = ssa::decode_attn_kernel<D, G>;
-  constexpr int smem = ssa::decode_attn_smem<D, G>();
-  const ssa_status s = ensure_smem(kernel, smem, &smem_done);
-  if (s != SSA_OK) return s;
-  kernel<<<items, ssa::kDecodeThreads, smem, st>>>(dp);
+  constexpr int kMaxSmem = 227 * 1024;
+  auto kernel = ssa::decode_kernel<D, G>;
+  const DecodeLaunch s = decode_launch_shape<D, G>(d);
+  if (s.smem > kMaxSmem) return SSA_ERR_UNSUPPORTED;
+  const ssa_status e0 = ensure_smem(kernel, kMaxSmem, &smem_done);
+  if (e0 != SSA_OK) return e0;
+  dp.ns = s.ns;
+  dp.slice_cap = s.slice_cap;
+  dp.cand_cap = s.cand_cap;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(d.B) * d.Hkv * s.ns);
+  cfg.blockDim = dim3(ssa::kDecodeThreads);
+  cfg.dynamicSmemBytes = s.smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = s.ns;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, dp);
+  g_launches.fetch_add(1);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return SSA_ERR_CUDA;
+  }
   return launch_result();
 }
 
 template <int D>
 ssa_status launch_decode(const Dims& d, const void* q, const void* k, const void* v, const float* kbar,
-                         const int32_t* len, void* o, float* lse, int32_t* idx_out, void* workspace,
-                         cudaStream_t st) {
-  const DecodeLayout L = decode_layout(d);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
+                         const int32_t* len, void* o, float* lse, int32_t* idx_out, cudaStream_t st) {
   ssa::DecodeParams dp;
   dp.B = d.B;
   dp.S = d.S;
@@ -571,42 +597,24 @@ ssa_status launch_decode(const Dims& d, const void* q, const void* k, const void
   dp.G = d.G;
   dp.n = d.n;
   dp.topk = d.topk;
+  dp.ns = 1;
+  dp.slice_cap = 0;
+  dp.cand_cap = 0;
   dp.scale_log2 = d.scale * 1.4426950408889634f;
   dp.q = static_cast<const __nv_bfloat16*>(q);
   dp.k = static_cast<const __nv_bfloat16*>(k);
   dp.v = static_cast<const __nv_bfloat16*>(v);
   dp.kbar = kbar;
   dp.len = len;
-  dp.idx = idx_out != nullptr ? idx_out : reinterpret_cast<int32_t*>(ws + L.idx);
-  dp.part = reinterpret_cast<float*>(ws + L.part);
+  dp.idx = idx_out;
   dp.o = static_cast<__nv_bfloat16*>(o);
   dp.lse = lse;
-  const unsigned bh = static_cast<unsigned>(d.B) * d.Hkv;
-  dp.keys = nullptr;
-  if (d.n >= kDecodeSplitBlocks) {
-    dp.keys = reinterpret_cast<uint32_t*>(ws + L.keys);
-    const dim3 grid((d.n - 1 + ssa::kDecodeSelThreads - 1) / ssa::kDecodeSelThreads, bh);
-    ssa::decode_score_kernel<D><<<grid, ssa::kDecodeSelThreads, 0, st>>>(dp);
-    const ssa_status s0 = launch_result();
-    if (s0 != SSA_OK) return s0;
-  }
-  ssa::decode_select_kernel<D><<<bh, ssa::kDecodeSelThreads, 4 * d.n, st>>>(dp);
-  ssa_status s = launch_result();
-  if (s != SSA_OK) return s;
-  const unsigned items = bh * static_cast<unsigned>(d.topk);
   switch (d.G) {
-    case 2: s = launch_decode_attn<D, 2>(items, dp, st); break;
-    case 4: s = launch_decode_attn<D, 4>(items, dp, st); break;
-    case 8: s = launch_decode_attn<D, 8>(items, dp, st); break;
-    default: s = launch_decode_attn<D, 16>(items, dp, st); break;
+    case 2: return launch_decode_g<D, 2>(d, dp, st);
+    case 4: return launch_decode_g<D, 4>(d, dp, st);
+    case 8: return launch_decode_g<D, 8>(d, dp, st);
+    default: return launch_decode_g<D, 16>(d, dp, st);
   }
-  if (s != SSA_OK) return s;
-  const unsigned rows = static_cast<unsigned>(d.B) * d.Hq;
-  if (d.topk >= 64)
-    ssa::decode_combine_kernel<D, 256><<<rows, 256, 0, st>>>(dp);
-  else
-    ssa::decode_combine_kernel<D, 64><<<rows, 64, 0, st>>>(dp);
-  return launch_result();
 }
 
 // ------------------------------------------------------------ host buffers
@@ -946,8 +954,8 @@ ssa_status ssa_sparse_attn_fwd_early_stop(const ssa_problem* p, const ssa_bf16* 
 
 size_t ssa_decode_attn_workspace(const ssa_problem* p) {
   Dims d;
-  if (check_problem(p, &d) != SSA_OK) return 0;
-  return decode_layout(d).total;
+  (void)check_problem(p, &d);
+  return 0;  // the selection and the partial softmax states stay on chip
 }
 
 ssa_status ssa_decode_attn(const ssa_problem* p, const ssa_bf16* q, const ssa_bf16* k_cache,
@@ -961,11 +969,11 @@ ssa_status ssa_decode_attn(const ssa_problem* p, const ssa_bf16* q, const ssa_bf
   for (const void* ptr : ptrs)
     if (ptr == nullptr || !aligned16(ptr)) return SSA_ERR_INVALID_ARG;
   if (block_idx != nullptr && !aligned16(block_idx)) return SSA_ERR_INVALID_ARG;
-  if (workspace == nullptr || !aligned16(workspace) || ws_bytes < decode_layout(d).total)
-    return SSA_ERR_WORKSPACE;
+  (void)workspace;  // none is needed (ssa_decode_attn_workspace returns 0)
+  (void)ws_bytes;
   auto st = reinterpret_cast<cudaStream_t>(stream);
-  return d.D == 64 ? launch_decode<64>(d, q, k_cache, v_cache, k_pooled, lengths, o, lse, block_idx, workspace, st)
-                   : launch_decode<128>(d, q, k_cache, v_cache, k_pooled, lengths, o, lse, block_idx, workspace, st);
+  return d.D == 64 ? launch_decode<64>(d, q, k_cache, v_cache, k_pooled, lengths, o, lse, block_idx, st)
+                   : launch_decode<128>(d, q, k_cache, v_cache, k_pooled, lengths, o, lse, block_idx, st);
 }
 
 // ------------------------------------------------------------ DashAttention

@@ -309,8 +309,9 @@ ssa_status ssa_sparse_attn_bwd_noalloc(const ssa_problem *p, const ssa_bf16 *q, 
                                        ssa_bf16 *dq, ssa_bf16 *dk, ssa_bf16 *dv,
                                        ssa_stream stream);
 
-/* Bytes of device workspace ssa_decode_attn needs for problem p (0 on an
- * invalid problem). */
+/* Bytes of device workspace ssa_decode_attn needs for problem p: 0, since
+ * the table and the partial softmax states stay in shared memory.  Kept so
+ * callers size every call's scratch the same way. */
 size_t ssa_decode_attn_workspace(const ssa_problem *p);
 
 /* One decoding step of the sparse stream against a KV cache ([SSA-it]
@@ -329,9 +330,12 @@ size_t ssa_decode_attn_workspace(const ssa_problem *p);
  *    block c (keys up to t), for each query head of the group.
  * k_cache, v_cache: [B][S][Hkv][D] bf16.  Outputs: o [B][Hq][D] bf16,
  * lse [B][Hq] fp32 (natural log), and, if block_idx is not NULL, the kept
- * blocks [B][Hkv][k] int32, ascending, -1 padded.  `workspace`: at least
- * ssa_decode_attn_workspace(p) bytes, 256-byte aligned.
- * Errors: INVALID_ARG / UNSUPPORTED / WORKSPACE as for the other calls.  A
+ * blocks [B][Hkv][k] int32, ascending, -1 padded.  `workspace` and
+ * `ws_bytes` are not read (ssa_decode_attn_workspace returns 0; NULL is fine).
+ * One launch: a cluster of up to 8 CTAs per (b, KV head) scores, selects,
+ * attends and merges; UNSUPPORTED if its shared memory (about 4 B per cached
+ * block plus the K/V ring) exceeds 227 KB.
+ * Errors: INVALID_ARG / UNSUPPORTED as for the other calls.  A
  * length outside 1..S is found on the device; that sequence's outputs become
  * 0 (lse -inf), and ssa_get_device_error then returns SSA_ERR_INVALID_ARG.
  * The pages have no decode kernel of their own; this call is the sparse

@@ -130,11 +130,11 @@ def test_alignment_backward_arguments_are_checked_before_launch(lib):
 def test_decode_arguments_are_checked_before_launch(lib):
     p = ctypes.byref(_p())
     f = FAKE
-    ws = lib.ssa_decode_attn_workspace(p)
-    assert ws > 0
-    assert lib.ssa_decode_attn(p, f, f, f, f, f, f, f, None, f, ws - 1, None) == WORKSPACE
-    assert lib.ssa_decode_attn(p, f, f, f, f, None, f, f, None, f, ws, None) == INVALID
-    assert lib.ssa_decode_attn(p, f, f, f, f, f, f, f, f + 4, f, ws, None) == INVALID
+    # the selection and the partial softmax states stay on chip: no workspace
+    assert lib.ssa_decode_attn_workspace(p) == 0
+    assert lib.ssa_decode_attn(p, f, f, f, f, None, f, f, None, None, 0, None) == INVALID
+    assert lib.ssa_decode_attn(p, f, f, f, f, f, f, f, f + 4, None, 0, None) == INVALID
+    assert lib.ssa_decode_attn(p, f, f, f, f, f, f, f + 4, None, None, 0, None) == INVALID
 
 
 def test_early_stop_arguments_are_checked_before_launch(lib):

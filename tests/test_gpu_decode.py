@@ -50,6 +50,8 @@ CASES = [
     (2, 4096, 8, 2, 64, 16, [1024, 1025]),          # 16 blocks: all kept; 17: the search
     (2, 8192, 8, 2, 64, 64, [4096, 8192]),          # 64 blocks: all kept; 128: the search
     (1, 16384, 8, 2, 64, 96, [16384]),              # a budget of 96 blocks: 96 partials per row
+    (64, 2048, 8, 4, 64, 8, None),                  # 256 (b, KV head) rows: one CTA each
+    (48, 4096, 16, 4, 128, 16, None),               # head_dim 128, one CTA per row
 ]
 
 
@@ -76,6 +78,16 @@ def test_decode_step_matches_oracle(case):
                 sl = slice(h * G, (h + 1) * G)
                 assert np.abs(go[b, sl] - oo[b, sl]).max() <= 2e-2
                 assert np.abs(gl[b, sl] - olse[b, sl]).max() <= 1e-3
+
+
+def test_decode_is_deterministic():
+    # the merge order of the warps' and CTAs' partials is fixed
+    for B, S, Hkv, topk in ((64, 2048, 4, 8), (2, 131072, 1, 16)):
+        x = gen.make_decode(B, S, 8, Hkv, 64, topk, seed=901 + B)
+        first = _run(x, topk)
+        again = _run(x, topk)
+        for a, b in zip(first[1:], again[1:]):
+            assert torch.equal(a, b)
 
 
 def test_decode_length_outside_the_cache_is_reported():
