@@ -194,6 +194,28 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS, EARLY, DASH>::THREADS,
     mbar_init(bar_qfree, C::ISS);  // one commit per issuer and unit
     *abort_flag = 0;
     fence_mbar_init();
+    if (PERSIST) {
+      // thread 0 is the producer: the first unit's Q and diagonal block do
+      // not depend on the index table, so they load before the wait below,
+      // while the selection kernel may still run (only the pooling and
+      // selection kernels let their dependents start early, and neither
+      // writes Q, K or V)
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_arrive_expect_tx(&bar_kfull[0], KVT);
+      for (int pn = 0; pn < NP; ++pn)
+        tma_load_4d(sK + pn * (64 * 128), &tm_k, &bar_kfull[0], 64 * pn, h, 64 * i, b);
+      mbar_arrive_expect_tx(&bar_vfull[0], KVT);
+      for (int pn = 0; pn < NP; ++pn)
+        tma_load_4d(sV + pn * (64 * 128), &tm_v, &bar_vfull[0], 64 * pn, h, 64 * i, b);
+      mbar_arrive_expect_tx(bar_q, T * QTILE);
+      for (int t = 0; t < T; ++t)
+        for (int hh = 0; hh < 2; ++hh)
+          for (int pn = 0; pn < NP; ++pn)
+            tma_load_4d(sQ + t * QTILE + pn * (128 * 128) + hh * (64 * 128), &tm_q, bar_q, 64 * pn,
+                        hq0 + 2 * t + hh, 64 * i, b);
+    }
   }
   // launched with programmatic serialization: the index table may still be
   // in flight from the selection kernel until here
@@ -241,17 +263,23 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS, EARLY, DASH>::THREADS,
         // per unit: its first K/V block, then its Q once the previous unit's
         // last score MMAs have read the old Q, then the rest of its blocks
         int g = 0, k = 0;  // K/V blocks and units loaded so far
-        int qk = -1;       // the last unit whose Q was loaded
+        int qk = 0;        // the last unit whose Q was loaded (unit 0: before the table wait)
         bool alive = true;
         for (int u = static_cast<int>(blockIdx.x); alive && u < n_units; u += gridDim.x, ++k) {
           const Unit w = unit_of(u);
+          // the diagonal block first (the table's last entry), then the others
+          // in table order
           for (int s = 0; s < w.nsel; ++s) {
             const int st = g % NS, use = g / NS;
+            if (k == 0 && s == 0) {  // issued with Q before the table wait
+              ++g;
+              continue;
+            }
             if (use > 0 && !mbar_wait(&bar_empty[st], (use - 1) & 1, abort_flag, tmo, 0x101)) {
               alive = false;
               break;
             }
-            const int j = w.idx_row[s];
+            const int j = s == 0 ? w.i : w.idx_row[s - 1];
             mbar_arrive_expect_tx(&bar_kfull[st], KVT);
             for (int pn = 0; pn < NP; ++pn)
               tma_load_4d(sK + st * KVT + pn * (64 * 128), &tm_k, &bar_kfull[st], 64 * pn, w.h, 64 * j, w.b);
@@ -478,9 +506,9 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS, EARLY, DASH>::THREADS,
         tc_fence_after();
         // warp-uniform: both warps of a head stop together
         const bool live = !EARLY || !hstop;
-        // the diagonal block comes last in the ascending table, first in the
-        // early-stop order
-        const bool diag = EARLY ? (jj == 0) : (jj == nb - 1);
+        // the diagonal block comes first in the plain (persistent) and the
+        // early-stop orders, last in the other modes' ascending orders
+        const bool diag = (EARLY || PERSIST) ? (jj == 0) : (jj == nb - 1);
         bool is_sel = true;
         if (MASS) is_sel = (selbits[jj >> 5] >> (jj & 31)) & 1u;
         // all 64 scores with one TMEM round trip, then the raw row maximum
