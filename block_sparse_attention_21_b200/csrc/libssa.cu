@@ -577,13 +577,11 @@ ssa_status launch_decode_g(const Dims& d, ssa::DecodeParams dp, cudaStream_t st)
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, dp);
-  g_launches.fetch_add(1);
-  if (e != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, kernel, dp) != cudaSuccess) {
     cudaGetLastError();
     return SSA_ERR_CUDA;
   }
-  return launch_result();
+  return launch_result();  // counts the launch
 }
 
 template <int D>
