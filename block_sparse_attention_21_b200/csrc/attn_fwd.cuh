@@ -154,14 +154,14 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS, EARLY, DASH>::THREADS,
   // other modes one unit per CTA
   constexpr bool PERSIST = !MASS && !EARLY && !DASH;
   const int per_i = p.B * p.Hkv * p.slices;
-  const int n_units = PERSIST ? p.n * per_i : static_cast<int>(blockIdx.x) + 1;
+  const int n_units = PERSIST ? (p.i_hi - p.i_lo) * per_i : static_cast<int>(blockIdx.x) + 1;
   struct Unit {
     int i, b, h, slice, hq0, nsel;
     const int32_t* idx_row;
   };
   auto unit_of = [&](int u) {
     Unit w;
-    w.i = p.n - 1 - u / per_i;
+    w.i = p.i_hi - 1 - u / per_i;
     int rem = u % per_i;
     w.slice = rem % p.slices;
     rem /= p.slices;
@@ -488,7 +488,7 @@ __global__ void __launch_bounds__(FwdConfig<D, T, MASS, EARLY, DASH>::THREADS,
     // parities count the CTA's blocks (g + jj) and units (k)
     int g = 0, k = 0;
     for (int u = static_cast<int>(blockIdx.x); ok && u < n_units; u += gridDim.x, ++k) {
-      const int nb = PERSIST ? min(p.topk, p.n - u / per_i) : nblk;
+      const int nb = PERSIST ? min(p.topk, p.i_hi - u / per_i) : nblk;
       float m_ref = -INFINITY;  // reference maximum, scaled (log2) units
       float l_sel = 0.f, l_uns = 0.f;
       // EARLY: each head of the tile (64-row half: warps wq 0-1 and 2-3)

@@ -162,14 +162,14 @@ __global__ void __launch_bounds__(PsFwdConfig<D, T, MASS, DASH, EARLY>::THREADS,
   // other modes one unit per CTA
   constexpr bool PERSIST = !MASS && !DASH && !EARLY;
   const int per_i = p.B * p.Hkv * p.slices;
-  const int n_units = PERSIST ? p.n * per_i : static_cast<int>(blockIdx.x) + 1;
+  const int n_units = PERSIST ? (p.i_hi - p.i_lo) * per_i : static_cast<int>(blockIdx.x) + 1;
   struct Unit {
     int i, b, h, slice, hq0, nsel;
     const int32_t* idx_row;
   };
   auto unit_of = [&](int u) {
     Unit w;
-    w.i = p.n - 1 - u / per_i;
+    w.i = p.i_hi - 1 - u / per_i;
     int rem = u % per_i;
     w.slice = rem % p.slices;
     rem /= p.slices;

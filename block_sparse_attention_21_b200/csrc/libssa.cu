@@ -7,6 +7,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <vector>
 #include <atomic>
 #include <cmath>
 #include <cstdlib>
@@ -164,9 +165,10 @@ ssa_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sm
   return cudaGetLastError() == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;
 }
 
+// blocks j0 .. j0 + nj - 1 (nj < 0: every block)
 template <int D>
 ssa_status launch_pool(const Dims& d, const void* k, const void* q, float* kb, float* qb,
-                       cudaStream_t st) {
+                       cudaStream_t st, int j0 = 0, int nj = -1) {
   ssa::PoolParams pp;
   pp.k = static_cast<const __nv_bfloat16*>(k);
   pp.q = static_cast<const __nv_bfloat16*>(q);
@@ -177,7 +179,9 @@ ssa_status launch_pool(const Dims& d, const void* k, const void* q, float* kb, f
   pp.Hkv = d.Hkv;
   pp.G = d.G;
   pp.n = d.n;
-  return launch_pdl(ssa::block_pool_kernel<D>, dim3(d.n, d.Hkv, d.B), dim3(ssa::PoolConfig<D>::THREADS), 0,
+  pp.j0 = j0;
+  if (nj < 0) nj = d.n;
+  return launch_pdl(ssa::block_pool_kernel<D>, dim3(nj, d.Hkv, d.B), dim3(ssa::PoolConfig<D>::THREADS), 0,
                     st, pp);
 }
 
@@ -187,7 +191,7 @@ ssa_status launch_select(const Dims& d, const ssa::SelectParams& sp, cudaStream_
   auto kernel = ssa::block_select_kernel<D, KPL>;
   const ssa_status s = ensure_smem(kernel, 200 * 1024, &done);
   if (s != SSA_OK) return s;
-  const dim3 grid((d.n + ssa::kSelectWarps - 1) / ssa::kSelectWarps, d.B * d.Hkv);
+  const dim3 grid((sp.i1 - sp.i0 + ssa::kSelectWarps - 1) / ssa::kSelectWarps, d.B * d.Hkv);
   return launch_pdl(kernel, grid, dim3(32 * ssa::kSelectWarps), ssa::SelectConfig<D>::smem_bytes(d.n), st,
                     sp);
 }
@@ -206,7 +210,7 @@ ssa_status launch_fwd(const Dims& d, const void* q, const void* k, const void* v
                       const int32_t* idx, void* o, float* lse, void* of, float* lsef,
                       float* dropped, cudaStream_t st, const float* qbar = nullptr,
                       const float* kbar = nullptr, float tau = 0.f, int32_t* visited = nullptr,
-                      DashIn dash = DashIn()) {
+                      DashIn dash = DashIn(), int i_lo = 0, int i_hi = -1) {
   using C = ssa::FwdConfig<D, T, MASS, EARLY, DASH>;
   static std::atomic<uint64_t> smem_done{0};
   auto kernel = ssa::attn_fwd_kernel<D, T, MASS, EARLY, DASH>;
@@ -225,6 +229,9 @@ ssa_status launch_fwd(const Dims& d, const void* q, const void* k, const void* v
   fp.n = d.n;
   fp.topk = d.topk;
   fp.slices = (d.G / 2) / T;
+  // query blocks i_lo .. i_hi - 1 (the plain mode only; the others take all)
+  fp.i_lo = (MASS || EARLY || DASH) ? 0 : i_lo;
+  fp.i_hi = (MASS || EARLY || DASH || i_hi < 0) ? d.n : i_hi;
   fp.scale_log2 = d.scale * 1.4426950408889634f;
   fp.idx = idx;
   fp.o = static_cast<__nv_bfloat16*>(o);
@@ -242,7 +249,7 @@ ssa_status launch_fwd(const Dims& d, const void* q, const void* k, const void* v
   fp.sigma = dash.sigma;
   // the plain sparse stream runs persistent CTAs, as many as are resident at
   // once, over the units; the other modes one CTA per unit
-  const unsigned units = static_cast<unsigned>(d.B) * d.Hkv * d.n * fp.slices;
+  const unsigned units = static_cast<unsigned>(d.B) * d.Hkv * (fp.i_hi - fp.i_lo) * fp.slices;
   const unsigned slots = static_cast<unsigned>(sm_count()) * C::MIN_CTAS;
   const bool persist = !MASS && !EARLY && !DASH;
   if (persist && slots == 0) return SSA_ERR_CUDA;
@@ -255,7 +262,8 @@ template <int D, int T, bool MASS, bool DASH = false, bool EARLY = false>
 ssa_status launch_psfwd(const Dims& d, const void* q, const void* k, const void* v,
                       const int32_t* idx, void* o, float* lse, void* of, float* lsef,
                       float* dropped, cudaStream_t st, DashIn dash = DashIn(), const float* qbar = nullptr,
-                      const float* kbar = nullptr, float tau = 0.f, int32_t* visited = nullptr) {
+                      const float* kbar = nullptr, float tau = 0.f, int32_t* visited = nullptr,
+                      int i_lo = 0, int i_hi = -1) {
   using C = ssa::PsFwdConfig<D, T, MASS, DASH, EARLY>;
   static std::atomic<uint64_t> smem_done{0};
   auto kernel = ssa::attn_fwd_psmem_kernel<D, T, MASS, DASH, EARLY>;
@@ -274,6 +282,9 @@ ssa_status launch_psfwd(const Dims& d, const void* q, const void* k, const void*
   fp.n = d.n;
   fp.topk = d.topk;
   fp.slices = (d.G / 2) / T;
+  // query blocks i_lo .. i_hi - 1 (the plain mode only; the others take all)
+  fp.i_lo = (MASS || EARLY || DASH) ? 0 : i_lo;
+  fp.i_hi = (MASS || EARLY || DASH || i_hi < 0) ? d.n : i_hi;
   fp.scale_log2 = d.scale * 1.4426950408889634f;
   fp.idx = idx;
   fp.o = static_cast<__nv_bfloat16*>(o);
@@ -291,7 +302,7 @@ ssa_status launch_psfwd(const Dims& d, const void* q, const void* k, const void*
   fp.sigma = dash.sigma;
   // the plain sparse stream runs persistent CTAs, one per SM, over the units;
   // the other modes one CTA per unit
-  const unsigned units = static_cast<unsigned>(d.B) * d.Hkv * d.n * fp.slices;
+  const unsigned units = static_cast<unsigned>(d.B) * d.Hkv * (fp.i_hi - fp.i_lo) * fp.slices;
   const unsigned sms = static_cast<unsigned>(sm_count());
   const bool persist = !MASS && !DASH && !EARLY;
   if (persist && sms == 0) return SSA_ERR_CUDA;
@@ -616,34 +627,73 @@ ssa_status launch_decode(const Dims& d, const void* q, const void* k, const void
 }
 
 // ------------------------------------------------------------ host buffers
-// ssa_sparse_attn_fwd_host: per (batch, KV head) unit, the unit's Q, K, V in
-// one of two device buffer sets, its pooled keys and queries, table, O, LSE.
-// K and V are copied whole first (contiguous, at full PCIe speed; their
-// per-unit rows of D values would be short strided copies) and each unit's
-// slice is taken from there on the device.
+// ssa_sparse_attn_fwd_host: device copies of Q, K, V, O and LSE whole, the
+// pooled keys and queries and the index table.  K and V are copied first and
+// pooled; then chunks of consecutive query blocks (all batch entries and
+// heads) stream through: a chunk's Q rows in (contiguous per batch entry),
+// its queries pooled, its rows selected and attended, its O rows and LSE
+// columns out, with the copies in, the kernels and the copies out of
+// neighbouring chunks overlapping.
 struct HostLayout {
-  size_t kall, vall, sets, q, k, v, kb, qb, idx, o, lse, set, total;
+  size_t kall, vall, qall, oall, lse, kb, qb, idx, total;
 };
 
 HostLayout host_layout(const Dims& d) {
   auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
-  const size_t S = d.S, G = d.G, D = d.D, n = d.n, k = d.topk;
-  const size_t kv_all = static_cast<size_t>(d.B) * S * d.Hkv * D * 2;
+  const size_t B = d.B, S = d.S, D = d.D, n = d.n, k = d.topk;
+  const size_t kv = B * S * d.Hkv * D * 2, qo = B * S * d.Hq * D * 2;
   HostLayout L;
   L.kall = 0;
-  L.vall = al(kv_all);
-  L.sets = L.vall + al(kv_all);
-  L.q = 0;
-  L.k = al(S * G * D * 2);
-  L.v = L.k + al(S * D * 2);
-  L.kb = L.v + al(S * D * 2);
-  L.qb = L.kb + al(n * D * 4);
-  L.idx = L.qb + al(n * D * 4);
-  L.o = L.idx + al(n * k * 4);
-  L.lse = L.o + al(S * G * D * 2);
-  L.set = L.lse + al(G * S * 4);
-  L.total = L.sets + 2 * L.set;
+  L.vall = L.kall + al(kv);
+  L.qall = L.vall + al(kv);
+  L.oall = L.qall + al(qo);
+  L.lse = L.oall + al(qo);
+  L.kb = L.lse + al(B * d.Hq * S * 4);
+  L.qb = L.kb + al(B * d.Hkv * n * D * 4);
+  L.idx = L.qb + al(B * d.Hkv * n * D * 4);
+  L.total = L.idx + al(B * d.Hkv * n * k * 4);
   return L;
+}
+
+// Query blocks per chunk of the host-buffer path: at least 8 MB of Q per
+// chunk (about 150 us of PCIe, which hides a chunk's launches and keeps many
+// work units per forward launch), and at most sixteen chunks.
+int host_chunk_blocks(const Dims& d) {
+  const size_t row_bytes = static_cast<size_t>(d.B) * 64 * d.Hq * d.D * 2;  // one query block, all heads
+  const int by_bytes = static_cast<int>(((8u << 20) + row_bytes - 1) / row_bytes);
+  return std::min(d.n, std::max(by_bytes, (d.n + 15) / 16));
+}
+
+// The plain sparse forward over query blocks i0 .. i1 - 1.
+ssa_status sparse_fwd_range(const Dims& d, const void* q, const void* k, const void* v, const int32_t* idx,
+                            void* o, float* lse, cudaStream_t st, int i0, int i1) {
+  if (d.D == 64)
+    return d.G >= 4 ? launch_fwd<64, 2, false>(d, q, k, v, idx, o, lse, nullptr, nullptr, nullptr, st, nullptr,
+                                               nullptr, 0.f, nullptr, DashIn(), i0, i1)
+                    : launch_fwd<64, 1, false>(d, q, k, v, idx, o, lse, nullptr, nullptr, nullptr, st, nullptr,
+                                               nullptr, 0.f, nullptr, DashIn(), i0, i1);
+  return d.G >= 4 ? launch_psfwd<128, 2, false>(d, q, k, v, idx, o, lse, nullptr, nullptr, nullptr, st, DashIn(),
+                                                nullptr, nullptr, 0.f, nullptr, i0, i1)
+                  : launch_psfwd<128, 1, false>(d, q, k, v, idx, o, lse, nullptr, nullptr, nullptr, st, DashIn(),
+                                                nullptr, nullptr, 0.f, nullptr, i0, i1);
+}
+
+// The selection of query blocks i0 .. i1 - 1.
+ssa_status select_range(const Dims& d, const float* qb, const float* kb, int32_t* idx, cudaStream_t st, int i0,
+                        int i1) {
+  ssa::SelectParams sp;
+  sp.qbar = qb;
+  sp.kbar = kb;
+  sp.idx = idx;
+  sp.n = d.n;
+  sp.topk = d.topk;
+  sp.i0 = i0;
+  sp.i1 = i1;
+  if (d.D == 64)
+    return d.n <= 128 ? launch_select<64, 4>(d, sp, st)
+                      : (d.n <= 512 ? launch_select<64, 16>(d, sp, st) : launch_select<64, 0>(d, sp, st));
+  return d.n <= 128 ? launch_select<128, 4>(d, sp, st)
+                    : (d.n <= 512 ? launch_select<128, 16>(d, sp, st) : launch_select<128, 0>(d, sp, st));
 }
 
 // The copy-in and copy-out streams of the host-buffer path, one pair per
@@ -710,6 +760,8 @@ ssa_status ssa_block_select(const ssa_problem* p, const float* q_pooled, const f
   sp.idx = block_idx;
   sp.n = d.n;
   sp.topk = d.topk;
+  sp.i0 = 0;
+  sp.i1 = d.n;
   auto st = reinterpret_cast<cudaStream_t>(stream);
   // keys in registers while a lane's share (n / 32) is small
   if (d.D == 64)
@@ -761,63 +813,63 @@ ssa_status ssa_sparse_attn_fwd_host(const ssa_problem* p, const ssa_bf16* q, con
   cudaStream_t sin = nullptr, sout = nullptr;
   s = pipe_streams(&sin, &sout);
   if (s != SSA_OK) return s;
-  // one unit = one batch entry and one KV head: its G query heads, its K and V
-  ssa_problem unit = *p;
-  unit.batch = 1;
-  unit.n_q_heads = d.G;
-  unit.n_kv_heads = 1;
-  cudaEvent_t ev[8];
-  for (auto& e : ev)
-    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return SSA_ERR_CUDA;
-  cudaEvent_t ev_start = ev[0], ev_end = ev[1], in_done[2] = {ev[2], ev[3]}, comp_done[2] = {ev[4], ev[5]},
-              out_done[2] = {ev[6], ev[7]};
-  const size_t S = d.S, D = d.D, G = d.G, Hq = d.Hq, Hkv = d.Hkv;
-  const size_t qrow = G * D * 2, krow = D * 2;  // bytes of a unit's token row
-  bool ok = cudaEventRecord(ev_start, sc) == cudaSuccess && cudaStreamWaitEvent(sin, ev_start, 0) == cudaSuccess &&
-            cudaStreamWaitEvent(sout, ev_start, 0) == cudaSuccess;
-  // K and V whole, ahead of the first unit's Q
+  const int cb = host_chunk_blocks(d), chunks = (d.n + cb - 1) / cb;
+  std::vector<cudaEvent_t> ev(3 + 2 * static_cast<size_t>(chunks), nullptr);
+  bool ok = true;
+  for (auto& e : ev) ok = ok && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) == cudaSuccess;
+  if (!ok) {
+    for (auto& e : ev)
+      if (e != nullptr) cudaEventDestroy(e);
+    return SSA_ERR_CUDA;
+  }
+  cudaEvent_t ev_start = ev[0], ev_kv = ev[1], ev_end = ev[2];
+  cudaEvent_t* in_done = ev.data() + 3;
+  cudaEvent_t* comp_done = in_done + chunks;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
+  auto* dk = reinterpret_cast<ssa_bf16*>(ws + L.kall);
+  auto* dv = reinterpret_cast<ssa_bf16*>(ws + L.vall);
+  auto* dq = reinterpret_cast<ssa_bf16*>(ws + L.qall);
+  auto* dout = reinterpret_cast<ssa_bf16*>(ws + L.oall);
+  auto* dlse = reinterpret_cast<float*>(ws + L.lse);
+  auto* dkb = reinterpret_cast<float*>(ws + L.kb);
+  auto* dqb = reinterpret_cast<float*>(ws + L.qb);
+  auto* didx = reinterpret_cast<int32_t*>(ws + L.idx);
+  const size_t S = d.S, D = d.D, Hq = d.Hq, Hkv = d.Hkv;
+  const size_t qtok = Hq * D * 2;  // bytes of one token's Q (or O) row, all heads
+  ok = cudaEventRecord(ev_start, sc) == cudaSuccess && cudaStreamWaitEvent(sin, ev_start, 0) == cudaSuccess &&
+       cudaStreamWaitEvent(sout, ev_start, 0) == cudaSuccess;
+  // K and V whole, then the pooled keys of every block
   const size_t kv_all = static_cast<size_t>(d.B) * S * Hkv * D * 2;
-  ok = ok && cudaMemcpyAsync(ws + L.kall, k, kv_all, cudaMemcpyHostToDevice, sin) == cudaSuccess &&
-       cudaMemcpyAsync(ws + L.vall, v, kv_all, cudaMemcpyHostToDevice, sin) == cudaSuccess;
-  const int units = d.B * d.Hkv;
-  for (int u = 0; ok && u < units; ++u) {
-    const int set = u & 1;
-    const size_t b = u / d.Hkv, h = u % d.Hkv;
-    uint8_t* base = ws + L.sets + set * L.set;
-    auto* uq = reinterpret_cast<ssa_bf16*>(base + L.q);
-    auto* uk = reinterpret_cast<ssa_bf16*>(base + L.k);
-    auto* uv = reinterpret_cast<ssa_bf16*>(base + L.v);
-    auto* ukb = reinterpret_cast<float*>(base + L.kb);
-    auto* uqb = reinterpret_cast<float*>(base + L.qb);
-    auto* uidx = reinterpret_cast<int32_t*>(base + L.idx);
-    auto* uo = reinterpret_cast<ssa_bf16*>(base + L.o);
-    auto* ulse = reinterpret_cast<float*>(base + L.lse);
-    // copy in, once unit u - 2's compute no longer reads this buffer set
-    const auto* hq_src = reinterpret_cast<const uint8_t*>(q) + ((b * S) * Hq + h * G) * D * 2;
-    const uint8_t* dk_src = ws + L.kall + ((b * S) * Hkv + h) * D * 2;
-    const uint8_t* dv_src = ws + L.vall + ((b * S) * Hkv + h) * D * 2;
-    ok = (u < 2 || cudaStreamWaitEvent(sin, comp_done[set], 0) == cudaSuccess) &&
-         cudaMemcpy2DAsync(uq, qrow, hq_src, Hq * D * 2, qrow, S, cudaMemcpyHostToDevice, sin) == cudaSuccess &&
-         cudaEventRecord(in_done[set], sin) == cudaSuccess;
-    // compute on the caller's stream, once the inputs landed (K and V whole
-    // came first on the same stream) and unit u - 2's outputs left this
-    // buffer set; the unit's K and V rows are gathered on the device
-    ok = ok && cudaStreamWaitEvent(sc, in_done[set], 0) == cudaSuccess &&
-         (u < 2 || cudaStreamWaitEvent(sc, out_done[set], 0) == cudaSuccess) &&
-         cudaMemcpy2DAsync(uk, krow, dk_src, Hkv * D * 2, krow, S, cudaMemcpyDeviceToDevice, sc) == cudaSuccess &&
-         cudaMemcpy2DAsync(uv, krow, dv_src, Hkv * D * 2, krow, S, cudaMemcpyDeviceToDevice, sc) == cudaSuccess;
-    if (ok) s = ssa_block_pool(&unit, uk, uq, ukb, uqb, stream);
-    if (ok && s == SSA_OK) s = ssa_block_select(&unit, uqb, ukb, uidx, stream);
-    if (ok && s == SSA_OK) s = ssa_sparse_attn_fwd(&unit, uq, uk, uv, uidx, uo, ulse, stream);
-    ok = ok && s == SSA_OK && cudaEventRecord(comp_done[set], sc) == cudaSuccess;
-    // copy out
-    auto* ho_dst = reinterpret_cast<uint8_t*>(o) + ((b * S) * Hq + h * G) * D * 2;
-    float* hl_dst = lse + (b * Hq + h * G) * S;
-    ok = ok && cudaStreamWaitEvent(sout, comp_done[set], 0) == cudaSuccess &&
-         cudaMemcpy2DAsync(ho_dst, Hq * D * 2, uo, qrow, qrow, S, cudaMemcpyDeviceToHost, sout) == cudaSuccess &&
-         cudaMemcpyAsync(hl_dst, ulse, G * S * 4, cudaMemcpyDeviceToHost, sout) == cudaSuccess &&
-         cudaEventRecord(out_done[set], sout) == cudaSuccess;
+  ok = ok && cudaMemcpyAsync(dk, k, kv_all, cudaMemcpyHostToDevice, sin) == cudaSuccess &&
+       cudaMemcpyAsync(dv, v, kv_all, cudaMemcpyHostToDevice, sin) == cudaSuccess &&
+       cudaEventRecord(ev_kv, sin) == cudaSuccess && cudaStreamWaitEvent(sc, ev_kv, 0) == cudaSuccess;
+  if (ok) s = d.D == 64 ? launch_pool<64>(d, dk, nullptr, dkb, nullptr, sc) : launch_pool<128>(d, dk, nullptr, dkb, nullptr, sc);
+  for (int c = 0; ok && s == SSA_OK && c < chunks; ++c) {
+    const int i0 = c * cb, i1 = std::min(d.n, i0 + cb);
+    const size_t t0 = 64 * static_cast<size_t>(i0), nt = 64 * static_cast<size_t>(i1 - i0);
+    // copy in: the chunk's Q rows of every batch entry
+    for (size_t b = 0; ok && b < static_cast<size_t>(d.B); ++b)
+      ok = cudaMemcpyAsync(reinterpret_cast<uint8_t*>(dq) + (b * S + t0) * qtok,
+                           reinterpret_cast<const uint8_t*>(q) + (b * S + t0) * qtok, nt * qtok,
+                           cudaMemcpyHostToDevice, sin) == cudaSuccess;
+    ok = ok && cudaEventRecord(in_done[c], sin) == cudaSuccess;
+    // compute on the caller's stream: the chunk's pooled queries, selection
+    // and attention
+    ok = ok && cudaStreamWaitEvent(sc, in_done[c], 0) == cudaSuccess;
+    if (ok) s = d.D == 64 ? launch_pool<64>(d, nullptr, dq, nullptr, dqb, sc, i0, i1 - i0)
+                          : launch_pool<128>(d, nullptr, dq, nullptr, dqb, sc, i0, i1 - i0);
+    if (ok && s == SSA_OK) s = select_range(d, dqb, dkb, didx, sc, i0, i1);
+    if (ok && s == SSA_OK) s = sparse_fwd_range(d, dq, dk, dv, didx, dout, dlse, sc, i0, i1);
+    ok = ok && s == SSA_OK && cudaEventRecord(comp_done[c], sc) == cudaSuccess;
+    // copy out: the chunk's O rows of every batch entry, and its LSE columns
+    // of every (batch entry, query head) row
+    ok = ok && cudaStreamWaitEvent(sout, comp_done[c], 0) == cudaSuccess;
+    for (size_t b = 0; ok && b < static_cast<size_t>(d.B); ++b)
+      ok = cudaMemcpyAsync(reinterpret_cast<uint8_t*>(o) + (b * S + t0) * qtok,
+                           reinterpret_cast<const uint8_t*>(dout) + (b * S + t0) * qtok, nt * qtok,
+                           cudaMemcpyDeviceToHost, sout) == cudaSuccess;
+    ok = ok && cudaMemcpy2DAsync(lse + t0, S * 4, dlse + t0, S * 4, nt * 4, static_cast<size_t>(d.B) * Hq,
+                                 cudaMemcpyDeviceToHost, sout) == cudaSuccess;
   }
   // the caller's stream continues after the last copies; copy-in waits too, so
   // a later call cannot overwrite buffers still being read

@@ -14,11 +14,12 @@
 namespace ssa {
 
 struct PoolParams {
-  const __nv_bfloat16* k;
-  const __nv_bfloat16* q;  // may be null
+  const __nv_bfloat16* k;  // may be null (queries only)
+  const __nv_bfloat16* q;  // may be null (keys only)
   float* kbar;
   float* qbar;  // may be null
   int S, Hq, Hkv, G, n;
+  int j0;       // the grid's first block (blocks j0 .. j0 + gridDim.x - 1)
 };
 
 __device__ __forceinline__ void add_bf16x8(float (&acc)[8], const uint4 v) {
@@ -84,10 +85,11 @@ __global__ void __launch_bounds__(PoolConfig<D>::THREADS, PoolConfig<D>::MIN_CTA
   __shared__ float partk[32 * C::KW][9];
   pdl_launch_dependents();
   pdl_wait();
-  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int j = p.j0 + static_cast<int>(blockIdx.x), h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x;
   const size_t out_off = ((static_cast<size_t>(b) * p.Hkv + h) * p.n + j) * D;
   const bool with_q = p.q != nullptr && p.qbar != nullptr;
+  const bool with_k = p.k != nullptr && p.kbar != nullptr;
   const int chq = p.G * D / 8, ntlq = 256 / chq;
   float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   if (tid < 256) {
@@ -103,7 +105,7 @@ __global__ void __launch_bounds__(PoolConfig<D>::THREADS, PoolConfig<D>::MIN_CTA
     }
 #pragma unroll
     for (int e = 0; e < 8; ++e) partq[tid][e] = acc[e];
-  } else {
+  } else if (with_k) {
     const int tk = tid - 256;
     const __nv_bfloat16* kbase =
         p.k + ((static_cast<size_t>(b) * p.S + 64 * j) * p.Hkv + h) * D + (tk % C::CHK) * 8;
@@ -118,10 +120,12 @@ __global__ void __launch_bounds__(PoolConfig<D>::THREADS, PoolConfig<D>::MIN_CTA
     for (int e = 0; e < 8; ++e) partk[tk][e] = acc[e];
   }
   __syncthreads();
-  for (int d = tid; d < D; d += C::THREADS) {
-    float s = 0.f;
-    for (int l = 0; l < C::KTL; ++l) s += partk[l * C::CHK + d / 8][d % 8];
-    p.kbar[out_off + d] = s * (1.0f / 64.0f);
+  if (with_k) {
+    for (int d = tid; d < D; d += C::THREADS) {
+      float s = 0.f;
+      for (int l = 0; l < C::KTL; ++l) s += partk[l * C::CHK + d / 8][d % 8];
+      p.kbar[out_off + d] = s * (1.0f / 64.0f);
+    }
   }
   if (with_q) {
     const float inv = 1.0f / (64.0f * static_cast<float>(p.G));
@@ -139,6 +143,7 @@ struct SelectParams {
   const float* kbar;
   int32_t* idx;
   int n, topk;
+  int i0, i1;  // rows i0 .. i1 - 1 (query blocks); the grid covers them in fours
 };
 
 constexpr int kSelectWarps = 4;
@@ -196,13 +201,13 @@ __global__ void __launch_bounds__(32 * kSelectWarps) block_select_kernel(const S
   pdl_wait();
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int bh = blockIdx.y;
-  const int i = blockIdx.x * kSelectWarps + warp;
-  const bool valid = i < p.n;
+  const int i = p.i0 + static_cast<int>(blockIdx.x) * kSelectWarps + warp;
+  const bool valid = i < p.i1;
   const bool active = valid && i + 1 > p.topk;  // needs a real selection
   int32_t* out = p.idx + (static_cast<size_t>(bh) * p.n + i) * p.topk;
   if (valid && !active)  // every causal block
     for (int r = lane; r < p.topk; r += 32) out[r] = (r <= i) ? r : -1;
-  const int imax = min(p.n - 1, static_cast<int>(blockIdx.x) * kSelectWarps + kSelectWarps - 1);
+  const int imax = min(p.i1 - 1, p.i0 + static_cast<int>(blockIdx.x) * kSelectWarps + kSelectWarps - 1);
   const int need_rows = (imax + 1 > p.topk) ? imax : 0;  // CTA-uniform
   if (need_rows == 0) return;
 

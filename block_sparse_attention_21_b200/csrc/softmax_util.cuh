@@ -14,6 +14,9 @@ constexpr int kDashMaxG = 16;
 
 struct FwdParams {
   int B, S, Hq, Hkv, G, n, topk, slices;
+  // the plain (persistent) sparse stream computes query blocks i_lo .. i_hi - 1
+  // only (0 .. n - 1 from the C entry points); the other modes use 0, n
+  int i_lo, i_hi;
   float scale_log2;  // softmax scale * log2(e)
   const int32_t* idx;
   __nv_bfloat16* o;      // sparse output

@@ -120,21 +120,23 @@ ssa_status ssa_sparse_attn_fwd(const ssa_problem *p, const ssa_bf16 *q, const ss
                                float *lse, ssa_stream stream);
 
 /* Bytes of device workspace ssa_sparse_attn_fwd_host needs for problem p (0
- * on an invalid problem): K and V whole, and two buffer sets of one (batch,
- * KV head) unit. */
+ * on an invalid problem): device copies of Q, K, V, O and LSE whole, the
+ * pooled keys and queries, and the index table. */
 size_t ssa_sparse_attn_fwd_host_workspace(const ssa_problem *p);
 
 /* ssa_block_pool, ssa_block_select and ssa_sparse_attn_fwd on HOST buffers:
  * q [B][S][Hq][D], k and v [B][S][Hkv][D] bf16 in, o [B][S][Hq][D] bf16 and
  * lse [B][Hq][S] fp32 out, all in host memory (page-locked, or the copies do
- * not overlap).  The work is split into B * Hkv units of one batch entry and
- * one KV head, processed in two device buffer sets of `workspace` (caller-
- * owned, >= ssa_sparse_attn_fwd_host_workspace(p) bytes, 256-byte aligned):
- * K and V are first copied whole; then a unit's Q is copied in (a strided
- * 2-D copy) on an internal stream while the previous unit is computed on
- * `stream` (its K and V rows gathered on the device first) and the one
- * before is copied out on a second internal stream, so both copy directions
- * and the kernels overlap.  The results equal the device-buffer calls bit for bit.
+ * not overlap).  `workspace` is caller-owned device memory of at least
+ * ssa_sparse_attn_fwd_host_workspace(p) bytes, 256-byte aligned.  K and V are
+ * copied in whole and the keys pooled; then the query blocks stream through
+ * in chunks of consecutive blocks (every batch entry and head; at least 8 MB
+ * of Q per chunk, at most sixteen chunks):
+ * a chunk's Q rows are copied in on an internal stream, its queries pooled,
+ * its rows selected and attended on `stream`, and its O rows and LSE columns
+ * copied out on a second internal stream, so both copy directions and the
+ * kernels of neighbouring chunks overlap.  The results equal the
+ * device-buffer calls bit for bit.
  * `stream` is ordered after everything before the call and waits for the
  * last copy out, so synchronising it makes o and lse valid on the host.
  * Not capturable in a CUDA graph.  Errors: INVALID_ARG for null pointers,

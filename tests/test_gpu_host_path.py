@@ -1,7 +1,8 @@
 """GPU check of ssa_sparse_attn_fwd_host, the pipelined host-buffer forward:
 its outputs must equal the device-buffer calls (ssa_block_pool,
 ssa_block_select, ssa_sparse_attn_fwd) bit for bit, since it runs the same
-kernels on one (batch, KV head) unit at a time."""
+kernels over chunks of consecutive query blocks (the last chunk may be
+shorter)."""
 import pytest
 import torch
 
@@ -22,7 +23,7 @@ def _built():
 
 
 @pytest.mark.parametrize("case", [(1, 2048, 8, 2, 64, 6), (2, 1280, 4, 2, 128, 5), (3, 1024, 16, 1, 64, 4),
-                                  (1, 8192, 32, 4, 64, 16)],
+                                  (1, 8192, 32, 4, 64, 16), (1, 4480, 32, 4, 64, 16), (1, 4096, 16, 2, 128, 8)],
                          ids=lambda c: "x".join(map(str, c)))
 def test_host_path_equals_device_path(case):
     B, S, Hq, Hkv, D, topk = case
