@@ -49,7 +49,7 @@ CASES = [
     (1, 65536, 4, 1, 128, 32, [65536]),             # 1024 blocks: scored by a grid of their own
     (2, 4096, 8, 2, 64, 16, [1024, 1025]),          # 16 blocks: all kept; 17: the search
     (2, 8192, 8, 2, 64, 64, [4096, 8192]),          # 64 blocks: all kept; 128: the search
-    (1, 16384, 8, 2, 64, 96, [16384]),              # a budget of 96: 95 candidates per cluster, radix pick
+    (1, 16384, 8, 2, 64, 96, [16384]),              # a budget of 96: all 255 blocks are candidates, radix pick
     (64, 2048, 8, 4, 64, 8, None),                  # 256 (b, KV head) rows: one CTA each
     (48, 4096, 16, 4, 128, 16, None),               # head_dim 128, one CTA per row
 ]
