@@ -557,10 +557,15 @@ struct DqConfig {
   static constexpr int QTILE = 128 * D * 2;
   static constexpr int KVT = 64 * D * 2;
   static constexpr int NS = (D == 64) ? 4 : 2;
-  static constexpr int TSTRIDE = 128 + D;      // S (dS over it) +0, dP +64, dQ +128
+  // SEP: dS in TMEM columns of its own (S +0, dP +64, dQ +128, dS +128 + D),
+  // so the next block's S and dP need only wait for S and dP to be read;
+  // else dS over S's first columns (S +0, dP +64, dQ +128)
+  static constexpr bool SEP = (D == 64);
+  static constexpr int DS_COL = 128 + D;
+  static constexpr int TSTRIDE = 128 + D + (SEP ? 32 : 0);
   static constexpr int TMEM_COLS = pow2_at_least(T * TSTRIDE);
   static constexpr int THREADS = 128 * (T + 1);
-  static constexpr int NBARS = 1 + 3 * NS + 3 * T + 1;
+  static constexpr int NBARS = 1 + 3 * NS + 5 * T + 1;
   static constexpr int SMEM_BYTES = 1024 + 2 * T * QTILE + 2 * NS * KVT + NBARS * 8 + 16;
   // two CTAs share an SM when both fit in TMEM and shared memory: one CTA's
   // prologue and epilogue overlap the other's main loop
@@ -574,9 +579,14 @@ struct DqConfig {
 //   issuer:      wait dS_t(jj);  dQ_t += dS_t(jj) K(jj);  S_t = Q_t K(jj+1)^T,
 //                dP_t = dO_t V(jj+1)^T
 //   elementwise: S_t, dP_t -> P = exp2(S scale log2e - LSE log2e),
-//                dS = P (dP - D) -> bf16 over S's first 32 TMEM columns.
-// dS(jj) is overwritten by S(jj+1) only after the dQ MMA read it (the tensor
-// pipe runs one thread's MMAs in issue order).
+//                dS = P (dP - D) -> bf16 into TMEM.
+// At head_dim 64 (SEP) dS has TMEM columns of its own: the issuer issues
+// S(jj+1) and dP(jj+1) as soon as the elementwise warps have loaded S(jj) and
+// dP(jj) (s_free), then dQ(jj) once dS(jj) is stored; the elementwise warps
+// store dS(jj+1) once the dQ MMAs of jj have read dS(jj) (ds_free).  So the
+// next block's score MMAs overlap this block's exponentials.  At head_dim 128
+// dS goes over S's first 32 columns, and S(jj+1) is issued after dQ(jj) (the
+// tensor pipe runs one thread's MMAs in issue order).
 template <int D, int T_>
 __global__ void __launch_bounds__(DqConfig<D, T_>::THREADS, DqConfig<D, T_>::MIN_CTAS)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -599,7 +609,9 @@ __global__ void __launch_bounds__(DqConfig<D, T_>::THREADS, DqConfig<D, T_>::MIN
   uint64_t* s_full = kv_empty + NS;    // [T]
   uint64_t* ds_full = s_full + T;      // [T]
   uint64_t* q_done = ds_full + T;      // [T] last dQ MMA completed
-  uint64_t* drain = q_done + T;
+  uint64_t* s_free = q_done + T;       // [T] SEP: S and dP read into registers
+  uint64_t* ds_free = s_free + T;      // [T] SEP: the dQ MMAs of the block read dS
+  uint64_t* drain = ds_free + T;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -626,6 +638,8 @@ __global__ void __launch_bounds__(DqConfig<D, T_>::THREADS, DqConfig<D, T_>::MIN
       mbar_init(&s_full[t], 1);
       mbar_init(&ds_full[t], 128);
       mbar_init(&q_done[t], 1);
+      mbar_init(&s_free[t], 128);
+      mbar_init(&ds_free[t], 1);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -712,22 +726,34 @@ __global__ void __launch_bounds__(DqConfig<D, T_>::THREADS, DqConfig<D, T_>::MIN
                      !mbar_wait(&v_full[st1], ((jj + 1) / NS) & 1, abort_flag, tmo, 0xc05)))
           break;
         for (int t = 0; t < T; ++t) {
+          const uint32_t tS = tmem + t * TS;
+          if (C::SEP && more) {
+            // the next block's S and dP once this block's are in registers
+            if (!mbar_wait(&s_free[t], jj & 1, abort_flag, tmo, 0xc07)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_scores(t, st1);
+            tc_commit(&s_full[t]);
+          }
           if (!mbar_wait(&ds_full[t], jj & 1, abort_flag, tmo, 0xc06)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t tS = tmem + t * TS;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t bd = sdesc_sw128(aK + st * KVT + kk * (16 * 128), 64 * 128, 1024);
-            mma_ts(tS + 128, tS + kk * 8, bd, idesc_dq, (jj == 0 && kk == 0) ? 0u : 1u);
+            mma_ts(tS + 128, tS + (C::SEP ? C::DS_COL : 0) + kk * 8, bd, idesc_dq, (jj == 0 && kk == 0) ? 0u : 1u);
           }
-          if (more) {
+          if (!more) {
+            tc_commit(&q_done[t]);
+          } else if (C::SEP) {
+            tc_commit(&ds_free[t]);
+          } else {
             issue_scores(t, st1);
             tc_commit(&s_full[t]);
-          } else {
-            tc_commit(&q_done[t]);
           }
         }
         if (!ok) break;
@@ -765,6 +791,10 @@ __global__ void __launch_bounds__(DqConfig<D, T_>::THREADS, DqConfig<D, T_>::MIN
       tmem_ld32_to(row + 32, s + 32);
       tmem_ld32_to(row + 64, dp);
       tmem_ld32_to(row + 96, dp + 32);
+      if (C::SEP) {  // S and dP are in registers: the next block's may be issued
+        tc_fence_before();
+        mbar_arrive(&s_free[t]);
+      }
       const bool diag = (jj == nblk - 1);
       uint32_t dd[32];
 #pragma unroll
@@ -776,7 +806,17 @@ __global__ void __launch_bounds__(DqConfig<D, T_>::THREADS, DqConfig<D, T_>::MIN
         }
         dd[c / 2] = pack_bf16x2(p0 * (dp[c] - dt), p1 * (dp[c + 1] - dt));
       }
-      tmem_st32(row, dd);  // dS (bf16 pairs) over S columns 0..31, already read
+      if (C::SEP) {
+        // dS into its own columns once the previous block's dQ MMAs read them
+        if (jj > 0 && !__all_sync(0xffffffffu, mbar_wait(&ds_free[t], (jj - 1) & 1, abort_flag, tmo, 0xd03))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        tmem_st32(row + C::DS_COL, dd);
+      } else {
+        tmem_st32(row, dd);  // dS (bf16 pairs) over S columns 0..31, already read
+      }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&ds_full[t]);
