@@ -155,6 +155,12 @@ def test_small_problems_every_row(shape):
     ov, lv = _rows_of(o, lse, rows)
     assert np.abs(ov - ref["o_sparse"])[same].max() <= O_TOL
     assert np.abs(lv - ref["lse_sparse"])[same].max() <= LSE_TOL
+    # the same launch on the oracle's own table: every row, none left out
+    otab = torch.from_numpy(np.ascontiguousarray(oidx, dtype=np.int32)).to(DEV)
+    o2, lse2 = _gpu_sparse(p, q, k, v, otab, pad=4096)
+    ov2, lv2 = _rows_of(o2, lse2, rows)
+    assert np.abs(ov2 - ref["o_sparse"]).max() <= O_TOL
+    assert np.abs(lv2 - ref["lse_sparse"]).max() <= LSE_TOL
     # the dense counterpart costs O(S^2) in the oracle: every row up to 2k
     # tokens, a sample (with whole first and last query blocks) beyond
     if S > 2048:
@@ -170,6 +176,13 @@ def test_small_problems_every_row(shape):
     assert np.abs(fov - ref["o_full"]).max() <= O_TOL
     assert np.abs(flv - ref["lse_full"]).max() <= LSE_TOL
     assert np.abs(dmv - ref["delta"])[same].max() <= DELTA_TOL
+    # on the oracle's own table: every row, none left out
+    mo2, ml2, _, _, mdm2 = _gpu_mass(p, q, k, v, otab)
+    mov2, mlv2 = _rows_of(mo2, ml2, rows)
+    _, dmv2 = _rows_of(mo2, mdm2, rows)
+    assert np.abs(mov2 - ref["o_sparse"]).max() <= O_TOL
+    assert np.abs(mlv2 - ref["lse_sparse"]).max() <= LSE_TOL
+    assert np.abs(dmv2 - ref["delta"]).max() <= DELTA_TOL
 
 
 def test_tiny_workload_every_row_and_deterministic():

@@ -2,12 +2,16 @@
 its outputs must equal the device-buffer calls (ssa_block_pool,
 ssa_block_select, ssa_sparse_attn_fwd) bit for bit, since it runs the same
 kernels over chunks of consecutive query blocks (the last chunk may be
-shorter)."""
+shorter).  Its host buffers are also checked against the fp64 oracle on
+sampled rows (max-abs 2e-2 for O, 1e-3 for LSE)."""
+import numpy as np
 import pytest
 import torch
 
 import block_sparse_attention_21_b200 as ssa
 import gen
+import oracle
+from conftest import same_table_rows
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -39,3 +43,22 @@ def test_host_path_equals_device_path(case):
     assert ssa.ssa_get_device_error() == 0
     assert torch.equal(ho.view(torch.int16), st.o.cpu().view(torch.int16))
     assert torch.equal(hl, st.lse.cpu())
+    # against the oracle: random rows plus every row of the first and last
+    # query blocks (batch 0, query head 0), where both tables hold the same row
+    n = S // 64
+    rng = np.random.Generator(np.random.PCG64(S + D))
+    rows = [np.stack([rng.integers(0, B, 400), rng.integers(0, Hq, 400), rng.integers(0, S, 400)], axis=1)]
+    for blk in (0, n - 1):
+        t = np.arange(64 * blk, 64 * blk + 64)
+        rows.append(np.stack([np.zeros_like(t), np.zeros_like(t), t], axis=1))
+    rows = np.concatenate(rows).astype(np.int64)
+    okb, oqb = oracle.block_pool(x.k, x.q)
+    oidx, _ = oracle.block_select(oqb, okb, topk)
+    same = same_table_rows(rows, st.block_idx.cpu().numpy(), oidx, Hq // Hkv)
+    assert same.mean() > 0.5
+    ref = oracle.attn_rows(x.q, x.k, x.v, oidx, rows, want_full=False)
+    b_, h_, t_ = rows[:, 0], rows[:, 1], rows[:, 2]
+    go = ho.float().numpy()[b_, t_, h_]
+    gl = hl.numpy()[b_, h_, t_]
+    assert np.abs(go - ref["o_sparse"])[same].max() <= 2e-2
+    assert np.abs(gl - ref["lse_sparse"])[same].max() <= 1e-3

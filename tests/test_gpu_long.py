@@ -81,6 +81,16 @@ def test_long_sequence_forward_and_backward(shape):
     gl = st.lse[r[:, 0], r[:, 1], r[:, 2]].cpu().numpy()
     assert np.abs(go - ref["o_sparse"])[same].max() <= 2e-2
     assert np.abs(gl - ref["lse_sparse"])[same].max() <= 1e-3
+    # the forward on the oracle's own table: every sampled row, none left out
+    otab = torch.from_numpy(np.ascontiguousarray(oidx, dtype=np.int32)).to(DEV)
+    o2, l2 = torch.empty_like(st.o), torch.empty_like(st.lse)
+    ssa.ssa_sparse_attn_fwd(p, q, k, v, otab, o2, l2)
+    torch.cuda.synchronize()
+    assert ssa.ssa_get_device_error() == 0
+    go2 = o2[r[:, 0], r[:, 2], r[:, 1]].float().cpu().numpy()
+    gl2 = l2[r[:, 0], r[:, 1], r[:, 2]].cpu().numpy()
+    assert np.abs(go2 - ref["o_sparse"]).max() <= 2e-2
+    assert np.abs(gl2 - ref["lse_sparse"]).max() <= 1e-3
 
     # sparse backward: repeatable bit for bit, sampled against the oracle
     dq, dk, dv = (t.clone() for t in st.backward(q, k, v, do))
