@@ -24,7 +24,8 @@
 //   bwd_dkdv_reduce_kernel  adds the partials in a fixed order into dK, dV.
 //   attn_bwd_dq_kernel one CTA per (batch, KV head, query block, head pairs):
 //                      walks the selected blocks like the forward; dS goes to
-//                      TMEM over S and dQ += dS K_j reads it as the A operand.
+//                      TMEM (columns of its own at head_dim 64, over S at 128)
+//                      and dQ += dS K_j reads it as the A operand.
 #pragma once
 
 #include "sm100.cuh"
