@@ -750,3 +750,39 @@ def test_dash_attention_maximises_score_minus_kl_to_the_prior():
             d[sup] -= d[sup].mean()
             eps = 0.2 * p[sup].min() / (np.abs(d).max() + 1e-30)
             assert F(p + eps * d) <= best + 1e-12
+
+
+def test_receptive_field_is_the_guides_figure():
+    # The guide's receptive fields (tests/golden/receptive_field.json) at
+    # 64-token blocks: k = rf / 64 kept blocks, the diagonal among them.  With
+    # one-hot values the sparse output row is the attention row, so its
+    # nonzero entries are the keys the query sees: every earlier kept block in
+    # full plus the diagonal block up to the query.  A query block with at
+    # least k earlier blocks then sees 64 (k - 1) + (t mod 64) + 1 keys, and
+    # its last row exactly the receptive field.
+    import json
+    import os
+    with open(os.path.join(os.path.dirname(__file__), "golden", "receptive_field.json")) as f:
+        fx = json.load(f)
+    assert fx["block_size"] == BS
+    for rf in fx["receptive_fields"]:
+        topk = rf // BS
+        S = BS * (topk + 1)              # the last block has k earlier blocks to choose from
+        q, k, _ = _tiny(1, S, 1, 1, S, seed=rf)
+        v = np.eye(S)[None, :, None, :]
+        kbar, qbar = oracle.block_pool(k, q)
+        idx, _ = oracle.block_select(qbar, kbar, topk)
+        n = S // BS
+        rows = np.array([[0, 0, t] for t in range(BS * (n - 2), S)], dtype=np.int64)
+        p = oracle.attn_rows(q, k, v, idx, rows, want_full=False)["o_sparse"]
+        seen = (p > 0).sum(axis=1)
+        t = rows[:, 2]
+        assert np.array_equal(seen, BS * (topk - 1) + t % BS + 1)
+        assert seen.max() == rf
+        np.testing.assert_allclose(p.sum(axis=1), 1.0, atol=1e-12)
+        # the last block drops exactly one earlier block: the one it did not select
+        last = p[-BS:]
+        dropped = [j for j in range(n - 1) if j not in idx[0, 0, n - 1]]
+        assert len(dropped) == 1
+        j = dropped[0]
+        assert np.all(last[:, BS * j:BS * j + BS] == 0)
