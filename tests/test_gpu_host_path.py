@@ -27,7 +27,8 @@ def _built():
 
 
 @pytest.mark.parametrize("case", [(1, 2048, 8, 2, 64, 6), (2, 1280, 4, 2, 128, 5), (3, 1024, 16, 1, 64, 4),
-                                  (1, 8192, 32, 4, 64, 16), (1, 4480, 32, 4, 64, 16), (1, 4096, 16, 2, 128, 8)],
+                                  (1, 8192, 32, 4, 64, 16), (1, 4480, 32, 4, 64, 16), (1, 4096, 16, 2, 128, 8),
+                                  (2, 4096, 32, 4, 64, 16)],   # B = 2 in four chunks
                          ids=lambda c: "x".join(map(str, c)))
 def test_host_path_equals_device_path(case):
     B, S, Hq, Hkv, D, topk = case
